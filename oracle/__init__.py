@@ -1,0 +1,180 @@
+"""fp64 CPU oracle for multi-dimensional local attention -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never loads it and shares no code with it.
+
+The arithmetic lives in ``na_oracle.c`` (plain C, fp64, dense mask per query);
+this module compiles it with gcc and marshals numpy arrays through ctypes.
+Definitions and sources are stated at the top of ``na_oracle.c``:
+softmax(QK^T/sqrt(d))V restricted to the window ("pi-Attention", section 3.1
+eqs. (1)-(3), section 3.2 eqs. (4)-(5)), with the window centred on the query's
+stride group and clamped inside the grid ("Generalized Neighborhood Attention"
+abstract; "ENA" sliding tile attention).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(_HERE, "na_oracle.c")
+LIB = os.path.join(_HERE, "libna_oracle.so")
+_lock = threading.Lock()
+_libs: dict[str, "OracleLib"] = {}
+
+
+def compile_lib(src: str, out: str) -> str:
+    """Compile an oracle source file into a shared library (gcc -O2, no fast-math)."""
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                           "-o", tmp, src, "-lm"])
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        compile_lib(SRC, LIB)
+    return LIB
+
+
+class OracleLib:
+    """ctypes view of one compiled oracle library (the real one, or a test mutant)."""
+
+    def __init__(self, path: str):
+        lib = ctypes.CDLL(path)
+        i32p = ctypes.POINTER(ctypes.c_int)
+        lib.na_oracle_window_start.argtypes = [ctypes.c_int] * 4
+        lib.na_oracle_window_start.restype = ctypes.c_int
+        lib.na_oracle_mask_row.argtypes = [ctypes.c_int, i32p, i32p, i32p, ctypes.c_longlong,
+                                           ctypes.c_void_p]
+        lib.na_oracle_mask_row.restype = ctypes.c_int
+        lib.na_oracle_forward.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong,
+            ctypes.c_int, i32p, i32p, i32p, ctypes.c_int, ctypes.c_double,
+            ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        lib.na_oracle_forward.restype = ctypes.c_int
+        lib.na_oracle_block_counts.argtypes = [ctypes.c_int, i32p, i32p, i32p, ctypes.c_longlong,
+                                               ctypes.c_void_p]
+        lib.na_oracle_block_counts.restype = ctypes.c_int
+        self.lib = lib
+        self.path = path
+
+    @staticmethod
+    def _ivec(vals):
+        vals = [int(x) for x in vals]
+        return (ctypes.c_int * len(vals))(*vals)
+
+    # -- window rule -------------------------------------------------------
+    def window_start(self, L: int, w: int, s: int, i: int) -> int:
+        r = self.lib.na_oracle_window_start(L, w, s, i)
+        if r < 0:
+            raise ValueError(f"invalid window arguments L={L} w={w} s={s} i={i}")
+        return r
+
+    def mask_row(self, grid, window, stride, token: int) -> np.ndarray:
+        grid, window, stride = _geom(grid, window, stride)
+        n = int(np.prod(grid))
+        out = np.zeros(n, dtype=np.uint8)
+        rc = self.lib.na_oracle_mask_row(len(grid), self._ivec(grid), self._ivec(window),
+                                         self._ivec(stride), int(token), out.ctypes.data)
+        if rc:
+            raise ValueError("na_oracle_mask_row: invalid arguments")
+        return out.astype(bool)
+
+    # -- forward -----------------------------------------------------------
+    def forward(self, q, k, v, grid, window, stride, *, dtype: str, rows=None,
+                scale: float = 0.0, threads: int | None = None):
+        """Exact forward in fp64.
+
+        q, k, v: arrays of shape [B, heads, *grid, d]; float32 values for
+        ``dtype="f32"`` or uint16 bfloat16 bit patterns for ``dtype="bf16"``.
+        rows: None for every query, else int64 global row ids (bh * N + token).
+        Returns (out [nrows, d] float64, lse [nrows] float64); with rows=None
+        out is reshaped to q's shape and lse to q's shape without d.
+        """
+        grid, window, stride = _geom(grid, window, stride)
+        want = np.float32 if dtype == "f32" else np.uint16
+        arrs = [np.ascontiguousarray(a) for a in (q, k, v)]
+        for a in arrs:
+            if a.dtype != want:
+                raise TypeError(f"oracle expects {want} arrays for dtype={dtype}")
+            if a.shape != arrs[0].shape:
+                raise ValueError("q, k, v shapes differ")
+        shape = arrs[0].shape
+        nd = len(grid)
+        if tuple(shape[2:2 + nd]) != tuple(grid) or len(shape) != nd + 3:
+            raise ValueError(f"tensor shape {shape} does not match grid {grid}")
+        BH = shape[0] * shape[1]
+        d = shape[-1]
+        N = int(np.prod(grid))
+        if rows is None:
+            nrows = BH * N
+            rows_ptr = None
+        else:
+            rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+            nrows = rows.size
+            rows_ptr = rows.ctypes.data
+        out = np.empty((nrows, d), dtype=np.float64)
+        lse = np.empty(nrows, dtype=np.float64)
+        rc = self.lib.na_oracle_forward(
+            arrs[0].ctypes.data, arrs[1].ctypes.data, arrs[2].ctypes.data,
+            0 if dtype == "f32" else 1, BH, nd, self._ivec(grid), self._ivec(window),
+            self._ivec(stride), d, float(scale), rows_ptr, nrows, out.ctypes.data,
+            lse.ctypes.data, int(threads or os.cpu_count() or 1))
+        if rc:
+            raise RuntimeError(f"na_oracle_forward failed with code {rc}")
+        if rows is None:
+            return out.reshape(shape).astype(np.float64), lse.reshape(shape[:-1])
+        return out, lse
+
+    # -- block counting ------------------------------------------------------
+    def block_counts(self, grid, window, stride, block: int):
+        """(empty, partial, full) blk x blk tiles of the row-major attention map."""
+        grid, window, stride = _geom(grid, window, stride)
+        counts = np.zeros(3, dtype=np.int64)
+        rc = self.lib.na_oracle_block_counts(len(grid), self._ivec(grid), self._ivec(window),
+                                             self._ivec(stride), int(block), counts.ctypes.data)
+        if rc:
+            raise ValueError("na_oracle_block_counts: invalid arguments")
+        return tuple(int(c) for c in counts)
+
+
+def _geom(grid, window, stride):
+    grid = [int(x) for x in grid]
+    window = [int(x) for x in window]
+    stride = [1] * len(grid) if stride is None else [int(x) for x in stride]
+    if not (len(grid) == len(window) == len(stride)):
+        raise ValueError("grid, window and stride must have the same length")
+    return grid, window, stride
+
+
+def load(path: str | None = None) -> OracleLib:
+    """The oracle library at ``path`` (default: the real one, built on demand)."""
+    with _lock:
+        if path is None:
+            path = build()
+        if path not in _libs:
+            _libs[path] = OracleLib(path)
+        return _libs[path]
+
+
+def window_start(L, w, s, i):
+    return load().window_start(L, w, s, i)
+
+
+def mask_row(grid, window, stride, token):
+    return load().mask_row(grid, window, stride, token)
+
+
+def forward(q, k, v, grid, window, stride, **kw):
+    return load().forward(q, k, v, grid, window, stride, **kw)
+
+
+def block_counts(grid, window, stride, block):
+    return load().block_counts(grid, window, stride, block)

@@ -1,0 +1,268 @@
+/*
+ * na_oracle.c -- TEST INFRASTRUCTURE ONLY.
+ *
+ * Plain, slow, fp64 CPU definition of the forward pass of multi-dimensional
+ * local ("generalized neighborhood" / "sliding tile") attention.  Only the
+ * tests, the package's smoke check and the benchmark's CPU-baseline leg may
+ * load this library; the product path never does.  It shares no code with the
+ * CUDA path: its window rule, mask, softmax and block counting are written
+ * here from the pages and from nothing else.
+ *
+ * What it computes, per (batch*head bh, query token i):
+ *   z_ij  = scale * <q_i, k_j>           for every key j in the window of i
+ *   m     = max_j z_ij
+ *   l     = sum_j exp(z_ij - m)
+ *   out_i = sum_j exp(z_ij - m) v_j / l
+ *   lse_i = m + ln l
+ * following "pi-Attention: Online Efficient Sparse Transformers for
+ * Long-Context Modeling", section 3.1 eqs. (1)-(3) (softmax(QK^T/sqrt(d_k))V,
+ * a weighted sum of values) and section 3.2 eq. (4) (pre-softmax score z_ij)
+ * with the sum restricted to the neighbourhood (text after eq. (5)).  The
+ * restriction is evaluated as a dense mask over all N keys of the row, the
+ * convention stated under eq. (34) of the same page (invalid positions get
+ * -inf before the softmax, which is the same as restricting the sum); the
+ * arithmetic is only done where the mask is true, which is identical because
+ * exp(-inf) = 0.
+ *
+ * Window rule (per grid dimension, window w, stride s, length L):
+ *   g     = floor(i / s)                 stride group of coordinate i
+ *   c     = g*s + floor(s/2)             the group's centre ("leader")
+ *   start = clamp(c - floor(w/2), 0, L - w)
+ *   window = [start, start + w)
+ * and the N-d window is the Cartesian product over dimensions.  Sources:
+ * "Generalized Neighborhood Attention: Multi-dimensional Sparse Attention at
+ * the Speed of Light" (abstract: one family covering sliding window, strided
+ * sliding window and blocked attention); "ENA: Efficient N-dimensional
+ * Attention" (the pith, "What carries the argument": tokens within one tile
+ * share a window that shifts tile by tile).  The pages print no formula; the
+ * reading used here (a window centred on the query's stride group and clamped
+ * inside the grid, so that every query sees exactly prod(w) keys) is the
+ * plainest one consistent with both pages.
+ *
+ * Block counting (empty / partial / full tiles of the N x N attention map in
+ * row-major token order) follows "Hilbert-Guided Sparse Local Attention",
+ * "Methodology in Plain English" (tiles labelled full, partial or empty).
+ *
+ * Inputs are read as the exact float32 values, or the exact bfloat16 values
+ * (16-bit patterns widened by a shift), that the GPU receives.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define NA_ORACLE_MAXDIM 3
+
+enum { IN_F32 = 0, IN_BF16 = 1 };
+
+/* ---------------------------------------------------------------- window -- */
+
+int na_oracle_window_start(int L, int w, int s, int i) {
+    if (L < 1 || w < 1 || w > L || s < 1 || s > w || i < 0 || i >= L) return -1;
+    int g = i / s;
+    int c = g * s + s / 2;
+    int start = c - w / 2;
+    if (start < 0) start = 0;
+    if (start > L - w) start = L - w;
+    return start;
+}
+
+static int check_geometry(int ndim, const int* L, const int* w, const int* s, long long* N) {
+    if (ndim < 1 || ndim > NA_ORACLE_MAXDIM || !L || !w || !s) return -1;
+    long long n = 1;
+    for (int a = 0; a < ndim; ++a) {
+        if (L[a] < 1 || w[a] < 1 || w[a] > L[a] || s[a] < 1 || s[a] > w[a]) return -1;
+        n *= L[a];
+    }
+    *N = n;
+    return 0;
+}
+
+static void unflatten(long long t, int ndim, const int* L, int* coord) {
+    for (int a = ndim - 1; a >= 0; --a) {
+        coord[a] = (int)(t % L[a]);
+        t /= L[a];
+    }
+}
+
+/* Dense membership row: mask[j] = 1 iff key token j is in the window of query token t. */
+int na_oracle_mask_row(int ndim, const int* L, const int* w, const int* s, long long t,
+                       uint8_t* mask) {
+    long long N;
+    if (check_geometry(ndim, L, w, s, &N) || t < 0 || t >= N || !mask) return -1;
+    int qi[NA_ORACLE_MAXDIM], ws[NA_ORACLE_MAXDIM], kj[NA_ORACLE_MAXDIM];
+    unflatten(t, ndim, L, qi);
+    for (int a = 0; a < ndim; ++a) ws[a] = na_oracle_window_start(L[a], w[a], s[a], qi[a]);
+    for (int a = 0; a < ndim; ++a) kj[a] = 0;
+    for (long long j = 0; j < N; ++j) {
+        int in = 1;
+        for (int a = 0; a < ndim; ++a)
+            if (kj[a] < ws[a] || kj[a] >= ws[a] + w[a]) in = 0;
+        mask[j] = (uint8_t)in;
+        for (int a = ndim - 1; a >= 0; --a) { /* advance the row-major key counter */
+            if (++kj[a] < L[a]) break;
+            kj[a] = 0;
+        }
+    }
+    return 0;
+}
+
+/* --------------------------------------------------------------- forward -- */
+
+static inline double load_in(const void* p, int dtype, size_t idx) {
+    if (dtype == IN_F32) return (double)((const float*)p)[idx];
+    uint32_t bits = (uint32_t)((const uint16_t*)p)[idx] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+typedef struct {
+    const void *q, *k, *v;
+    int dtype, ndim, d;
+    const int *L, *w, *s;
+    long long N, BH, W;
+    double scale;
+    const long long* rows;
+    long long r_begin, r_end;
+    double *out, *lse;
+    int status;
+} fwd_job;
+
+static void* fwd_worker(void* arg) {
+    fwd_job* J = (fwd_job*)arg;
+    const int ndim = J->ndim, d = J->d;
+    const long long N = J->N;
+    double* z = (double*)malloc(sizeof(double) * (size_t)J->W);
+    long long* idx = (long long*)malloc(sizeof(long long) * (size_t)J->W);
+    uint8_t* mask = (uint8_t*)malloc((size_t)N);
+    double* acc = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!z || !idx || !mask || !acc) {
+        J->status = -2;
+        goto done;
+    }
+    for (long long r = J->r_begin; r < J->r_end; ++r) {
+        long long row = J->rows ? J->rows[r] : r;
+        if (row < 0 || row >= J->BH * N) { J->status = -1; break; }
+        long long bh = row / N, t = row % N;
+        na_oracle_mask_row(ndim, J->L, J->w, J->s, t, mask);
+        size_t qoff = (size_t)row * (size_t)d;
+        long long cnt = 0;
+        for (long long j = 0; j < N; ++j) {
+            if (!mask[j]) continue;
+            if (cnt >= J->W) { J->status = -3; goto done; }
+            size_t koff = ((size_t)bh * (size_t)N + (size_t)j) * (size_t)d;
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c)
+                dot += load_in(J->q, J->dtype, qoff + c) * load_in(J->k, J->dtype, koff + c);
+            z[cnt] = J->scale * dot;
+            idx[cnt] = j;
+            ++cnt;
+        }
+        if (cnt != J->W) { J->status = -3; goto done; } /* every query sees prod(w) keys */
+        double m = -INFINITY;
+        for (long long e = 0; e < cnt; ++e) if (z[e] > m) m = z[e];
+        double l = 0.0;
+        for (long long e = 0; e < cnt; ++e) l += exp(z[e] - m);
+        for (int c = 0; c < d; ++c) acc[c] = 0.0;
+        for (long long e = 0; e < cnt; ++e) {
+            double p = exp(z[e] - m) / l;
+            size_t voff = ((size_t)bh * (size_t)N + (size_t)idx[e]) * (size_t)d;
+            for (int c = 0; c < d; ++c) acc[c] += p * load_in(J->v, J->dtype, voff + c);
+        }
+        for (int c = 0; c < d; ++c) J->out[(size_t)r * (size_t)d + c] = acc[c];
+        J->lse[r] = m + log(l);
+    }
+done:
+    free(z);
+    free(idx);
+    free(mask);
+    free(acc);
+    return NULL;
+}
+
+/*
+ * q, k, v: [BH, N, d] with the N tokens in row-major grid order (last grid
+ * dimension fastest), float32 (in_dtype 0) or bfloat16 bit patterns (1).
+ * rows: NULL for every row 0..BH*N-1 (then nrows must be BH*N), else a list
+ * of global row indices bh*N + token.  out: [nrows, d] fp64; lse: [nrows] fp64.
+ * scale <= 0 means 1/sqrt(d).  Returns 0, or a negative code on bad input
+ * (-1), allocation failure (-2) or a window that does not hold prod(w) keys (-3).
+ */
+int na_oracle_forward(const void* q, const void* k, const void* v, int in_dtype, long long BH,
+                      int ndim, const int* L, const int* w, const int* s, int d, double scale,
+                      const long long* rows, long long nrows, double* out, double* lse,
+                      int nthreads) {
+    long long N;
+    if (!q || !k || !v || !out || !lse || BH < 1 || d < 1 || nrows < 0) return -1;
+    if (in_dtype != IN_F32 && in_dtype != IN_BF16) return -1;
+    if (check_geometry(ndim, L, w, s, &N)) return -1;
+    if (!rows && nrows != BH * N) return -1;
+    long long W = 1;
+    for (int a = 0; a < ndim; ++a) W *= w[a];
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (nthreads > nrows) nthreads = (int)(nrows > 0 ? nrows : 1);
+    fwd_job jobs[256];
+    pthread_t th[256];
+    long long per = (nrows + nthreads - 1) / nthreads;
+    for (int t = 0; t < nthreads; ++t) {
+        fwd_job* J = &jobs[t];
+        J->q = q; J->k = k; J->v = v;
+        J->dtype = in_dtype; J->ndim = ndim; J->d = d;
+        J->L = L; J->w = w; J->s = s;
+        J->N = N; J->BH = BH; J->W = W;
+        J->scale = scale;
+        J->rows = rows;
+        J->r_begin = per * t < nrows ? per * t : nrows;
+        J->r_end = per * (t + 1) < nrows ? per * (t + 1) : nrows;
+        J->out = out; J->lse = lse;
+        J->status = 0;
+    }
+    for (int t = 1; t < nthreads; ++t)
+        if (pthread_create(&th[t], NULL, fwd_worker, &jobs[t]) != 0) {
+            fwd_worker(&jobs[t]);
+            th[t] = 0;
+        }
+    fwd_worker(&jobs[0]);
+    for (int t = 1; t < nthreads; ++t)
+        if (th[t]) pthread_join(th[t], NULL);
+    for (int t = 0; t < nthreads; ++t)
+        if (jobs[t].status) return jobs[t].status;
+    return 0;
+}
+
+/* --------------------------------------------------------- block counts -- */
+
+/*
+ * Cut the N x N attention map (tokens in row-major grid order) into blk x blk
+ * tiles and count empty (no query-key pair in a window), full (every pair in
+ * a window) and partial tiles.  counts[0..2] = {empty, partial, full}.
+ */
+int na_oracle_block_counts(int ndim, const int* L, const int* w, const int* s, long long blk,
+                           long long* counts) {
+    long long N;
+    if (check_geometry(ndim, L, w, s, &N) || blk < 1 || !counts) return -1;
+    long long nb = (N + blk - 1) / blk;
+    long long* members = (long long*)calloc((size_t)(nb * nb), sizeof(long long));
+    uint8_t* mask = (uint8_t*)malloc((size_t)N);
+    if (!members || !mask) { free(members); free(mask); return -2; }
+    for (long long t = 0; t < N; ++t) {
+        na_oracle_mask_row(ndim, L, w, s, t, mask);
+        long long* rowblk = members + (t / blk) * nb;
+        for (long long j = 0; j < N; ++j) rowblk[j / blk] += mask[j];
+    }
+    counts[0] = counts[1] = counts[2] = 0;
+    for (long long a = 0; a < nb; ++a)
+        for (long long b = 0; b < nb; ++b) {
+            long long ra = (a + 1) * blk <= N ? blk : N - a * blk;
+            long long cb = (b + 1) * blk <= N ? blk : N - b * blk;
+            long long m = members[a * nb + b];
+            counts[m == 0 ? 0 : (m == ra * cb ? 2 : 1)] += 1;
+        }
+    free(members);
+    free(mask);
+    return 0;
+}

@@ -1,0 +1,341 @@
+"""Pins for the fp64 oracle: checks against facts that do not come from the
+oracle itself -- values the pages print, closed forms, invariants, special
+cases that reduce to a dense library routine, and brute-force enumeration.
+
+Each ``pin_*`` function takes an ``oracle.OracleLib`` and raises
+``AssertionError`` on a mismatch, so the same set can be run against the real
+oracle (``test_oracle_pins.py``) and against deliberately broken copies of it
+(``test_oracle_mutants.py``), which must each fail at least one pin.
+"""
+from __future__ import annotations
+
+import itertools
+import math
+import os
+
+import numpy as np
+
+import seeded_inputs
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ---------------------------------------------------------------- helpers --
+
+def _dense_attention(q, k, v, scale):
+    """Full softmax attention of one head with numpy matmuls (fp64):
+    softmax(q k^T * scale) v and the row log-sum-exp."""
+    s = (q @ k.T) * scale
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = e.sum(axis=1, keepdims=True)
+    return (e / l) @ v, (m + np.log(l))[:, 0]
+
+
+def _randn(seed, shape):
+    return seeded_inputs.normal_f32(seed, shape, threads=1)
+
+
+def _leader_start(L, w, s, i):
+    """Brute force: among all w-long windows that fit in [0, L), the one whose
+    start is nearest to (leader - floor(w/2)), leader = member floor(s/2) of the
+    stride group of i.  Exhaustive search, no clamp arithmetic."""
+    g = i // s
+    target = g * s + s // 2 - w // 2
+    best = None
+    for a in range(0, L - w + 1):
+        if best is None or abs(a - target) < abs(best - target):
+            best = a
+    return best
+
+
+def _nearest_set(L, w, i):
+    """The w grid positions nearest to i (odd w, no ties possible)."""
+    order = sorted(range(L), key=lambda j: (abs(j - i), j))
+    return set(order[:w])
+
+
+def _window_sets(grid, window, stride):
+    """Per-dimension window start for every coordinate, by brute force."""
+    return [[_leader_start(L, w, s, i) for i in range(L)] for L, w, s in zip(grid, window, stride)]
+
+
+def _brute_mask(grid, window, stride, token):
+    starts = _window_sets(grid, window, stride)
+    coords = np.unravel_index(token, grid)
+    N = int(np.prod(grid))
+    keys = np.array(np.unravel_index(np.arange(N), grid))
+    ok = np.ones(N, dtype=bool)
+    for a, (L, w) in enumerate(zip(grid, window)):
+        st = starts[a][coords[a]]
+        ok &= (keys[a] >= st) & (keys[a] < st + w)
+    return ok
+
+
+# ------------------------------------------------------------------- pins --
+
+def pin_window_bruteforce(lib):
+    """Window start vs exhaustive nearest-feasible-window search, every
+    (L <= 12, 1 <= w <= L, 1 <= s <= w, i)."""
+    for L in range(1, 13):
+        for w in range(1, L + 1):
+            for s in range(1, w + 1):
+                for i in range(L):
+                    got = lib.window_start(L, w, s, i)
+                    assert got == _leader_start(L, w, s, i), (L, w, s, i, got)
+
+
+def pin_window_geometric_centre(lib):
+    """When stride and window have the same parity and no clamping happens,
+    the window's centre equals the centre of the query's stride group."""
+    for L in range(2, 40):
+        for w in range(1, L + 1):
+            for s in range(1, w + 1):
+                if (w - s) % 2:
+                    continue
+                for i in range(L):
+                    g = i // s
+                    start = g * s + (s - w) // 2
+                    if start < 0 or start + w > L:
+                        continue
+                    got = lib.window_start(L, w, s, i)
+                    assert 2 * got + (w - 1) == 2 * g * s + (s - 1), (L, w, s, i, got)
+
+
+def pin_window_neighbourhood_metric(lib):
+    """stride 1, odd w: the window is the set of the w positions nearest to i
+    (neighborhood attention's clamped neighbourhood)."""
+    for L in range(1, 30):
+        for w in range(1, L + 1, 2):
+            for i in range(L):
+                st = lib.window_start(L, w, 1, i)
+                assert set(range(st, st + w)) == _nearest_set(L, w, i), (L, w, i)
+
+
+def pin_window_sliding_tile(lib):
+    """Sliding tile attention: stride = tile t, window = n*t with n odd, t | L.
+    Every query of tile g sees whole tiles g-(n-1)/2 .. g+(n-1)/2, shifted
+    inside the grid at the borders."""
+    for t in range(1, 9):
+        for T in range(1, 9):
+            L = t * T
+            for n in range(1, T + 1, 2):
+                w = n * t
+                for i in range(L):
+                    g = i // t
+                    first_tile = min(max(g - (n - 1) // 2, 0), T - n)
+                    assert lib.window_start(L, w, t, i) == t * first_tile, (t, T, n, i)
+
+
+def pin_window_blocked(lib):
+    """stride = window dividing the grid: non-overlapping blocks."""
+    for w in range(1, 9):
+        for nb in range(1, 7):
+            L = w * nb
+            for i in range(L):
+                assert lib.window_start(L, w, w, i) == (i // w) * w
+
+
+def pin_mask_bruteforce(lib):
+    """Dense mask rows vs brute-force per-dimension membership (2D and 3D)."""
+    cases = [([5, 7], [3, 4], [1, 2]), ([6, 5], [6, 2], [3, 1]), ([3, 4, 5], [2, 3, 3], [1, 3, 2]),
+             ([4, 4, 6], [4, 2, 6], [2, 2, 3])]
+    for grid, window, stride in cases:
+        N = int(np.prod(grid))
+        for t in range(N):
+            got = lib.mask_row(grid, window, stride, t)
+            assert np.array_equal(got, _brute_mask(grid, window, stride, t)), (grid, t)
+            assert got.sum() == int(np.prod(window))
+
+
+def pin_full_attention(lib):
+    """window = whole grid: equals dense softmax attention (numpy matmuls)."""
+    for grid, stride, d, dtype in [([7, 5], [2, 3], 16, "f32"), ([3, 4, 5], [1, 2, 5], 8, "f32"),
+                                   ([23], [1], 12, "bf16")]:
+        B, H = 2, 1
+        shape = (B, H, *grid, d)
+        if dtype == "f32":
+            q, k, v = (_randn(70 + t, shape) for t in range(3))
+            qf, kf, vf = q, k, v
+        else:
+            q, k, v = (seeded_inputs.normal_bf16_bits(80 + t, shape, threads=1) for t in range(3))
+            qf, kf, vf = (seeded_inputs.bf16_bits_to_f32(a) for a in (q, k, v))
+        out, lse = lib.forward(q, k, v, grid, grid, stride, dtype=dtype)
+        N = int(np.prod(grid))
+        for b in range(B):
+            ref_o, ref_l = _dense_attention(qf[b, 0].reshape(N, d).astype(np.float64),
+                                            kf[b, 0].reshape(N, d).astype(np.float64),
+                                            vf[b, 0].reshape(N, d).astype(np.float64),
+                                            1.0 / math.sqrt(d))
+            np.testing.assert_allclose(out[b, 0].reshape(N, d), ref_o, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(lse[b, 0].reshape(N), ref_l, rtol=0, atol=1e-12)
+
+
+def pin_blocked_attention(lib):
+    """stride = window dividing the grid: each block attends densely inside
+    itself (reshape into blocks, numpy dense attention per block)."""
+    for grid, window, d in [([6, 8], [3, 4], 8), ([4, 6, 6], [2, 3, 2], 4)]:
+        shape = (1, 2, *grid, d)
+        q, k, v = (_randn(90 + t, shape) for t in range(3))
+        out, lse = lib.forward(q, k, v, grid, window, window, dtype="f32")
+        nd = len(grid)
+        blocks = [range(L // w) for L, w in zip(grid, window)]
+        for h in range(2):
+            for bidx in itertools.product(*blocks):
+                sl = tuple(slice(bi * w, (bi + 1) * w) for bi, w in zip(bidx, window))
+                qs, ks, vs = (a[0, h][sl].reshape(-1, d).astype(np.float64) for a in (q, k, v))
+                ref_o, ref_l = _dense_attention(qs, ks, vs, 1.0 / math.sqrt(d))
+                np.testing.assert_allclose(out[0, h][sl].reshape(-1, d), ref_o, atol=1e-12, rtol=0)
+                np.testing.assert_allclose(lse[0, h][sl].reshape(-1), ref_l, atol=1e-12, rtol=0)
+        assert nd in (2, 3)
+
+
+def pin_probability_rows(lib):
+    """One-hot values expose the attention row itself: it sums to 1, its
+    support is exactly the brute-force window, and on the support it equals a
+    softmax of numpy-computed scores."""
+    grid, window, stride = [4, 5], [3, 2], [1, 2]
+    N = 20
+    d = 32
+    q = _randn(11, (1, 1, *grid, d))
+    k = _randn(12, (1, 1, *grid, d))
+    v = np.zeros((1, 1, *grid, d), dtype=np.float32)
+    v.reshape(N, d)[np.arange(N), np.arange(N)] = 1.0
+    out, lse = lib.forward(q, k, v, grid, window, stride, dtype="f32")
+    P = out.reshape(N, d)[:, :N]
+    qm = q.reshape(N, d).astype(np.float64)
+    km = k.reshape(N, d).astype(np.float64)
+    for t in range(N):
+        sup = _brute_mask(grid, window, stride, t)
+        assert abs(P[t].sum() - 1.0) < 1e-12
+        assert np.all(P[t][~sup] == 0.0)
+        assert np.all(P[t][sup] > 0.0)
+        z = (km[sup] @ qm[t]) / math.sqrt(d)
+        ref = np.exp(z - z.max()) / np.exp(z - z.max()).sum()
+        np.testing.assert_allclose(P[t][sup], ref, atol=1e-13, rtol=0)
+        np.testing.assert_allclose(lse.reshape(N)[t], z.max() + math.log(np.exp(z - z.max()).sum()),
+                                   atol=1e-12, rtol=0)
+
+
+def pin_uniform_queries(lib):
+    """q = 0: every score is 0, so out = mean of v over the window and
+    lse = ln(prod w) exactly; with v = key coordinates the output recovers the
+    window start, start + (w-1)/2 per dimension."""
+    for grid, window, stride in [([9, 7], [5, 4], [1, 2]), ([5, 6, 7], [3, 6, 2], [3, 2, 1])]:
+        nd = len(grid)
+        d = 4
+        N = int(np.prod(grid))
+        q = np.zeros((1, 1, *grid, d), dtype=np.float32)
+        k = _randn(21, (1, 1, *grid, d))
+        v = np.zeros((1, 1, *grid, d), dtype=np.float32)
+        coords = np.array(np.unravel_index(np.arange(N), grid)).T
+        v.reshape(N, d)[:, :nd] = coords
+        v.reshape(N, d)[:, nd] = 7.0
+        out, lse = lib.forward(q, k, v, grid, window, stride, dtype="f32")
+        W = int(np.prod(window))
+        np.testing.assert_allclose(lse.reshape(N), math.log(W), atol=1e-13, rtol=0)
+        starts = _window_sets(grid, window, stride)
+        for t in range(N):
+            c = coords[t]
+            expect = [starts[a][c[a]] + (window[a] - 1) / 2 for a in range(nd)]
+            np.testing.assert_allclose(out.reshape(N, d)[t, :nd], expect, atol=1e-12, rtol=0)
+            assert abs(out.reshape(N, d)[t, nd] - 7.0) < 1e-13
+
+
+def pin_single_key(lib):
+    """w = 1 (stride 1): each query sees only itself: out_i = v_i and
+    lse_i = scale * <q_i, k_i>."""
+    grid, d = [3, 4, 5], 8
+    N = 60
+    q, k, v = (_randn(31 + t, (1, 2, *grid, d)) for t in range(3))
+    out, lse = lib.forward(q, k, v, grid, [1, 1, 1], [1, 1, 1], dtype="f32")
+    np.testing.assert_allclose(out, v.astype(np.float64), atol=0, rtol=0)
+    ref = (q.astype(np.float64) * k.astype(np.float64)).sum(-1) / math.sqrt(d)
+    np.testing.assert_allclose(lse, ref, atol=1e-13, rtol=0)
+    assert N == int(np.prod(grid))
+
+
+def pin_constant_values(lib):
+    """v the same vector at every key: out = that vector whatever the scores."""
+    grid, d = [6, 9], 16
+    q, k = (_randn(41 + t, (2, 1, *grid, d)) for t in range(2))
+    row = _randn(43, (d,))
+    v = np.broadcast_to(row, (2, 1, *grid, d)).copy()
+    out, _ = lib.forward(q, k, v, grid, [3, 5], [1, 1], dtype="f32")
+    np.testing.assert_allclose(out, np.broadcast_to(row.astype(np.float64), out.shape),
+                               atol=1e-14, rtol=0)
+
+
+def pin_explicit_scale(lib):
+    """An explicit scale equal to 1/sqrt(d) gives the default result; scale 2x
+    doubles every score, which the one-element window (w = 1) exposes in lse."""
+    grid, d = [5, 5], 8
+    q, k, v = (_randn(51 + t, (1, 1, *grid, d)) for t in range(3))
+    o1, l1 = lib.forward(q, k, v, grid, [3, 3], [1, 1], dtype="f32")
+    o2, l2 = lib.forward(q, k, v, grid, [3, 3], [1, 1], dtype="f32", scale=1 / math.sqrt(d))
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    _, l3 = lib.forward(q, k, v, grid, [1, 1], [1, 1], dtype="f32", scale=2 / math.sqrt(d))
+    ref = 2 * (q.astype(np.float64) * k.astype(np.float64)).sum(-1) / math.sqrt(d)
+    np.testing.assert_allclose(l3, ref, atol=1e-13, rtol=0)
+
+
+def pin_row_subset(lib):
+    """Computing a list of rows gives the same values as the full run."""
+    grid, d = [6, 7], 8
+    q, k, v = (_randn(61 + t, (2, 3, *grid, d)) for t in range(3))
+    of, lf = lib.forward(q, k, v, grid, [3, 5], [1, 2], dtype="f32")
+    rows = np.array([0, 5, 41, 42, 100, 251], dtype=np.int64)
+    o, l = lib.forward(q, k, v, grid, [3, 5], [1, 2], dtype="f32", rows=rows)
+    np.testing.assert_array_equal(o, of.reshape(-1, d)[rows])
+    np.testing.assert_array_equal(l, lf.reshape(-1)[rows])
+
+
+def pin_wsa_empty_blocks_golden(lib):
+    """The empty-block ratios the Hilbert page prints for row-major window
+    attention (Table 1, Table 2) reproduce exactly from the oracle's mask."""
+    rows = _read_golden("wsa_empty_block_ratio.txt")
+    for side, win, blk, pct in rows:
+        e, p, f = lib.block_counts([int(side)] * 2, [int(win)] * 2, [int(win)] * 2, int(blk))
+        assert round(100.0 * e / (e + p + f), 2) == round(pct, 2), (side, win, blk, e, p, f)
+
+
+def pin_block_counts_closed_forms(lib):
+    """Full attention has only full tiles; blocked attention whose block equals
+    the tile is block-diagonal (full on the diagonal, empty elsewhere)."""
+    e, p, f = lib.block_counts([8, 8], [8, 8], [1, 1], 16)
+    assert (e, p, f) == (0, 0, 16)
+    e, p, f = lib.block_counts([64], [16], [16], 16)
+    assert (e, p, f) == (12, 0, 4)
+
+
+def pin_ena_density_golden(lib):
+    """ENA's example window (48x24 on a 4096-token 64x64 grid) covers about
+    30% of the tokens for every query."""
+    for gh, gw, wh, ww, dens, tol in _read_golden("ena_window_density.txt"):
+        grid, win = [int(gh), int(gw)], [int(wh), int(ww)]
+        for t in (0, 1000, 2080, 4095):
+            frac = lib.mask_row(grid, win, [1, 1], t).mean()
+            assert abs(frac - dens) <= tol, (t, frac)
+
+
+def _read_golden(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append([float(x) for x in line.split()])
+    return rows
+
+
+ALL_PINS = [
+    pin_window_bruteforce, pin_window_geometric_centre, pin_window_neighbourhood_metric,
+    pin_window_sliding_tile, pin_window_blocked, pin_mask_bruteforce, pin_full_attention,
+    pin_blocked_attention, pin_probability_rows, pin_uniform_queries, pin_single_key,
+    pin_constant_values, pin_explicit_scale, pin_row_subset, pin_wsa_empty_blocks_golden,
+    pin_block_counts_closed_forms, pin_ena_density_golden,
+]
+
+# The golden-file pins take a few seconds each; mutant runs use the fast ones.
+FAST_PINS = [p for p in ALL_PINS if p not in (pin_wsa_empty_blocks_golden,)]

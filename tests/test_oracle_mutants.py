@@ -1,0 +1,52 @@
+"""Plausible mistakes planted in copies of the oracle (on the CPU) must each
+fail at least one pin: evidence that the pins can catch a dropped term, a
+wrong sign or index, or a transposed operand."""
+import os
+import shutil
+
+import pytest
+
+import oracle
+from oracle_pins import FAST_PINS
+
+# (name, text in na_oracle.c, replacement)
+MUTANTS = [
+    ("leader_at_group_start", "int c = g * s + s / 2;", "int c = g * s;"),
+    ("window_off_by_one", "int start = c - w / 2;", "int start = c - w / 2 + 1;"),
+    ("window_not_centred", "int start = c - w / 2;", "int start = c - w;"),
+    ("no_upper_clamp", "if (start > L - w) start = L - w;", ""),
+    ("dropped_scale", "z[cnt] = J->scale * dot;", "z[cnt] = dot;"),
+    ("key_index_is_query", "load_in(J->k, J->dtype, koff + c)", "load_in(J->k, J->dtype, qoff + c)"),
+    ("value_of_query", "(size_t)N + (size_t)idx[e]) * (size_t)d;", "(size_t)N + (size_t)t) * (size_t)d;"),
+    ("lse_without_max", "J->lse[r] = m + log(l);", "J->lse[r] = log(l);"),
+    ("lse_log2", "J->lse[r] = m + log(l);", "J->lse[r] = m + log2(l);"),
+    ("unnormalised", "double p = exp(z[e] - m) / l;", "double p = exp(z[e] - m);"),
+    ("sign_flip_exp", "double p = exp(z[e] - m) / l;", "double p = exp(m - z[e]) / l;"),
+    ("column_major_tokens", "for (int a = ndim - 1; a >= 0; --a) {\n        coord[a]",
+     "for (int a = 0; a < ndim; ++a) {\n        coord[a]"),
+    ("mask_upper_inclusive", "kj[a] >= ws[a] + w[a]) in = 0;", "kj[a] > ws[a] + w[a]) in = 0;"),
+    ("full_partial_swapped", "m == ra * cb ? 2 : 1", "m == ra * cb ? 1 : 2"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(name, old, new, tmp_path):
+    src = open(oracle.SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mpath = tmp_path / f"mut_{name}.c"
+    mpath.write_text(src.replace(old, new))
+    lib_path = str(tmp_path / f"libmut_{name}.so")
+    oracle.compile_lib(str(mpath), lib_path)
+    lib = oracle.OracleLib(lib_path)
+    pins = list(FAST_PINS)
+    if name == "full_partial_swapped":
+        from oracle_pins import pin_block_counts_closed_forms
+        pins = [pin_block_counts_closed_forms]
+    caught = []
+    for pin in pins:
+        try:
+            pin(lib)
+        except (AssertionError, RuntimeError, ValueError):
+            caught.append(pin.__name__)
+            break
+    assert caught, f"mutant {name} passed every pin"
