@@ -1,0 +1,360 @@
+"""Benchmark of the forward pass on the 3-D sliding tile attention workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (one step = one forward pass over one batch): B=1, heads=24,
+head_dim=128, grid T x H x W = 30 x 48 x 80 (115,200 tokens), tile 6x8x8,
+window 18x24x40 (3x3x5 tiles), stride = tile, bf16 inputs drawn N(0, 1) from
+fixed seeds.  Metric: effective TFLOP/s = 4 * d * B * heads * N * prod(window)
+/ time, i.e. only the (query, key) pairs inside windows count.
+
+Our arm times the tensor-core kernel through the C ABI with inputs resident in
+HBM (q, k, v total 2.1 GB, larger than the 126 MB L2, so no flush is needed),
+plus an end-to-end figure with pinned-host inputs copied in and outputs copied
+out inside the timed region.  The reference arm (--impl reference) times the
+fp64 CPU oracle on a bounded sample of query rows on the host cores.
+
+With N > 1 (torchrun), every rank runs its own replica of the workload (weak
+scaling; the problem has no exchange step), the timed region is bracketed by
+barriers, and the time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "effective TFLOP/s and % of B200 bf16 tensor peak, 3D sliding-tile attn fwd"
+WORKLOAD = dict(workload="3D sliding tile attention fwd", B=1, heads=24, head_dim=128,
+                grid=[30, 48, 80], tile=[6, 8, 8], window=[18, 24, 40], stride=[6, 8, 8])
+SEED = 4000
+FALLBACK_PEAK_TFLOPS = 1590.0
+KERNEL_SOURCES = ["neighborhood_attention_b200/csrc/na_fwd_sm100.cu",
+                  "neighborhood_attention_b200/csrc/na_ptx.cuh",
+                  "neighborhood_attention_b200/csrc/na_sched.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "na_fwd_tc_sta3d_traffic.txt")
+
+
+def flops_per_step(w=WORKLOAD):
+    N = int(np.prod(w["grid"]))
+    W = int(np.prod(w["window"]))
+    return 4.0 * w["head_dim"] * w["B"] * w["heads"] * N * W
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    try:
+        kv = {}
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) == 2 and not line.startswith("#"):
+                    kv[parts[0]] = parts[1]
+        if kv.get("kernel_hash") == kernel_hash():
+            return float(kv["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        pass
+    return None
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 0) or 0), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_PEAK_TFLOPS, 0.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU side --
+def oracle_sample_rows(n_rows, seed=1):
+    w = WORKLOAD
+    N = int(np.prod(w["grid"]))
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(w["B"] * w["heads"] * N, size=n_rows, replace=False)).astype(np.int64)
+
+
+def host_qkv():
+    import seeded_inputs
+    w = WORKLOAD
+    return seeded_inputs.qkv(SEED, w["B"], w["heads"], w["grid"], w["head_dim"], "bf16")
+
+
+def time_oracle(qkv, n_rows, threads):
+    import oracle
+    w = WORKLOAD
+    rows = oracle_sample_rows(n_rows)
+    t0 = time.perf_counter()
+    oracle.forward(*qkv, w["grid"], w["window"], w["stride"], dtype="bf16", rows=rows,
+                   threads=threads)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * w["head_dim"] * int(np.prod(w["window"])) * n_rows
+    return flops / dt / 1e12, dt
+
+
+def cpu_baseline(qkv, target_s=15.0):
+    threads = os.cpu_count() or 1
+    probe = max(64, threads * 8)
+    _, dt = time_oracle(qkv, probe, threads)
+    n = int(min(200000, max(probe, probe * target_s / max(dt, 1e-3))))
+    val, dt = time_oracle(qkv, n, threads)
+    return {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} query rows drawn uniformly from the workload's {int(np.prod(WORKLOAD['grid'])) * WORKLOAD['heads']} "
+                      f"(fp64 dense-mask oracle, {dt:.1f} s)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    qkv = host_qkv()
+    threads = os.cpu_count() or 1
+    probe = max(64, threads * 8)
+    _, dt = time_oracle(qkv, probe, threads)
+    # each step a bounded sample sized so that warm-up + timed steps end within minutes
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    n = int(max(probe, probe * min(budget, 20.0) / max(dt, 1e-3)))
+    for _ in range(args.warmup):
+        time_oracle(qkv, n, threads)
+    vals, tot = [], 0.0
+    for _ in range(args.steps):
+        v, dt = time_oracle(qkv, n, threads)
+        vals.append(v)
+        tot += dt
+    flops = 4.0 * WORKLOAD["head_dim"] * int(np.prod(WORKLOAD["window"])) * n * args.steps
+    value = flops / tot / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(WORKLOAD, sample_rows_per_step=n),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{n} query rows per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU side --
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import neighborhood_attention_b200 as na
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOAD
+    qkv_host = host_qkv()
+    pinned = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory() for a in qkv_host]
+    q, k, v = (t.to(dev) for t in pinned)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=dev)
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        na.na_forward(q, k, v, out, lse, w["window"], w["stride"], w["tile"], stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    na.na_sync_status(stream)
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    na.na_sync_status(stream)
+    total_ms = t_start.elapsed_time(t_end)
+    per_launch_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+
+    # end to end through the public API: pinned host -> device, forward, device -> host
+    h2d = sum(t.numel() * t.element_size() for t in pinned)
+    d2h = out_host.numel() * out_host.element_size() + lse_host.numel() * lse_host.element_size()
+
+    def e2e_step():
+        q.copy_(pinned[0], non_blocking=True)
+        k.copy_(pinned[1], non_blocking=True)
+        v.copy_(pinned[2], non_blocking=True)
+        step()
+        out_host.copy_(out, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+
+    for _ in range(min(args.warmup, 2)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    na.na_sync_status(stream)
+    e2e_ms = e0.elapsed_time(e1)
+
+    times = torch.tensor([total_ms, e2e_ms, per_launch_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms, per_launch_ms = (float(x) for x in times.tolist())
+
+    flops = flops_per_step()
+    value = flops * args.steps * world / (total_ms / 1e3) / 1e12
+    e2e_value = flops * args.steps * world / (e2e_ms / 1e3) / 1e12
+    peak, peak_sustained, peak_kind = read_peaks()
+    achieved = flops / (per_launch_ms / 1e3) / 1e12
+    plan = na.na_plan(w["grid"], w["window"], w["stride"], w["tile"], w["head_dim"], na.NA_BF16)
+    if rank != 0:
+        return 0
+    base = cpu_baseline(qkv_host) if world == 1 and not args.no_cpu_baseline else None
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": dict(w, l2=f"inputs ({h2d / 1e9:.2f} GB) larger than the 126 MB L2; no flush",
+                       qblock=plan["qblock"], kvchunk=plan["kvchunk"],
+                       parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "pct_of_peak": 100.0 * value / world / peak,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": read_traffic(),
+                     "peak_kind": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"},
+        "cpu_baseline": base,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "kernel_ms": per_launch_ms,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

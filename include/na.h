@@ -1,0 +1,169 @@
+/*
+ * na.h -- C ABI of the B200 forward pass of multi-dimensional local attention
+ * (generalized neighborhood attention / sliding tile attention).
+ *
+ * Operation.  For every (batch b, head h) and every query token i of a 1-, 2-
+ * or 3-D token grid of extents L, the library computes
+ *     out_i = sum_{j in W(i)} softmax_j( <q_i, k_j> * scale ) v_j
+ *     lse_i = ln sum_{j in W(i)} exp( <q_i, k_j> * scale )
+ * i.e. softmax(QK^T / sqrt(d)) V of "pi-Attention: Online Efficient Sparse
+ * Transformers for Long-Context Modeling" (section 3.1, eqs. (1)-(3)) with the
+ * sum restricted to a neighbourhood (section 3.2, eqs. (4)-(5)), plus the log
+ * of eq. (2)'s denominator.  The neighbourhood W(i) is the product over grid
+ * dimensions of the 1-D windows
+ *     g = i / s,  c = g*s + s/2,  start = clamp(c - w/2, 0, L - w),
+ *     window = [start, start + w)
+ * (window w, stride s): centred on the query's stride group and clamped
+ * inside the grid, so every query sees exactly prod(w) keys.  stride 1 is
+ * neighborhood attention; stride = tile with an odd number of tiles per
+ * window is the sliding tile attention of "ENA: Efficient N-dimensional
+ * Attention"; stride = window dividing the grid is blocked attention -- the
+ * family named in the abstract of "Generalized Neighborhood Attention:
+ * Multi-dimensional Sparse Attention at the Speed of Light".
+ *
+ * Layout.  q, k, v and out are dense row-major [B, heads, X1, .., Xn, d]
+ * (n = ndim, last grid dimension fastest, then d); lse is [B, heads, X1..Xn].
+ *
+ * Ownership.  Every tensor is caller-owned device memory.  The library keeps
+ * one 4-byte device status word per device, allocated on that device's first
+ * call (so make the first call outside any stream capture), and nothing else.
+ *
+ * Asynchrony.  Calls enqueue work on `stream` (a cudaStream_t; NULL = legacy
+ * default stream) and return once it is queued.  Argument errors are returned
+ * at once.  Errors that only the device can see (a bounded in-kernel wait that
+ * ran out) are reported by na_sync_status().
+ *
+ * Determinism.  Identical inputs give bit-identical outputs run to run (fixed
+ * reduction order, no atomics on data).
+ */
+#ifndef NA_H_
+#define NA_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NA_OK = 0,
+  NA_ERR_INVALID_ARG = 1,  /* a pointer, size or window/stride violates the contract */
+  NA_ERR_UNSUPPORTED = 2,  /* valid, but outside what the kernels implement */
+  NA_ERR_CUDA = 3,         /* a CUDA runtime call failed; na_last_error() has the text */
+  NA_ERR_TIMEOUT = 4       /* a bounded in-kernel wait expired (reported by na_sync_status) */
+} na_status;
+
+typedef enum { NA_F32 = 0, NA_BF16 = 1 } na_dtype;
+
+typedef enum {
+  NA_KERNEL_AUTO = 0,  /* tensor-core kernel where it applies, else the CUDA-core kernel */
+  NA_KERNEL_SIMT = 1,  /* CUDA-core kernel (fp32 and bf16, head_dim 32/64/128) */
+  NA_KERNEL_TC = 2     /* tcgen05 tensor-core kernel (bf16, head_dim 64/128) */
+} na_kernel;
+
+/*
+ * na_forward -- enqueue one forward pass.
+ *   q, k, v   device pointers, [B, heads, X1..Xn, d], dtype `dtype`, 16-byte aligned.
+ *   out       device pointer, same shape and dtype as q (written).
+ *   lse       device pointer, float32 [B, heads, X1..Xn] (written).
+ *   B, heads  >= 1.
+ *   dims      {ndim, head_dim}: ndim in 1..3; head_dim in {32, 64, 128}.
+ *   grid      ndim extents X1..Xn (>= 1).
+ *   window    ndim window sizes, 1 <= window[i] <= grid[i].
+ *   stride    ndim strides, 1 <= stride[i] <= window[i]; NULL = all 1.
+ *   tile      ndim query-tile shape, or NULL for the library's choice.  It only
+ *             groups queries for scheduling (results do not depend on it): the
+ *             tensor-core path splits a tile of >= 128 tokens into 128-query
+ *             blocks, or joins tiles of < 128 tokens into such blocks.
+ *   dtype     NA_F32 (CUDA-core kernel) or NA_BF16 (tensor-core kernel when
+ *             head_dim is 64 or 128).
+ *   stream    cudaStream_t.
+ * Returns NA_OK once the work is queued, NA_ERR_INVALID_ARG / NA_ERR_UNSUPPORTED
+ * without touching the device, or NA_ERR_CUDA.  Scale is 1/sqrt(head_dim).
+ */
+na_status na_forward(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                     int heads, const int dims[2], const int* grid, const int* window,
+                     const int* stride, const int* tile, na_dtype dtype, void* stream);
+
+typedef struct {
+  float scale;              /* <= 0: 1/sqrt(head_dim) */
+  int kernel;               /* na_kernel */
+  int qblock[3];            /* 0s: automatic; else the query block shape, padded to 3 dims
+                               (outermost first; product 128 for NA_KERNEL_TC) */
+  int kvchunk[3];           /* 0s: automatic; else the key chunk shape (product 128 for TC,
+                               32 for SIMT) */
+  long long wait_timeout_ns;/* bound on each in-kernel wait; <= 0: 4 s (or env NA_WAIT_TIMEOUT_MS) */
+  int debug_flags;          /* testing hook, 0 in normal use.  1: the tensor-core kernel's
+                               loader withholds the first key chunk, so the consumer's bounded
+                               wait expires and the timeout path (NA_ERR_TIMEOUT from
+                               na_sync_status) is exercised without any fault or hang. */
+} na_options;
+
+/* na_options with every field at its default (automatic) value. */
+na_options na_default_options(void);
+
+/* na_forward with explicit options (NULL = defaults).  Same contract otherwise. */
+na_status na_forward_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                        int heads, const int dims[2], const int* grid, const int* window,
+                        const int* stride, const int* tile, na_dtype dtype,
+                        const na_options* opt, void* stream);
+
+/*
+ * na_sync_status -- synchronise `stream`, then read and clear this device's
+ * status word.  NA_ERR_TIMEOUT if a kernel since the last call gave up on a
+ * bounded wait (its outputs are then undefined); NA_ERR_CUDA if the
+ * synchronisation itself failed; else NA_OK.
+ */
+na_status na_sync_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* na_status_string(na_status s);
+
+/* Detail of the last failure on the calling thread ("" if none).  Thread-local, static storage. */
+const char* na_last_error(void);
+
+/*
+ * Schedule statistics for one (batch, head), computed on the host with the
+ * same scheduler the kernels run: the chosen block / chunk shapes and how much
+ * work they imply.  Units: (query, key) pairs unless noted.
+ */
+typedef struct {
+  int kernel;               /* na_kernel actually chosen */
+  int qblock[3];            /* query block shape (3-d padded, outermost first) */
+  int kvchunk[3];           /* key chunk shape */
+  int tile[3];              /* query tile shape used to order blocks */
+  long long query_blocks;   /* blocks per head */
+  long long ctas;           /* CTAs per head */
+  long long chunks_loaded;  /* key chunks staged per head */
+  long long units_full;     /* (block, chunk) products with no mask */
+  long long units_partial;  /* (block, chunk) products with an element mask */
+  long long computed_pairs; /* (units_full + units_partial) * block rows * chunk keys */
+  long long useful_pairs;   /* N * prod(window) */
+} na_plan_info;
+
+/* Fill *info for the given problem without touching the device. */
+na_status na_plan(const int dims[2], const int* grid, const int* window, const int* stride,
+                  const int* tile, na_dtype dtype, const na_options* opt, na_plan_info* info);
+
+/* The 1-D window start used by the kernels (host copy), -1 on invalid input. */
+int na_window_start(int L, int w, int s, int i);
+
+/*
+ * Key box and chunk classification of one query block, for tests: the
+ * block's origin and valid extent, the union [lo, hi) and intersection
+ * [ilo, ihi) of its queries' windows (3-d padded), and per key chunk of the
+ * block's own key box (row-major over the chunk grid) its status 0 = empty,
+ * 1 = partial, 2 = full.  `status` holds up to `max_chunks` entries; the
+ * number of chunks is returned in *nchunks.
+ */
+na_status na_block_schedule(const int dims[2], const int* grid, const int* window,
+                            const int* stride, const int qblock[3], const int kvchunk[3],
+                            long long block, int origin[3], int extent[3], int lo[3], int hi[3],
+                            int ilo[3], int ihi[3], int* status, int max_chunks, int* nchunks);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int na_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NA_H_ */

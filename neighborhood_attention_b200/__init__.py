@@ -1,0 +1,234 @@
+"""Python binding of the B200 multi-dimensional local attention library.
+
+Argument marshalling only: every step of the forward pass runs in the CUDA
+kernels of ``libna.so`` (built in-tree by ``neighborhood_attention_b200.build``).
+Importing this package without the built library raises ImportError; there is
+no fallback of any kind.
+
+Functions keep the C-ABI names (``include/na.h``): ``na_forward``,
+``na_forward_ex``, ``na_sync_status``, ``na_plan``, ``na_window_start``,
+``na_block_schedule``, ``na_status_string``, ``na_last_error``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libna.so")
+
+NA_OK, NA_ERR_INVALID_ARG, NA_ERR_UNSUPPORTED, NA_ERR_CUDA, NA_ERR_TIMEOUT = range(5)
+NA_F32, NA_BF16 = 0, 1
+NA_KERNEL_AUTO, NA_KERNEL_SIMT, NA_KERNEL_TC = 0, 1, 2
+KERNEL_NAMES = {NA_KERNEL_AUTO: "auto", NA_KERNEL_SIMT: "simt", NA_KERNEL_TC: "tc"}
+
+
+class NaError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{_status_name(status)}: {detail}")
+        self.status = status
+        self.detail = detail
+
+
+class na_options(ctypes.Structure):
+    _fields_ = [("scale", ctypes.c_float), ("kernel", ctypes.c_int),
+                ("qblock", ctypes.c_int * 3), ("kvchunk", ctypes.c_int * 3),
+                ("wait_timeout_ns", ctypes.c_longlong), ("debug_flags", ctypes.c_int)]
+
+
+class na_plan_info(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_int), ("qblock", ctypes.c_int * 3),
+                ("kvchunk", ctypes.c_int * 3), ("tile", ctypes.c_int * 3),
+                ("query_blocks", ctypes.c_longlong), ("ctas", ctypes.c_longlong),
+                ("chunks_loaded", ctypes.c_longlong), ("units_full", ctypes.c_longlong),
+                ("units_partial", ctypes.c_longlong), ("computed_pairs", ctypes.c_longlong),
+                ("useful_pairs", ctypes.c_longlong)]
+
+    def as_dict(self):
+        out = {}
+        for name, _ in self._fields_:
+            v = getattr(self, name)
+            out[name] = list(v) if isinstance(v, ctypes.Array) else v
+        out["kernel"] = KERNEL_NAMES.get(out["kernel"], out["kernel"])
+        return out
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: run `python -m neighborhood_attention_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    i32p = ctypes.POINTER(ctypes.c_int)
+    vp = ctypes.c_void_p
+    lib.na_forward.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int, i32p, i32p, i32p,
+                               i32p, i32p, ctypes.c_int, vp]
+    lib.na_forward.restype = ctypes.c_int
+    lib.na_forward_ex.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int, i32p, i32p,
+                                  i32p, i32p, i32p, ctypes.c_int, ctypes.POINTER(na_options), vp]
+    lib.na_forward_ex.restype = ctypes.c_int
+    lib.na_default_options.argtypes = []
+    lib.na_default_options.restype = na_options
+    lib.na_sync_status.argtypes = [vp]
+    lib.na_sync_status.restype = ctypes.c_int
+    lib.na_status_string.argtypes = [ctypes.c_int]
+    lib.na_status_string.restype = ctypes.c_char_p
+    lib.na_last_error.argtypes = []
+    lib.na_last_error.restype = ctypes.c_char_p
+    lib.na_plan.argtypes = [i32p, i32p, i32p, i32p, i32p, ctypes.c_int,
+                            ctypes.POINTER(na_options), ctypes.POINTER(na_plan_info)]
+    lib.na_plan.restype = ctypes.c_int
+    lib.na_window_start.argtypes = [ctypes.c_int] * 4
+    lib.na_window_start.restype = ctypes.c_int
+    lib.na_block_schedule.argtypes = [i32p, i32p, i32p, i32p, i32p, i32p, ctypes.c_longlong,
+                                      i32p, i32p, i32p, i32p, i32p, i32p, i32p, ctypes.c_int, i32p]
+    lib.na_block_schedule.restype = ctypes.c_int
+    lib.na_version.argtypes = []
+    lib.na_version.restype = ctypes.c_int
+    return lib
+
+
+_lib = _load()
+
+
+def _status_name(s: int) -> str:
+    return _lib.na_status_string(int(s)).decode()
+
+
+def _ivec(vals):
+    if vals is None:
+        return None
+    vals = [int(x) for x in vals]
+    return (ctypes.c_int * len(vals))(*vals)
+
+
+def _check(status: int):
+    if status != NA_OK:
+        raise NaError(status, _lib.na_last_error().decode())
+
+
+def na_status_string(status: int) -> str:
+    return _status_name(status)
+
+
+def na_last_error() -> str:
+    return _lib.na_last_error().decode()
+
+
+def na_version() -> int:
+    return int(_lib.na_version())
+
+
+def na_default_options() -> na_options:
+    return _lib.na_default_options()
+
+
+def make_options(kernel: int = NA_KERNEL_AUTO, scale: float = 0.0, qblock=None, kvchunk=None,
+                 wait_timeout_ns: int = 0, debug_flags: int = 0) -> na_options:
+    o = na_default_options()
+    o.kernel = int(kernel)
+    o.scale = float(scale)
+    if qblock is not None:
+        for i, x in enumerate(qblock):
+            o.qblock[i] = int(x)
+    if kvchunk is not None:
+        for i, x in enumerate(kvchunk):
+            o.kvchunk[i] = int(x)
+    o.wait_timeout_ns = int(wait_timeout_ns)
+    o.debug_flags = int(debug_flags)
+    return o
+
+
+def _dtype_of(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return NA_BF16
+    if t.dtype == torch.float32:
+        return NA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16 or torch.float32")
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def na_forward_ex(q, k, v, out, lse, window, stride=None, tile=None, options=None, stream=None,
+                  ndim=None):
+    """Enqueue na_forward_ex on torch CUDA tensors.
+
+    q, k, v, out: [B, heads, X1..Xn, d] contiguous on one CUDA device; lse:
+    float32 [B, heads, X1..Xn].  ``ndim`` defaults to len(window).
+    """
+    nd = len(window) if ndim is None else int(ndim)
+    shape = tuple(q.shape)
+    if len(shape) != nd + 3:
+        raise ValueError(f"q has shape {shape}; expected [B, heads, {nd} grid dims, d]")
+    for name, t in (("k", k), ("v", v), ("out", out)):
+        if tuple(t.shape) != shape or t.dtype != q.dtype:
+            raise ValueError(f"{name} must match q in shape and dtype")
+    import torch
+    if tuple(lse.shape) != shape[:-1] or lse.dtype != torch.float32:
+        raise ValueError("lse must be float32 with q's shape minus head_dim")
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    dims = _ivec([nd, shape[-1]])
+    st = _lib.na_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                            lse.data_ptr(), shape[0], shape[1], dims, _ivec(shape[2:2 + nd]),
+                            _ivec(window), _ivec(stride), _ivec(tile), _dtype_of(q),
+                            ctypes.byref(options) if options is not None else None,
+                            _stream_ptr(stream))
+    _check(st)
+    return out, lse
+
+
+def na_forward(q, k, v, out, lse, window, stride=None, tile=None, stream=None):
+    """Enqueue na_forward (scale 1/sqrt(d), automatic kernel choice)."""
+    return na_forward_ex(q, k, v, out, lse, window, stride, tile, None, stream)
+
+
+def na_sync_status(stream=None):
+    """Synchronise the stream and raise NaError if a kernel's bounded wait expired."""
+    _check(_lib.na_sync_status(_stream_ptr(stream)))
+
+
+def na_plan(grid, window, stride=None, tile=None, head_dim=128, dtype=NA_BF16, options=None):
+    """Schedule statistics of one (batch, head) as a dict (host only, no device)."""
+    info = na_plan_info()
+    dims = _ivec([len(grid), head_dim])
+    st = _lib.na_plan(dims, _ivec(grid), _ivec(window), _ivec(stride), _ivec(tile), int(dtype),
+                      ctypes.byref(options) if options is not None else None, ctypes.byref(info))
+    _check(st)
+    return info.as_dict()
+
+
+def na_window_start(L: int, w: int, s: int, i: int) -> int:
+    return int(_lib.na_window_start(L, w, s, i))
+
+
+def na_block_schedule(grid, window, stride, qblock, kvchunk, block: int, max_chunks: int = 4096):
+    """Key box and per-chunk status (0 empty, 1 partial, 2 full) of one query block."""
+    arrs = {n: (ctypes.c_int * 3)() for n in ("origin", "extent", "lo", "hi", "ilo", "ihi")}
+    status = (ctypes.c_int * max_chunks)()
+    n = ctypes.c_int(0)
+    dims = _ivec([len(grid), 32])
+    st = _lib.na_block_schedule(dims, _ivec(grid), _ivec(window), _ivec(stride), _ivec(qblock),
+                                _ivec(kvchunk), int(block), arrs["origin"], arrs["extent"],
+                                arrs["lo"], arrs["hi"], arrs["ilo"], arrs["ihi"], status,
+                                max_chunks, ctypes.byref(n))
+    _check(st)
+    out = {k: list(v) for k, v in arrs.items()}
+    out["nchunks"] = n.value
+    out["status"] = list(status[: min(n.value, max_chunks)])
+    return out
+
+
+def forward(q, k, v, window, stride=None, tile=None, options=None, stream=None):
+    """Allocate out / lse with torch and enqueue the forward pass; returns (out, lse)."""
+    import torch
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    return na_forward_ex(q, k, v, out, lse, window, stride, tile, options, stream)

@@ -1,0 +1,472 @@
+// C-ABI layer: argument validation, schedule planning, kernel dispatch and
+// the device status word.  Declarations and the contract are in include/na.h.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <array>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include "../../include/na.h"
+#include "na_internal.h"
+
+using namespace na;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+na_status fail(na_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+constexpr int MAX_DEVICES = 64;
+std::mutex g_status_mu;
+int* g_status[MAX_DEVICES] = {nullptr};
+
+// ------------------------------------------------------------ problem --
+struct Problem {
+  int ndim = 0, D = 0;
+  Geom g{};
+  int tile[3] = {0, 0, 0};   // 0 = none given
+  int dtype = NA_BF16;
+  na_options opt{};
+};
+
+struct Plan {
+  int kernel = NA_KERNEL_SIMT;
+  QTiling t{};
+  int kb[3] = {1, 1, 1};
+};
+
+na_status read_problem(const int dims[2], const int* grid, const int* window, const int* stride,
+                       const int* tile, na_dtype dtype, const na_options* opt, Problem& P) {
+  if (!dims) return fail(NA_ERR_INVALID_ARG, "dims is NULL");
+  const int nd = dims[0], D = dims[1];
+  if (nd < 1 || nd > 3) return fail(NA_ERR_INVALID_ARG, "ndim=%d not in 1..3", nd);
+  if (D <= 0) return fail(NA_ERR_INVALID_ARG, "head_dim=%d must be positive", D);
+  if (D != 32 && D != 64 && D != 128)
+    return fail(NA_ERR_UNSUPPORTED, "head_dim=%d not in {32, 64, 128}", D);
+  if (!grid || !window) return fail(NA_ERR_INVALID_ARG, "grid or window is NULL");
+  if (dtype != NA_F32 && dtype != NA_BF16) return fail(NA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  P.ndim = nd;
+  P.D = D;
+  P.dtype = dtype;
+  const int pad = 3 - nd;
+  for (int d = 0; d < 3; ++d) {
+    P.g.L[d] = P.g.w[d] = P.g.s[d] = 1;
+    P.tile[d] = tile ? 1 : 0;
+  }
+  long long N = 1;
+  for (int i = 0; i < nd; ++i) {
+    const int L = grid[i], w = window[i], s = stride ? stride[i] : 1;
+    if (L < 1) return fail(NA_ERR_INVALID_ARG, "grid[%d]=%d must be >= 1", i, L);
+    if (w < 1 || w > L)
+      return fail(NA_ERR_INVALID_ARG, "window[%d]=%d must be in 1..grid[%d]=%d", i, w, i, L);
+    if (s < 1 || s > w)
+      return fail(NA_ERR_INVALID_ARG, "stride[%d]=%d must be in 1..window[%d]=%d", i, s, i, w);
+    if (tile && tile[i] < 1) return fail(NA_ERR_INVALID_ARG, "tile[%d]=%d must be >= 1", i, tile[i]);
+    P.g.L[pad + i] = L;
+    P.g.w[pad + i] = w;
+    P.g.s[pad + i] = s;
+    if (tile) P.tile[pad + i] = tile[i];
+    N *= L;
+    if (N > (1LL << 31)) return fail(NA_ERR_UNSUPPORTED, "grid has more than 2^31 tokens");
+  }
+  P.opt = opt ? *opt : na_default_options();
+  if (P.opt.kernel < NA_KERNEL_AUTO || P.opt.kernel > NA_KERNEL_TC)
+    return fail(NA_ERR_INVALID_ARG, "unknown kernel selector %d", P.opt.kernel);
+  return NA_OK;
+}
+
+// Shapes of `prod` tokens (powers of two per dimension, <= 256 each), with
+// extent 1 on dimensions the problem does not have.
+std::vector<std::array<int, 3>> shape_candidates(const Problem& P, int prod) {
+  std::vector<std::array<int, 3>> out;
+  int lp = 0;
+  while ((1 << lp) < prod) ++lp;
+  for (int e0 = 0; e0 <= lp; ++e0)
+    for (int e1 = 0; e0 + e1 <= lp; ++e1) {
+      const int e2 = lp - e0 - e1;
+      const int e[3] = {e0, e1, e2};
+      bool okc = true;
+      for (int d = 0; d < 3; ++d) {
+        if (P.g.L[d] == 1 && e[d] != 0) okc = false;
+        if (e[d] > 8) okc = false;
+      }
+      if (okc) out.push_back({1 << e0, 1 << e1, 1 << e2});
+    }
+  return out;
+}
+
+struct Cost {
+  double cost = 0;
+  long long loads = 0, full = 0, partial = 0;
+};
+
+// Walk the CTA work items exactly like the kernels do.  group = 2 for the
+// tensor-core kernel (a CTA owns a pair of blocks), 1 for the CUDA-core one.
+Cost walk(const Geom& g, const QTiling& t, const int kb[3], int group, int max_items) {
+  Cost c;
+  const int items = (t.nblocks + group - 1) / group;
+  const int n = (max_items > 0 && items > max_items) ? max_items : items;
+  for (int i = 0; i < n; ++i) {
+    const int it = (n == items) ? i : (int)((long long)i * items / n);
+    BlockInfo bi[2];
+    for (int b = 0; b < group; ++b) block_info(g, t, it * group + b, bi[b]);
+    ChunkGrid cg;
+    chunk_grid_for(bi, group, kb, cg);
+    for (int ch = 0; ch < cg.total; ++ch) {
+      int a[3];
+      chunk_origin(cg, kb, ch, a);
+      int active = 0;
+      for (int b = 0; b < group; ++b) {
+        const int st = chunk_status(bi[b], a, kb);
+        if (st == CHUNK_EMPTY) continue;
+        ++active;
+        if (st == CHUNK_FULL) ++c.full; else ++c.partial;
+        c.cost += (st == CHUNK_FULL) ? 1.0 : 1.3;
+      }
+      if (active) {
+        ++c.loads;
+        c.cost += 0.2 + ((group == 2 && active == 1) ? 0.5 : 0.0);
+      }
+    }
+  }
+  if (n != items && n > 0) c.cost *= (double)items / n;
+  return c;
+}
+
+bool build_tiling(const Problem& P, const int qb[3], int kernel, QTiling& t) {
+  int tl[3] = {qb[0], qb[1], qb[2]};
+  if (P.tile[0] && kernel == NA_KERNEL_TC) {
+    const int tprod = P.tile[0] * P.tile[1] * P.tile[2];
+    if (tprod >= qb[0] * qb[1] * qb[2]) {
+      bool nest = true;
+      for (int d = 0; d < 3; ++d)
+        if (P.tile[d] % qb[d]) nest = false;
+      if (nest)
+        for (int d = 0; d < 3; ++d) tl[d] = P.tile[d];
+      else
+        return false;
+    } else {
+      for (int d = 0; d < 3; ++d)
+        if (qb[d] % P.tile[d]) return false;
+    }
+  }
+  return make_tiling(P.g, qb, tl, t) == 0;
+}
+
+std::mutex g_plan_mu;
+std::map<std::vector<long long>, Plan> g_plans;
+
+na_status make_plan(const Problem& P, Plan& out) {
+  int kernel = P.opt.kernel;
+  if (kernel == NA_KERNEL_AUTO)
+    kernel = (P.dtype == NA_BF16 && (P.D == 64 || P.D == 128)) ? NA_KERNEL_TC : NA_KERNEL_SIMT;
+  if (kernel == NA_KERNEL_TC && P.dtype != NA_BF16)
+    return fail(NA_ERR_UNSUPPORTED, "the tensor-core kernel takes bf16 only");
+  if (kernel == NA_KERNEL_TC && P.D != 64 && P.D != 128)
+    return fail(NA_ERR_UNSUPPORTED, "the tensor-core kernel takes head_dim 64 or 128");
+
+  std::vector<long long> key = {P.ndim, P.D, P.dtype, kernel};
+  for (int d = 0; d < 3; ++d) {
+    key.insert(key.end(), {P.g.L[d], P.g.w[d], P.g.s[d], P.tile[d], P.opt.qblock[d],
+                           P.opt.kvchunk[d]});
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_plan_mu);
+    auto it = g_plans.find(key);
+    if (it != g_plans.end()) {
+      out = it->second;
+      return NA_OK;
+    }
+  }
+  const int qprod = kernel == NA_KERNEL_TC ? 128 : 128 / (P.D / 32);
+  const int kprod = kernel == NA_KERNEL_TC ? 128 : 32;
+  const int group = kernel == NA_KERNEL_TC ? 2 : 1;
+
+  std::vector<std::array<int, 3>> qcands, kcands;
+  if (P.opt.qblock[0] > 0) {
+    const int* q = P.opt.qblock;
+    if (q[0] * q[1] * q[2] != qprod)
+      return fail(NA_ERR_UNSUPPORTED, "qblock product must be %d for this kernel", qprod);
+    qcands.push_back({q[0], q[1], q[2]});
+  } else {
+    qcands = shape_candidates(P, qprod);
+  }
+  if (P.opt.kvchunk[0] > 0) {
+    const int* k = P.opt.kvchunk;
+    if (k[0] * k[1] * k[2] != kprod)
+      return fail(NA_ERR_UNSUPPORTED, "kvchunk product must be %d for this kernel", kprod);
+    for (int d = 0; d < 3; ++d)
+      if (k[d] > 256) return fail(NA_ERR_UNSUPPORTED, "kvchunk extents must be <= 256");
+    kcands.push_back({k[0], k[1], k[2]});
+  } else {
+    kcands = shape_candidates(P, kprod);
+  }
+
+  bool found = false;
+  Plan best;
+  double best_cost = 0;
+  for (int pass = 0; pass < 2 && !found; ++pass) {
+    // pass 0 honours the tile hint; pass 1 drops it (it only orders queries).
+    Problem Q = P;
+    if (pass == 1) Q.tile[0] = Q.tile[1] = Q.tile[2] = 0;
+    for (const auto& qb : qcands) {
+      QTiling t;
+      if (!build_tiling(Q, qb.data(), kernel, t)) continue;
+      for (const auto& kb : kcands) {
+        const Cost c = walk(Q.g, t, kb.data(), group, 48);
+        if (!found || c.cost < best_cost - 1e-9) {
+          found = true;
+          best_cost = c.cost;
+          best.kernel = kernel;
+          best.t = t;
+          for (int d = 0; d < 3; ++d) best.kb[d] = kb[d];
+        }
+      }
+    }
+  }
+  if (!found) return fail(NA_ERR_UNSUPPORTED, "no query block / key chunk shape fits this grid");
+  {
+    std::lock_guard<std::mutex> lk(g_plan_mu);
+    g_plans[key] = best;
+  }
+  out = best;
+  return NA_OK;
+}
+
+long long default_timeout_ns() {
+  const char* e = getenv("NA_WAIT_TIMEOUT_MS");
+  if (e) {
+    const long long ms = atoll(e);
+    if (ms > 0) return ms * 1000000LL;
+  }
+  return 4000LL * 1000000LL;
+}
+
+na_status status_word(int** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= MAX_DEVICES) return fail(NA_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status[dev]) {
+    int* p = nullptr;
+    e = cudaMalloc(&p, sizeof(int));
+    if (e != cudaSuccess) return fail(NA_ERR_CUDA, "cudaMalloc(status): %s", cudaGetErrorString(e));
+    e = cudaMemset(p, 0, sizeof(int));
+    if (e != cudaSuccess) return fail(NA_ERR_CUDA, "cudaMemset(status): %s", cudaGetErrorString(e));
+    g_status[dev] = p;
+  }
+  *out = g_status[dev];
+  return NA_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+na_options na_default_options(void) {
+  na_options o;
+  memset(&o, 0, sizeof o);
+  o.scale = 0.f;
+  o.kernel = NA_KERNEL_AUTO;
+  o.wait_timeout_ns = 0;
+  return o;
+}
+
+const char* na_status_string(na_status s) {
+  switch (s) {
+    case NA_OK: return "NA_OK";
+    case NA_ERR_INVALID_ARG: return "NA_ERR_INVALID_ARG";
+    case NA_ERR_UNSUPPORTED: return "NA_ERR_UNSUPPORTED";
+    case NA_ERR_CUDA: return "NA_ERR_CUDA";
+    case NA_ERR_TIMEOUT: return "NA_ERR_TIMEOUT";
+  }
+  return "NA_ERR_UNKNOWN";
+}
+
+const char* na_last_error(void) { return g_err; }
+
+int na_version(void) { return 100; }
+
+int na_window_start(int L, int w, int s, int i) {
+  if (L < 1 || w < 1 || w > L || s < 1 || s > w || i < 0 || i >= L) return -1;
+  return window_start(L, w, s, i);
+}
+
+na_status na_forward_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                        int heads, const int dims[2], const int* grid, const int* window,
+                        const int* stride, const int* tile, na_dtype dtype,
+                        const na_options* opt, void* stream) {
+  g_err[0] = 0;
+  if (!q || !k || !v || !out || !lse) return fail(NA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  if (B < 1 || heads < 1) return fail(NA_ERR_INVALID_ARG, "B=%d heads=%d must be >= 1", B, heads);
+  Problem P;
+  na_status st = read_problem(dims, grid, window, stride, tile, dtype, opt, P);
+  if (st != NA_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(lse, 4))
+    return fail(NA_ERR_INVALID_ARG, "q, k, v, out must be 16-byte aligned and lse 4-byte aligned");
+  const long long BH = (long long)B * heads;
+  if (BH > (1LL << 30)) return fail(NA_ERR_UNSUPPORTED, "B*heads too large");
+  Plan plan;
+  st = make_plan(P, plan);
+  if (st != NA_OK) return st;
+  const long long N = (long long)P.g.L[0] * P.g.L[1] * P.g.L[2];
+  const float scale = P.opt.scale > 0.f ? P.opt.scale : 1.0f / sqrtf((float)P.D);
+  const float log2e = 1.4426950408889634f;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  if (plan.kernel == NA_KERNEL_TC) {
+    int* status = nullptr;
+    st = status_word(&status);
+    if (st != NA_OK) return st;
+    TcLaunch L;
+    L.g = P.g;
+    L.t = plan.t;
+    for (int d = 0; d < 3; ++d) L.kb[d] = plan.kb[d];
+    L.BH = (int)BH;
+    L.N = (int)N;
+    L.D = P.D;
+    L.scale_log2 = scale * log2e;
+    L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
+    L.status = status;
+    L.timeout_ns = P.opt.wait_timeout_ns > 0 ? P.opt.wait_timeout_ns : default_timeout_ns();
+    L.debug_flags = P.opt.debug_flags;
+    char msg[256] = "";
+    cudaError_t e = launch_tc(L, s, msg, sizeof msg);
+    if (e == cudaErrorNotSupported)
+      return fail(NA_ERR_UNSUPPORTED, "tensor-core kernel does not take this shape");
+    if (e != cudaSuccess)
+      return fail(NA_ERR_CUDA, "tensor-core launch: %s %s", cudaGetErrorString(e), msg);
+    return NA_OK;
+  }
+  SimtLaunch L;
+  L.g = P.g;
+  L.t = plan.t;
+  for (int d = 0; d < 3; ++d) L.kb[d] = plan.kb[d];
+  L.BH = (int)BH;
+  L.N = (int)N;
+  L.D = P.D;
+  L.bf16 = P.dtype == NA_BF16;
+  L.scale_log2 = scale * log2e;
+  L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
+  cudaError_t e = launch_simt(L, s);
+  if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "CUDA-core kernel: shape");
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "CUDA-core launch: %s", cudaGetErrorString(e));
+  return NA_OK;
+}
+
+na_status na_forward(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                     int heads, const int dims[2], const int* grid, const int* window,
+                     const int* stride, const int* tile, na_dtype dtype, void* stream) {
+  return na_forward_ex(q, k, v, out, lse, B, heads, dims, grid, window, stride, tile, dtype,
+                       nullptr, stream);
+}
+
+na_status na_sync_status(void* stream) {
+  g_err[0] = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return NA_OK;
+  int* p = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_status_mu);
+    p = g_status[dev];
+  }
+  if (!p) return NA_OK;
+  int h = 0;
+  e = cudaMemcpy(&h, p, sizeof h, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "reading status word: %s", cudaGetErrorString(e));
+  if (h != DEV_OK) {
+    cudaMemset(p, 0, sizeof(int));
+    return fail(NA_ERR_TIMEOUT, "a bounded in-kernel wait expired (code %d)", h);
+  }
+  return NA_OK;
+}
+
+na_status na_plan(const int dims[2], const int* grid, const int* window, const int* stride,
+                  const int* tile, na_dtype dtype, const na_options* opt, na_plan_info* info) {
+  g_err[0] = 0;
+  if (!info) return fail(NA_ERR_INVALID_ARG, "info is NULL");
+  Problem P;
+  na_status st = read_problem(dims, grid, window, stride, tile, dtype, opt, P);
+  if (st != NA_OK) return st;
+  Plan plan;
+  st = make_plan(P, plan);
+  if (st != NA_OK) return st;
+  const int group = plan.kernel == NA_KERNEL_TC ? 2 : 1;
+  const Cost c = walk(P.g, plan.t, plan.kb, group, 0);
+  memset(info, 0, sizeof *info);
+  info->kernel = plan.kernel;
+  for (int d = 0; d < 3; ++d) {
+    info->qblock[d] = plan.t.qb[d];
+    info->kvchunk[d] = plan.kb[d];
+    info->tile[d] = plan.t.tl[d];
+  }
+  const long long rows = (long long)plan.t.qb[0] * plan.t.qb[1] * plan.t.qb[2];
+  const long long keys = (long long)plan.kb[0] * plan.kb[1] * plan.kb[2];
+  info->query_blocks = plan.t.nblocks;
+  info->ctas = (plan.t.nblocks + group - 1) / group;
+  info->chunks_loaded = c.loads;
+  info->units_full = c.full;
+  info->units_partial = c.partial;
+  info->computed_pairs = (c.full + c.partial) * rows * keys;
+  info->useful_pairs = (long long)P.g.L[0] * P.g.L[1] * P.g.L[2] *
+                       ((long long)P.g.w[0] * P.g.w[1] * P.g.w[2]);
+  return NA_OK;
+}
+
+na_status na_block_schedule(const int dims[2], const int* grid, const int* window,
+                            const int* stride, const int qblock[3], const int kvchunk[3],
+                            long long block, int origin[3], int extent[3], int lo[3], int hi[3],
+                            int ilo[3], int ihi[3], int* status, int max_chunks, int* nchunks) {
+  g_err[0] = 0;
+  Problem P;
+  na_status st = read_problem(dims, grid, window, stride, nullptr, NA_BF16, nullptr, P);
+  if (st != NA_OK) return st;
+  if (!qblock || !kvchunk || !nchunks) return fail(NA_ERR_INVALID_ARG, "NULL argument");
+  for (int d = 0; d < 3; ++d)
+    if (qblock[d] < 1 || kvchunk[d] < 1) return fail(NA_ERR_INVALID_ARG, "shapes must be >= 1");
+  QTiling t;
+  if (make_tiling(P.g, qblock, qblock, t)) return fail(NA_ERR_INVALID_ARG, "bad qblock");
+  if (block < 0 || block >= t.nblocks) return fail(NA_ERR_INVALID_ARG, "block out of range");
+  BlockInfo b;
+  block_info(P.g, t, (int)block, b);
+  ChunkGrid cg;
+  chunk_grid_for(&b, 1, kvchunk, cg);
+  for (int d = 0; d < 3; ++d) {
+    if (origin) origin[d] = b.o[d];
+    if (extent) extent[d] = b.n[d];
+    if (lo) lo[d] = b.lo[d];
+    if (hi) hi[d] = b.hi[d];
+    if (ilo) ilo[d] = b.ilo[d];
+    if (ihi) ihi[d] = b.ihi[d];
+  }
+  *nchunks = cg.total;
+  for (int c = 0; c < cg.total && c < max_chunks && status; ++c) {
+    int a[3];
+    chunk_origin(cg, kvchunk, c, a);
+    status[c] = chunk_status(b, a, kvchunk);
+  }
+  return NA_OK;
+}
+
+}  // extern "C"

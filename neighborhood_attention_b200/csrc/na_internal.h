@@ -1,0 +1,45 @@
+// Internal interface between the C-ABI layer (na_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "na_sched.cuh"
+
+namespace na {
+
+// Device status word values (written by kernels, read by na_sync_status).
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_SCHEDULE = 2 };
+
+struct SimtLaunch {
+  Geom g;
+  QTiling t;
+  int kb[3];
+  int BH, N, D;
+  int bf16;              // 1: bf16 in/out, 0: fp32 in/out
+  float scale_log2;      // scale * log2(e)
+  const void *q, *k, *v;
+  void* out;
+  float* lse;
+};
+
+struct TcLaunch {
+  Geom g;
+  QTiling t;
+  int kb[3];
+  int BH, N, D;
+  float scale_log2;
+  const void *q, *k, *v;
+  void* out;
+  float* lse;
+  int* status;           // device status word
+  long long timeout_ns;  // bound on every in-kernel wait
+  int debug_flags;       // 1: withhold the first key chunk (timeout-path test)
+};
+
+cudaError_t launch_simt(const SimtLaunch& L, cudaStream_t stream);
+
+// Returns cudaErrorNotSupported when the shape is outside the kernel's range.
+cudaError_t launch_tc(const TcLaunch& L, cudaStream_t stream, char* err, int errlen);
+
+}  // namespace na

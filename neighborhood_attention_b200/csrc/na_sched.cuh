@@ -1,0 +1,161 @@
+// Window rule and tile scheduler of the CUDA path, usable on host and device.
+//
+// Geometry is always held in three dimensions (X1, X2, X3), X3 innermost in
+// memory; a 1-D problem is (1, 1, L) and a 2-D problem (1, H, W).
+//
+// Window rule (per dimension; window w, stride s, length L): the query at
+// coordinate i belongs to stride group g = i / s whose centre member is
+// c = g*s + s/2; its window is [start, start + w) with
+//   start = clamp(c - w/2, 0, L - w),
+// so every query sees exactly prod(w) keys.  Stride 1 is neighborhood
+// attention; stride equal to the tile with w an odd multiple of it is sliding
+// tile attention ("Generalized Neighborhood Attention: Multi-dimensional
+// Sparse Attention at the Speed of Light", abstract: sliding, strided sliding
+// and blocked windows; "ENA: Efficient N-dimensional Attention", sliding tile
+// attention: tokens of a tile share one window that shifts tile by tile).
+//
+// Schedule: queries are processed in blocks (boxes of the grid); a block's
+// keys lie in the per-dimension union of its queries' windows, which is a box
+// because the window start is monotone in the query coordinate and the N-d
+// window is a product of 1-D windows.  That key box is walked in chunks
+// (boxes of kb tokens).  A chunk is EMPTY for a block when it misses the
+// block's key box, FULL when it lies inside the intersection of all the
+// block's windows (no mask needed), else PARTIAL (element mask) -- the
+// empty / partial / full block taxonomy of "Hilbert-Guided Sparse Local
+// Attention" (Methodology in Plain English), with masks only on partial tiles.
+#pragma once
+
+#ifdef __CUDACC__
+#define NA_HD __host__ __device__ __forceinline__
+#else
+#define NA_HD inline
+#endif
+
+namespace na {
+
+enum ChunkStatus : int { CHUNK_EMPTY = 0, CHUNK_PARTIAL = 1, CHUNK_FULL = 2 };
+
+NA_HD int imin(int a, int b) { return a < b ? a : b; }
+NA_HD int imax(int a, int b) { return a > b ? a : b; }
+NA_HD int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+NA_HD int window_start(int L, int w, int s, int i) {
+  int g = i / s;
+  int c = g * s + s / 2;
+  int start = c - w / 2;
+  start = imax(start, 0);
+  start = imin(start, L - w);
+  return start;
+}
+
+struct Geom {
+  int L[3], w[3], s[3];
+};
+
+// Tiling of the queries: tiles of tl tokens per dim, each split into blocks
+// of qb tokens (qb divides tl).  Blocks are numbered tile by tile, row-major
+// over the tile grid and row-major over the blocks inside a tile, so that
+// consecutive block ids stay inside one tile where possible.
+struct QTiling {
+  int qb[3];      // block shape
+  int tl[3];      // tile shape (multiple of qb per dim)
+  int nt[3];      // tiles per dim = ceil(L / tl)
+  int bt[3];      // blocks per tile per dim = tl / qb
+  int bpt;        // blocks per tile
+  int nblocks;    // blocks per (batch, head)
+};
+
+// Per-dimension extents of one query block.
+struct BlockInfo {
+  int exists;      // 1 if the block holds at least one query inside the grid
+  int o[3];        // origin (grid coordinates of row 0)
+  int n[3];        // valid extent per dim (rows inside the grid)
+  int lo[3], hi[3];    // union of the valid queries' windows: [lo, hi)
+  int ilo[3], ihi[3];  // intersection of their windows: [ilo, ihi) (may be empty)
+};
+
+NA_HD void block_info(const Geom& g, const QTiling& t, int blk, BlockInfo& b) {
+  b.exists = 0;
+  if (blk < 0 || blk >= t.nblocks) return;
+  int tile = blk / t.bpt, sub = blk % t.bpt;
+  int tc[3], sc[3];
+  tc[2] = tile % t.nt[2]; tile /= t.nt[2];
+  tc[1] = tile % t.nt[1]; tc[0] = tile / t.nt[1];
+  sc[2] = sub % t.bt[2]; sub /= t.bt[2];
+  sc[1] = sub % t.bt[1]; sc[0] = sub / t.bt[1];
+  b.exists = 1;
+  for (int d = 0; d < 3; ++d) {
+    b.o[d] = tc[d] * t.tl[d] + sc[d] * t.qb[d];
+    b.n[d] = imin(t.qb[d], g.L[d] - b.o[d]);
+    if (b.n[d] <= 0) { b.exists = 0; b.n[d] = 0; continue; }
+    int first = window_start(g.L[d], g.w[d], g.s[d], b.o[d]);
+    int last = window_start(g.L[d], g.w[d], g.s[d], b.o[d] + b.n[d] - 1);
+    b.lo[d] = first;
+    b.hi[d] = last + g.w[d];
+    b.ilo[d] = last;
+    b.ihi[d] = first + g.w[d];
+  }
+}
+
+// Key box walked for a group of blocks (a CTA's blocks), in chunks of kb.
+struct ChunkGrid {
+  int org[3];     // origin of chunk (0,0,0)
+  int nc[3];      // chunks per dim
+  int total;
+};
+
+NA_HD void chunk_grid_for(const BlockInfo* bs, int nb, const int kb[3], ChunkGrid& cg) {
+  int lo[3] = {0, 0, 0}, hi[3] = {0, 0, 0};
+  int any = 0;
+  for (int i = 0; i < nb; ++i) {
+    if (!bs[i].exists) continue;
+    for (int d = 0; d < 3; ++d) {
+      lo[d] = any ? imin(lo[d], bs[i].lo[d]) : bs[i].lo[d];
+      hi[d] = any ? imax(hi[d], bs[i].hi[d]) : bs[i].hi[d];
+    }
+    any = 1;
+  }
+  cg.total = any ? 1 : 0;
+  for (int d = 0; d < 3; ++d) {
+    cg.org[d] = lo[d];
+    cg.nc[d] = any ? cdiv(hi[d] - lo[d], kb[d]) : 0;
+    cg.total *= cg.nc[d];
+  }
+}
+
+NA_HD void chunk_origin(const ChunkGrid& cg, const int kb[3], int c, int a[3]) {
+  int c2 = c % cg.nc[2]; c /= cg.nc[2];
+  int c1 = c % cg.nc[1]; int c0 = c / cg.nc[1];
+  a[0] = cg.org[0] + c0 * kb[0];
+  a[1] = cg.org[1] + c1 * kb[1];
+  a[2] = cg.org[2] + c2 * kb[2];
+}
+
+NA_HD int chunk_status(const BlockInfo& b, const int a[3], const int kb[3]) {
+  if (!b.exists) return CHUNK_EMPTY;
+  int full = 1;
+  for (int d = 0; d < 3; ++d) {
+    int c0 = a[d], c1 = a[d] + kb[d];
+    if (c1 <= b.lo[d] || c0 >= b.hi[d]) return CHUNK_EMPTY;
+    if (!(c0 >= b.ilo[d] && c1 <= b.ihi[d])) full = 0;
+  }
+  return full ? CHUNK_FULL : CHUNK_PARTIAL;
+}
+
+NA_HD int make_tiling(const Geom& g, const int qb[3], const int tl[3], QTiling& t) {
+  t.bpt = 1;
+  int ntiles = 1;
+  for (int d = 0; d < 3; ++d) {
+    t.qb[d] = qb[d];
+    t.tl[d] = tl[d];
+    if (qb[d] < 1 || tl[d] < qb[d] || tl[d] % qb[d]) return -1;
+    t.nt[d] = cdiv(g.L[d], tl[d]);
+    t.bt[d] = tl[d] / qb[d];
+    t.bpt *= t.bt[d];
+    ntiles *= t.nt[d];
+  }
+  t.nblocks = ntiles * t.bpt;
+  return 0;
+}
+
+}  // namespace na

@@ -1,0 +1,79 @@
+"""The C-ABI library loads on a machine without a GPU, exports every entry
+point include/na.h declares, and rejects bad arguments before touching any
+device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"\b(na_[a-z_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol():
+    import neighborhood_attention_b200 as na
+    lib = ctypes.CDLL(na.LIB_PATH)
+    names = _declared_functions()
+    assert "na_forward" in names and "na_sync_status" in names
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, f"declared but not exported: {missing}"
+
+
+def test_status_strings():
+    import neighborhood_attention_b200 as na
+    assert na.na_status_string(na.NA_OK) == "NA_OK"
+    assert na.na_status_string(na.NA_ERR_TIMEOUT) == "NA_ERR_TIMEOUT"
+    assert na.na_status_string(99) == "NA_ERR_UNKNOWN"
+    assert na.na_version() >= 100
+
+
+def _call(lib, q=16, dims=(2, 64), grid=(8, 8), window=(3, 3), stride=None, tile=None,
+          dtype=1, B=1, heads=1):
+    iv = lambda xs: None if xs is None else (ctypes.c_int * len(xs))(*xs)
+    p = lambda x: ctypes.c_void_p(x) if x else None
+    lib.na_forward.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_int] + \
+        [ctypes.POINTER(ctypes.c_int)] * 5 + [ctypes.c_int, ctypes.c_void_p]
+    return lib.na_forward(p(q), p(16), p(16), p(16), p(16), B, heads, iv(dims), iv(grid),
+                          iv(window), iv(stride), iv(tile), dtype, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=0), 1),                                 # NULL pointer
+    (dict(q=8), 1),                                 # misaligned pointer
+    (dict(B=0), 1),
+    (dict(dims=(4, 64)), 1),                        # ndim out of range
+    (dict(dims=(2, 0)), 1),
+    (dict(dims=(2, 48)), 2),                        # head_dim not supported
+    (dict(grid=(0, 8)), 1),
+    (dict(window=(9, 3)), 1),                       # window larger than grid
+    (dict(window=(0, 3)), 1),
+    (dict(stride=(4, 1)), 1),                       # stride larger than window
+    (dict(stride=(0, 1)), 1),
+    (dict(tile=(0, 4)), 1),
+    (dict(dtype=7), 1),
+])
+def test_argument_errors_need_no_device(kw, expect):
+    import neighborhood_attention_b200 as na
+    lib = ctypes.CDLL(na.LIB_PATH)
+    assert _call(lib, **kw) == expect
+    lib.na_last_error.restype = ctypes.c_char_p
+    assert lib.na_last_error().decode() != ""
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    import neighborhood_attention_b200 as na
+    q = torch.zeros(1, 1, 8, 8, 64, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 1, 8, 8)
+    with pytest.raises(ValueError):
+        na.na_forward(q, q, q, q.clone(), lse, window=(3, 3))

@@ -1,0 +1,104 @@
+"""The CUDA path's host-side tile scheduler against brute force: the window
+rule, each query block's key box, and every chunk's empty / partial / full
+label, checked pair by pair with the oracle's dense mask."""
+import itertools
+
+import numpy as np
+import pytest
+
+import neighborhood_attention_b200 as na
+
+
+def test_window_rule_matches_oracle(oracle_lib):
+    for L in range(1, 14):
+        for w in range(1, L + 1):
+            for s in range(1, w + 1):
+                for i in range(L):
+                    assert na.na_window_start(L, w, s, i) == oracle_lib.window_start(L, w, s, i)
+    assert na.na_window_start(5, 6, 1, 0) == -1
+    assert na.na_window_start(5, 3, 4, 0) == -1
+
+
+CASES = [
+    # grid, window, stride, qblock(3-d padded), kvchunk(3-d padded)
+    ([16, 16], [5, 5], [1, 1], [1, 4, 8], [1, 4, 8]),
+    ([12, 20], [7, 6], [2, 3], [1, 4, 4], [1, 2, 8]),
+    ([32, 32], [16, 16], [8, 8], [1, 8, 16], [1, 16, 8]),
+    ([6, 8, 10], [3, 4, 5], [3, 2, 5], [2, 2, 4], [1, 4, 4]),
+    ([9, 7, 5], [5, 7, 3], [1, 1, 1], [2, 4, 2], [4, 2, 2]),
+    ([40], [11], [3], [1, 1, 16], [1, 1, 8]),
+]
+
+
+@pytest.mark.parametrize("grid,window,stride,qb,kb", CASES)
+def test_block_schedule_bruteforce(grid, window, stride, qb, kb, oracle_lib):
+    nd = len(grid)
+    pad = 3 - nd
+    g3 = [1] * pad + list(grid)
+    N = int(np.prod(grid))
+    nblocks = int(np.prod([-(-g3[d] // qb[d]) for d in range(3)]))
+    masks = np.stack([oracle_lib.mask_row(grid, window, stride, t) for t in range(N)])
+    mask3 = masks.reshape([N] + g3)
+    for blk in range(nblocks):
+        s = na.na_block_schedule(grid, window, stride, qb, kb, blk)
+        o, n = s["origin"], s["extent"]
+        rows = [np.ravel_multi_index(tuple(c[pad:]), grid) if nd else 0
+                for c in itertools.product(*[range(o[d], o[d] + n[d]) for d in range(3)])]
+        assert len(rows) == int(np.prod(n)) > 0
+        m = mask3[rows]                                   # [rows, X1, X2, X3]
+        keys_any = m.any(axis=0)
+        keys_all = m.all(axis=0)
+        # key box = bounding box of the union of the windows (which is a box)
+        idx = np.nonzero(keys_any)
+        for d in range(3):
+            assert s["lo"][d] == idx[d].min() and s["hi"][d] == idx[d].max() + 1, (blk, d)
+        box = tuple(slice(s["lo"][d], s["hi"][d]) for d in range(3))
+        assert keys_any[box].all()
+        # chunks of the block's own key box, row-major
+        nc = [-(-(s["hi"][d] - s["lo"][d]) // kb[d]) for d in range(3)]
+        assert s["nchunks"] == int(np.prod(nc))
+        for c, cc in enumerate(itertools.product(*[range(x) for x in nc])):
+            a = [s["lo"][d] + cc[d] * kb[d] for d in range(3)]
+            inside = all(a[d] + kb[d] <= g3[d] for d in range(3))
+            sl = tuple(slice(a[d], min(a[d] + kb[d], g3[d])) for d in range(3))
+            sub_any, sub_all = keys_any[sl], keys_all[sl]
+            if not sub_any.any():
+                expect = 0
+            elif inside and sub_all.all():
+                expect = 2
+            else:
+                expect = 1
+            assert s["status"][c] == expect, (blk, c, a)
+
+
+def _cfg(i):
+    return {
+        1: dict(grid=[16, 16], window=[5, 5], stride=[1, 1], tile=None, d=32, dtype=na.NA_F32),
+        2: dict(grid=[64, 64], window=[13, 13], stride=[1, 1], tile=None, d=64, dtype=na.NA_BF16),
+        3: dict(grid=[128, 128], window=[32, 32], stride=[8, 8], tile=[8, 8], d=64,
+                dtype=na.NA_BF16),
+        4: dict(grid=[30, 48, 80], window=[18, 24, 40], stride=[6, 8, 8], tile=[6, 8, 8], d=128,
+                dtype=na.NA_BF16),
+        5: dict(grid=[16, 32, 32], window=[12, 20, 20], stride=[4, 4, 4], tile=[4, 4, 4], d=64,
+                dtype=na.NA_BF16),
+    }[i]
+
+
+@pytest.mark.parametrize("i", [1, 2, 3, 4, 5])
+def test_plan_statistics(i):
+    c = _cfg(i)
+    p = na.na_plan(c["grid"], c["window"], c["stride"], c["tile"], c["d"], c["dtype"])
+    N = int(np.prod(c["grid"]))
+    W = int(np.prod(c["window"]))
+    assert p["useful_pairs"] == N * W
+    assert p["computed_pairs"] >= p["useful_pairs"]
+    if i == 1:
+        assert p["kernel"] == "simt"
+    else:
+        assert p["kernel"] == "tc"
+        assert np.prod(p["qblock"]) == 128 and np.prod(p["kvchunk"]) == 128
+    if i == 4:
+        # sliding tile attention with tile-aligned windows: every chunk is
+        # full, nothing computed is masked out
+        assert p["units_partial"] == 0
+        assert p["computed_pairs"] == p["useful_pairs"]
