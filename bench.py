@@ -211,6 +211,23 @@ def run_reference(args, rank, world):
     return 0
 
 
+# ------------------------------------------------------------ rank logic --
+def max_over_ranks(values, world, device):
+    """Element-wise maximum of a list of floats over all ranks (identity when world == 1)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tflops(flops_per_rank_step, steps, world, max_ms):
+    """Whole-job throughput: the work every rank did (each rank runs one replica
+    of the workload per step) over the slowest rank's time."""
+    return flops_per_rank_step * steps * world / (max_ms / 1e3) / 1e12
+
+
 # ---------------------------------------------------------------- GPU side --
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -289,14 +306,11 @@ def run_ours(args, rank, world, local_rank):
     na.na_sync_status(stream)
     e2e_ms = e0.elapsed_time(e1)
 
-    times = torch.tensor([total_ms, e2e_ms, per_launch_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms, per_launch_ms = (float(x) for x in times.tolist())
+    total_ms, e2e_ms, per_launch_ms = max_over_ranks([total_ms, e2e_ms, per_launch_ms], world, dev)
 
     flops = flops_per_step()
-    value = flops * args.steps * world / (total_ms / 1e3) / 1e12
-    e2e_value = flops * args.steps * world / (e2e_ms / 1e3) / 1e12
+    value = whole_job_tflops(flops, args.steps, world, total_ms)
+    e2e_value = whole_job_tflops(flops, args.steps, world, e2e_ms)
     peak, peak_sustained, peak_kind = read_peaks()
     achieved = flops / (per_launch_ms / 1e3) / 1e12
     plan = na.na_plan(w["grid"], w["window"], w["stride"], w["tile"], w["head_dim"], na.NA_BF16)
@@ -333,9 +347,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="profiling only: run the workload with this many heads instead of 24 "
+                         "(the JSON line then reports that smaller workload)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.heads > 0:
+        WORKLOAD["heads"] = args.heads
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

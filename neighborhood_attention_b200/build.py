@@ -1,6 +1,9 @@
 """Build the CUDA library ``libna.so`` in-tree with nvcc for sm_100a.
 
-    python -m neighborhood_attention_b200.build [--force]
+    python neighborhood_attention_b200/build.py [--force] [-v]
+
+Run it by path (or load it with ``load_builder()`` from ``__graft_entry__``):
+importing the package itself requires the built library.
 
 The CUDA runtime is linked statically; the tensor-map encoder is reached
 through cudaGetDriverEntryPoint, so the library needs no -lcuda.

@@ -1,7 +1,7 @@
 """Helpers for the GPU parity tests: seeded inputs on both sides, the CUDA path
-through the C ABI, the fp64 oracle on the same host buffers, and the
-tolerances (from the problem statement: bf16 in / fp32 accumulate,
-max |out - oracle| <= 1e-2, mean <= 1e-3, |lse - oracle| <= 1e-3)."""
+through the C ABI, the fp64 oracle on the same host buffers, and the parity
+bar for bf16 inputs with fp32 accumulation on N(0, 1) data:
+max |out - oracle| <= 1e-2, mean |out - oracle| <= 1e-3, |lse - oracle| <= 1e-3."""
 from __future__ import annotations
 
 import numpy as np
