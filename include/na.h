@@ -162,6 +162,43 @@ na_status na_block_schedule(const int dims[2], const int* grid, const int* windo
 /* Library version, major*10000 + minor*100 + patch. */
 int na_version(void);
 
+/*
+ * na_forward_noalloc -- na_forward_ex for callers that must not allocate
+ * device memory.  The paper has no counterpart: this is a deployment entry
+ * point, not part of the method.
+ *
+ * Who needs it: hosts that own all device memory themselves -- for example a
+ * serving engine that reserves nearly all of HBM for its own pools up front,
+ * where a stray cudaMalloc would fail or slip past its memory accounting, or a
+ * latency-critical loop that cannot afford cudaMalloc's implicit device-wide
+ * synchronisation.  na_forward allocates one 4-byte status word per device on
+ * its first call; this entry point instead keeps that word in a fixed
+ * 256-byte array compiled into the library (every GPU that loads the library
+ * holds it until the process exits) and calls no cudaMalloc, cudaFree or other
+ * device-allocating routine.  Host-side planning may still use the C++ heap.
+ *
+ * Same arguments and layouts as na_forward_ex; the caller still passes q, k,
+ * v, out and lse.  It runs the tensor-core kernel only (bf16, head_dim 64 or
+ * 128; opt->kernel must be NA_KERNEL_AUTO or NA_KERNEL_TC), else returns
+ * NA_ERR_UNSUPPORTED.  The kernel's scratch need (4 bytes) is checked against
+ * the array's size and refused with NA_ERR_UNSUPPORTED if it ever exceeded it.
+ *
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture.
+ *
+ * Sharing: all calls on a device use the same array, which keeps the last
+ * call's contents.  Each call clears the status word on `stream` before its
+ * kernel, so calls whose kernels overlap on the GPU (different streams, no
+ * ordering between them) race on it.  A bounded in-kernel wait that expires
+ * leaves out/lse undefined and is not reported here (na_sync_status reads only
+ * na_forward's status word); use na_forward when that report is needed.
+ */
+na_status na_forward_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                             int B, int heads, const int dims[2], const int* grid,
+                             const int* window, const int* stride, const int* tile,
+                             na_dtype dtype, const na_options* opt, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -55,7 +55,7 @@ class na_plan_info(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: run `python -m neighborhood_attention_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: run `python neighborhood_attention_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     i32p = ctypes.POINTER(ctypes.c_int)
     vp = ctypes.c_void_p
@@ -83,6 +83,8 @@ def _load():
     lib.na_block_schedule.restype = ctypes.c_int
     lib.na_version.argtypes = []
     lib.na_version.restype = ctypes.c_int
+    lib.na_forward_noalloc.argtypes = lib.na_forward_ex.argtypes
+    lib.na_forward_noalloc.restype = ctypes.c_int
     return lib
 
 
@@ -188,6 +190,35 @@ def na_forward_ex(q, k, v, out, lse, window, stride=None, tile=None, options=Non
 def na_forward(q, k, v, out, lse, window, stride=None, tile=None, stream=None):
     """Enqueue na_forward (scale 1/sqrt(d), automatic kernel choice)."""
     return na_forward_ex(q, k, v, out, lse, window, stride, tile, None, stream)
+
+
+def na_forward_noalloc(q, k, v, out, lse, window, stride=None, tile=None, options=None,
+                       stream=None):
+    """Enqueue na_forward_noalloc: the tensor-core forward pass with its device
+    scratch in a fixed array inside the library, for callers that must not
+    allocate device memory (see include/na.h).  Same tensor contract as
+    na_forward_ex; allocates nothing (the caller passes out and lse)."""
+    import torch
+    nd = len(window)
+    shape = tuple(q.shape)
+    if len(shape) != nd + 3:
+        raise ValueError(f"q has shape {shape}; expected [B, heads, {nd} grid dims, d]")
+    for name, t in (("k", k), ("v", v), ("out", out)):
+        if tuple(t.shape) != shape or t.dtype != q.dtype:
+            raise ValueError(f"{name} must match q in shape and dtype")
+    if tuple(lse.shape) != shape[:-1] or lse.dtype != torch.float32:
+        raise ValueError("lse must be float32 with q's shape minus head_dim")
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    st = _lib.na_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr(), shape[0], shape[1], _ivec([nd, shape[-1]]),
+                                 _ivec(shape[2:2 + nd]), _ivec(window), _ivec(stride),
+                                 _ivec(tile), _dtype_of(q),
+                                 ctypes.byref(options) if options is not None else None,
+                                 _stream_ptr(stream))
+    _check(st)
+    return out, lse
 
 
 def na_sync_status(stream=None):

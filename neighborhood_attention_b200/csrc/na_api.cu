@@ -276,6 +276,38 @@ na_status status_word(int** out) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// ---------------------------------------------- allocation-free variant --
+// Device scratch of na_forward_noalloc: a fixed array in the library's own
+// device image instead of memory from cudaMalloc.  Every GPU that loads the
+// library holds these bytes until the process exits.  The tensor-core kernel
+// needs one 4-byte status word of it.
+constexpr size_t NOALLOC_SCRATCH_BYTES = 256;
+constexpr size_t TC_SCRATCH_BYTES = sizeof(int);
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[MAX_DEVICES] = {nullptr};
+
+// The device address of g_noalloc_scratch on the current device, looked up
+// once per device.  On the host the array's name is only a stand-in for the
+// device copy, so kernels must be given this address, never &g_noalloc_scratch.
+na_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= MAX_DEVICES) return fail(NA_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(NA_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return NA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -466,6 +498,59 @@ na_status na_block_schedule(const int dims[2], const int* grid, const int* windo
     chunk_origin(cg, kvchunk, c, a);
     status[c] = chunk_status(b, a, kvchunk);
   }
+  return NA_OK;
+}
+
+na_status na_forward_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                             int B, int heads, const int dims[2], const int* grid,
+                             const int* window, const int* stride, const int* tile,
+                             na_dtype dtype, const na_options* opt, void* stream) {
+  g_err[0] = 0;
+  if (!q || !k || !v || !out || !lse) return fail(NA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  if (B < 1 || heads < 1) return fail(NA_ERR_INVALID_ARG, "B=%d heads=%d must be >= 1", B, heads);
+  Problem P;
+  na_status st = read_problem(dims, grid, window, stride, tile, dtype, opt, P);
+  if (st != NA_OK) return st;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(lse, 4))
+    return fail(NA_ERR_INVALID_ARG, "q, k, v, out must be 16-byte aligned and lse 4-byte aligned");
+  const long long BH = (long long)B * heads;
+  if (BH > (1LL << 30)) return fail(NA_ERR_UNSUPPORTED, "B*heads too large");
+  if (P.opt.kernel == NA_KERNEL_SIMT)
+    return fail(NA_ERR_UNSUPPORTED, "na_forward_noalloc runs the tensor-core kernel only");
+  P.opt.kernel = NA_KERNEL_TC;
+  Plan plan;
+  st = make_plan(P, plan);
+  if (st != NA_OK) return st;
+  if (TC_SCRATCH_BYTES > NOALLOC_SCRATCH_BYTES)
+    return fail(NA_ERR_UNSUPPORTED, "needs %zu bytes of scratch; the static array holds %zu",
+                TC_SCRATCH_BYTES, NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != NA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // The array keeps the previous call's contents: the status word must start at 0.
+  cudaError_t e = cudaMemsetAsync(scratch, 0, TC_SCRATCH_BYTES, s);
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "clearing scratch: %s", cudaGetErrorString(e));
+  const float scale = P.opt.scale > 0.f ? P.opt.scale : 1.0f / sqrtf((float)P.D);
+  TcLaunch L;
+  L.g = P.g;
+  L.t = plan.t;
+  for (int d = 0; d < 3; ++d) L.kb[d] = plan.kb[d];
+  L.BH = (int)BH;
+  L.N = P.g.L[0] * P.g.L[1] * P.g.L[2];
+  L.D = P.D;
+  L.scale_log2 = scale * 1.4426950408889634f;
+  L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
+  L.status = static_cast<int*>(scratch);
+  L.timeout_ns = P.opt.wait_timeout_ns > 0 ? P.opt.wait_timeout_ns : default_timeout_ns();
+  L.debug_flags = P.opt.debug_flags;
+  char msg[256] = "";
+  e = launch_tc(L, s, msg, sizeof msg);
+  if (e == cudaErrorNotSupported)
+    return fail(NA_ERR_UNSUPPORTED, "tensor-core kernel does not take this shape");
+  if (e != cudaSuccess)
+    return fail(NA_ERR_CUDA, "tensor-core launch: %s %s", cudaGetErrorString(e), msg);
   return NA_OK;
 }
 
