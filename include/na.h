@@ -163,6 +163,15 @@ na_status na_block_schedule(const int dims[2], const int* grid, const int* windo
 int na_version(void);
 
 /*
+ * na_selftest_exp2 -- y[i] = 2^x[i] computed by the FMA-pipe polynomial the
+ * tensor-core kernel uses for part of its softmax exponentials (degree-3
+ * minimax fit of 2^f on [-1/2, 1/2], relative error <= 1.02e-4 for
+ * -125 <= x <= 8).  x and y are device float arrays of n elements; enqueued on
+ * `stream`.  For tests: it checks the device arithmetic against exact values.
+ */
+na_status na_selftest_exp2(const float* x, float* y, int n, void* stream);
+
+/*
  * na_forward_noalloc -- na_forward_ex for callers that must not allocate
  * device memory.  The paper has no counterpart: this is a deployment entry
  * point, not part of the method.

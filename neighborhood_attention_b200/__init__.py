@@ -85,6 +85,8 @@ def _load():
     lib.na_version.restype = ctypes.c_int
     lib.na_forward_noalloc.argtypes = lib.na_forward_ex.argtypes
     lib.na_forward_noalloc.restype = ctypes.c_int
+    lib.na_selftest_exp2.argtypes = [vp, vp, ctypes.c_int, vp]
+    lib.na_selftest_exp2.restype = ctypes.c_int
     return lib
 
 
@@ -219,6 +221,15 @@ def na_forward_noalloc(q, k, v, out, lse, window, stride=None, tile=None, option
                                  _stream_ptr(stream))
     _check(st)
     return out, lse
+
+
+def na_selftest_exp2(x, y, stream=None):
+    """y = 2^x by the kernel's FMA-pipe polynomial (float32 CUDA tensors)."""
+    import torch
+    if x.dtype != torch.float32 or y.dtype != torch.float32 or x.numel() != y.numel():
+        raise ValueError("x and y must be float32 tensors of the same size")
+    _check(_lib.na_selftest_exp2(x.data_ptr(), y.data_ptr(), x.numel(), _stream_ptr(stream)))
+    return y
 
 
 def na_sync_status(stream=None):

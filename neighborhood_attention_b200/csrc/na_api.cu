@@ -336,6 +336,14 @@ const char* na_last_error(void) { return g_err; }
 
 int na_version(void) { return 100; }
 
+na_status na_selftest_exp2(const float* x, float* y, int n, void* stream) {
+  g_err[0] = 0;
+  if (n < 0 || (n > 0 && (!x || !y))) return fail(NA_ERR_INVALID_ARG, "bad self-test arguments");
+  cudaError_t e = launch_exp2_selftest(x, y, n, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "exp2 self-test: %s", cudaGetErrorString(e));
+  return NA_OK;
+}
+
 int na_window_start(int L, int w, int s, int i) {
   if (L < 1 || w < 1 || w > L || s < 1 || s > w || i < 0 || i >= L) return -1;
   return window_start(L, w, s, i);

@@ -6,7 +6,7 @@
 // PARTIAL or FULL per block (na_sched.cuh), so masks are applied only on
 // partial chunks and a block skips chunks it does not see.
 //
-// Roles (12 warps):
+// Roles (12 warps, three warpgroups):
 //   warp 0     TMA producer: Q blocks once, then K and V chunks through an
 //              NS-slot shared-memory ring (128-byte swizzled, token-tile-major:
 //              each tile is a multi-dimensional box of the grid);
@@ -18,7 +18,11 @@
 //              TMEM as bf16 over its S, O rescaled in TMEM when the max moves;
 //              then the epilogue (O / l -> bf16, lse).
 // Two blocks ping-pong: while one block's softmax runs, the tensor core works
-// on the other block.
+// on the other block.  Warpgroup 0 hands most of its registers to the two
+// softmax warpgroups (setmaxnreg).  The softmax can evaluate a fixed share of
+// its exponentials on the FMA pipe (polynomial, EMU_NUM / EMU_DEN) instead of
+// the MUFU unit.  The MMA issuer learns each chunk's per-block status from the
+// producer (slot info written with the K tile), so its loop is straight-line.
 //
 // The arithmetic is the restricted softmax attention of "pi-Attention",
 // section 3.1 eqs. (1)-(3) and section 3.2 eq. (4), computed tile by tile
@@ -44,6 +48,19 @@ constexpr int TC_THREADS = 384;
 constexpr int BLOCK_M = 128;     // query rows per block
 constexpr int CHUNK_N = 128;     // keys per chunk
 constexpr int HALF_BYTES = 128 * 128;  // one 128-row x 64-element bf16 box (16 KB)
+constexpr int REGS_LOADER = 56;        // warpgroup 0 after setmaxnreg.dec
+constexpr int REGS_SOFTMAX = 216;      // warpgroups 1 and 2 after setmaxnreg.inc
+constexpr int REGS_NEEDED = 128 * REGS_LOADER + 256 * REGS_SOFTMAX;  // must fit the launch
+// Exponentials of P pair j go to the FMA-pipe polynomial when
+// (j * EMU_NUM) % EMU_DEN < EMU_NUM, i.e. EMU_NUM / EMU_DEN of them.  Measured
+// on the sliding-tile workload: 0/5 978, 1/5 913, 2/5 890, 3/5 857 TFLOP/s --
+// the softmax here is latency-bound in one warp per sub-partition, not
+// MUFU-bound, so every exponential currently stays on the MUFU unit.
+constexpr int EMU_NUM = 0;
+constexpr int EMU_DEN = 5;
+
+__host__ __device__ constexpr bool emulate_pair(int j) { return (j * EMU_NUM) % EMU_DEN < EMU_NUM; }
+constexpr uint32_t INFO_END = 0xFFFFu;   // slot info: no more chunks
 
 template <int D>
 struct TcCfg {
@@ -67,6 +84,9 @@ struct Bars {
   uint64_t o_done;
   uint32_t tmem_base;
   int abort;
+  volatile uint32_t info[NS];  // per K slot: chunk status of block 0 | block 1 << 2
+  BlockInfo bi[2];   // this CTA's two query blocks
+  ChunkGrid cg;      // and the chunk grid over their key box
 };
 
 template <int D>
@@ -75,18 +95,61 @@ constexpr size_t smem_bytes() {
          sizeof(Bars<TcCfg<D>::NS>);
 }
 
-// Next chunk index >= c that is non-empty for at least one block.
-__device__ __forceinline__ int next_chunk(const ChunkGrid& cg, const int* kb, const BlockInfo* bi,
-                                          int c, int& st0, int& st1) {
-  for (; c < cg.total; ++c) {
-    int a[3];
-    chunk_origin(cg, kb, c, a);
-    st0 = chunk_status(bi[0], a, kb);
-    st1 = chunk_status(bi[1], a, kb);
-    if (st0 != CHUNK_EMPTY || st1 != CHUNK_EMPTY) return c;
+// Advance `it` to the first chunk (at or after it) that is non-empty for at
+// least one of the two blocks; it.idx == cg.total when there is none.
+__device__ __forceinline__ void seek_pair(const ChunkGrid& cg, const int* kb, const BlockInfo* bi,
+                                          ChunkIter& it, int& st0, int& st1) {
+  for (; it.idx < cg.total; iter_next(cg, kb, it)) {
+    st0 = chunk_status(bi[0], it.a, kb);
+    st1 = chunk_status(bi[1], it.a, kb);
+    if (st0 != CHUNK_EMPTY || st1 != CHUNK_EMPTY) return;
   }
   st0 = st1 = CHUNK_EMPTY;
-  return cg.total;
+}
+
+// Bits i of 32-bit word w that mark keys j = 32w + i with (j mod period) in
+// [a, b): one grid dimension's window range laid over a chunk's key order.
+__device__ __forceinline__ uint32_t periodic_range_word(int w, int period, int a, int b) {
+  uint32_t m = 0;
+  const int base = 32 * w;
+  for (int p0 = base - base % period; p0 < base + 32; p0 += period) {
+    const int lo = imax(p0 + a, base) - base;
+    const int hi = imin(p0 + b, base + 32) - base;
+    if (lo < hi) m |= (hi - lo == 32 ? 0xffffffffu : ((1u << (hi - lo)) - 1u) << lo);
+  }
+  return m;
+}
+
+// Validity of the 128 keys of a chunk for one query: key j (chunk-local
+// coordinates (j >> sh0, (j >> sh1) & (kb1-1), j & (kb2-1))) is inside the
+// query's window [ws_d, ws_d + w_d) in every dimension.
+__device__ __forceinline__ void chunk_key_mask(const int a[3], const int ws[3], const int w[3],
+                                               const int kb[3], const int kbl[3], uint32_t (&mk)[4]) {
+  int lo[3], hi[3], stride[3];
+  stride[2] = 1;
+  stride[1] = 1 << kbl[2];
+  stride[0] = 1 << (kbl[1] + kbl[2]);
+  for (int d = 0; d < 3; ++d) {
+    lo[d] = imin(imax(ws[d] - a[d], 0), kb[d]);
+    hi[d] = imin(imax(ws[d] + w[d] - a[d], 0), kb[d]);
+  }
+#pragma unroll
+  for (int wd = 0; wd < 4; ++wd) {
+    uint32_t m = 0xffffffffu;
+    for (int d = 0; d < 3; ++d)
+      m &= periodic_range_word(wd, kb[d] * stride[d], lo[d] * stride[d], hi[d] * stride[d]);
+    mk[wd] = m;
+  }
+}
+
+// Same for one block: the status of the chunk found (CHUNK_EMPTY at the end).
+__device__ __forceinline__ int seek_block(const ChunkGrid& cg, const int* kb, const BlockInfo& b,
+                                          ChunkIter& it) {
+  for (; it.idx < cg.total; iter_next(cg, kb, it)) {
+    const int st = chunk_status(b, it.a, kb);
+    if (st != CHUNK_EMPTY) return st;
+  }
+  return CHUNK_EMPTY;
 }
 
 template <int D>
@@ -110,13 +173,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int npairs = (t.nblocks + 1) >> 1;
   const int bh = blockIdx.x / npairs;
   const int pair = blockIdx.x % npairs;
-  BlockInfo bi[2];
-  block_info(P.g, t, 2 * pair, bi[0]);
-  block_info(P.g, t, 2 * pair + 1, bi[1]);
-  ChunkGrid cg;
-  chunk_grid_for(bi, 2, P.kb, cg);
+  // Block descriptors and chunk grid live in shared memory, so no role holds
+  // them in registers across its main loop.
+  BlockInfo* bi = bars->bi;
+  const ChunkGrid& cg = bars->cg;
 
   if (threadIdx.x == 0) {
+    block_info(P.g, t, 2 * pair, bars->bi[0]);
+    block_info(P.g, t, 2 * pair + 1, bars->bi[1]);
+    chunk_grid_for(bars->bi, 2, P.kb, bars->cg);
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&bars->q_full[b], 1);
       ptx::mbar_init(&bars->s_full[b], 1);
@@ -146,6 +211,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   ctl.status = P.status;
   ctl.timeout_ns = (uint64_t)P.timeout_ns;
 
+  if (warp < 4) {
+  // Warpgroup 0: loader warps.  Each warpgroup rebalances registers at the top
+  // of its own branch so the compiler can apply each limit to its code only.
+  ptx::regs_dec<REGS_LOADER>();
   if (warp == 0) {
     // =========================== TMA producer ===========================
     if (lane == 0) {
@@ -160,26 +229,39 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           ptx::tma_load_5d(sQ + b * C::TILE_BYTES + h * HALF_BYTES, &tm_q, &bars->q_full[b],
                            h * 64, bi[b].o[2], bi[b].o[1], bi[b].o[0], bh);
       }
+      ChunkIter it;
+      iter_begin(cg, it);
       int st0, st1;
-      for (int c = next_chunk(cg, P.kb, bi, 0, st0, st1); c < cg.total;
-           c = next_chunk(cg, P.kb, bi, c + 1, st0, st1)) {
-        int a[3];
-        chunk_origin(cg, P.kb, c, a);
-        bool ok = true;
+      bool ok = true;
+      for (seek_pair(cg, P.kb, bi, it, st0, st1); ok && it.idx < cg.total;
+           iter_next(cg, P.kb, it), seek_pair(cg, P.kb, bi, it, st0, st1)) {
         for (int kv = 0; kv < 2 && ok; ++kv) {
           const int slot = seq % NS;
           if (seq >= NS) ok = ptx::wait(&bars->empty[slot], ((seq / NS) - 1) & 1, ctl);
           if (!ok) break;
+          // The K tile carries the chunk's per-block status to the MMA issuer
+          // (published by the arrive below, read after its wait on `full`).
+          if (kv == 0) bars->info[slot] = (uint32_t)st0 | ((uint32_t)st1 << 2);
           if (!((P.debug_flags & 1) && seq == 0)) {  // testing hook: withhold chunk 0's K
             ptx::mbar_expect_tx(&bars->full[slot], C::TILE_BYTES);
             for (int h = 0; h < C::HALVES; ++h)
               ptx::tma_load_5d(ring + slot * C::TILE_BYTES + h * HALF_BYTES, kv ? &tm_v : &tm_k,
-                               &bars->full[slot], h * 64, a[2], a[1], a[0], bh);
+                               &bars->full[slot], h * 64, it.a[2], it.a[1], it.a[0], bh);
             ++issued[slot];
           }
           ++seq;
         }
-        if (!ok) break;
+      }
+      if (ok) {
+        // End-of-stream marker in the slot where the next K tile would go.
+        const int slot = seq % NS;
+        if (seq >= NS) ok = ptx::wait(&bars->empty[slot], ((seq / NS) - 1) & 1, ctl);
+        if (ok) {
+          bars->info[slot] = INFO_END;
+          ptx::mbar_arrive(&bars->full[slot]);
+          ++issued[slot];
+          ++seq;
+        }
       }
       // Drain: every issued copy must land before the CTA can exit.
       for (int s = 0; s < NS; ++s)
@@ -193,14 +275,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint32_t sQa = ptx::smem_u32(sQ);
       const uint32_t ringa = ptx::smem_u32(ring);
       bool ok = true;
-      for (int b = 0; b < 2 && ok; ++b)
-        if (bi[b].exists) ok = ptx::wait(&bars->q_full[b], 0, ctl);
-      int pcount[2] = {0, 0};
-      bool have_pv[2] = {false, false};
-      int seq = 0;
-      int st0 = CHUNK_EMPTY, st1 = CHUNK_EMPTY;
-      int cur = ok ? next_chunk(cg, P.kb, bi, 0, st0, st1) : cg.total;
-      int cst[2] = {st0, st1};
+      if (bi[0].exists) ok = ptx::wait(&bars->q_full[0], 0, ctl);
+      if (ok && bi[1].exists) ok = ptx::wait(&bars->q_full[1], 0, ctl);
 
       // S = Q K^T for one block into its S columns.
       auto issue_s = [&](int b, int kslot) {
@@ -225,72 +301,67 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       };
 
-      if (cur < cg.total) {
-        const int kslot = seq % NS;
-        ok = ptx::wait(&bars->full[kslot], (seq / NS) & 1, ctl);
-        ++seq;
+      // Straight-line issue loop: per-block state in scalars, chunk statuses
+      // read from the slot info the producer wrote with each K tile.
+      int seq = 0;
+      uint32_t ph0 = 0, ph1 = 0;          // p_ready phases consumed per block
+      bool acc0 = false, acc1 = false;    // O of the block already written once
+      uint32_t cinfo = INFO_END;
+      if (ok) {
+        ok = ptx::wait(&bars->full[0], 0, ctl);  // first K tile (or the end marker)
+        seq = 1;
         if (ok) {
+          cinfo = bars->info[0];
           ptx::tc_fence_after();
-          for (int b = 0; b < 2; ++b)
-            if (cst[b] != CHUNK_EMPTY) {
-              issue_s(b, kslot);
-              ptx::tc_commit(&bars->s_full[b]);
-            }
-          ptx::tc_commit(&bars->empty[kslot]);
+          if (cinfo != INFO_END) {
+            if (cinfo & 3u) { issue_s(0, 0); ptx::tc_commit(&bars->s_full[0]); }
+            if (cinfo >> 2) { issue_s(1, 0); ptx::tc_commit(&bars->s_full[1]); }
+          }
+          ptx::tc_commit(&bars->empty[0]);
         }
       }
-      while (ok && cur < cg.total) {
-        const int vslot = seq % NS;
-        const int vseq = seq++;
-        int nst0, nst1;
-        const int nxt = next_chunk(cg, P.kb, bi, cur + 1, nst0, nst1);
-        const int nst[2] = {nst0, nst1};
-        int kslot = -1, kseq = -1;
-        bool k_ready = false;
-        if (nxt < cg.total) { kslot = seq % NS; kseq = seq++; }
+      while (ok && cinfo != INFO_END) {
+        const int vslot = seq % NS, vseq = seq++;
+        const int kslot = seq % NS, kseq = seq++;   // next K tile or the end marker
         ok = ptx::wait(&bars->full[vslot], (vseq / NS) & 1, ctl);
         if (!ok) break;
         ptx::tc_fence_after();
-        for (int b = 0; b < 2 && ok; ++b) {
-          if (cst[b] != CHUNK_EMPTY) {
-            ok = ptx::wait(&bars->p_ready[b], pcount[b] & 1, ctl);
-            if (!ok) break;
-            ++pcount[b];
-            ptx::tc_fence_after();
-            issue_pv(b, vslot, have_pv[b]);
-            have_pv[b] = true;
-          }
-          if (nxt < cg.total && nst[b] != CHUNK_EMPTY) {
-            if (!k_ready) {
-              ok = ptx::wait(&bars->full[kslot], (kseq / NS) & 1, ctl);
-              if (!ok) break;
-              ptx::tc_fence_after();
-              k_ready = true;
-            }
-            issue_s(b, kslot);
-            ptx::tc_commit(&bars->s_full[b]);
-          }
+        if (cinfo & 3u) {
+          ok = ptx::wait(&bars->p_ready[0], ph0 & 1, ctl);
+          if (!ok) break;
+          ++ph0;
+          ptx::tc_fence_after();
+          issue_pv(0, vslot, acc0);
+          acc0 = true;
         }
+        ok = ptx::wait(&bars->full[kslot], (kseq / NS) & 1, ctl);
         if (!ok) break;
-        ptx::tc_commit(&bars->empty[vslot]);
-        if (nxt < cg.total) {
-          if (!k_ready) {
-            ok = ptx::wait(&bars->full[kslot], (kseq / NS) & 1, ctl);
-            if (!ok) break;
-          }
-          ptx::tc_commit(&bars->empty[kslot]);
+        const uint32_t ninfo = bars->info[kslot];
+        ptx::tc_fence_after();
+        const bool more = ninfo != INFO_END;
+        if (more && (ninfo & 3u)) { issue_s(0, kslot); ptx::tc_commit(&bars->s_full[0]); }
+        if (cinfo >> 2) {
+          ok = ptx::wait(&bars->p_ready[1], ph1 & 1, ctl);
+          if (!ok) break;
+          ++ph1;
+          ptx::tc_fence_after();
+          issue_pv(1, vslot, acc1);
+          acc1 = true;
         }
-        cur = nxt;
-        cst[0] = nst[0];
-        cst[1] = nst[1];
+        if (more && (ninfo >> 2)) { issue_s(1, kslot); ptx::tc_commit(&bars->s_full[1]); }
+        ptx::tc_commit(&bars->empty[vslot]);
+        ptx::tc_commit(&bars->empty[kslot]);
+        cinfo = ninfo;
       }
       // All MMAs done (normal or unwinding): release the epilogue, then make
       // sure nothing still writes tensor memory before it is freed.
       ptx::tc_commit(&bars->o_done);
       ptx::wait_drain(&bars->o_done, 0, ctl);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
     // ===================== softmax + epilogue (per block) =====================
+    ptx::regs_inc<REGS_SOFTMAX>();
     const int b = (warp - 4) >> 2;
     const BlockInfo& B = bi[b];
     const int quarter = warp & 3;
@@ -299,16 +370,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const uint32_t tS = tmem + lane_base + C::S_COL0 + b * 128;
     const uint32_t tO = tmem + lane_base + C::O_COL0 + b * D;
 
-    // Query coordinates of this row (row-major over the block box).
-    const int r2 = row % t.qb[2];
-    const int r1 = (row / t.qb[2]) % t.qb[1];
-    const int r0 = row / (t.qb[2] * t.qb[1]);
-    const int g0 = B.o[0] + r0, g1 = B.o[1] + r1, g2 = B.o[2] + r2;
-    const bool valid = B.exists && g0 < P.g.L[0] && g1 < P.g.L[1] && g2 < P.g.L[2];
-    const int ws0 = window_start(P.g.L[0], P.g.w[0], P.g.s[0], imin(g0, P.g.L[0] - 1));
-    const int ws1 = window_start(P.g.L[1], P.g.w[1], P.g.s[1], imin(g1, P.g.L[1] - 1));
-    const int ws2 = window_start(P.g.L[2], P.g.w[2], P.g.s[2], imin(g2, P.g.L[2] - 1));
-    const int kb2 = P.kb[2], kb12 = P.kb[1] * P.kb[2];
+    // Grid coordinates of this thread's query (row-major over the block box);
+    // recomputed in the epilogue rather than kept live across the main loop.
+    auto query_coord = [&](int rr, int g[3]) {
+      g[2] = B.o[2] + rr % t.qb[2];
+      g[1] = B.o[1] + (rr / t.qb[2]) % t.qb[1];
+      g[0] = B.o[0] + rr / (t.qb[2] * t.qb[1]);
+    };
+    int ws[3];
+    {
+      int g[3];
+      query_coord(row, g);
+      for (int d = 0; d < 3; ++d)
+        ws[d] = window_start(P.g.L[d], P.g.w[d], P.g.s[d], imin(g[d], P.g.L[d] - 1));
+    }
     const float sl2 = P.scale_log2;
 
     float m = -INFINITY;   // reference max, log2 domain
@@ -317,11 +392,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     bool had_pv = false;
     bool ok = true;
     if (B.exists) {
-      int st0, st1;
-      for (int c = next_chunk(cg, P.kb, bi, 0, st0, st1); c < cg.total;
-           c = next_chunk(cg, P.kb, bi, c + 1, st0, st1)) {
-        const int st = b ? st1 : st0;
-        if (st == CHUNK_EMPTY) continue;
+      ChunkIter it;
+      iter_begin(cg, it);
+      for (int st = seek_block(cg, P.kb, B, it); it.idx < cg.total;
+           iter_next(cg, P.kb, it), st = seek_block(cg, P.kb, B, it)) {
         bool got = ptx::wait(&bars->s_full[b], scount & 1, ctl);
         got = __all_sync(0xffffffffu, got);
         if (!got) { ok = false; break; }
@@ -345,22 +419,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           ptx::reg_fence(s3);
         }
         if (st == CHUNK_PARTIAL) {
-          int a[3];
-          chunk_origin(cg, P.kb, c, a);
-          const int d0 = a[0] - ws0, d1 = a[1] - ws1, d2 = a[2] - ws2;
+          uint32_t mk[4];
+          chunk_key_mask(it.a, ws, P.g.w, P.kb, P.kb_log2, mk);
 #pragma unroll
-          for (int j = 0; j < 128; ++j) {
-            const int k2 = j % kb2, k1 = (j % kb12) / kb2, k0 = j / kb12;
-            const bool in = (unsigned)(d0 + k0) < (unsigned)P.g.w[0] &&
-                            (unsigned)(d1 + k1) < (unsigned)P.g.w[1] &&
-                            (unsigned)(d2 + k2) < (unsigned)P.g.w[2];
-            if (!in) s[j] = __float_as_uint(-INFINITY);
-          }
+          for (int j = 0; j < 128; ++j)
+            if (!((mk[j >> 5] >> (j & 31)) & 1u)) s[j] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < 128; ++j) mx = fmaxf(mx, __uint_as_float(s[j]));
-        const float mx2 = mx * sl2;
+        for (int j = 0; j < 128; j += 8) {
+          a0 = ptx::max3(a0, __uint_as_float(s[j]), __uint_as_float(s[j + 1]));
+          a1 = ptx::max3(a1, __uint_as_float(s[j + 2]), __uint_as_float(s[j + 3]));
+          a2 = ptx::max3(a2, __uint_as_float(s[j + 4]), __uint_as_float(s[j + 5]));
+          a3 = ptx::max3(a3, __uint_as_float(s[j + 6]), __uint_as_float(s[j + 7]));
+        }
+        const float mx2 = ptx::max3(a0, a1, fmaxf(a2, a3)) * sl2;
         // Move the reference max only when the new max exceeds it by more
         // than 2^8: P stays <= 256, exact after the final division by l.
         const bool need = mx2 > m + 8.f;
@@ -369,12 +442,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const float alpha = need ? ptx::ex2(m - m_use) : 1.f;
         const bool warp_need = __any_sync(0xffffffffu, need);
 
-        float sum = 0.f;
+        const uint64_t scale2 = ptx::f2(sl2, sl2);
+        const uint64_t negm2 = ptx::f2(-m_use, -m_use);
+        uint64_t acc0 = ptx::f2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
 #pragma unroll
         for (int j = 0; j < 64; ++j) {
-          const float p0 = ptx::ex2(fmaf(__uint_as_float(s[2 * j]), sl2, -m_use));
-          const float p1 = ptx::ex2(fmaf(__uint_as_float(s[2 * j + 1]), sl2, -m_use));
-          sum += p0 + p1;
+          const uint64_t x = ptx::f2_fma(
+              ptx::f2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), scale2, negm2);
+          float x0, x1, p0, p1;
+          ptx::f2_split(x, x0, x1);
+          if (emulate_pair(j)) {
+            ptx::exp2_poly_x2(x0, x1, p0, p1);
+          } else {
+            p0 = ptx::ex2(x0);
+            p1 = ptx::ex2(x1);
+          }
+          const uint64_t p = ptx::f2(p0, p1);
+          switch (j & 3) {
+            case 0: acc0 = ptx::f2_add(acc0, p); break;
+            case 1: acc1 = ptx::f2_add(acc1, p); break;
+            case 2: acc2 = ptx::f2_add(acc2, p); break;
+            default: acc3 = ptx::f2_add(acc3, p); break;
+          }
           s[j] = ptx::pack_bf16(p0, p1);
         }
         {
@@ -395,6 +484,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             ptx::tmem_st32(tO + cc * 32, o);
           }
         }
+        float q0, q1, q2, q3, q4, q5, q6, q7;
+        ptx::f2_split(acc0, q0, q1);
+        ptx::f2_split(acc1, q2, q3);
+        ptx::f2_split(acc2, q4, q5);
+        ptx::f2_split(acc3, q6, q7);
+        const float sum = ((q0 + q1) + (q2 + q3)) + ((q4 + q5) + (q6 + q7));
         l = l * alpha + sum;
         m = m_new;
         ptx::tmem_st_wait();
@@ -409,7 +504,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       got = __all_sync(0xffffffffu, got);
       if (got) {
         ptx::tc_fence_after();
-        const long long token = ((long long)g0 * P.g.L[1] + g1) * P.g.L[2] + g2;
+        int rr = row;
+        asm volatile("" : "+r"(rr));  // recompute, do not carry the coordinates
+        int g[3];
+        query_coord(rr, g);
+        const bool valid = B.exists && g[0] < P.g.L[0] && g[1] < P.g.L[1] && g[2] < P.g.L[2];
+        const long long token = ((long long)g[0] * P.g.L[1] + g[1]) * P.g.L[2] + g[2];
         const size_t rbase = ((size_t)bh * P.N + (size_t)(valid ? token : 0)) * D;
         const float inv_l = 1.f / l;
         uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(P.out) + rbase);
@@ -441,6 +541,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+__global__ void exp2_poly_selftest_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    ptx::exp2_poly_x2(x[i], x[i + 1], y[i], y[i + 1]);
+  } else if (i < n) {
+    float dummy;
+    ptx::exp2_poly_x2(x[i], 0.f, y[i], dummy);
   }
 }
 
@@ -491,8 +601,18 @@ cudaError_t launch_d(const TcLaunch& L, cudaStream_t stream, char* err, int errl
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(tc_fwd_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // setmaxnreg.inc waits for registers that the .dec of warpgroup 0 frees;
+    // refuse to launch if the compiled register count could not cover the split.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, tc_fwd_kernel<D>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * TC_THREADS < REGS_NEEDED) {
+      snprintf(err, errlen, "kernel compiled with %d registers/thread; the register split needs %d",
+               fa.numRegs, (REGS_NEEDED + TC_THREADS - 1) / TC_THREADS);
+      return cudaErrorInvalidConfiguration;
+    }
+    e = cudaFuncSetAttribute(tc_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
@@ -505,9 +625,22 @@ cudaError_t launch_d(const TcLaunch& L, cudaStream_t stream, char* err, int errl
 
 }  // namespace
 
-cudaError_t launch_tc(const TcLaunch& L, cudaStream_t stream, char* err, int errlen) {
+cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const int threads = 256;
+  const int blocks = ((n + 1) / 2 + threads - 1) / threads;
+  exp2_poly_selftest_kernel<<<blocks, threads, 0, stream>>>(x, y, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tc(const TcLaunch& L0, cudaStream_t stream, char* err, int errlen) {
+  TcLaunch L = L0;
   for (int d = 0; d < 3; ++d) {
     if (L.t.qb[d] > 256 || L.kb[d] > 256) return cudaErrorNotSupported;
+    if (L.kb[d] & (L.kb[d] - 1)) return cudaErrorNotSupported;  // powers of two only
+    int lg = 0;
+    while ((1 << lg) < L.kb[d]) ++lg;
+    L.kb_log2[d] = lg;
   }
   if (L.t.qb[0] * L.t.qb[1] * L.t.qb[2] != BLOCK_M || L.kb[0] * L.kb[1] * L.kb[2] != CHUNK_N)
     return cudaErrorNotSupported;

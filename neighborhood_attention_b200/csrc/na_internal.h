@@ -27,6 +27,7 @@ struct TcLaunch {
   Geom g;
   QTiling t;
   int kb[3];
+  int kb_log2[3];        // filled by launch_tc (chunk extents are powers of two)
   int BH, N, D;
   float scale_log2;
   const void *q, *k, *v;
@@ -38,6 +39,9 @@ struct TcLaunch {
 };
 
 cudaError_t launch_simt(const SimtLaunch& L, cudaStream_t stream);
+
+// y[i] = the tensor-core kernel's FMA-pipe 2^x applied to x[i] (self-test).
+cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t stream);
 
 // Returns cudaErrorNotSupported when the shape is outside the kernel's range.
 cudaError_t launch_tc(const TcLaunch& L, cudaStream_t stream, char* err, int errlen);

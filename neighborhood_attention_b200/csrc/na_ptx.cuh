@@ -54,7 +54,7 @@ struct WaitCtl {
   uint64_t timeout_ns;
 };
 
-__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, const WaitCtl& c,
+__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, const WaitCtl& c,
                                        bool honour_abort) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -193,6 +193,75 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed pairs of fp32 (sm_100 f32x2 instructions: two lanes of work per
+// issued instruction on the FMA pipe).
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair, on the FMA pipe instead of the MUFU unit (which the
+// softmax otherwise saturates).  Range reduction x = j + f with j the nearest
+// integer (adding 1.5 * 2^23 leaves j in the low mantissa bits) and
+// |f| <= 1/2; 2^f from p(f) = 1 + c1 f + c2 f^2 + c3 f^3, the minimax
+// relative-error fit on [-1/2, 1/2] with p(0) = 1 exactly (so 2^0 = 1 stays
+// exact), computed as a linear program on a dense grid by exp2_poly_fit.py:
+// max relative error 1.01e-4, well below bf16's 2^-9 rounding step of P.
+// 2^j is added into the exponent field.  Inputs are clamped to >= -126 so the
+// exponent cannot wrap; callers guarantee x <= 8.
+__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, float& y1) {
+  const float kShift = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = f2_add(x, f2(kShift, kShift));
+  const uint64_t j = f2_add(t, f2(-kShift, -kShift));
+  const uint64_t f = f2_fma(j, f2(-1.f, -1.f), x);
+  uint64_t p = f2_fma(f2(0.055008927149527376f, 0.055008927149527376f), f,
+                      f2(0.242210960010335f, 0.242210960010335f));
+  p = f2_fma(p, f, f2(0.6932829282143407f, 0.6932829282143407f));
+  p = f2_fma(p, f, f2(1.0f, 1.0f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
+// Re-balance the register file between warpgroups (sm_90+): every warp of a
+// warpgroup must execute the same instruction.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // Two floats to a packed bf16x2 (round-to-nearest-even); `lo` in bits 0..15.

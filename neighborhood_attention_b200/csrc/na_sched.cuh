@@ -131,6 +131,33 @@ NA_HD void chunk_origin(const ChunkGrid& cg, const int kb[3], int c, int a[3]) {
   a[2] = cg.org[2] + c2 * kb[2];
 }
 
+// Row-major walk over a chunk grid without divisions.
+struct ChunkIter {
+  int idx;      // linear chunk index; == ChunkGrid::total when exhausted
+  int c[3];     // chunk coordinates
+  int a[3];     // chunk origin in grid coordinates
+};
+
+NA_HD void iter_begin(const ChunkGrid& cg, ChunkIter& it) {
+  it.idx = 0;
+  for (int d = 0; d < 3; ++d) {
+    it.c[d] = 0;
+    it.a[d] = cg.org[d];
+  }
+}
+
+NA_HD void iter_next(const ChunkGrid& cg, const int kb[3], ChunkIter& it) {
+  ++it.idx;
+  if (++it.c[2] < cg.nc[2]) { it.a[2] += kb[2]; return; }
+  it.c[2] = 0;
+  it.a[2] = cg.org[2];
+  if (++it.c[1] < cg.nc[1]) { it.a[1] += kb[1]; return; }
+  it.c[1] = 0;
+  it.a[1] = cg.org[1];
+  ++it.c[0];
+  it.a[0] += kb[0];
+}
+
 NA_HD int chunk_status(const BlockInfo& b, const int a[3], const int kb[3]) {
   if (!b.exists) return CHUNK_EMPTY;
   int full = 1;
