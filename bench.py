@@ -91,7 +91,7 @@ def read_peaks():
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -106,12 +106,15 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
 
-    def stop(self):
+    def stop(self, windows=()):
+        """Median SM clock and throttle reasons over the samples taken inside
+        the given (start, end) wall-clock windows (all samples if none)."""
+        import datetime
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -124,14 +127,20 @@ class ClockSampler:
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    smax.append(float(parts[2]))
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    ts = None
+                if windows and (ts is None or not any(a <= ts <= b for a, b in windows)):
+                    continue
+                try:
+                    sm.append(float(parts[2]))
+                    smax.append(float(parts[3]))
                 except ValueError:
                     continue
-                for n, val in zip(names, parts[5:9]):
+                for n, val in zip(names, parts[6:10]):
                     if val.lower() == "active":
                         reasons.add(n)
         os.unlink(self.path)
@@ -255,10 +264,11 @@ def run_ours(args, rank, world, local_rank):
 
     sampler = ClockSampler(local_rank)
     sampler.start()
-    time.sleep(0.3)
+    time.sleep(1.0)   # let nvidia-smi start sampling before the timed region
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    w0 = time.time()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
@@ -270,9 +280,9 @@ def run_ours(args, rank, world, local_rank):
         ev[i][1].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
+    w1 = time.time()
     if world > 1:
         dist.barrier()
-    clocks = sampler.stop()
     na.na_sync_status(stream)
     total_ms = t_start.elapsed_time(t_end)
     per_launch_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
@@ -296,11 +306,14 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    w2 = time.time()
     e0.record(stream)
     for _ in range(args.steps):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
+    w3 = time.time()
+    clocks = sampler.stop(windows=[(w0, w1), (w2, w3)])
     if world > 1:
         dist.barrier()
     na.na_sync_status(stream)
@@ -343,7 +356,7 @@ def run_ours(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
