@@ -10,7 +10,10 @@ Definitions and sources are stated at the top of ``na_oracle.c``:
 softmax(QK^T/sqrt(d))V restricted to the window ("pi-Attention", section 3.1
 eqs. (1)-(3), section 3.2 eqs. (4)-(5)), with the window centred on the query's
 stride group and clamped inside the grid ("Generalized Neighborhood Attention"
-abstract; "ENA" sliding tile attention).
+abstract; "ENA" sliding tile attention).  Per grid dimension the window may
+instead be truncated at the grid border or causal ("pi-Attention" section 3.2
+eq. (5)); ``mode`` arguments take "clamped" / "truncated" / "causal" (or 0 / 1
+/ 2) per dimension, None meaning all clamped.
 """
 from __future__ import annotations
 
@@ -51,22 +54,26 @@ class OracleLib:
         i32p = ctypes.POINTER(ctypes.c_int)
         lib.na_oracle_window_start.argtypes = [ctypes.c_int] * 4
         lib.na_oracle_window_start.restype = ctypes.c_int
-        lib.na_oracle_mask_row.argtypes = [ctypes.c_int, i32p, i32p, i32p, ctypes.c_longlong,
-                                           ctypes.c_void_p]
-        lib.na_oracle_mask_row.restype = ctypes.c_int
+        lib.na_oracle_window.argtypes = [ctypes.c_int] * 5 + [i32p, i32p]
+        lib.na_oracle_window.restype = ctypes.c_int
+        lib.na_oracle_mask_row.argtypes = [ctypes.c_int, i32p, i32p, i32p, i32p,
+                                           ctypes.c_longlong, ctypes.c_void_p]
+        lib.na_oracle_mask_row.restype = ctypes.c_longlong
         lib.na_oracle_forward.argtypes = [
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong,
-            ctypes.c_int, i32p, i32p, i32p, ctypes.c_int, ctypes.c_double,
+            ctypes.c_int, i32p, i32p, i32p, i32p, ctypes.c_int, ctypes.c_double,
             ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
         lib.na_oracle_forward.restype = ctypes.c_int
-        lib.na_oracle_block_counts.argtypes = [ctypes.c_int, i32p, i32p, i32p, ctypes.c_longlong,
-                                               ctypes.c_void_p]
+        lib.na_oracle_block_counts.argtypes = [ctypes.c_int, i32p, i32p, i32p, i32p,
+                                               ctypes.c_longlong, ctypes.c_void_p]
         lib.na_oracle_block_counts.restype = ctypes.c_int
         self.lib = lib
         self.path = path
 
     @staticmethod
     def _ivec(vals):
+        if vals is None:
+            return None
         vals = [int(x) for x in vals]
         return (ctypes.c_int * len(vals))(*vals)
 
@@ -77,19 +84,29 @@ class OracleLib:
             raise ValueError(f"invalid window arguments L={L} w={w} s={s} i={i}")
         return r
 
-    def mask_row(self, grid, window, stride, token: int) -> np.ndarray:
+    def window(self, L: int, w: int, s: int, mode, i: int) -> tuple[int, int]:
+        """The 1-D window [lo, hi) of coordinate i under ``mode``."""
+        lo, hi = ctypes.c_int(), ctypes.c_int()
+        r = self.lib.na_oracle_window(L, w, s, _modes([mode], 1)[0], i, ctypes.byref(lo),
+                                      ctypes.byref(hi))
+        if r < 0:
+            raise ValueError(f"invalid window arguments L={L} w={w} s={s} mode={mode} i={i}")
+        return lo.value, hi.value
+
+    def mask_row(self, grid, window, stride, token: int, mode=None) -> np.ndarray:
         grid, window, stride = _geom(grid, window, stride)
         n = int(np.prod(grid))
         out = np.zeros(n, dtype=np.uint8)
         rc = self.lib.na_oracle_mask_row(len(grid), self._ivec(grid), self._ivec(window),
-                                         self._ivec(stride), int(token), out.ctypes.data)
-        if rc:
+                                         self._ivec(stride), self._ivec(_modes(mode, len(grid))),
+                                         int(token), out.ctypes.data)
+        if rc < 0:
             raise ValueError("na_oracle_mask_row: invalid arguments")
         return out.astype(bool)
 
     # -- forward -----------------------------------------------------------
     def forward(self, q, k, v, grid, window, stride, *, dtype: str, rows=None,
-                scale: float = 0.0, threads: int | None = None):
+                scale: float = 0.0, threads: int | None = None, mode=None):
         """Exact forward in fp64.
 
         q, k, v: arrays of shape [B, heads, *grid, d]; float32 values for
@@ -125,8 +142,8 @@ class OracleLib:
         rc = self.lib.na_oracle_forward(
             arrs[0].ctypes.data, arrs[1].ctypes.data, arrs[2].ctypes.data,
             0 if dtype == "f32" else 1, BH, nd, self._ivec(grid), self._ivec(window),
-            self._ivec(stride), d, float(scale), rows_ptr, nrows, out.ctypes.data,
-            lse.ctypes.data, int(threads or os.cpu_count() or 1))
+            self._ivec(stride), self._ivec(_modes(mode, nd)), d, float(scale), rows_ptr, nrows,
+            out.ctypes.data, lse.ctypes.data, int(threads or os.cpu_count() or 1))
         if rc:
             raise RuntimeError(f"na_oracle_forward failed with code {rc}")
         if rows is None:
@@ -134,12 +151,13 @@ class OracleLib:
         return out, lse
 
     # -- block counting ------------------------------------------------------
-    def block_counts(self, grid, window, stride, block: int):
+    def block_counts(self, grid, window, stride, block: int, mode=None):
         """(empty, partial, full) blk x blk tiles of the row-major attention map."""
         grid, window, stride = _geom(grid, window, stride)
         counts = np.zeros(3, dtype=np.int64)
         rc = self.lib.na_oracle_block_counts(len(grid), self._ivec(grid), self._ivec(window),
-                                             self._ivec(stride), int(block), counts.ctypes.data)
+                                             self._ivec(stride), self._ivec(_modes(mode, len(grid))),
+                                             int(block), counts.ctypes.data)
         if rc:
             raise ValueError("na_oracle_block_counts: invalid arguments")
         return tuple(int(c) for c in counts)
@@ -152,6 +170,21 @@ def _geom(grid, window, stride):
     if not (len(grid) == len(window) == len(stride)):
         raise ValueError("grid, window and stride must have the same length")
     return grid, window, stride
+
+
+MODES = {"clamped": 0, "truncated": 1, "causal": 2}
+
+
+def _modes(mode, nd):
+    """Per-dimension window modes as ints (None stays None: all clamped)."""
+    if mode is None:
+        return None
+    if isinstance(mode, (str, int)):
+        mode = [mode] * nd
+    out = [MODES[m] if isinstance(m, str) else int(m) for m in mode]
+    if len(out) != nd:
+        raise ValueError(f"{len(out)} window modes for {nd} dimensions")
+    return out
 
 
 def load(path: str | None = None) -> OracleLib:
@@ -168,13 +201,17 @@ def window_start(L, w, s, i):
     return load().window_start(L, w, s, i)
 
 
-def mask_row(grid, window, stride, token):
-    return load().mask_row(grid, window, stride, token)
+def window(L, w, s, mode, i):
+    return load().window(L, w, s, mode, i)
+
+
+def mask_row(grid, window, stride, token, mode=None):
+    return load().mask_row(grid, window, stride, token, mode)
 
 
 def forward(q, k, v, grid, window, stride, **kw):
     return load().forward(q, k, v, grid, window, stride, **kw)
 
 
-def block_counts(grid, window, stride, block):
-    return load().block_counts(grid, window, stride, block)
+def block_counts(grid, window, stride, block, mode=None):
+    return load().block_counts(grid, window, stride, block, mode)

@@ -39,6 +39,23 @@
  * inside the grid, so that every query sees exactly prod(w) keys) is the
  * plainest one consistent with both pages.
  *
+ * Window modes (chosen per grid dimension; the rule above is "clamped"):
+ *   truncated  the clamped rule's window taken before the clamp and cut to
+ *              the grid: [c - floor(w/2), c - floor(w/2) + w) intersected
+ *              with [0, L).  With s = 1 and w = 2k + 1 this is the
+ *              bidirectional neighbourhood {j : |j - i| <= k} of
+ *              "pi-Attention", section 3.2 eq. (5); queries near a border see
+ *              fewer keys instead of a shifted window.
+ *   causal     the w positions ending with the last position of the query's
+ *              stride group, cut to the grid: [(g+1)*s - w, (g+1)*s)
+ *              intersected with [0, L).  With s = 1 and w = k + 1 this is the
+ *              causal neighbourhood {j : max(0, i - k) <= j <= i} of eq. (5)
+ *              (self included, as the text after eq. (5) states).  For s > 1
+ *              every query of a group sees the whole group (block causal).
+ *   Eq. (5) has no stride; the stride readings above are this oracle's
+ *   (truncated: the same centring as the clamped rule; causal: the group as
+ *   the unit of causality) and coincide with eq. (5) at s = 1.
+ *
  * Block counting (empty / partial / full tiles of the N x N attention map in
  * row-major token order) follows "Hilbert-Guided Sparse Local Attention",
  * "Methodology in Plain English" (tiles labelled full, partial or empty).
@@ -55,6 +72,7 @@
 #define NA_ORACLE_MAXDIM 3
 
 enum { IN_F32 = 0, IN_BF16 = 1 };
+enum { WIN_CLAMPED = 0, WIN_TRUNCATED = 1, WIN_CAUSAL = 2 };
 
 /* ---------------------------------------------------------------- window -- */
 
@@ -68,11 +86,37 @@ int na_oracle_window_start(int L, int w, int s, int i) {
     return start;
 }
 
-static int check_geometry(int ndim, const int* L, const int* w, const int* s, long long* N) {
+/*
+ * Window of coordinate i in one dimension as the half-open range [*lo, *hi),
+ * for mode WIN_CLAMPED, WIN_TRUNCATED or WIN_CAUSAL (definitions above).
+ */
+int na_oracle_window(int L, int w, int s, int mode, int i, int* lo, int* hi) {
+    if (L < 1 || w < 1 || w > L || s < 1 || s > w || i < 0 || i >= L || !lo || !hi) return -1;
+    if (mode == WIN_CLAMPED) {
+        *lo = na_oracle_window_start(L, w, s, i);
+        *hi = *lo + w;
+        return 0;
+    }
+    int g = i / s;
+    int a;
+    if (mode == WIN_TRUNCATED)
+        a = g * s + s / 2 - w / 2;
+    else if (mode == WIN_CAUSAL)
+        a = (g + 1) * s - w;
+    else
+        return -1;
+    *lo = a < 0 ? 0 : a;
+    *hi = a + w > L ? L : a + w;
+    return 0;
+}
+
+static int check_geometry(int ndim, const int* L, const int* w, const int* s, const int* mode,
+                          long long* N) {
     if (ndim < 1 || ndim > NA_ORACLE_MAXDIM || !L || !w || !s) return -1;
     long long n = 1;
     for (int a = 0; a < ndim; ++a) {
         if (L[a] < 1 || w[a] < 1 || w[a] > L[a] || s[a] < 1 || s[a] > w[a]) return -1;
+        if (mode && (mode[a] < WIN_CLAMPED || mode[a] > WIN_CAUSAL)) return -1;
         n *= L[a];
     }
     *N = n;
@@ -86,26 +130,33 @@ static void unflatten(long long t, int ndim, const int* L, int* coord) {
     }
 }
 
-/* Dense membership row: mask[j] = 1 iff key token j is in the window of query token t. */
-int na_oracle_mask_row(int ndim, const int* L, const int* w, const int* s, long long t,
-                       uint8_t* mask) {
+/*
+ * Dense membership row: mask[j] = 1 iff key token j is in the window of query
+ * token t.  mode: per-dimension window modes, NULL = all clamped.  Returns the
+ * number of keys in the window (> 0), or -1 on invalid input.
+ */
+long long na_oracle_mask_row(int ndim, const int* L, const int* w, const int* s, const int* mode,
+                             long long t, uint8_t* mask) {
     long long N;
-    if (check_geometry(ndim, L, w, s, &N) || t < 0 || t >= N || !mask) return -1;
-    int qi[NA_ORACLE_MAXDIM], ws[NA_ORACLE_MAXDIM], kj[NA_ORACLE_MAXDIM];
+    if (check_geometry(ndim, L, w, s, mode, &N) || t < 0 || t >= N || !mask) return -1;
+    int qi[NA_ORACLE_MAXDIM], lo[NA_ORACLE_MAXDIM], hi[NA_ORACLE_MAXDIM], kj[NA_ORACLE_MAXDIM];
     unflatten(t, ndim, L, qi);
-    for (int a = 0; a < ndim; ++a) ws[a] = na_oracle_window_start(L[a], w[a], s[a], qi[a]);
+    for (int a = 0; a < ndim; ++a)
+        na_oracle_window(L[a], w[a], s[a], mode ? mode[a] : WIN_CLAMPED, qi[a], &lo[a], &hi[a]);
     for (int a = 0; a < ndim; ++a) kj[a] = 0;
+    long long count = 0;
     for (long long j = 0; j < N; ++j) {
         int in = 1;
         for (int a = 0; a < ndim; ++a)
-            if (kj[a] < ws[a] || kj[a] >= ws[a] + w[a]) in = 0;
+            if (kj[a] < lo[a] || kj[a] >= hi[a]) in = 0;
+        count += in;
         mask[j] = (uint8_t)in;
         for (int a = ndim - 1; a >= 0; --a) { /* advance the row-major key counter */
             if (++kj[a] < L[a]) break;
             kj[a] = 0;
         }
     }
-    return 0;
+    return count;
 }
 
 /* --------------------------------------------------------------- forward -- */
@@ -121,7 +172,7 @@ static inline double load_in(const void* p, int dtype, size_t idx) {
 typedef struct {
     const void *q, *k, *v;
     int dtype, ndim, d;
-    const int *L, *w, *s;
+    const int *L, *w, *s, *mode;
     long long N, BH, W;
     double scale;
     const long long* rows;
@@ -146,7 +197,7 @@ static void* fwd_worker(void* arg) {
         long long row = J->rows ? J->rows[r] : r;
         if (row < 0 || row >= J->BH * N) { J->status = -1; break; }
         long long bh = row / N, t = row % N;
-        na_oracle_mask_row(ndim, J->L, J->w, J->s, t, mask);
+        const long long inwin = na_oracle_mask_row(ndim, J->L, J->w, J->s, J->mode, t, mask);
         size_t qoff = (size_t)row * (size_t)d;
         long long cnt = 0;
         for (long long j = 0; j < N; ++j) {
@@ -160,7 +211,8 @@ static void* fwd_worker(void* arg) {
             idx[cnt] = j;
             ++cnt;
         }
-        if (cnt != J->W) { J->status = -3; goto done; } /* every query sees prod(w) keys */
+        /* clamped windows hold exactly prod(w) keys; every window at least one */
+        if (cnt != inwin || cnt < 1 || (!J->mode && cnt != J->W)) { J->status = -3; goto done; }
         double m = -INFINITY;
         for (long long e = 0; e < cnt; ++e) if (z[e] > m) m = z[e];
         double l = 0.0;
@@ -185,19 +237,21 @@ done:
 /*
  * q, k, v: [BH, N, d] with the N tokens in row-major grid order (last grid
  * dimension fastest), float32 (in_dtype 0) or bfloat16 bit patterns (1).
+ * mode: per-dimension window modes (WIN_*), or NULL for all clamped.
  * rows: NULL for every row 0..BH*N-1 (then nrows must be BH*N), else a list
  * of global row indices bh*N + token.  out: [nrows, d] fp64; lse: [nrows] fp64.
  * scale <= 0 means 1/sqrt(d).  Returns 0, or a negative code on bad input
- * (-1), allocation failure (-2) or a window that does not hold prod(w) keys (-3).
+ * (-1), allocation failure (-2) or a window whose key count is inconsistent (-3).
  */
 int na_oracle_forward(const void* q, const void* k, const void* v, int in_dtype, long long BH,
-                      int ndim, const int* L, const int* w, const int* s, int d, double scale,
+                      int ndim, const int* L, const int* w, const int* s, const int* mode, int d,
+                      double scale,
                       const long long* rows, long long nrows, double* out, double* lse,
                       int nthreads) {
     long long N;
     if (!q || !k || !v || !out || !lse || BH < 1 || d < 1 || nrows < 0) return -1;
     if (in_dtype != IN_F32 && in_dtype != IN_BF16) return -1;
-    if (check_geometry(ndim, L, w, s, &N)) return -1;
+    if (check_geometry(ndim, L, w, s, mode, &N)) return -1;
     if (!rows && nrows != BH * N) return -1;
     long long W = 1;
     for (int a = 0; a < ndim; ++a) W *= w[a];
@@ -212,7 +266,7 @@ int na_oracle_forward(const void* q, const void* k, const void* v, int in_dtype,
         fwd_job* J = &jobs[t];
         J->q = q; J->k = k; J->v = v;
         J->dtype = in_dtype; J->ndim = ndim; J->d = d;
-        J->L = L; J->w = w; J->s = s;
+        J->L = L; J->w = w; J->s = s; J->mode = mode;
         J->N = N; J->BH = BH; J->W = W;
         J->scale = scale;
         J->rows = rows;
@@ -241,16 +295,16 @@ int na_oracle_forward(const void* q, const void* k, const void* v, int in_dtype,
  * tiles and count empty (no query-key pair in a window), full (every pair in
  * a window) and partial tiles.  counts[0..2] = {empty, partial, full}.
  */
-int na_oracle_block_counts(int ndim, const int* L, const int* w, const int* s, long long blk,
-                           long long* counts) {
+int na_oracle_block_counts(int ndim, const int* L, const int* w, const int* s, const int* mode,
+                           long long blk, long long* counts) {
     long long N;
-    if (check_geometry(ndim, L, w, s, &N) || blk < 1 || !counts) return -1;
+    if (check_geometry(ndim, L, w, s, mode, &N) || blk < 1 || !counts) return -1;
     long long nb = (N + blk - 1) / blk;
     long long* members = (long long*)calloc((size_t)(nb * nb), sizeof(long long));
     uint8_t* mask = (uint8_t*)malloc((size_t)N);
     if (!members || !mask) { free(members); free(mask); return -2; }
     for (long long t = 0; t < N; ++t) {
-        na_oracle_mask_row(ndim, L, w, s, t, mask);
+        na_oracle_mask_row(ndim, L, w, s, mode, t, mask);
         long long* rowblk = members + (t / blk) * nb;
         for (long long j = 0; j < N; ++j) rowblk[j / blk] += mask[j];
     }

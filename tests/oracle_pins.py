@@ -319,6 +319,158 @@ def pin_ena_density_golden(lib):
             assert abs(frac - dens) <= tol, (t, frac)
 
 
+# ------------------------------------------------- truncated / causal modes --
+
+def _eq5_set(L, k, i, causal):
+    """"pi-Attention" section 3.2 eq. (5) written out: the causal
+    neighbourhood {j : max(0, i-k) <= j <= i} or the bidirectional one
+    {j : |j - i| <= k}, restricted to the grid [0, L)."""
+    if causal:
+        return {j for j in range(L) if max(0, i - k) <= j <= i}
+    return {j for j in range(L) if abs(j - i) <= k}
+
+
+def _mode_set(L, w, s, mode, i):
+    """Brute-force 1-D window of coordinate i for every mode.
+    clamped:   the brute-force nearest feasible window (_leader_start).
+    truncated: the clamped window of the same query on a grid padded by a
+               multiple of s on both sides (wide enough that nothing is
+               clamped there), mapped back and cut to [0, L).
+    causal:    the w positions ending with the largest coordinate of i's
+               stride group, cut to [0, L)."""
+    if mode == "clamped":
+        st = _leader_start(L, w, s, i)
+        return set(range(st, st + w))
+    if mode == "truncated":
+        P = s * (w + 1)
+        st = _leader_start(L + 2 * P, w, s, i + P) - P
+        return {j for j in range(st, st + w) if 0 <= j < L}
+    last = max(m for m in range(i, i + s) if m // s == i // s)
+    return {j for j in range(L) if 0 <= last - j < w}
+
+
+def _mode_mask(grid, window, stride, modes, token):
+    coords = np.unravel_index(token, grid)
+    N = int(np.prod(grid))
+    keys = np.array(np.unravel_index(np.arange(N), grid))
+    ok = np.ones(N, dtype=bool)
+    for a, (L, w, s, m) in enumerate(zip(grid, window, stride, modes)):
+        ok &= np.isin(keys[a], sorted(_mode_set(L, w, s, m, int(coords[a]))))
+    return ok
+
+
+def pin_truncated_eq5(lib):
+    """stride 1, w = 2k + 1: the truncated window is eq. (5)'s bidirectional
+    neighbourhood |j - i| <= k cut to the grid."""
+    for L in range(1, 24):
+        for w in range(1, L + 1, 2):
+            for i in range(L):
+                lo, hi = lib.window(L, w, 1, "truncated", i)
+                assert set(range(lo, hi)) == _eq5_set(L, (w - 1) // 2, i, False), (L, w, i)
+
+
+def pin_causal_eq5(lib):
+    """stride 1, w = k + 1: the causal window is eq. (5)'s causal
+    neighbourhood max(0, i-k) <= j <= i (self included)."""
+    for L in range(1, 24):
+        for w in range(1, L + 1):
+            for i in range(L):
+                lo, hi = lib.window(L, w, 1, "causal", i)
+                assert set(range(lo, hi)) == _eq5_set(L, w - 1, i, True), (L, w, i)
+
+
+def pin_modes_strided(lib):
+    """Every mode, stride and window on short grids vs the brute-force sets:
+    truncated = the unclamped centred window cut to the grid, causal = the w
+    positions ending with the query's stride group."""
+    for L in range(1, 15):
+        for w in range(1, L + 1):
+            for s in range(1, w + 1):
+                for i in range(L):
+                    for mode in ("clamped", "truncated", "causal"):
+                        lo, hi = lib.window(L, w, s, mode, i)
+                        assert set(range(lo, hi)) == _mode_set(L, w, s, mode, i), \
+                            (L, w, s, mode, i)
+
+
+def pin_mode_mask_bruteforce(lib):
+    """Dense mask rows with a different mode per dimension vs the product of
+    the brute-force 1-D sets."""
+    cases = [([7, 6], [5, 3], [1, 1], ["truncated", "causal"]),
+             ([6, 8], [4, 5], [2, 1], ["causal", "clamped"]),
+             ([4, 5, 6], [3, 3, 4], [1, 3, 2], ["causal", "truncated", "truncated"]),
+             ([9], [4], [2], ["causal"])]
+    for grid, window, stride, modes in cases:
+        N = int(np.prod(grid))
+        for t in range(N):
+            got = lib.mask_row(grid, window, stride, t, mode=modes)
+            assert np.array_equal(got, _mode_mask(grid, window, stride, modes, t)), (grid, t)
+
+
+def pin_causal_full_sdpa(lib):
+    """A causal window as long as the grid is causal attention: equals
+    torch's scaled_dot_product_attention(is_causal=True) in fp64.  Causal in
+    the outer dimension only, with whole-grid windows elsewhere, is
+    frame-causal attention: SDPA with a block lower-triangular boolean mask."""
+    import torch
+    import torch.nn.functional as F
+    d = 16
+    L = 37
+    q, k, v = (_randn(100 + t, (2, 3, L, d)) for t in range(3))
+    out, lse = lib.forward(q, k, v, [L], [L], [1], dtype="f32", mode=["causal"])
+    qt, kt, vt = (torch.from_numpy(a.astype(np.float64)) for a in (q, k, v))
+    ref = F.scaled_dot_product_attention(qt, kt, vt, is_causal=True).numpy()
+    np.testing.assert_allclose(out, ref, atol=1e-12, rtol=0)
+    s = (qt @ kt.transpose(-1, -2)) / math.sqrt(d)
+    s = s.masked_fill(~torch.ones(L, L, dtype=torch.bool).tril(), -math.inf)
+    np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), atol=1e-12, rtol=0)
+
+    grid = [5, 3, 4]
+    N = 60
+    q, k, v = (_randn(110 + t, (1, 2, *grid, d)) for t in range(3))
+    out, _ = lib.forward(q, k, v, grid, grid, [1, 1, 1], dtype="f32",
+                         mode=["causal", "clamped", "clamped"])
+    frame = torch.arange(N) // 12
+    mask = frame[None, :] <= frame[:, None]
+    qt, kt, vt = (torch.from_numpy(a.reshape(1, 2, N, d).astype(np.float64)) for a in (q, k, v))
+    ref = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask).numpy()
+    np.testing.assert_allclose(out.reshape(1, 2, N, d), ref, atol=1e-12, rtol=0)
+
+
+def pin_mode_uniform_queries(lib):
+    """q = 0 with cut windows: every row averages v over its own (smaller)
+    window, so lse = ln(window size) and the mean key coordinate is the centre
+    of the brute-force set, per row."""
+    for grid, window, stride, modes in [([9, 8], [5, 4], [1, 2], ["truncated", "causal"]),
+                                        ([6, 5, 7], [3, 5, 3], [3, 1, 1],
+                                         ["causal", "clamped", "truncated"])]:
+        nd = len(grid)
+        d = 4
+        N = int(np.prod(grid))
+        q = np.zeros((1, 1, *grid, d), dtype=np.float32)
+        k = _randn(121, (1, 1, *grid, d))
+        v = np.zeros((1, 1, *grid, d), dtype=np.float32)
+        coords = np.array(np.unravel_index(np.arange(N), grid)).T
+        v.reshape(N, d)[:, :nd] = coords
+        out, lse = lib.forward(q, k, v, grid, window, stride, dtype="f32", mode=modes)
+        for t in range(N):
+            sets = [_mode_set(grid[a], window[a], stride[a], modes[a], int(coords[t][a]))
+                    for a in range(nd)]
+            count = int(np.prod([len(x) for x in sets]))
+            assert abs(lse.reshape(N)[t] - math.log(count)) < 1e-13, (t, count)
+            expect = [np.mean(sorted(x)) for x in sets]
+            np.testing.assert_allclose(out.reshape(N, d)[t, :nd], expect, atol=1e-12, rtol=0)
+
+
+def pin_sa_empty_blocks_golden(lib):
+    """The Hilbert page's empty-block ratio for row-major slide attention
+    (Table 3, SA (Flex) at 96x96) reproduces from the truncated window."""
+    for side, win, blk, pct in _read_golden("sa_empty_block_ratio.txt"):
+        e, p, f = lib.block_counts([int(side)] * 2, [int(win)] * 2, [1, 1], int(blk),
+                                   mode="truncated")
+        assert round(100.0 * e / (e + p + f), 2) == round(pct, 2), (side, win, blk, e, p, f)
+
+
 def _read_golden(name):
     rows = []
     with open(os.path.join(GOLDEN, name)) as f:
@@ -334,8 +486,11 @@ ALL_PINS = [
     pin_window_sliding_tile, pin_window_blocked, pin_mask_bruteforce, pin_full_attention,
     pin_blocked_attention, pin_probability_rows, pin_uniform_queries, pin_single_key,
     pin_constant_values, pin_explicit_scale, pin_row_subset, pin_wsa_empty_blocks_golden,
-    pin_block_counts_closed_forms, pin_ena_density_golden,
+    pin_block_counts_closed_forms, pin_ena_density_golden, pin_truncated_eq5, pin_causal_eq5,
+    pin_modes_strided, pin_mode_mask_bruteforce, pin_causal_full_sdpa, pin_mode_uniform_queries,
+    pin_sa_empty_blocks_golden,
 ]
 
 # The golden-file pins take a few seconds each; mutant runs use the fast ones.
-FAST_PINS = [p for p in ALL_PINS if p not in (pin_wsa_empty_blocks_golden,)]
+FAST_PINS = [p for p in ALL_PINS if p not in (pin_wsa_empty_blocks_golden,
+                                              pin_sa_empty_blocks_golden)]

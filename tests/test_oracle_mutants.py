@@ -24,8 +24,14 @@ MUTANTS = [
     ("sign_flip_exp", "double p = exp(z[e] - m) / l;", "double p = exp(m - z[e]) / l;"),
     ("column_major_tokens", "for (int a = ndim - 1; a >= 0; --a) {\n        coord[a]",
      "for (int a = 0; a < ndim; ++a) {\n        coord[a]"),
-    ("mask_upper_inclusive", "kj[a] >= ws[a] + w[a]) in = 0;", "kj[a] > ws[a] + w[a]) in = 0;"),
+    ("mask_upper_inclusive", "kj[a] >= hi[a]) in = 0;", "kj[a] > hi[a]) in = 0;"),
     ("full_partial_swapped", "m == ra * cb ? 2 : 1", "m == ra * cb ? 1 : 2"),
+    ("causal_excludes_self", "a = (g + 1) * s - w;", "a = g * s - w;"),
+    ("causal_looks_ahead", "a = (g + 1) * s - w;", "a = g * s;"),
+    ("truncated_not_centred", "a = g * s + s / 2 - w / 2;", "a = g * s - w / 2;"),
+    ("truncated_as_clamped", "if (mode == WIN_CLAMPED) {", "if (mode != WIN_CAUSAL) {"),
+    ("cut_upper_short", "*hi = a + w > L ? L : a + w;", "*hi = a + w > L ? L - 1 : a + w;"),
+    ("mode_ignored_in_mask", "mode ? mode[a] : WIN_CLAMPED", "WIN_CLAMPED"),
 ]
 
 
