@@ -21,6 +21,17 @@
  * family named in the abstract of "Generalized Neighborhood Attention:
  * Multi-dimensional Sparse Attention at the Speed of Light".
  *
+ * Window modes (na_options.window_mode, per grid dimension) replace the
+ * clamp by a cut at the grid border, after "pi-Attention" section 3.2
+ * eq. (5):
+ *     truncated  [c - w/2, c - w/2 + w) intersected with [0, L)
+ *                (s = 1, w = 2k+1: the bidirectional |j - i| <= k)
+ *     causal     [(g+1)*s - w, (g+1)*s) intersected with [0, L)
+ *                (s = 1, w = k+1: the causal max(0, i-k) <= j <= i)
+ * so queries near a border (or near the start, for causal) see fewer keys.
+ * With s > 1 a causal window covers the query's whole stride group (block
+ * causal).
+ *
  * Layout.  q, k, v and out are dense row-major [B, heads, X1, .., Xn, d]
  * (n = ndim, last grid dimension fastest, then d); lse is [B, heads, X1..Xn].
  *
@@ -52,6 +63,13 @@ typedef enum {
 } na_status;
 
 typedef enum { NA_F32 = 0, NA_BF16 = 1 } na_dtype;
+
+/* Per-dimension window rule (see the top of this file). */
+typedef enum {
+  NA_WINDOW_CLAMPED = 0,    /* shifted inside the grid: always w keys (default) */
+  NA_WINDOW_TRUNCATED = 1,  /* centred, cut at the grid border */
+  NA_WINDOW_CAUSAL = 2      /* ending with the query's stride group, cut at 0 */
+} na_window_mode;
 
 typedef enum {
   NA_KERNEL_AUTO = 0,  /* tensor-core kernel where it applies, else the CUDA-core kernel */
@@ -95,6 +113,8 @@ typedef struct {
                                loader withholds the first key chunk, so the consumer's bounded
                                wait expires and the timeout path (NA_ERR_TIMEOUT from
                                na_sync_status) is exercised without any fault or hang. */
+  int window_mode[3];       /* na_window_mode of grid dimension i (i < ndim, the order of
+                               `window`); entries from ndim on are ignored.  0 = clamped. */
 } na_options;
 
 /* na_options with every field at its default (automatic) value. */
@@ -136,28 +156,35 @@ typedef struct {
   long long units_full;     /* (block, chunk) products with no mask */
   long long units_partial;  /* (block, chunk) products with an element mask */
   long long computed_pairs; /* (units_full + units_partial) * block rows * chunk keys */
-  long long useful_pairs;   /* N * prod(window) */
+  long long useful_pairs;   /* sum over queries of the window size (N * prod(window) when
+                               every dimension is clamped) */
 } na_plan_info;
 
 /* Fill *info for the given problem without touching the device. */
 na_status na_plan(const int dims[2], const int* grid, const int* window, const int* stride,
                   const int* tile, na_dtype dtype, const na_options* opt, na_plan_info* info);
 
-/* The 1-D window start used by the kernels (host copy), -1 on invalid input. */
+/* The 1-D clamped window start used by the kernels (host copy), -1 on invalid input. */
 int na_window_start(int L, int w, int s, int i);
+
+/* The 1-D window [*lo, *hi) of coordinate i under na_window_mode `mode`, as the
+ * kernels compute it (host copy).  Returns 0, or -1 on invalid input. */
+int na_window_range(int L, int w, int s, int mode, int i, int* lo, int* hi);
 
 /*
  * Key box and chunk classification of one query block, for tests: the
  * block's origin and valid extent, the union [lo, hi) and intersection
  * [ilo, ihi) of its queries' windows (3-d padded), and per key chunk of the
  * block's own key box (row-major over the chunk grid) its status 0 = empty,
- * 1 = partial, 2 = full.  `status` holds up to `max_chunks` entries; the
- * number of chunks is returned in *nchunks.
+ * 1 = partial, 2 = full.  window_mode: ndim na_window_mode values, or NULL
+ * for all clamped.  `status` holds up to `max_chunks` entries; the number of
+ * chunks is returned in *nchunks.
  */
 na_status na_block_schedule(const int dims[2], const int* grid, const int* window,
-                            const int* stride, const int qblock[3], const int kvchunk[3],
-                            long long block, int origin[3], int extent[3], int lo[3], int hi[3],
-                            int ilo[3], int ihi[3], int* status, int max_chunks, int* nchunks);
+                            const int* stride, const int* window_mode, const int qblock[3],
+                            const int kvchunk[3], long long block, int origin[3], int extent[3],
+                            int lo[3], int hi[3], int ilo[3], int ihi[3], int* status,
+                            int max_chunks, int* nchunks);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int na_version(void);

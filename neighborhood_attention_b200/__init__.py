@@ -7,7 +7,7 @@ no fallback of any kind.
 
 Functions keep the C-ABI names (``include/na.h``): ``na_forward``,
 ``na_forward_ex``, ``na_sync_status``, ``na_plan``, ``na_window_start``,
-``na_block_schedule``, ``na_status_string``, ``na_last_error``.
+``na_window_range``, ``na_block_schedule``, ``na_status_string``, ``na_last_error``.
 """
 from __future__ import annotations
 
@@ -21,6 +21,9 @@ NA_OK, NA_ERR_INVALID_ARG, NA_ERR_UNSUPPORTED, NA_ERR_CUDA, NA_ERR_TIMEOUT = ran
 NA_F32, NA_BF16 = 0, 1
 NA_KERNEL_AUTO, NA_KERNEL_SIMT, NA_KERNEL_TC = 0, 1, 2
 KERNEL_NAMES = {NA_KERNEL_AUTO: "auto", NA_KERNEL_SIMT: "simt", NA_KERNEL_TC: "tc"}
+NA_WINDOW_CLAMPED, NA_WINDOW_TRUNCATED, NA_WINDOW_CAUSAL = range(3)
+WINDOW_MODES = {"clamped": NA_WINDOW_CLAMPED, "truncated": NA_WINDOW_TRUNCATED,
+                "causal": NA_WINDOW_CAUSAL}
 
 
 class NaError(RuntimeError):
@@ -33,7 +36,8 @@ class NaError(RuntimeError):
 class na_options(ctypes.Structure):
     _fields_ = [("scale", ctypes.c_float), ("kernel", ctypes.c_int),
                 ("qblock", ctypes.c_int * 3), ("kvchunk", ctypes.c_int * 3),
-                ("wait_timeout_ns", ctypes.c_longlong), ("debug_flags", ctypes.c_int)]
+                ("wait_timeout_ns", ctypes.c_longlong), ("debug_flags", ctypes.c_int),
+                ("window_mode", ctypes.c_int * 3)]
 
 
 class na_plan_info(ctypes.Structure):
@@ -78,8 +82,11 @@ def _load():
     lib.na_plan.restype = ctypes.c_int
     lib.na_window_start.argtypes = [ctypes.c_int] * 4
     lib.na_window_start.restype = ctypes.c_int
-    lib.na_block_schedule.argtypes = [i32p, i32p, i32p, i32p, i32p, i32p, ctypes.c_longlong,
-                                      i32p, i32p, i32p, i32p, i32p, i32p, i32p, ctypes.c_int, i32p]
+    lib.na_window_range.argtypes = [ctypes.c_int] * 5 + [i32p, i32p]
+    lib.na_window_range.restype = ctypes.c_int
+    lib.na_block_schedule.argtypes = [i32p, i32p, i32p, i32p, i32p, i32p, i32p,
+                                      ctypes.c_longlong, i32p, i32p, i32p, i32p, i32p, i32p, i32p,
+                                      ctypes.c_int, i32p]
     lib.na_block_schedule.restype = ctypes.c_int
     lib.na_version.argtypes = []
     lib.na_version.restype = ctypes.c_int
@@ -125,9 +132,31 @@ def na_default_options() -> na_options:
     return _lib.na_default_options()
 
 
+def window_modes(mode, ndim: int):
+    """Per-dimension na_window_mode values from None (all clamped), one mode
+    for every dimension, or a sequence of ndim modes ("clamped", "truncated",
+    "causal" or the enum values)."""
+    if mode is None:
+        return [NA_WINDOW_CLAMPED] * ndim
+    if isinstance(mode, (str, int)):
+        mode = [mode] * ndim
+    out = [WINDOW_MODES[m] if isinstance(m, str) else int(m) for m in mode]
+    if len(out) != ndim:
+        raise ValueError(f"{len(out)} window modes for {ndim} grid dimensions")
+    return out
+
+
 def make_options(kernel: int = NA_KERNEL_AUTO, scale: float = 0.0, qblock=None, kvchunk=None,
-                 wait_timeout_ns: int = 0, debug_flags: int = 0) -> na_options:
+                 wait_timeout_ns: int = 0, debug_flags: int = 0, window_mode=None,
+                 ndim: int | None = None) -> na_options:
+    """na_options from keyword values; ``window_mode`` as in window_modes()
+    (a single mode needs ``ndim``, or applies to all three slots)."""
     o = na_default_options()
+    if window_mode is not None:
+        modes = window_modes(window_mode, ndim if ndim is not None else
+                             (3 if isinstance(window_mode, (str, int)) else len(window_mode)))
+        for i, m in enumerate(modes):
+            o.window_mode[i] = m
     o.kernel = int(kernel)
     o.scale = float(scale)
     if qblock is not None:
@@ -251,14 +280,25 @@ def na_window_start(L: int, w: int, s: int, i: int) -> int:
     return int(_lib.na_window_start(L, w, s, i))
 
 
-def na_block_schedule(grid, window, stride, qblock, kvchunk, block: int, max_chunks: int = 4096):
+def na_window_range(L: int, w: int, s: int, mode, i: int):
+    """The kernels' 1-D window (lo, hi) of coordinate i; None on invalid input."""
+    lo, hi = ctypes.c_int(), ctypes.c_int()
+    m = window_modes([mode], 1)[0]
+    if _lib.na_window_range(L, w, s, m, i, ctypes.byref(lo), ctypes.byref(hi)) != 0:
+        return None
+    return lo.value, hi.value
+
+
+def na_block_schedule(grid, window, stride, qblock, kvchunk, block: int, max_chunks: int = 4096,
+                      window_mode=None):
     """Key box and per-chunk status (0 empty, 1 partial, 2 full) of one query block."""
     arrs = {n: (ctypes.c_int * 3)() for n in ("origin", "extent", "lo", "hi", "ilo", "ihi")}
     status = (ctypes.c_int * max_chunks)()
     n = ctypes.c_int(0)
     dims = _ivec([len(grid), 32])
-    st = _lib.na_block_schedule(dims, _ivec(grid), _ivec(window), _ivec(stride), _ivec(qblock),
-                                _ivec(kvchunk), int(block), arrs["origin"], arrs["extent"],
+    modes = None if window_mode is None else _ivec(window_modes(window_mode, len(grid)))
+    st = _lib.na_block_schedule(dims, _ivec(grid), _ivec(window), _ivec(stride), modes,
+                                _ivec(qblock), _ivec(kvchunk), int(block), arrs["origin"], arrs["extent"],
                                 arrs["lo"], arrs["hi"], arrs["ilo"], arrs["ihi"], status,
                                 max_chunks, ctypes.byref(n))
     _check(st)
@@ -268,9 +308,16 @@ def na_block_schedule(grid, window, stride, qblock, kvchunk, block: int, max_chu
     return out
 
 
-def forward(q, k, v, window, stride=None, tile=None, options=None, stream=None):
-    """Allocate out / lse with torch and enqueue the forward pass; returns (out, lse)."""
+def forward(q, k, v, window, stride=None, tile=None, options=None, stream=None,
+            window_mode=None):
+    """Allocate out / lse with torch and enqueue the forward pass; returns (out, lse).
+    ``window_mode`` (as in window_modes()) overrides options.window_mode."""
     import torch
+    if window_mode is not None:
+        if options is None:
+            options = na_default_options()
+        for i, m in enumerate(window_modes(window_mode, len(window))):
+            options.window_mode[i] = m
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
     return na_forward_ex(q, k, v, out, lse, window, stride, tile, options, stream)

@@ -65,6 +65,7 @@ na_status read_problem(const int dims[2], const int* grid, const int* window, co
   const int pad = 3 - nd;
   for (int d = 0; d < 3; ++d) {
     P.g.L[d] = P.g.w[d] = P.g.s[d] = 1;
+    P.g.m[d] = WIN_CLAMPED;
     P.tile[d] = tile ? 1 : 0;
   }
   long long N = 1;
@@ -86,6 +87,12 @@ na_status read_problem(const int dims[2], const int* grid, const int* window, co
   P.opt = opt ? *opt : na_default_options();
   if (P.opt.kernel < NA_KERNEL_AUTO || P.opt.kernel > NA_KERNEL_TC)
     return fail(NA_ERR_INVALID_ARG, "unknown kernel selector %d", P.opt.kernel);
+  for (int i = 0; i < nd; ++i) {
+    const int m = P.opt.window_mode[i];
+    if (m < NA_WINDOW_CLAMPED || m > NA_WINDOW_CAUSAL)
+      return fail(NA_ERR_INVALID_ARG, "window_mode[%d]=%d is not a na_window_mode", i, m);
+    P.g.m[pad + i] = m;
+  }
   return NA_OK;
 }
 
@@ -181,7 +188,7 @@ na_status make_plan(const Problem& P, Plan& out) {
 
   std::vector<long long> key = {P.ndim, P.D, P.dtype, kernel};
   for (int d = 0; d < 3; ++d) {
-    key.insert(key.end(), {P.g.L[d], P.g.w[d], P.g.s[d], P.tile[d], P.opt.qblock[d],
+    key.insert(key.end(), {P.g.L[d], P.g.w[d], P.g.s[d], P.g.m[d], P.tile[d], P.opt.qblock[d],
                            P.opt.kvchunk[d]});
   }
   {
@@ -349,6 +356,13 @@ int na_window_start(int L, int w, int s, int i) {
   return window_start(L, w, s, i);
 }
 
+int na_window_range(int L, int w, int s, int mode, int i, int* lo, int* hi) {
+  if (L < 1 || w < 1 || w > L || s < 1 || s > w || i < 0 || i >= L || !lo || !hi) return -1;
+  if (mode < NA_WINDOW_CLAMPED || mode > NA_WINDOW_CAUSAL) return -1;
+  window_range(L, w, s, mode, i, *lo, *hi);
+  return 0;
+}
+
 na_status na_forward_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                         int heads, const int dims[2], const int* grid, const int* window,
                         const int* stride, const int* tile, na_dtype dtype,
@@ -469,18 +483,33 @@ na_status na_plan(const int dims[2], const int* grid, const int* window, const i
   info->units_full = c.full;
   info->units_partial = c.partial;
   info->computed_pairs = (c.full + c.partial) * rows * keys;
-  info->useful_pairs = (long long)P.g.L[0] * P.g.L[1] * P.g.L[2] *
-                       ((long long)P.g.w[0] * P.g.w[1] * P.g.w[2]);
+  // sum over queries of the window size = product over dimensions of the sum
+  // over coordinates of the 1-D window length (the window is a product).
+  long long useful = 1;
+  for (int d = 0; d < 3; ++d) {
+    long long sum = 0;
+    for (int i = 0; i < P.g.L[d]; ++i) {
+      int lo, hi;
+      window_range(P.g.L[d], P.g.w[d], P.g.s[d], P.g.m[d], i, lo, hi);
+      sum += hi - lo;
+    }
+    useful *= sum;
+  }
+  info->useful_pairs = useful;
   return NA_OK;
 }
 
 na_status na_block_schedule(const int dims[2], const int* grid, const int* window,
-                            const int* stride, const int qblock[3], const int kvchunk[3],
-                            long long block, int origin[3], int extent[3], int lo[3], int hi[3],
-                            int ilo[3], int ihi[3], int* status, int max_chunks, int* nchunks) {
+                            const int* stride, const int* window_mode, const int qblock[3],
+                            const int kvchunk[3], long long block, int origin[3], int extent[3],
+                            int lo[3], int hi[3], int ilo[3], int ihi[3], int* status,
+                            int max_chunks, int* nchunks) {
   g_err[0] = 0;
+  na_options o = na_default_options();
+  if (window_mode && dims && dims[0] >= 1 && dims[0] <= 3)
+    for (int i = 0; i < dims[0]; ++i) o.window_mode[i] = window_mode[i];
   Problem P;
-  na_status st = read_problem(dims, grid, window, stride, nullptr, NA_BF16, nullptr, P);
+  na_status st = read_problem(dims, grid, window, stride, nullptr, NA_BF16, &o, P);
   if (st != NA_OK) return st;
   if (!qblock || !kvchunk || !nchunks) return fail(NA_ERR_INVALID_ARG, "NULL argument");
   for (int d = 0; d < 3; ++d)

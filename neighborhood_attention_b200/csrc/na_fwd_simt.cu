@@ -48,12 +48,14 @@ __global__ void __launch_bounds__(SIMT_THREADS) simt_fwd_kernel(const SimtLaunch
   r[2] = qi % t.qb[2];
   r[1] = (qi / t.qb[2]) % t.qb[1];
   r[0] = qi / (t.qb[2] * t.qb[1]);
-  int gc[3], ws[3];
+  int gc[3], wlo[3], wn[3];  // this query's window: [wlo, wlo + wn) per dimension
   bool valid = qi < QPB;
   for (int d = 0; d < 3; ++d) {
     gc[d] = bi.o[d] + r[d];
     if (gc[d] >= g.L[d]) valid = false;
-    ws[d] = window_start(g.L[d], g.w[d], g.s[d], imin(gc[d], g.L[d] - 1));
+    int whi;
+    window_range(g.L[d], g.w[d], g.s[d], g.m[d], imin(gc[d], g.L[d] - 1), wlo[d], whi);
+    wn[d] = whi - wlo[d];
   }
   const long long token = ((long long)gc[0] * g.L[1] + gc[1]) * g.L[2] + gc[2];
   const size_t head_off = (size_t)bh * (size_t)P.N * D;
@@ -100,9 +102,9 @@ __global__ void __launch_bounds__(SIMT_THREADS) simt_fwd_kernel(const SimtLaunch
       float sv = dot * P.scale_log2;
       if (st == CHUNK_PARTIAL) {
         const int k2 = kk % P.kb[2], k1 = (kk / P.kb[2]) % P.kb[1], k0 = kk / (P.kb[2] * P.kb[1]);
-        const bool in = (unsigned)(a[0] + k0 - ws[0]) < (unsigned)g.w[0] &&
-                        (unsigned)(a[1] + k1 - ws[1]) < (unsigned)g.w[1] &&
-                        (unsigned)(a[2] + k2 - ws[2]) < (unsigned)g.w[2];
+        const bool in = (unsigned)(a[0] + k0 - wlo[0]) < (unsigned)wn[0] &&
+                        (unsigned)(a[1] + k1 - wlo[1]) < (unsigned)wn[1] &&
+                        (unsigned)(a[2] + k2 - wlo[2]) < (unsigned)wn[2];
         if (!in) sv = -INFINITY;
       }
       s[kk] = sv;

@@ -122,16 +122,16 @@ __device__ __forceinline__ uint32_t periodic_range_word(int w, int period, int a
 
 // Validity of the 128 keys of a chunk for one query: key j (chunk-local
 // coordinates (j >> sh0, (j >> sh1) & (kb1-1), j & (kb2-1))) is inside the
-// query's window [ws_d, ws_d + w_d) in every dimension.
-__device__ __forceinline__ void chunk_key_mask(const int a[3], const int ws[3], const int w[3],
+// query's window [wlo_d, whi_d) in every dimension.
+__device__ __forceinline__ void chunk_key_mask(const int a[3], const int wlo[3], const int whi[3],
                                                const int kb[3], const int kbl[3], uint32_t (&mk)[4]) {
   int lo[3], hi[3], stride[3];
   stride[2] = 1;
   stride[1] = 1 << kbl[2];
   stride[0] = 1 << (kbl[1] + kbl[2]);
   for (int d = 0; d < 3; ++d) {
-    lo[d] = imin(imax(ws[d] - a[d], 0), kb[d]);
-    hi[d] = imin(imax(ws[d] + w[d] - a[d], 0), kb[d]);
+    lo[d] = imin(imax(wlo[d] - a[d], 0), kb[d]);
+    hi[d] = imin(imax(whi[d] - a[d], 0), kb[d]);
   }
 #pragma unroll
   for (int wd = 0; wd < 4; ++wd) {
@@ -377,12 +377,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       g[1] = B.o[1] + (rr / t.qb[2]) % t.qb[1];
       g[0] = B.o[0] + rr / (t.qb[2] * t.qb[1]);
     };
-    int ws[3];
+    int wlo[3], whi[3];   // this row's window [wlo, whi) per dimension
     {
       int g[3];
       query_coord(row, g);
       for (int d = 0; d < 3; ++d)
-        ws[d] = window_start(P.g.L[d], P.g.w[d], P.g.s[d], imin(g[d], P.g.L[d] - 1));
+        window_range(P.g.L[d], P.g.w[d], P.g.s[d], P.g.m[d], imin(g[d], P.g.L[d] - 1), wlo[d],
+                     whi[d]);
     }
     const float sl2 = P.scale_log2;
 
@@ -420,7 +421,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         if (st == CHUNK_PARTIAL) {
           uint32_t mk[4];
-          chunk_key_mask(it.a, ws, P.g.w, P.kb, P.kb_log2, mk);
+          chunk_key_mask(it.a, wlo, whi, P.kb, P.kb_log2, mk);
 #pragma unroll
           for (int j = 0; j < 128; ++j)
             if (!((mk[j >> 5] >> (j & 31)) & 1u)) s[j] = __float_as_uint(-INFINITY);

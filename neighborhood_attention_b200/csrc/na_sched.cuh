@@ -7,7 +7,7 @@
 // coordinate i belongs to stride group g = i / s whose centre member is
 // c = g*s + s/2; its window is [start, start + w) with
 //   start = clamp(c - w/2, 0, L - w),
-// so every query sees exactly prod(w) keys.  Stride 1 is neighborhood
+// so every query sees exactly prod(w) keys ("clamped" mode).  Stride 1 is neighborhood
 // attention; stride equal to the tile with w an odd multiple of it is sliding
 // tile attention ("Generalized Neighborhood Attention: Multi-dimensional
 // Sparse Attention at the Speed of Light", abstract: sliding, strided sliding
@@ -34,6 +34,7 @@
 namespace na {
 
 enum ChunkStatus : int { CHUNK_EMPTY = 0, CHUNK_PARTIAL = 1, CHUNK_FULL = 2 };
+enum WindowMode : int { WIN_CLAMPED = 0, WIN_TRUNCATED = 1, WIN_CAUSAL = 2 };
 
 NA_HD int imin(int a, int b) { return a < b ? a : b; }
 NA_HD int imax(int a, int b) { return a > b ? a : b; }
@@ -48,8 +49,22 @@ NA_HD int window_start(int L, int w, int s, int i) {
   return start;
 }
 
+// Window [lo, hi) of coordinate i in one dimension under `mode`.
+NA_HD void window_range(int L, int w, int s, int mode, int i, int& lo, int& hi) {
+  if (mode == WIN_CLAMPED) {
+    lo = window_start(L, w, s, i);
+    hi = lo + w;
+    return;
+  }
+  const int g = i / s;
+  const int a = (mode == WIN_TRUNCATED) ? g * s + s / 2 - w / 2 : (g + 1) * s - w;
+  lo = imax(a, 0);
+  hi = imin(a + w, L);
+}
+
 struct Geom {
   int L[3], w[3], s[3];
+  int m[3];  // WindowMode per dimension
 };
 
 // Tiling of the queries: tiles of tl tokens per dim, each split into blocks
@@ -88,12 +103,13 @@ NA_HD void block_info(const Geom& g, const QTiling& t, int blk, BlockInfo& b) {
     b.o[d] = tc[d] * t.tl[d] + sc[d] * t.qb[d];
     b.n[d] = imin(t.qb[d], g.L[d] - b.o[d]);
     if (b.n[d] <= 0) { b.exists = 0; b.n[d] = 0; continue; }
-    int first = window_start(g.L[d], g.w[d], g.s[d], b.o[d]);
-    int last = window_start(g.L[d], g.w[d], g.s[d], b.o[d] + b.n[d] - 1);
-    b.lo[d] = first;
-    b.hi[d] = last + g.w[d];
-    b.ilo[d] = last;
-    b.ihi[d] = first + g.w[d];
+    int flo, fhi, llo, lhi;  // windows of the first and last valid query
+    window_range(g.L[d], g.w[d], g.s[d], g.m[d], b.o[d], flo, fhi);
+    window_range(g.L[d], g.w[d], g.s[d], g.m[d], b.o[d] + b.n[d] - 1, llo, lhi);
+    b.lo[d] = flo;
+    b.hi[d] = lhi;
+    b.ilo[d] = llo;
+    b.ihi[d] = fhi;
   }
 }
 

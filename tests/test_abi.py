@@ -77,3 +77,21 @@ def test_binding_refuses_cpu_tensors():
     lse = torch.zeros(1, 1, 8, 8)
     with pytest.raises(ValueError):
         na.na_forward(q, q, q, q.clone(), lse, window=(3, 3))
+
+
+@pytest.mark.parametrize("mode", [3, -1, 100])
+def test_bad_window_mode_is_refused(mode):
+    """An unknown na_window_mode is NA_ERR_INVALID_ARG, found on the host."""
+    import neighborhood_attention_b200 as na
+    opts = na.make_options(window_mode=[0, mode])
+    with pytest.raises(na.NaError) as e:
+        na.na_plan([8, 8], [3, 3], None, None, 64, na.NA_BF16, options=opts)
+    assert e.value.status == na.NA_ERR_INVALID_ARG
+    assert "window_mode[1]" in e.value.detail
+
+
+def test_window_mode_beyond_ndim_is_ignored():
+    import neighborhood_attention_b200 as na
+    opts = na.make_options(window_mode=[2, 1, 77])
+    p = na.na_plan([8, 8], [3, 3], None, None, 64, na.NA_BF16, options=opts)
+    assert p["useful_pairs"] > 0

@@ -19,6 +19,18 @@ def test_window_rule_matches_oracle(oracle_lib):
     assert na.na_window_start(5, 3, 4, 0) == -1
 
 
+def test_window_range_matches_oracle(oracle_lib):
+    for L in range(1, 14):
+        for w in range(1, L + 1):
+            for s in range(1, w + 1):
+                for i in range(L):
+                    for mode in ("clamped", "truncated", "causal"):
+                        assert na.na_window_range(L, w, s, mode, i) == \
+                            oracle_lib.window(L, w, s, mode, i), (L, w, s, mode, i)
+    assert na.na_window_range(5, 3, 1, 3, 0) is None
+    assert na.na_window_range(5, 3, 1, -1, 0) is None
+
+
 CASES = [
     # grid, window, stride, qblock(3-d padded), kvchunk(3-d padded)
     ([16, 16], [5, 5], [1, 1], [1, 4, 8], [1, 4, 8]),
@@ -28,19 +40,29 @@ CASES = [
     ([9, 7, 5], [5, 7, 3], [1, 1, 1], [2, 4, 2], [4, 2, 2]),
     ([40], [11], [3], [1, 1, 16], [1, 1, 8]),
 ]
+# the same with truncated / causal windows (mode per dimension)
+MODE_CASES = [
+    ([16, 16], [5, 5], [1, 1], [1, 4, 8], [1, 4, 8], ["truncated", "truncated"]),
+    ([12, 20], [7, 6], [2, 3], [1, 4, 4], [1, 2, 8], ["causal", "truncated"]),
+    ([6, 8, 10], [3, 4, 5], [3, 2, 5], [2, 2, 4], [1, 4, 4], ["causal", "clamped", "truncated"]),
+    ([9, 7, 5], [5, 7, 3], [1, 1, 1], [2, 4, 2], [4, 2, 2], ["truncated", "causal", "causal"]),
+    ([40], [11], [3], [1, 1, 16], [1, 1, 8], ["causal"]),
+    ([64], [17], [1], [1, 1, 16], [1, 1, 16], ["causal"]),
+]
 
 
-@pytest.mark.parametrize("grid,window,stride,qb,kb", CASES)
-def test_block_schedule_bruteforce(grid, window, stride, qb, kb, oracle_lib):
+@pytest.mark.parametrize("grid,window,stride,qb,kb,modes",
+                         [c + (None,) for c in map(tuple, CASES)] + [tuple(c) for c in MODE_CASES])
+def test_block_schedule_bruteforce(grid, window, stride, qb, kb, modes, oracle_lib):
     nd = len(grid)
     pad = 3 - nd
     g3 = [1] * pad + list(grid)
     N = int(np.prod(grid))
     nblocks = int(np.prod([-(-g3[d] // qb[d]) for d in range(3)]))
-    masks = np.stack([oracle_lib.mask_row(grid, window, stride, t) for t in range(N)])
+    masks = np.stack([oracle_lib.mask_row(grid, window, stride, t, mode=modes) for t in range(N)])
     mask3 = masks.reshape([N] + g3)
     for blk in range(nblocks):
-        s = na.na_block_schedule(grid, window, stride, qb, kb, blk)
+        s = na.na_block_schedule(grid, window, stride, qb, kb, blk, window_mode=modes)
         o, n = s["origin"], s["extent"]
         rows = [np.ravel_multi_index(tuple(c[pad:]), grid) if nd else 0
                 for c in itertools.product(*[range(o[d], o[d] + n[d]) for d in range(3)])]
@@ -102,3 +124,19 @@ def test_plan_statistics(i):
         # full, nothing computed is masked out
         assert p["units_partial"] == 0
         assert p["computed_pairs"] == p["useful_pairs"]
+
+
+@pytest.mark.parametrize("grid,window,stride,modes", [
+    ([12, 10], [5, 3], [1, 1], ["truncated", "causal"]),
+    ([6, 8, 9], [3, 4, 5], [3, 2, 1], ["causal", "clamped", "truncated"]),
+    ([50], [17], [1], ["causal"]),
+])
+def test_plan_useful_pairs_with_modes(grid, window, stride, modes, oracle_lib):
+    """useful_pairs = the number of (query, key) pairs the oracle's masks hold."""
+    N = int(np.prod(grid))
+    expect = sum(int(oracle_lib.mask_row(grid, window, stride, t, mode=modes).sum())
+                 for t in range(N))
+    opts = na.make_options(window_mode=modes)
+    p = na.na_plan(grid, window, stride, None, 64, na.NA_BF16, options=opts)
+    assert p["useful_pairs"] == expect
+    assert p["computed_pairs"] >= expect
