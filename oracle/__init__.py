@@ -67,6 +67,8 @@ class OracleLib:
         lib.na_oracle_block_counts.argtypes = [ctypes.c_int, i32p, i32p, i32p, i32p,
                                                ctypes.c_longlong, ctypes.c_void_p]
         lib.na_oracle_block_counts.restype = ctypes.c_int
+        lib.na_oracle_f16_value.argtypes = [ctypes.c_uint16]
+        lib.na_oracle_f16_value.restype = ctypes.c_double
         self.lib = lib
         self.path = path
 
@@ -110,13 +112,18 @@ class OracleLib:
         """Exact forward in fp64.
 
         q, k, v: arrays of shape [B, heads, *grid, d]; float32 values for
-        ``dtype="f32"`` or uint16 bfloat16 bit patterns for ``dtype="bf16"``.
+        ``dtype="f32"``, uint16 bfloat16 bit patterns for ``dtype="bf16"`` or
+        float16 values for ``dtype="f16"`` (decoded by the C code from their
+        bit patterns).
         rows: None for every query, else int64 global row ids (bh * N + token).
         Returns (out [nrows, d] float64, lse [nrows] float64); with rows=None
         out is reshaped to q's shape and lse to q's shape without d.
         """
         grid, window, stride = _geom(grid, window, stride)
-        want = np.float32 if dtype == "f32" else np.uint16
+        codes = {"f32": (np.float32, 0), "bf16": (np.uint16, 1), "f16": (np.float16, 2)}
+        if dtype not in codes:
+            raise ValueError(f"unknown dtype {dtype!r}")
+        want, code = codes[dtype]
         arrs = [np.ascontiguousarray(a) for a in (q, k, v)]
         for a in arrs:
             if a.dtype != want:
@@ -141,7 +148,7 @@ class OracleLib:
         lse = np.empty(nrows, dtype=np.float64)
         rc = self.lib.na_oracle_forward(
             arrs[0].ctypes.data, arrs[1].ctypes.data, arrs[2].ctypes.data,
-            0 if dtype == "f32" else 1, BH, nd, self._ivec(grid), self._ivec(window),
+            code, BH, nd, self._ivec(grid), self._ivec(window),
             self._ivec(stride), self._ivec(_modes(mode, nd)), d, float(scale), rows_ptr, nrows,
             out.ctypes.data, lse.ctypes.data, int(threads or os.cpu_count() or 1))
         if rc:
@@ -149,6 +156,10 @@ class OracleLib:
         if rows is None:
             return out.reshape(shape).astype(np.float64), lse.reshape(shape[:-1])
         return out, lse
+
+    def f16_value(self, bits: int) -> float:
+        """The oracle's decoding of one binary16 bit pattern."""
+        return float(self.lib.na_oracle_f16_value(int(bits)))
 
     # -- block counting ------------------------------------------------------
     def block_counts(self, grid, window, stride, block: int, mode=None):

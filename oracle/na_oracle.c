@@ -60,8 +60,9 @@
  * row-major token order) follows "Hilbert-Guided Sparse Local Attention",
  * "Methodology in Plain English" (tiles labelled full, partial or empty).
  *
- * Inputs are read as the exact float32 values, or the exact bfloat16 values
- * (16-bit patterns widened by a shift), that the GPU receives.
+ * Inputs are read as the exact float32 values, the exact bfloat16 values
+ * (16-bit patterns widened by a shift) or the exact IEEE 754 binary16 values
+ * (decoded below from the format's definition) that the GPU receives.
  */
 #include <math.h>
 #include <pthread.h>
@@ -71,7 +72,7 @@
 
 #define NA_ORACLE_MAXDIM 3
 
-enum { IN_F32 = 0, IN_BF16 = 1 };
+enum { IN_F32 = 0, IN_BF16 = 1, IN_F16 = 2 };
 enum { WIN_CLAMPED = 0, WIN_TRUNCATED = 1, WIN_CAUSAL = 2 };
 
 /* ---------------------------------------------------------------- window -- */
@@ -161,8 +162,26 @@ long long na_oracle_mask_row(int ndim, const int* L, const int* w, const int* s,
 
 /* --------------------------------------------------------------- forward -- */
 
+/*
+ * Value of an IEEE 754 binary16 bit pattern: sign bit, 5-bit exponent field e
+ * (bias 15), 10-bit fraction f.  e = 0: subnormal f * 2^-24; e = 31: infinity
+ * (f = 0) or NaN; otherwise (1024 + f) * 2^(e - 25) = (1 + f/1024) * 2^(e - 15).
+ */
+double na_oracle_f16_value(uint16_t h) {
+    const int e = (h >> 10) & 0x1f, f = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + f), e - 25);
+    return (h & 0x8000) ? -v : v;
+}
+
 static inline double load_in(const void* p, int dtype, size_t idx) {
     if (dtype == IN_F32) return (double)((const float*)p)[idx];
+    if (dtype == IN_F16) return na_oracle_f16_value(((const uint16_t*)p)[idx]);
     uint32_t bits = (uint32_t)((const uint16_t*)p)[idx] << 16;
     float f;
     memcpy(&f, &bits, sizeof f);
@@ -236,7 +255,8 @@ done:
 
 /*
  * q, k, v: [BH, N, d] with the N tokens in row-major grid order (last grid
- * dimension fastest), float32 (in_dtype 0) or bfloat16 bit patterns (1).
+ * dimension fastest), float32 (in_dtype 0), bfloat16 bit patterns (1) or
+ * binary16 bit patterns (2).
  * mode: per-dimension window modes (WIN_*), or NULL for all clamped.
  * rows: NULL for every row 0..BH*N-1 (then nrows must be BH*N), else a list
  * of global row indices bh*N + token.  out: [nrows, d] fp64; lse: [nrows] fp64.
@@ -250,7 +270,7 @@ int na_oracle_forward(const void* q, const void* k, const void* v, int in_dtype,
                       int nthreads) {
     long long N;
     if (!q || !k || !v || !out || !lse || BH < 1 || d < 1 || nrows < 0) return -1;
-    if (in_dtype != IN_F32 && in_dtype != IN_BF16) return -1;
+    if (in_dtype != IN_F32 && in_dtype != IN_BF16 && in_dtype != IN_F16) return -1;
     if (check_geometry(ndim, L, w, s, mode, &N)) return -1;
     if (!rows && nrows != BH * N) return -1;
     long long W = 1;

@@ -3,9 +3,10 @@ CUDA side of every test and of the benchmark.
 
 This module holds no attention arithmetic.  It only maps (seed, element index)
 to a standard-normal sample through a counter-based SplitMix64 generator and a
-Box-Muller transform (see ``gen.c``), then rounds to float32 or bfloat16
-(round-to-nearest-even).  Both sides receive the very same host buffers, so the
-oracle reads exactly the bf16/fp32 values that the GPU receives.
+Box-Muller transform (see ``gen.c``), then rounds to float32, bfloat16 or
+float16 (round-to-nearest-even; float16 by numpy's conversion).  Both sides
+receive the very same host buffers, so the oracle reads exactly the values
+that the GPU receives.
 """
 from __future__ import annotations
 
@@ -85,15 +86,21 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32)
 
 
+def normal_f16(seed: int, shape, scale: float = 1.0, threads: int | None = None) -> np.ndarray:
+    """The float32 samples of ``normal_f32`` rounded to float16 (nearest even)."""
+    return normal_f32(seed, shape, scale, threads).astype(np.float16)
+
+
 def qkv(seed_base: int, B: int, heads: int, grid, head_dim: int, dtype: str,
         threads: int | None = None):
     """(q, k, v) host arrays of shape [B, heads, *grid, head_dim].
 
-    ``dtype`` is "f32" (float32 arrays) or "bf16" (uint16 bit-pattern arrays).
-    Streams ``seed_base + 0/1/2`` feed q, k and v respectively.
+    ``dtype`` is "f32" (float32 arrays), "bf16" (uint16 bit-pattern arrays) or
+    "f16" (float16 arrays).  Streams ``seed_base + 0/1/2`` feed q, k and v.
     """
     shape = (B, heads, *tuple(grid), head_dim)
-    gen = normal_f32 if dtype == "f32" else normal_bf16_bits
-    if dtype not in ("f32", "bf16"):
+    gens = {"f32": normal_f32, "bf16": normal_bf16_bits, "f16": normal_f16}
+    if dtype not in gens:
         raise ValueError(f"unknown dtype {dtype!r}")
+    gen = gens[dtype]
     return tuple(gen(seed_base + t, shape, threads=threads) for t in range(3))

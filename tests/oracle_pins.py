@@ -151,12 +151,15 @@ def pin_mask_bruteforce(lib):
 def pin_full_attention(lib):
     """window = whole grid: equals dense softmax attention (numpy matmuls)."""
     for grid, stride, d, dtype in [([7, 5], [2, 3], 16, "f32"), ([3, 4, 5], [1, 2, 5], 8, "f32"),
-                                   ([23], [1], 12, "bf16")]:
+                                   ([23], [1], 12, "bf16"), ([6, 7], [3, 1], 16, "f16")]:
         B, H = 2, 1
         shape = (B, H, *grid, d)
         if dtype == "f32":
             q, k, v = (_randn(70 + t, shape) for t in range(3))
             qf, kf, vf = q, k, v
+        elif dtype == "f16":
+            q, k, v = (seeded_inputs.normal_f16(85 + t, shape, threads=1) for t in range(3))
+            qf, kf, vf = (a.astype(np.float64) for a in (q, k, v))
         else:
             q, k, v = (seeded_inputs.normal_bf16_bits(80 + t, shape, threads=1) for t in range(3))
             qf, kf, vf = (seeded_inputs.bf16_bits_to_f32(a) for a in (q, k, v))
@@ -317,6 +320,18 @@ def pin_ena_density_golden(lib):
         for t in (0, 1000, 2080, 4095):
             frac = lib.mask_row(grid, win, [1, 1], t).mean()
             assert abs(frac - dens) <= tol, (t, frac)
+
+
+def pin_f16_decoding(lib):
+    """The oracle's binary16 decoding equals numpy's float16 -> float64
+    conversion for all 65,536 bit patterns (NaN patterns decode to NaN)."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([lib.f16_value(int(b)) for b in bits])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
 
 
 # ------------------------------------------------- truncated / causal modes --
@@ -488,7 +503,7 @@ ALL_PINS = [
     pin_constant_values, pin_explicit_scale, pin_row_subset, pin_wsa_empty_blocks_golden,
     pin_block_counts_closed_forms, pin_ena_density_golden, pin_truncated_eq5, pin_causal_eq5,
     pin_modes_strided, pin_mode_mask_bruteforce, pin_causal_full_sdpa, pin_mode_uniform_queries,
-    pin_sa_empty_blocks_golden,
+    pin_sa_empty_blocks_golden, pin_f16_decoding,
 ]
 
 # The golden-file pins take a few seconds each; mutant runs use the fast ones.

@@ -32,6 +32,9 @@ MUTANTS = [
     ("truncated_as_clamped", "if (mode == WIN_CLAMPED) {", "if (mode != WIN_CAUSAL) {"),
     ("cut_upper_short", "*hi = a + w > L ? L : a + w;", "*hi = a + w > L ? L - 1 : a + w;"),
     ("mode_ignored_in_mask", "mode ? mode[a] : WIN_CLAMPED", "WIN_CLAMPED"),
+    ("f16_exponent_bias", "ldexp((double)(1024 + f), e - 25)", "ldexp((double)(1024 + f), e - 24)"),
+    ("f16_subnormal_as_normal", "v = ldexp((double)f, -24);", "v = ldexp((double)(1024 + f), -25);"),
+    ("f16_read_as_bf16", "if (dtype == IN_F16) return", "if (dtype == -1) return"),
 ]
 
 
