@@ -369,7 +369,7 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_sustained, peak_kind = read_peaks()
     achieved = flops / (per_launch_ms / 1e3) / 1e12
     plan = na.na_plan(w["grid"], w["window"], w["stride"], w["tile"], w["head_dim"],
-                      na.NA_BF16 if w["dtype"] == "bf16" else na.NA_F32)
+                      {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32}[w["dtype"]])
     if rank != 0:
         return 0
     base = cpu_baseline(qkv_host) if world == 1 and not args.no_cpu_baseline else None
@@ -388,7 +388,10 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak,
                      "traffic": read_traffic() if TRAFFIC_APPLIES else None,
-                     "peak_kind": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)" if peak_kind == "measured" else "fallback"},
+                     "peak_kind": (f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)"
+                                   + (" x 1: f16 and bf16 share the nominal dense rate"
+                                      if w["dtype"] == "f16" else "")
+                                   if peak_kind == "measured" else "fallback")},
         "cpu_baseline": base,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -410,6 +413,8 @@ def main():
     ap.add_argument("--config", type=int, default=4, choices=sorted(WORKLOADS),
                     help="workload: 4 (default) is the 3-D sliding tile one the metric is "
                          "quoted on; 1, 2, 3, 5 are the other parity workloads")
+    ap.add_argument("--dtype", choices=["bf16", "f16"], default=None,
+                    help="input type of a 16-bit workload (default: the workload's own, bf16)")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling only: run the workload with this many heads instead of 24 "
                          "(the JSON line then reports that smaller workload)")
@@ -423,6 +428,12 @@ def main():
         TRAFFIC_APPLIES = False
     if args.heads > 0:
         WORKLOAD["heads"] = args.heads
+        TRAFFIC_APPLIES = False
+    if args.dtype and args.dtype != WORKLOAD["dtype"]:
+        if WORKLOAD["dtype"] == "f32":
+            ap.error("--dtype applies to the 16-bit workloads only")
+        WORKLOAD = dict(WORKLOAD, dtype=args.dtype)
+        METRIC = f"effective TFLOP/s, {WORKLOAD['workload']}, {args.dtype} inputs"
         TRAFFIC_APPLIES = False
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -62,7 +62,7 @@ typedef enum {
   NA_ERR_TIMEOUT = 4       /* a bounded in-kernel wait expired (reported by na_sync_status) */
 } na_status;
 
-typedef enum { NA_F32 = 0, NA_BF16 = 1 } na_dtype;
+typedef enum { NA_F32 = 0, NA_BF16 = 1, NA_F16 = 2 } na_dtype;
 
 /* Per-dimension window rule (see the top of this file). */
 typedef enum {
@@ -73,8 +73,8 @@ typedef enum {
 
 typedef enum {
   NA_KERNEL_AUTO = 0,  /* tensor-core kernel where it applies, else the CUDA-core kernel */
-  NA_KERNEL_SIMT = 1,  /* CUDA-core kernel (fp32 and bf16, head_dim 32/64/128) */
-  NA_KERNEL_TC = 2     /* tcgen05 tensor-core kernel (bf16, head_dim 64/128) */
+  NA_KERNEL_SIMT = 1,  /* CUDA-core kernel (fp32, bf16 and f16, head_dim 32/64/128) */
+  NA_KERNEL_TC = 2     /* tcgen05 tensor-core kernel (bf16 or f16, head_dim 64/128) */
 } na_kernel;
 
 /*
@@ -91,8 +91,10 @@ typedef enum {
  *             groups queries for scheduling (results do not depend on it): the
  *             tensor-core path splits a tile of >= 128 tokens into 128-query
  *             blocks, or joins tiles of < 128 tokens into such blocks.
- *   dtype     NA_F32 (CUDA-core kernel) or NA_BF16 (tensor-core kernel when
- *             head_dim is 64 or 128).
+ *   dtype     NA_F32 (CUDA-core kernel), NA_BF16 or NA_F16 (tensor-core kernel
+ *             when head_dim is 64 or 128; out is written in the input type and
+ *             P, the softmax weights fed to the second product, are rounded to
+ *             it as well).
  *   stream    cudaStream_t.
  * Returns NA_OK once the work is queued, NA_ERR_INVALID_ARG / NA_ERR_UNSUPPORTED
  * without touching the device, or NA_ERR_CUDA.  Scale is 1/sqrt(head_dim).
@@ -215,7 +217,8 @@ na_status na_selftest_exp2(const float* x, float* y, int n, void* stream);
  *
  * Same arguments and layouts as na_forward_ex; the caller still passes q, k,
  * v, out and lse.  It runs the tensor-core kernel only (bf16, head_dim 64 or
- * 128; opt->kernel must be NA_KERNEL_AUTO or NA_KERNEL_TC), else returns
+ * 128, or f16 with the same head dims; opt->kernel must be NA_KERNEL_AUTO or
+ * NA_KERNEL_TC), else returns
  * NA_ERR_UNSUPPORTED.  The kernel's scratch need (4 bytes) is checked against
  * the array's size and refused with NA_ERR_UNSUPPORTED if it ever exceeded it.
  *

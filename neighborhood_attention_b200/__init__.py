@@ -18,7 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libna.so")
 
 NA_OK, NA_ERR_INVALID_ARG, NA_ERR_UNSUPPORTED, NA_ERR_CUDA, NA_ERR_TIMEOUT = range(5)
-NA_F32, NA_BF16 = 0, 1
+NA_F32, NA_BF16, NA_F16 = 0, 1, 2
 NA_KERNEL_AUTO, NA_KERNEL_SIMT, NA_KERNEL_TC = 0, 1, 2
 KERNEL_NAMES = {NA_KERNEL_AUTO: "auto", NA_KERNEL_SIMT: "simt", NA_KERNEL_TC: "tc"}
 NA_WINDOW_CLAMPED, NA_WINDOW_TRUNCATED, NA_WINDOW_CAUSAL = range(3)
@@ -174,9 +174,12 @@ def _dtype_of(t) -> int:
     import torch
     if t.dtype == torch.bfloat16:
         return NA_BF16
+    if t.dtype == torch.float16:
+        return NA_F16
     if t.dtype == torch.float32:
         return NA_F32
-    raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16 or torch.float32")
+    raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16, torch.float16 or "
+                    "torch.float32")
 
 
 def _stream_ptr(stream) -> int:

@@ -58,7 +58,8 @@ na_status read_problem(const int dims[2], const int* grid, const int* window, co
   if (D != 32 && D != 64 && D != 128)
     return fail(NA_ERR_UNSUPPORTED, "head_dim=%d not in {32, 64, 128}", D);
   if (!grid || !window) return fail(NA_ERR_INVALID_ARG, "grid or window is NULL");
-  if (dtype != NA_F32 && dtype != NA_BF16) return fail(NA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (dtype != NA_F32 && dtype != NA_BF16 && dtype != NA_F16)
+    return fail(NA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
   P.ndim = nd;
   P.D = D;
   P.dtype = dtype;
@@ -179,10 +180,11 @@ std::map<std::vector<long long>, Plan> g_plans;
 
 na_status make_plan(const Problem& P, Plan& out) {
   int kernel = P.opt.kernel;
+  const bool half = P.dtype == NA_BF16 || P.dtype == NA_F16;
   if (kernel == NA_KERNEL_AUTO)
-    kernel = (P.dtype == NA_BF16 && (P.D == 64 || P.D == 128)) ? NA_KERNEL_TC : NA_KERNEL_SIMT;
-  if (kernel == NA_KERNEL_TC && P.dtype != NA_BF16)
-    return fail(NA_ERR_UNSUPPORTED, "the tensor-core kernel takes bf16 only");
+    kernel = (half && (P.D == 64 || P.D == 128)) ? NA_KERNEL_TC : NA_KERNEL_SIMT;
+  if (kernel == NA_KERNEL_TC && !half)
+    return fail(NA_ERR_UNSUPPORTED, "the tensor-core kernel takes bf16 or f16 only");
   if (kernel == NA_KERNEL_TC && P.D != 64 && P.D != 128)
     return fail(NA_ERR_UNSUPPORTED, "the tensor-core kernel takes head_dim 64 or 128");
 
@@ -397,6 +399,7 @@ na_status na_forward_ex(const void* q, const void* k, const void* v, void* out, 
     L.BH = (int)BH;
     L.N = (int)N;
     L.D = P.D;
+    L.f16 = P.dtype == NA_F16;
     L.scale_log2 = scale * log2e;
     L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
     L.status = status;
@@ -417,7 +420,7 @@ na_status na_forward_ex(const void* q, const void* k, const void* v, void* out, 
   L.BH = (int)BH;
   L.N = (int)N;
   L.D = P.D;
-  L.bf16 = P.dtype == NA_BF16;
+  L.dtype = P.dtype;
   L.scale_log2 = scale * log2e;
   L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
   cudaError_t e = launch_simt(L, s);
@@ -577,6 +580,7 @@ na_status na_forward_noalloc(const void* q, const void* k, const void* v, void* 
   L.BH = (int)BH;
   L.N = P.g.L[0] * P.g.L[1] * P.g.L[2];
   L.D = P.D;
+  L.f16 = P.dtype == NA_F16;
   L.scale_log2 = scale * 1.4426950408889634f;
   L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
   L.status = static_cast<int*>(scratch);

@@ -1,4 +1,4 @@
-// CUDA-core (SIMT) forward kernel: fp32 and bf16 inputs, any window / stride /
+// CUDA-core (SIMT) forward kernel: fp32, bf16 and f16 inputs, any window / stride /
 // grid, head_dim 32, 64 or 128.  It serves the fp32 path (no exact fp32
 // tensor-core contraction exists) and shapes the tensor-core kernel does not
 // take.  Per query block it walks the key box of the block's windows in
@@ -7,6 +7,7 @@
 // softmax of "pi-Attention", section 3.1 eqs. (1)-(3) and section 3.2, with
 // the tile-by-tile on-chip accumulation that page's section 3.4 describes).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "na_internal.h"
 
@@ -16,16 +17,21 @@ namespace {
 constexpr int SIMT_THREADS = 128;
 constexpr int SIMT_CHUNK = 32;
 
-template <bool BF16>
+// Element types, numbered as na_dtype.
+enum : int { ELEM_F32 = 0, ELEM_BF16 = 1, ELEM_F16 = 2 };
+
+template <int T>
 __device__ __forceinline__ float load_elem(const void* p, size_t i) {
-  if constexpr (BF16) {
+  if constexpr (T == ELEM_BF16) {
     return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+  } else if constexpr (T == ELEM_F16) {
+    return __half2float(reinterpret_cast<const __half*>(p)[i]);
   } else {
     return reinterpret_cast<const float*>(p)[i];
   }
 }
 
-template <int D, bool BF16>
+template <int D, int T>
 __global__ void __launch_bounds__(SIMT_THREADS) simt_fwd_kernel(const SimtLaunch P) {
   constexpr int TPQ = D / 32;               // threads per query row
   constexpr int QPB = SIMT_THREADS / TPQ;   // queries per block
@@ -63,7 +69,7 @@ __global__ void __launch_bounds__(SIMT_THREADS) simt_fwd_kernel(const SimtLaunch
   float qr[32], acc[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
-    qr[c] = valid ? load_elem<BF16>(P.q, head_off + (size_t)token * D + gg * 32 + c) : 0.f;
+    qr[c] = valid ? load_elem<T>(P.q, head_off + (size_t)token * D + gg * 32 + c) : 0.f;
     acc[c] = 0.f;
   }
   float m = -INFINITY, l = 0.f;
@@ -81,8 +87,8 @@ __global__ void __launch_bounds__(SIMT_THREADS) simt_fwd_kernel(const SimtLaunch
       float kv = 0.f, vv = 0.f;
       if (x0 < g.L[0] && x1 < g.L[1] && x2 < g.L[2]) {
         const size_t off = head_off + (((size_t)x0 * g.L[1] + x1) * g.L[2] + x2) * D + ch;
-        kv = load_elem<BF16>(P.k, off);
-        vv = load_elem<BF16>(P.v, off);
+        kv = load_elem<T>(P.k, off);
+        vv = load_elem<T>(P.v, off);
       }
       const int si = key * D + (ch % 32) * TPQ + ch / 32;
       Ks[si] = kv;
@@ -129,10 +135,14 @@ __global__ void __launch_bounds__(SIMT_THREADS) simt_fwd_kernel(const SimtLaunch
   if (!valid) return;
   const float inv_l = 1.f / l;
   const size_t obase = head_off + (size_t)token * D + gg * 32;
-  if constexpr (BF16) {
+  if constexpr (T == ELEM_BF16) {
     __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(P.out) + obase;
 #pragma unroll
     for (int cc = 0; cc < 32; ++cc) o[cc] = __float2bfloat16_rn(acc[cc] * inv_l);
+  } else if constexpr (T == ELEM_F16) {
+    __half* o = reinterpret_cast<__half*>(P.out) + obase;
+#pragma unroll
+    for (int cc = 0; cc < 32; ++cc) o[cc] = __float2half_rn(acc[cc] * inv_l);
   } else {
     float* o = reinterpret_cast<float*>(P.out) + obase;
 #pragma unroll
@@ -145,10 +155,19 @@ template <int D>
 cudaError_t launch_d(const SimtLaunch& L, cudaStream_t stream) {
   const long long blocks = (long long)L.BH * L.t.nblocks;
   if (blocks <= 0 || blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  if (L.bf16)
-    simt_fwd_kernel<D, true><<<(unsigned)blocks, SIMT_THREADS, 0, stream>>>(L);
-  else
-    simt_fwd_kernel<D, false><<<(unsigned)blocks, SIMT_THREADS, 0, stream>>>(L);
+  switch (L.dtype) {
+    case ELEM_F32:
+      simt_fwd_kernel<D, ELEM_F32><<<(unsigned)blocks, SIMT_THREADS, 0, stream>>>(L);
+      break;
+    case ELEM_BF16:
+      simt_fwd_kernel<D, ELEM_BF16><<<(unsigned)blocks, SIMT_THREADS, 0, stream>>>(L);
+      break;
+    case ELEM_F16:
+      simt_fwd_kernel<D, ELEM_F16><<<(unsigned)blocks, SIMT_THREADS, 0, stream>>>(L);
+      break;
+    default:
+      return cudaErrorNotSupported;
+  }
   return cudaGetLastError();
 }
 

@@ -1,5 +1,5 @@
-// Tensor-core forward kernel for sm_100a (bf16 in, fp32 accumulate, bf16 out,
-// fp32 log-sum-exp).
+// Tensor-core forward kernel for sm_100a (bf16 or f16 in, fp32 accumulate,
+// output in the input type, fp32 log-sum-exp).
 //
 // One CTA owns a pair of 128-query blocks of one (batch, head).  It walks the
 // key box of the pair's windows in chunks of 128 keys; every chunk is EMPTY,
@@ -15,8 +15,8 @@
 //   warps 4-7  softmax for block 0, warps 8-11 softmax for block 1: one query
 //              row per thread (tcgen05.ld 32x32b), online softmax in the log2
 //              domain with a lazily moved reference max, P written back to
-//              TMEM as bf16 over its S, O rescaled in TMEM when the max moves;
-//              then the epilogue (O / l -> bf16, lse).
+//              TMEM in the input type over its S, O rescaled in TMEM when the
+//              max moves; then the epilogue (O / l -> input type, lse).
 // Two blocks ping-pong: while one block's softmax runs, the tensor core works
 // on the other block.  Warpgroup 0 hands most of its registers to the two
 // softmax warpgroups (setmaxnreg).  The softmax can evaluate a fixed share of
@@ -62,7 +62,7 @@ constexpr int EMU_DEN = 5;
 __host__ __device__ constexpr bool emulate_pair(int j) { return (j * EMU_NUM) % EMU_DEN < EMU_NUM; }
 constexpr uint32_t INFO_END = 0xFFFFu;   // slot info: no more chunks
 
-template <int D>
+template <int D, bool F16 = false>
 struct TcCfg {
   static constexpr int TILE_BYTES = 128 * D * 2;             // Q block or K/V chunk
   static constexpr int NS = (D == 128) ? 5 : 8;              // ring slots
@@ -70,8 +70,8 @@ struct TcCfg {
   static constexpr int TMEM_COLS = 512;
   static constexpr int S_COL0 = 0;
   static constexpr int O_COL0 = 256;
-  static constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(BLOCK_M, CHUNK_N, false, false);
-  static constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(BLOCK_M, D, false, true);
+  static constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(BLOCK_M, CHUNK_N, false, false, F16);
+  static constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(BLOCK_M, D, false, true, F16);
 };
 
 template <int NS>
@@ -152,11 +152,11 @@ __device__ __forceinline__ int seek_block(const ChunkGrid& cg, const int* kb, co
   return CHUNK_EMPTY;
 }
 
-template <int D>
+template <int D, bool F16>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const TcLaunch P) {
-  using C = TcCfg<D>;
+  using C = TcCfg<D, F16>;
   constexpr int NS = C::NS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
@@ -465,7 +465,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             case 2: acc2 = ptx::f2_add(acc2, p); break;
             default: acc3 = ptx::f2_add(acc3, p); break;
           }
-          s[j] = ptx::pack_bf16(p0, p1);
+          s[j] = ptx::pack_half2<F16>(p0, p1);
         }
         {
           uint32_t (&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
@@ -524,7 +524,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             uint32_t pk[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              pk[j] = ptx::pack_bf16(__uint_as_float(o[2 * j]) * inv_l,
+              pk[j] = ptx::pack_half2<F16>(__uint_as_float(o[2 * j]) * inv_l,
                                      __uint_as_float(o[2 * j + 1]) * inv_l);
 #pragma unroll
             for (int v = 0; v < 4; ++v)
@@ -570,8 +570,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
   return fn;
 }
 
-// [BH, X1, X2, X3, D] bf16 as a 5-d tensor (D, X3, X2, X1, BH), 64-element
-// inner box with 128-byte swizzle.
+// [BH, X1, X2, X3, D] bf16 / f16 as a 5-d tensor (D, X3, X2, X1, BH),
+// 64-element inner box with 128-byte swizzle.
 bool encode_map(CUtensorMap* m, const void* ptr, const TcLaunch& L, const int box[3]) {
   auto enc = get_encoder();
   if (!enc) return false;
@@ -583,13 +583,14 @@ bool encode_map(CUtensorMap* m, const void* ptr, const TcLaunch& L, const int bo
                            (cuuint64_t)L.N * L.D * es};
   cuuint32_t boxd[5] = {64, (cuuint32_t)box[2], (cuuint32_t)box[1], (cuuint32_t)box[0], 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides,
+  CUresult r = enc(m, L.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   5, const_cast<void*>(ptr), dims, strides,
                    boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool F16>
 cudaError_t launch_d(const TcLaunch& L, cudaStream_t stream, char* err, int errlen) {
   CUtensorMap mq, mk, mv;
   if (!encode_map(&mq, L.q, L, L.t.qb) || !encode_map(&mk, L.k, L, L.kb) ||
@@ -605,14 +606,14 @@ cudaError_t launch_d(const TcLaunch& L, cudaStream_t stream, char* err, int errl
     // setmaxnreg.inc waits for registers that the .dec of warpgroup 0 frees;
     // refuse to launch if the compiled register count could not cover the split.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, tc_fwd_kernel<D>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, tc_fwd_kernel<D, F16>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs * TC_THREADS < REGS_NEEDED) {
       snprintf(err, errlen, "kernel compiled with %d registers/thread; the register split needs %d",
                fa.numRegs, (REGS_NEEDED + TC_THREADS - 1) / TC_THREADS);
       return cudaErrorInvalidConfiguration;
     }
-    e = cudaFuncSetAttribute(tc_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(tc_fwd_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
@@ -620,7 +621,7 @@ cudaError_t launch_d(const TcLaunch& L, cudaStream_t stream, char* err, int errl
   const long long npairs = (L.t.nblocks + 1) / 2;
   const long long grid = npairs * L.BH;
   if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  tc_fwd_kernel<D><<<(unsigned)grid, TC_THREADS, smem, stream>>>(mq, mk, mv, L);
+  tc_fwd_kernel<D, F16><<<(unsigned)grid, TC_THREADS, smem, stream>>>(mq, mk, mv, L);
   return cudaGetLastError();
 }
 
@@ -646,8 +647,12 @@ cudaError_t launch_tc(const TcLaunch& L0, cudaStream_t stream, char* err, int er
   if (L.t.qb[0] * L.t.qb[1] * L.t.qb[2] != BLOCK_M || L.kb[0] * L.kb[1] * L.kb[2] != CHUNK_N)
     return cudaErrorNotSupported;
   switch (L.D) {
-    case 64: return launch_d<64>(L, stream, err, errlen);
-    case 128: return launch_d<128>(L, stream, err, errlen);
+    case 64:
+      return L.f16 ? launch_d<64, true>(L, stream, err, errlen)
+                   : launch_d<64, false>(L, stream, err, errlen);
+    case 128:
+      return L.f16 ? launch_d<128, true>(L, stream, err, errlen)
+                   : launch_d<128, false>(L, stream, err, errlen);
     default: return cudaErrorNotSupported;
   }
 }

@@ -16,7 +16,7 @@ struct SimtLaunch {
   QTiling t;
   int kb[3];
   int BH, N, D;
-  int bf16;              // 1: bf16 in/out, 0: fp32 in/out
+  int dtype;             // na_dtype of q, k, v and out (fp32, bf16 or f16)
   float scale_log2;      // scale * log2(e)
   const void *q, *k, *v;
   void* out;
@@ -29,6 +29,7 @@ struct TcLaunch {
   int kb[3];
   int kb_log2[3];        // filled by launch_tc (chunk extents are powers of two)
   int BH, N, D;
+  int f16;               // 1: f16 in/out, 0: bf16 in/out
   float scale_log2;
   const void *q, *k, *v;
   void* out;

@@ -271,6 +271,20 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return r;
 }
 
+// Two floats to a packed f16x2 (round-to-nearest-even); `lo` in bits 0..15.
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// The 16-bit input type's packer: f16 when F16, else bf16.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  if constexpr (F16) return pack_f16(lo, hi);
+  else return pack_bf16(lo, hi);
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: start
 // address, leading and stride byte offsets in 16-byte units, version 1 at
 // bit 46, layout type 2 = SWIZZLE_128B at bits 61..63).
@@ -280,12 +294,13 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo_byte
          ((uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
+// Instruction descriptor for kind::f16 with fp32 D and A/B both bf16 (or
+// both f16 when `f16`: format code 0 instead of 1).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
-                                                      bool b_mn_major) {
+                                                      bool b_mn_major, bool f16 = false) {
   return (1u << 4)                        // D format: f32
-         | (1u << 7)                      // A format: bf16
-         | (1u << 10)                     // B format: bf16
+         | ((f16 ? 0u : 1u) << 7)         // A format: f16 / bf16
+         | ((f16 ? 0u : 1u) << 10)        // B format: f16 / bf16
          | ((a_mn_major ? 1u : 0u) << 15) // A major
          | ((b_mn_major ? 1u : 0u) << 16) // B major
          | ((uint32_t)(N >> 3) << 17)     // N / 8

@@ -13,6 +13,9 @@ TOL = {
     "bf16": dict(out_max=1e-2, out_mean=1e-3, lse_max=1e-3),
     # fp32 inputs and outputs with fp32 accumulation: rounding of ~W-term sums
     "f32": dict(out_max=5e-5, out_mean=5e-6, lse_max=5e-5),
+    # f16 in and out: output rounding (half an ulp, <= 2^-10 for |out| < 2,
+    # 2^-9 below 4) plus P rounded to f16 (relative 2^-11 per weight)
+    "f16": dict(out_max=4e-3, out_mean=4e-4, lse_max=1e-3),
 }
 
 # The five workloads: 2-D neighborhood attention (fp32 and bf16), 2-D strided
@@ -43,7 +46,7 @@ def to_device(arr, dtype):
     if dtype == "bf16":
         t = torch.from_numpy(arr.view(np.int16)).view(torch.bfloat16)
     else:
-        t = torch.from_numpy(arr)
+        t = torch.from_numpy(arr)  # float32 or float16 values as they are
     return t.cuda()
 
 
