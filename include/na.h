@@ -160,6 +160,14 @@ typedef struct {
   long long computed_pairs; /* (units_full + units_partial) * block rows * chunk keys */
   long long useful_pairs;   /* sum over queries of the window size (N * prod(window) when
                                every dimension is clamped) */
+  long long dense_pairs;    /* N * N: the pairs of full self attention */
+  long long dense_units;    /* (block, chunk) products of full self attention under the
+                               same block and chunk shapes */
+  double speedup_bound;     /* dense_units / (units_full + units_partial): the speedup over
+                               the same kernel run densely that tile-granular skipping
+                               allows at most, a partial tile costing as much as a full
+                               one -- the "realistic speedup upper bound" of the simulator
+                               in the abstract of "Generalized Neighborhood Attention" */
 } na_plan_info;
 
 /* Fill *info for the given problem without touching the device. */

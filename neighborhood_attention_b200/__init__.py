@@ -46,7 +46,8 @@ class na_plan_info(ctypes.Structure):
                 ("query_blocks", ctypes.c_longlong), ("ctas", ctypes.c_longlong),
                 ("chunks_loaded", ctypes.c_longlong), ("units_full", ctypes.c_longlong),
                 ("units_partial", ctypes.c_longlong), ("computed_pairs", ctypes.c_longlong),
-                ("useful_pairs", ctypes.c_longlong)]
+                ("useful_pairs", ctypes.c_longlong), ("dense_pairs", ctypes.c_longlong),
+                ("dense_units", ctypes.c_longlong), ("speedup_bound", ctypes.c_double)]
 
     def as_dict(self):
         out = {}

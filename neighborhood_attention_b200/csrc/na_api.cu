@@ -499,6 +499,21 @@ na_status na_plan(const int dims[2], const int* grid, const int* window, const i
     useful *= sum;
   }
   info->useful_pairs = useful;
+  // Speedup bound: dense attention (every window the whole grid) under the
+  // same block / chunk shapes computes every (block, chunk) unit; this
+  // schedule computes only the non-empty ones, each at full tile cost.
+  Geom dense = P.g;
+  for (int d = 0; d < 3; ++d) {
+    dense.w[d] = dense.L[d];
+    dense.s[d] = 1;
+    dense.m[d] = WIN_CLAMPED;
+  }
+  const Cost cd = walk(dense, plan.t, plan.kb, group, 0);
+  const long long N = (long long)P.g.L[0] * P.g.L[1] * P.g.L[2];
+  info->dense_pairs = N * N;
+  info->dense_units = cd.full + cd.partial;
+  const long long units = c.full + c.partial;
+  info->speedup_bound = units > 0 ? (double)info->dense_units / (double)units : 0.0;
   return NA_OK;
 }
 

@@ -140,3 +140,23 @@ def test_plan_useful_pairs_with_modes(grid, window, stride, modes, oracle_lib):
     p = na.na_plan(grid, window, stride, None, 64, na.NA_BF16, options=opts)
     assert p["useful_pairs"] == expect
     assert p["computed_pairs"] >= expect
+
+
+def test_speedup_bound_simulator(oracle_lib):
+    """The speedup-bound simulator in na_plan: dense units over computed units.
+    Perfectly block-sparse sliding tile attention reaches N / prod(w); full
+    attention is 1; 1-D blocked attention with 128-token blocks agrees with
+    the oracle's count of non-empty 128 x 128 tiles."""
+    p = na.na_plan([30, 48, 80], [18, 24, 40], [6, 8, 8], [6, 8, 8], 128)
+    assert p["units_partial"] == 0
+    assert p["speedup_bound"] == pytest.approx(115200 / 17280)
+    assert p["dense_pairs"] == 115200 ** 2
+    p = na.na_plan([24, 40], [24, 40], [1, 1], None, 64)
+    assert p["speedup_bound"] == pytest.approx(1.0)
+    assert p["units_full"] + p["units_partial"] == p["dense_units"]
+    p = na.na_plan([1024], [128], [128], None, 64, options=na.make_options(
+        qblock=[1, 1, 128], kvchunk=[1, 1, 128]))
+    e, part, full = oracle_lib.block_counts([1024], [128], [128], 128)
+    assert p["dense_units"] == e + part + full == 64
+    assert p["units_full"] + p["units_partial"] == part + full == 8
+    assert p["speedup_bound"] == pytest.approx(8.0)
