@@ -62,6 +62,7 @@ KERNEL_SOURCES = ["neighborhood_attention_b200/csrc/na_fwd_sm100.cu",
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "na_fwd_tc_sta3d_traffic.txt")
 TRAFFIC_APPLIES = True     # the traffic file covers only the default 24-head workload
 L2_BYTES = 126 * 10**6
+DENSE_STEPS = 3
 FLUSH_BYTES = 256 * 2**20
 
 
@@ -361,7 +362,30 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = (float(np.sum([a.elapsed_time(b) for a, b in e_ev])) if flush
               else e0.elapsed_time(e1))
 
-    total_ms, e2e_ms, per_launch_ms = max_over_ranks([total_ms, e2e_ms, per_launch_ms], world, dev)
+    # Measured speedup over dense attention run through the same kernel (window
+    # = the whole grid), after the timed regions: the counterpart of the
+    # scheduler's speedup bound (na_plan_info.speedup_bound).
+    dense_ms = 0.0
+    if not args.no_speedup:
+        nd = len(w["grid"])
+
+        def dense_step():
+            na.na_forward(q, k, v, out, lse, w["grid"], [1] * nd, None, stream=stream)
+
+        dense_step()
+        d_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(DENSE_STEPS)]
+        for i in range(DENSE_STEPS):
+            flush_l2(i)
+            d_ev[i][0].record(stream)
+            dense_step()
+            d_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        na.na_sync_status(stream)
+        dense_ms = float(np.mean([a.elapsed_time(b) for a, b in d_ev]))
+
+    total_ms, e2e_ms, per_launch_ms, dense_ms = max_over_ranks(
+        [total_ms, e2e_ms, per_launch_ms, dense_ms], world, dev)
 
     flops = flops_per_step()
     value = whole_job_tflops(flops, args.steps, world, total_ms)
@@ -395,6 +419,12 @@ def run_ours(args, rank, world, local_rank):
         "cpu_baseline": base,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
+        "speedup": None if args.no_speedup else {
+            "bound": plan["speedup_bound"], "measured": dense_ms / per_launch_ms,
+            "ideal": plan["dense_pairs"] / plan["useful_pairs"], "dense_ms": dense_ms,
+            "kernel_ms": per_launch_ms,
+            "note": "dense = the same kernel with the window set to the whole grid, timed "
+                    "after the timed region; bound = dense tile units / computed tile units"},
         "gpu_launches": args.steps,
         "clocks": clocks,
         "kernel_ms": per_launch_ms,
@@ -410,6 +440,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-speedup", action="store_true",
+                    help="skip timing dense attention for the measured speedup")
     ap.add_argument("--config", type=int, default=4, choices=sorted(WORKLOADS),
                     help="workload: 4 (default) is the 3-D sliding tile one the metric is "
                          "quoted on; 1, 2, 3, 5 are the other parity workloads")

@@ -61,6 +61,10 @@ constexpr int EMU_DEN = 5;
 
 __host__ __device__ constexpr bool emulate_pair(int j) { return (j * EMU_NUM) % EMU_DEN < EMU_NUM; }
 constexpr uint32_t INFO_END = 0xFFFFu;   // slot info: no more chunks
+// Largest row sum of P accepted against a stale reference max: the sum bounds
+// every P of the row, so P <= 2^14 -- inside bf16's and f16's range, and
+// harmless to the fp32 accumulators -- while the reference rarely moves.
+constexpr float P_LIMIT = 16384.f;
 
 template <int D, bool F16 = false>
 struct TcCfg {
@@ -404,11 +408,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         ptx::tc_fence_after();
 
         uint32_t s[128];
-        {
-          uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
-          uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
-          uint32_t (&s2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[64]);
-          uint32_t (&s3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[96]);
+        uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
+        uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
+        uint32_t (&s2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[64]);
+        uint32_t (&s3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[96]);
+        // Scores of the chunk into registers (and -inf outside the row's
+        // window on partial chunks).
+        auto load_scores = [&]() {
           ptx::tmem_ld32(tS + 0, s0);
           ptx::tmem_ld32(tS + 32, s1);
           ptx::tmem_ld32(tS + 64, s2);
@@ -418,61 +424,89 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           ptx::reg_fence(s1);
           ptx::reg_fence(s2);
           ptx::reg_fence(s3);
-        }
-        if (st == CHUNK_PARTIAL) {
-          uint32_t mk[4];
-          chunk_key_mask(it.a, wlo, whi, P.kb, P.kb_log2, mk);
+          if (st == CHUNK_PARTIAL) {
+            uint32_t mk[4];
+            chunk_key_mask(it.a, wlo, whi, P.kb, P.kb_log2, mk);
 #pragma unroll
-          for (int j = 0; j < 128; ++j)
-            if (!((mk[j >> 5] >> (j & 31)) & 1u)) s[j] = __float_as_uint(-INFINITY);
-        }
-        float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
+            for (int j = 0; j < 128; ++j)
+              if (!((mk[j >> 5] >> (j & 31)) & 1u)) s[j] = __float_as_uint(-INFINITY);
+          }
+        };
+        // Maximum of the row's scores, log2 domain.
+        auto row_max = [&]() {
+          float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < 128; j += 8) {
-          a0 = ptx::max3(a0, __uint_as_float(s[j]), __uint_as_float(s[j + 1]));
-          a1 = ptx::max3(a1, __uint_as_float(s[j + 2]), __uint_as_float(s[j + 3]));
-          a2 = ptx::max3(a2, __uint_as_float(s[j + 4]), __uint_as_float(s[j + 5]));
-          a3 = ptx::max3(a3, __uint_as_float(s[j + 6]), __uint_as_float(s[j + 7]));
+          for (int j = 0; j < 128; j += 8) {
+            a0 = ptx::max3(a0, __uint_as_float(s[j]), __uint_as_float(s[j + 1]));
+            a1 = ptx::max3(a1, __uint_as_float(s[j + 2]), __uint_as_float(s[j + 3]));
+            a2 = ptx::max3(a2, __uint_as_float(s[j + 4]), __uint_as_float(s[j + 5]));
+            a3 = ptx::max3(a3, __uint_as_float(s[j + 6]), __uint_as_float(s[j + 7]));
+          }
+          return ptx::max3(a0, a1, fmaxf(a2, a3)) * sl2;
+        };
+        // P = 2^(score * scale - m_ref), packed in place into s[0..63]; returns
+        // the row sum of P.
+        auto exp_pass = [&](float m_ref) {
+          const uint64_t scale2 = ptx::f2(sl2, sl2);
+          const uint64_t negm2 = ptx::f2(-m_ref, -m_ref);
+          uint64_t acc0 = ptx::f2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
+#pragma unroll
+          for (int j = 0; j < 64; ++j) {
+            const uint64_t x = ptx::f2_fma(
+                ptx::f2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), scale2, negm2);
+            float x0, x1, p0, p1;
+            ptx::f2_split(x, x0, x1);
+            if (emulate_pair(j)) {
+              ptx::exp2_poly_x2(x0, x1, p0, p1);
+            } else {
+              p0 = ptx::ex2(x0);
+              p1 = ptx::ex2(x1);
+            }
+            const uint64_t p = ptx::f2(p0, p1);
+            switch (j & 3) {
+              case 0: acc0 = ptx::f2_add(acc0, p); break;
+              case 1: acc1 = ptx::f2_add(acc1, p); break;
+              case 2: acc2 = ptx::f2_add(acc2, p); break;
+              default: acc3 = ptx::f2_add(acc3, p); break;
+            }
+            s[j] = ptx::pack_half2<F16>(p0, p1);
+          }
+          float q0, q1, q2, q3, q4, q5, q6, q7;
+          ptx::f2_split(acc0, q0, q1);
+          ptx::f2_split(acc1, q2, q3);
+          ptx::f2_split(acc2, q4, q5);
+          ptx::f2_split(acc3, q6, q7);
+          return ((q0 + q1) + (q2 + q3)) + ((q4 + q5) + (q6 + q7));
+        };
+        // With a reference m from earlier chunks the exponentials start at
+        // once; the reference is moved (and the chunk redone from the scores
+        // still in TMEM) only when a row's sum -- an upper bound of its largest
+        // P -- exceeds P_LIMIT.  Without a reference yet (first chunk, or rows
+        // masked so far) the chunk's own maximum becomes the reference first.
+        load_scores();
+        float m_new = m, alpha = 1.f, sum;
+        bool need = false;
+        if (__any_sync(0xffffffffu, m == -INFINITY)) {
+          const float mx2 = row_max();
+          need = mx2 > m;
+          m_new = need ? mx2 : m;
+          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+          alpha = need ? ptx::ex2(m - m_use) : 1.f;
+          sum = exp_pass(m_use);
+        } else {
+          sum = exp_pass(m);
+          if (__any_sync(0xffffffffu, !(sum <= P_LIMIT))) {
+            load_scores();
+            const float mx2 = row_max();
+            need = mx2 > m;
+            m_new = need ? mx2 : m;
+            alpha = need ? ptx::ex2(m - m_new) : 1.f;
+            sum = exp_pass(m_new);
+          }
         }
-        const float mx2 = ptx::max3(a0, a1, fmaxf(a2, a3)) * sl2;
-        // Move the reference max only when the new max exceeds it by more
-        // than 2^8: P stays <= 256, exact after the final division by l.
-        const bool need = mx2 > m + 8.f;
-        const float m_new = need ? mx2 : m;
-        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = need ? ptx::ex2(m - m_use) : 1.f;
         const bool warp_need = __any_sync(0xffffffffu, need);
-
-        const uint64_t scale2 = ptx::f2(sl2, sl2);
-        const uint64_t negm2 = ptx::f2(-m_use, -m_use);
-        uint64_t acc0 = ptx::f2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const uint64_t x = ptx::f2_fma(
-              ptx::f2(__uint_as_float(s[2 * j]), __uint_as_float(s[2 * j + 1])), scale2, negm2);
-          float x0, x1, p0, p1;
-          ptx::f2_split(x, x0, x1);
-          if (emulate_pair(j)) {
-            ptx::exp2_poly_x2(x0, x1, p0, p1);
-          } else {
-            p0 = ptx::ex2(x0);
-            p1 = ptx::ex2(x1);
-          }
-          const uint64_t p = ptx::f2(p0, p1);
-          switch (j & 3) {
-            case 0: acc0 = ptx::f2_add(acc0, p); break;
-            case 1: acc1 = ptx::f2_add(acc1, p); break;
-            case 2: acc2 = ptx::f2_add(acc2, p); break;
-            default: acc3 = ptx::f2_add(acc3, p); break;
-          }
-          s[j] = ptx::pack_half2<F16>(p0, p1);
-        }
-        {
-          uint32_t (&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
-          uint32_t (&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
-          ptx::tmem_st32(tS + 0, p0);
-          ptx::tmem_st32(tS + 32, p1);
-        }
+        ptx::tmem_st32(tS + 0, s0);
+        ptx::tmem_st32(tS + 32, s1);
         if (warp_need && had_pv) {
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
@@ -485,12 +519,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             ptx::tmem_st32(tO + cc * 32, o);
           }
         }
-        float q0, q1, q2, q3, q4, q5, q6, q7;
-        ptx::f2_split(acc0, q0, q1);
-        ptx::f2_split(acc1, q2, q3);
-        ptx::f2_split(acc2, q4, q5);
-        ptx::f2_split(acc3, q6, q7);
-        const float sum = ((q0 + q1) + (q2 + q3)) + ((q4 + q5) + (q6 + q7));
         l = l * alpha + sum;
         m = m_new;
         ptx::tmem_st_wait();
