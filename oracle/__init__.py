@@ -67,6 +67,11 @@ class OracleLib:
         lib.na_oracle_block_counts.argtypes = [ctypes.c_int, i32p, i32p, i32p, i32p,
                                                ctypes.c_longlong, ctypes.c_void_p]
         lib.na_oracle_block_counts.restype = ctypes.c_int
+        lib.na_oracle_backward.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+            ctypes.c_longlong, ctypes.c_int, i32p, i32p, i32p, i32p, ctypes.c_int, ctypes.c_double,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        lib.na_oracle_backward.restype = ctypes.c_int
         lib.na_oracle_f16_value.argtypes = [ctypes.c_uint16]
         lib.na_oracle_f16_value.restype = ctypes.c_double
         self.lib = lib
@@ -157,6 +162,37 @@ class OracleLib:
             return out.reshape(shape).astype(np.float64), lse.reshape(shape[:-1])
         return out, lse
 
+    def backward(self, q, k, v, dout, grid, window, stride, *, dtype: str, scale: float = 0.0,
+                 threads: int | None = None, mode=None):
+        """Exact gradients (dq, dk, dv) in fp64 for upstream gradient dout.
+
+        q, k, v, dout: arrays of shape [B, heads, *grid, d] in the encoding of
+        ``forward``'s dtype.  Returns three float64 arrays of q's shape."""
+        grid, window, stride = _geom(grid, window, stride)
+        codes = {"f32": (np.float32, 0), "bf16": (np.uint16, 1), "f16": (np.float16, 2)}
+        if dtype not in codes:
+            raise ValueError(f"unknown dtype {dtype!r}")
+        want, code = codes[dtype]
+        arrs = [np.ascontiguousarray(a) for a in (q, k, v, dout)]
+        for a in arrs:
+            if a.dtype != want or a.shape != arrs[0].shape:
+                raise TypeError(f"oracle expects four {want} arrays of one shape")
+        shape = arrs[0].shape
+        nd = len(grid)
+        if tuple(shape[2:2 + nd]) != tuple(grid) or len(shape) != nd + 3:
+            raise ValueError(f"tensor shape {shape} does not match grid {grid}")
+        BH = shape[0] * shape[1]
+        d = shape[-1]
+        outs = [np.empty(shape, dtype=np.float64) for _ in range(3)]
+        rc = self.lib.na_oracle_backward(
+            arrs[0].ctypes.data, arrs[1].ctypes.data, arrs[2].ctypes.data, arrs[3].ctypes.data,
+            code, BH, nd, self._ivec(grid), self._ivec(window), self._ivec(stride),
+            self._ivec(_modes(mode, nd)), d, float(scale), outs[0].ctypes.data,
+            outs[1].ctypes.data, outs[2].ctypes.data, int(threads or os.cpu_count() or 1))
+        if rc:
+            raise RuntimeError(f"na_oracle_backward failed with code {rc}")
+        return tuple(outs)
+
     def f16_value(self, bits: int) -> float:
         """The oracle's decoding of one binary16 bit pattern."""
         return float(self.lib.na_oracle_f16_value(int(bits)))
@@ -222,6 +258,10 @@ def mask_row(grid, window, stride, token, mode=None):
 
 def forward(q, k, v, grid, window, stride, **kw):
     return load().forward(q, k, v, grid, window, stride, **kw)
+
+
+def backward(q, k, v, dout, grid, window, stride, **kw):
+    return load().backward(q, k, v, dout, grid, window, stride, **kw)
 
 
 def block_counts(grid, window, stride, block, mode=None):

@@ -56,6 +56,15 @@
  *   (truncated: the same centring as the clamped rule; causal: the group as
  *   the unit of causality) and coincide with eq. (5) at s = 1.
  *
+ * Backward (the gradients of the forward pass for an upstream gradient dO of
+ * out): the pages give only the forward; the gradients here are its
+ * vector-Jacobian product written out with P_ij = exp(z_ij - lse_i) over the
+ * same windows:
+ *   dV_j  = sum_{i : j in W(i)} P_ij dO_i
+ *   dP_ij = <dO_i, v_j>,  D_i = sum_j P_ij dP_ij  (= <dO_i, out_i>)
+ *   dZ_ij = P_ij (dP_ij - D_i)
+ *   dQ_i  = scale * sum_j dZ_ij k_j,   dK_j = scale * sum_{i : j in W(i)} dZ_ij q_i
+ *
  * Block counting (empty / partial / full tiles of the N x N attention map in
  * row-major token order) follows "Hilbert-Guided Sparse Local Attention",
  * "Methodology in Plain English" (tiles labelled full, partial or empty).
@@ -301,6 +310,136 @@ int na_oracle_forward(const void* q, const void* k, const void* v, int in_dtype,
             th[t] = 0;
         }
     fwd_worker(&jobs[0]);
+    for (int t = 1; t < nthreads; ++t)
+        if (th[t]) pthread_join(th[t], NULL);
+    for (int t = 0; t < nthreads; ++t)
+        if (jobs[t].status) return jobs[t].status;
+    return 0;
+}
+
+/* -------------------------------------------------------------- backward -- */
+
+typedef struct {
+    const void *q, *k, *v, *dout;
+    int dtype, ndim, d;
+    const int *L, *w, *s, *mode;
+    long long N, W;
+    double scale;
+    long long bh_begin, bh_end;
+    double *dq, *dk, *dv;
+    int status;
+} bwd_job;
+
+static void* bwd_worker(void* arg) {
+    bwd_job* J = (bwd_job*)arg;
+    const int d = J->d;
+    const long long N = J->N;
+    double* z = (double*)malloc(sizeof(double) * (size_t)J->W);
+    long long* idx = (long long*)malloc(sizeof(long long) * (size_t)J->W);
+    uint8_t* mask = (uint8_t*)malloc((size_t)N);
+    double* o = (double*)malloc(sizeof(double) * (size_t)d);
+    double* g = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!z || !idx || !mask || !o || !g) { J->status = -2; goto done; }
+    for (long long bh = J->bh_begin; bh < J->bh_end; ++bh) {
+        const size_t hoff = (size_t)bh * (size_t)N * (size_t)d;
+        for (long long t = 0; t < N; ++t) {
+            const long long inwin = na_oracle_mask_row(J->ndim, J->L, J->w, J->s, J->mode, t, mask);
+            const size_t qoff = hoff + (size_t)t * (size_t)d;
+            long long cnt = 0;
+            for (long long j = 0; j < N; ++j) {
+                if (!mask[j]) continue;
+                if (cnt >= J->W) { J->status = -3; goto done; }
+                const size_t koff = hoff + (size_t)j * (size_t)d;
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) {
+                    const double qc = load_in(J->q, J->dtype, qoff + c);
+                    dot += qc * load_in(J->k, J->dtype, koff + (size_t)c);
+                }
+                z[cnt] = dot * J->scale;
+                idx[cnt] = j;
+                ++cnt;
+            }
+            if (cnt != inwin || cnt < 1) { J->status = -3; goto done; }
+            double m = -INFINITY;
+            for (long long e = 0; e < cnt; ++e) if (z[e] > m) m = z[e];
+            double l = 0.0;
+            for (long long e = 0; e < cnt; ++e) l += exp(z[e] - m);
+            const double lse = m + log(l);
+            /* out_i and D_i = <dO_i, out_i> */
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            for (long long e = 0; e < cnt; ++e) {
+                const double p = exp(z[e] - lse);
+                const size_t voff = hoff + (size_t)idx[e] * (size_t)d;
+                for (int c = 0; c < d; ++c) o[c] += p * load_in(J->v, J->dtype, voff + c);
+            }
+            double Di = 0.0;
+            for (int c = 0; c < d; ++c) Di += load_in(J->dout, J->dtype, qoff + c) * o[c];
+            for (int c = 0; c < d; ++c) g[c] = 0.0;
+            for (long long e = 0; e < cnt; ++e) {
+                const double p = exp(z[e] - lse);
+                const size_t koff = hoff + (size_t)idx[e] * (size_t)d;
+                double dp = 0.0;
+                for (int c = 0; c < d; ++c)
+                    dp += load_in(J->dout, J->dtype, qoff + c) * load_in(J->v, J->dtype, koff + c);
+                const double dz = p * (dp - Di);
+                for (int c = 0; c < d; ++c) {
+                    g[c] += J->scale * dz * load_in(J->k, J->dtype, koff + (size_t)c);
+                    J->dk[koff + c] += J->scale * dz * load_in(J->q, J->dtype, qoff + c);
+                    J->dv[koff + c] += p * load_in(J->dout, J->dtype, qoff + c);
+                }
+            }
+            for (int c = 0; c < d; ++c) J->dq[qoff + c] = g[c];
+        }
+    }
+done:
+    free(z); free(idx); free(mask); free(o); free(g);
+    return NULL;
+}
+
+/*
+ * Gradients of the forward pass for upstream gradient dout (same layout and
+ * dtype as q): dq, dk, dv are [BH, N, d] fp64 (written).  mode: per-dimension
+ * window modes or NULL (all clamped).  scale <= 0 means 1/sqrt(d).  Threads
+ * split the BH (batch, head) slices, so dk and dv need no reduction across
+ * threads.  Returns 0 or a negative code as na_oracle_forward.
+ */
+int na_oracle_backward(const void* q, const void* k, const void* v, const void* dout, int in_dtype,
+                       long long BH, int ndim, const int* L, const int* w, const int* s,
+                       const int* mode, int d, double scale, double* dq, double* dk, double* dv,
+                       int nthreads) {
+    long long N;
+    if (!q || !k || !v || !dout || !dq || !dk || !dv || BH < 1 || d < 1) return -1;
+    if (in_dtype != IN_F32 && in_dtype != IN_BF16 && in_dtype != IN_F16) return -1;
+    if (check_geometry(ndim, L, w, s, mode, &N)) return -1;
+    long long W = 1;
+    for (int a = 0; a < ndim; ++a) W *= w[a];
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+    memset(dq, 0, sizeof(double) * (size_t)(BH * N * d));
+    memset(dk, 0, sizeof(double) * (size_t)(BH * N * d));
+    memset(dv, 0, sizeof(double) * (size_t)(BH * N * d));
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (nthreads > BH) nthreads = (int)BH;
+    bwd_job jobs[256];
+    pthread_t th[256];
+    const long long per = (BH + nthreads - 1) / nthreads;
+    for (int t = 0; t < nthreads; ++t) {
+        bwd_job* J = &jobs[t];
+        J->q = q; J->k = k; J->v = v; J->dout = dout;
+        J->dtype = in_dtype; J->ndim = ndim; J->d = d;
+        J->L = L; J->w = w; J->s = s; J->mode = mode;
+        J->N = N; J->W = W; J->scale = scale;
+        J->bh_begin = per * t < BH ? per * t : BH;
+        J->bh_end = per * (t + 1) < BH ? per * (t + 1) : BH;
+        J->dq = dq; J->dk = dk; J->dv = dv;
+        J->status = 0;
+    }
+    for (int t = 1; t < nthreads; ++t)
+        if (pthread_create(&th[t], NULL, bwd_worker, &jobs[t]) != 0) {
+            bwd_worker(&jobs[t]);
+            th[t] = 0;
+        }
+    bwd_worker(&jobs[0]);
     for (int t = 1; t < nthreads; ++t)
         if (th[t]) pthread_join(th[t], NULL);
     for (int t = 0; t < nthreads; ++t)

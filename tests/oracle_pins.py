@@ -486,6 +486,75 @@ def pin_sa_empty_blocks_golden(lib):
         assert round(100.0 * e / (e + p + f), 2) == round(pct, 2), (side, win, blk, e, p, f)
 
 
+# --------------------------------------------------------------- backward --
+
+def pin_backward_finite_differences(lib):
+    """Gradients of L = sum(out * dO) against central differences of the
+    oracle's own (pinned) forward: every element of dq, dk and dv on a small
+    2-D problem with mixed window modes and a stride.  The perturbation is
+    measured on the float32 values actually fed in."""
+    grid, window, stride, modes = [4, 5], [3, 3], [1, 2], ["clamped", "causal"]
+    d = 3
+    shape = (1, 1, *grid, d)
+    q, k, v, do = (_randn(150 + t, shape).astype(np.float64).astype(np.float32) for t in range(4))
+    dq, dk, dv = lib.backward(q, k, v, do, grid, window, stride, dtype="f32", mode=modes)
+
+    def loss(qq, kk, vv):
+        out, _ = lib.forward(qq, kk, vv, grid, window, stride, dtype="f32", mode=modes)
+        return float((out * do.astype(np.float64)).sum())
+
+    h = 1e-2
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        for idx in np.ndindex(*shape):
+            args = [q.copy(), k.copy(), v.copy()]
+            x0 = args[which][idx]
+            args[which][idx] = np.float32(x0 + h)
+            up = args[which][idx]
+            fp = loss(*args)
+            args[which][idx] = np.float32(x0 - h)
+            dn = args[which][idx]
+            fm = loss(*args)
+            num = (fp - fm) / (float(up) - float(dn))
+            assert abs(num - grad[idx]) <= 2e-4 * max(1.0, abs(num)), (which, idx, num, grad[idx])
+
+
+def pin_backward_full_attention_autograd(lib):
+    """Window = whole grid: the gradients equal torch autograd through dense
+    softmax attention in fp64."""
+    import torch
+    grid, d = [3, 7], 8
+    N = 21
+    shape = (2, 1, *grid, d)
+    q, k, v, do = (_randn(160 + t, shape) for t in range(4))
+    dq, dk, dv = lib.backward(q, k, v, do, grid, grid, [1, 1], dtype="f32")
+    qt, kt, vt = (torch.from_numpy(a.reshape(2, N, d).astype(np.float64)).requires_grad_()
+                  for a in (q, k, v))
+    att = torch.softmax((qt @ kt.transpose(1, 2)) / math.sqrt(d), dim=-1)
+    (att @ vt).backward(torch.from_numpy(do.reshape(2, N, d).astype(np.float64)))
+    for got, ref in ((dq, qt.grad), (dk, kt.grad), (dv, vt.grad)):
+        np.testing.assert_allclose(got.reshape(2, N, d), ref.numpy(), atol=1e-12, rtol=0)
+
+
+def pin_backward_invariants(lib):
+    """Closed forms: the rows of P sum to one, so the dv of all keys sums to
+    the dO of all queries; identical keys make every dq zero (each row of dZ
+    sums to zero); a one-key window (w = 1) gives dv = dO and dq = dk = 0."""
+    grid, window, stride, d = [6, 5], [3, 4], [2, 1], 4
+    shape = (1, 2, *grid, d)
+    q, k, v, do = (_randn(170 + t, shape) for t in range(4))
+    dq, dk, dv = lib.backward(q, k, v, do, grid, window, stride, dtype="f32",
+                              mode=["truncated", "clamped"])
+    np.testing.assert_allclose(dv.sum(axis=(2, 3)), do.astype(np.float64).sum(axis=(2, 3)),
+                               atol=1e-12, rtol=0)
+    kc = np.broadcast_to(k[:, :, :1, :1, :], k.shape).copy()
+    dq2, _, _ = lib.backward(q, kc, v, do, grid, window, stride, dtype="f32")
+    np.testing.assert_allclose(dq2, 0.0, atol=1e-13, rtol=0)
+    dq3, dk3, dv3 = lib.backward(q, k, v, do, grid, [1, 1], [1, 1], dtype="f32")
+    np.testing.assert_allclose(dv3, do.astype(np.float64), atol=0, rtol=0)
+    np.testing.assert_allclose(dq3, 0.0, atol=1e-14, rtol=0)
+    np.testing.assert_allclose(dk3, 0.0, atol=1e-14, rtol=0)
+
+
 def _read_golden(name):
     rows = []
     with open(os.path.join(GOLDEN, name)) as f:
@@ -503,7 +572,8 @@ ALL_PINS = [
     pin_constant_values, pin_explicit_scale, pin_row_subset, pin_wsa_empty_blocks_golden,
     pin_block_counts_closed_forms, pin_ena_density_golden, pin_truncated_eq5, pin_causal_eq5,
     pin_modes_strided, pin_mode_mask_bruteforce, pin_causal_full_sdpa, pin_mode_uniform_queries,
-    pin_sa_empty_blocks_golden, pin_f16_decoding,
+    pin_sa_empty_blocks_golden, pin_f16_decoding, pin_backward_finite_differences,
+    pin_backward_full_attention_autograd, pin_backward_invariants,
 ]
 
 # The golden-file pins take a few seconds each; mutant runs use the fast ones.

@@ -35,6 +35,15 @@ MUTANTS = [
     ("f16_exponent_bias", "ldexp((double)(1024 + f), e - 25)", "ldexp((double)(1024 + f), e - 24)"),
     ("f16_subnormal_as_normal", "v = ldexp((double)f, -24);", "v = ldexp((double)(1024 + f), -25);"),
     ("f16_read_as_bf16", "if (dtype == IN_F16) return", "if (dtype == -1) return"),
+    ("bwd_no_delta", "const double dz = p * (dp - Di);", "const double dz = p * dp;"),
+    ("bwd_dk_from_k", "J->dk[koff + c] += J->scale * dz * load_in(J->q, J->dtype, qoff + c);",
+     "J->dk[koff + c] += J->scale * dz * load_in(J->k, J->dtype, koff + c);"),
+    ("bwd_dv_without_p", "J->dv[koff + c] += p * load_in(J->dout, J->dtype, qoff + c);",
+     "J->dv[koff + c] += load_in(J->dout, J->dtype, qoff + c);"),
+    ("bwd_dq_unscaled", "g[c] += J->scale * dz * load_in(J->k, J->dtype, koff + (size_t)c);",
+     "g[c] += dz * load_in(J->k, J->dtype, koff + (size_t)c);"),
+    ("bwd_delta_from_v", "Di += load_in(J->dout, J->dtype, qoff + c) * o[c];",
+     "Di += load_in(J->dout, J->dtype, qoff + c) * load_in(J->v, J->dtype, qoff + c);"),
 ]
 
 
