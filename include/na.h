@@ -129,6 +129,32 @@ na_status na_forward_ex(const void* q, const void* k, const void* v, void* out, 
                         const na_options* opt, void* stream);
 
 /*
+ * na_backward -- enqueue the backward pass: the gradients of the forward's
+ * `out` with respect to q, k and v for an upstream gradient `dout`.  The pages
+ * give only the forward pass; these are its vector-Jacobian product over the
+ * same windows (softmax weights recomputed from the forward's lse):
+ *     P_ij  = exp(scale <q_i, k_j> - lse_i),   D_i = <dout_i, out_i>
+ *     dZ_ij = P_ij (<dout_i, v_j> - D_i)
+ *     dq_i  = scale sum_j dZ_ij k_j
+ *     dk_j  = scale sum_{i : j in W(i)} dZ_ij q_i
+ *     dv_j  = sum_{i : j in W(i)} P_ij dout_i
+ *   q, k, v, out, lse  the forward's inputs and outputs (out and lse as
+ *                      na_forward wrote them for the same arguments and options).
+ *   dout              device, same shape / dtype as q.
+ *   dq, dk, dv        device, same shape / dtype as q (written; every row once,
+ *                     no atomics, deterministic).
+ *   delta             device float32 [B, heads, X1..Xn] workspace (written: D_i).
+ * Other arguments, options (scale, window_mode) and errors as na_forward_ex.
+ * Runs CUDA-core kernels (fp32 arithmetic); opt->kernel = NA_KERNEL_TC is
+ * NA_ERR_UNSUPPORTED.
+ */
+na_status na_backward(const void* q, const void* k, const void* v, const void* out,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                      float* delta, int B, int heads, const int dims[2], const int* grid,
+                      const int* window, const int* stride, const int* tile, na_dtype dtype,
+                      const na_options* opt, void* stream);
+
+/*
  * na_sync_status -- synchronise `stream`, then read and clear this device's
  * status word.  NA_ERR_TIMEOUT if a kernel since the last call gave up on a
  * bounded wait (its outputs are then undefined); NA_ERR_CUDA if the

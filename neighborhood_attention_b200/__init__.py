@@ -7,7 +7,8 @@ no fallback of any kind.
 
 Functions keep the C-ABI names (``include/na.h``): ``na_forward``,
 ``na_forward_ex``, ``na_sync_status``, ``na_plan``, ``na_window_start``,
-``na_window_range``, ``na_block_schedule``, ``na_status_string``, ``na_last_error``.
+``na_window_range``, ``na_block_schedule``, ``na_backward``, ``na_status_string``,
+``na_last_error``.
 """
 from __future__ import annotations
 
@@ -93,6 +94,9 @@ def _load():
     lib.na_version.restype = ctypes.c_int
     lib.na_forward_noalloc.argtypes = lib.na_forward_ex.argtypes
     lib.na_forward_noalloc.restype = ctypes.c_int
+    lib.na_backward.argtypes = [vp] * 10 + [ctypes.c_int, ctypes.c_int, i32p, i32p, i32p, i32p,
+                                            i32p, ctypes.c_int, ctypes.POINTER(na_options), vp]
+    lib.na_backward.restype = ctypes.c_int
     lib.na_selftest_exp2.argtypes = [vp, vp, ctypes.c_int, vp]
     lib.na_selftest_exp2.restype = ctypes.c_int
     return lib
@@ -254,6 +258,54 @@ def na_forward_noalloc(q, k, v, out, lse, window, stride=None, tile=None, option
                                  _stream_ptr(stream))
     _check(st)
     return out, lse
+
+
+def na_backward(q, k, v, out, dout, lse, dq, dk, dv, delta, window, stride=None, tile=None,
+                options=None, stream=None):
+    """Enqueue na_backward on torch CUDA tensors (see include/na.h): dq, dk, dv
+    (same shape / dtype as q) and the float32 workspace delta (lse's shape)
+    are written."""
+    nd = len(window)
+    shape = tuple(q.shape)
+    if len(shape) != nd + 3:
+        raise ValueError(f"q has shape {shape}; expected [B, heads, {nd} grid dims, d]")
+    import torch
+    for name, t in (("k", k), ("v", v), ("out", out), ("dout", dout), ("dq", dq), ("dk", dk),
+                    ("dv", dv)):
+        if tuple(t.shape) != shape or t.dtype != q.dtype:
+            raise ValueError(f"{name} must match q in shape and dtype")
+    for name, t in (("lse", lse), ("delta", delta)):
+        if tuple(t.shape) != shape[:-1] or t.dtype != torch.float32:
+            raise ValueError(f"{name} must be float32 with q's shape minus head_dim")
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("lse", lse),
+                    ("dq", dq), ("dk", dk), ("dv", dv), ("delta", delta)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    st = _lib.na_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                          dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                          dv.data_ptr(), delta.data_ptr(), shape[0], shape[1],
+                          _ivec([nd, shape[-1]]), _ivec(shape[2:2 + nd]), _ivec(window),
+                          _ivec(stride), _ivec(tile), _dtype_of(q),
+                          ctypes.byref(options) if options is not None else None,
+                          _stream_ptr(stream))
+    _check(st)
+    return dq, dk, dv
+
+
+def backward(q, k, v, out, lse, dout, window, stride=None, tile=None, options=None, stream=None,
+             window_mode=None):
+    """Allocate dq, dk, dv (and the delta workspace) with torch and enqueue the
+    backward pass; returns (dq, dk, dv)."""
+    import torch
+    if window_mode is not None:
+        if options is None:
+            options = na_default_options()
+        for i, m in enumerate(window_modes(window_mode, len(window))):
+            options.window_mode[i] = m
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    delta = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    return na_backward(q, k, v, out, dout, lse, dq, dk, dv, delta, window, stride, tile, options,
+                       stream)
 
 
 def na_selftest_exp2(x, y, stream=None):

@@ -436,6 +436,50 @@ na_status na_forward(const void* q, const void* k, const void* v, void* out, flo
                        nullptr, stream);
 }
 
+na_status na_backward(const void* q, const void* k, const void* v, const void* out,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                      float* delta, int B, int heads, const int dims[2], const int* grid,
+                      const int* window, const int* stride, const int* tile, na_dtype dtype,
+                      const na_options* opt, void* stream) {
+  g_err[0] = 0;
+  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !delta)
+    return fail(NA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  if (B < 1 || heads < 1) return fail(NA_ERR_INVALID_ARG, "B=%d heads=%d must be >= 1", B, heads);
+  Problem P;
+  na_status st = read_problem(dims, grid, window, stride, tile, dtype, opt, P);
+  if (st != NA_OK) return st;
+  const void* ptrs[] = {q, k, v, out, dout, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return fail(NA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (!aligned(lse, 4) || !aligned(delta, 4))
+    return fail(NA_ERR_INVALID_ARG, "lse and delta must be 4-byte aligned");
+  if (P.opt.kernel == NA_KERNEL_TC)
+    return fail(NA_ERR_UNSUPPORTED, "the backward pass runs on the CUDA-core kernels");
+  const long long BH = (long long)B * heads;
+  if (BH > (1LL << 30)) return fail(NA_ERR_UNSUPPORTED, "B*heads too large");
+  P.opt.kernel = NA_KERNEL_SIMT;
+  Plan plan;
+  st = make_plan(P, plan);
+  if (st != NA_OK) return st;
+  const float scale = P.opt.scale > 0.f ? P.opt.scale : 1.0f / sqrtf((float)P.D);
+  BwdLaunch L;
+  L.g = P.g;
+  L.t = plan.t;
+  for (int d = 0; d < 3; ++d) L.kb[d] = plan.kb[d];
+  L.BH = (int)BH;
+  L.N = P.g.L[0] * P.g.L[1] * P.g.L[2];
+  L.D = P.D;
+  L.dtype = P.dtype;
+  L.scale = scale;
+  L.scale_log2 = scale * 1.4426950408889634f;
+  L.q = q; L.k = k; L.v = v; L.out = out; L.dout = dout; L.lse = lse; L.delta = delta;
+  L.dq = dq; L.dk = dk; L.dv = dv;
+  cudaError_t e = launch_bwd_simt(L, reinterpret_cast<cudaStream_t>(stream));
+  if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "backward: shape");
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
+  return NA_OK;
+}
+
 na_status na_sync_status(void* stream) {
   g_err[0] = 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -39,7 +39,23 @@ struct TcLaunch {
   int debug_flags;       // 1: withhold the first key chunk (timeout-path test)
 };
 
+// Backward pass (CUDA-core kernels): dq, dk, dv of the forward for upstream dout.
+struct BwdLaunch {
+  Geom g;
+  QTiling t;             // query blocks (dQ) and key blocks (dK, dV)
+  int kb[3];             // key chunks (dQ) and query chunks (dK, dV), 32 tokens
+  int BH, N, D;
+  int dtype;             // na_dtype of q, k, v, out, dout and the gradients
+  float scale;           // softmax scale
+  float scale_log2;      // scale * log2(e)
+  const void *q, *k, *v, *out, *dout;
+  const float* lse;      // forward log-sum-exp (natural log)
+  float* delta;          // [BH, N] workspace: <dout_i, out_i>
+  void *dq, *dk, *dv;
+};
+
 cudaError_t launch_simt(const SimtLaunch& L, cudaStream_t stream);
+cudaError_t launch_bwd_simt(const BwdLaunch& L, cudaStream_t stream);
 
 // y[i] = the tensor-core kernel's FMA-pipe 2^x applied to x[i] (self-test).
 cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t stream);

@@ -1,0 +1,100 @@
+"""GPU parity of the backward pass: dq, dk, dv from the CUDA kernels (through
+the C ABI, after the CUDA forward produced out and lse) against the fp64
+oracle's gradients on identical seeded inputs, element by element.
+
+Bar, from the arithmetic: 16-bit gradients are rounded once to the input
+type (half an ulp, 2^-9 relative for bf16, 2^-12 for f16), and the forward's
+16-bit out enters D_i = <dO_i, out_i>; fp32 accumulation adds far less.  So
+max |g - oracle| <= 2^-8 max|oracle| + 2e-3 and mean <= 2^-10 mean|oracle| + 2e-4
+for bf16 / f16; fp32 inputs: max <= 1e-4 max(1, max|oracle|), mean <= 1e-5."""
+import zlib
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # pragma: no cover - CPU machines skip the module
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import neighborhood_attention_b200 as na  # noqa: E402
+import oracle  # noqa: E402
+import seeded_inputs  # noqa: E402
+from gpu_parity import to_device  # noqa: E402
+
+
+def _case(grid, window, stride, d, dtype="bf16", B=1, heads=2, mode=None, tile=None):
+    return dict(B=B, heads=heads, grid=tuple(grid), window=tuple(window), stride=tuple(stride),
+                d=d, dtype=dtype, mode=mode, tile=tile)
+
+
+CASES = {
+    "na2d_ragged_d64": _case((21, 27), (7, 5), (1, 1), 64),
+    "na2d_d128": _case((13, 17), (5, 7), (1, 1), 128),
+    "gna2d_strided": _case((24, 20), (12, 8), (4, 2), 64),
+    "sta3d_small": _case((6, 8, 16), (6, 8, 8), (2, 4, 4), 64, tile=(2, 4, 4)),
+    "na1d_long": _case((700,), (65,), (1,), 64),
+    "causal1d": _case((500,), (97,), (1,), 128, mode=["causal"]),
+    "truncated_mixed3d": _case((5, 9, 11), (3, 5, 7), (1, 2, 1), 32,
+                               mode=["truncated", "causal", "clamped"], B=2, heads=1),
+    "full_attention": _case((12, 16), (12, 16), (1, 1), 64),
+    "fp32_d32": _case((16, 16), (5, 5), (1, 1), 32, dtype="f32", heads=3),
+    "f16_d64": _case((18, 22), (7, 9), (2, 1), 64, dtype="f16"),
+    "sta3d_medium_d128": _case((6, 16, 40), (6, 12, 24), (2, 4, 8), 128, tile=(2, 4, 8)),
+}
+
+
+def _run(c, seed):
+    shape = (c["B"], c["heads"], *c["grid"], c["d"])
+    q, k, v = seeded_inputs.qkv(seed, c["B"], c["heads"], c["grid"], c["d"], c["dtype"])
+    gen = {"f32": seeded_inputs.normal_f32, "bf16": seeded_inputs.normal_bf16_bits,
+           "f16": seeded_inputs.normal_f16}[c["dtype"]]
+    do = gen(seed + 7, shape, threads=1)
+    qd, kd, vd, dod = (to_device(a, c["dtype"]) for a in (q, k, v, do))
+    opts = na.make_options(window_mode=c["mode"], ndim=len(c["grid"])) if c["mode"] else None
+    out, lse = na.forward(qd, kd, vd, c["window"], c["stride"], c["tile"], options=opts)
+    dq, dk, dv = na.backward(qd, kd, vd, out, lse, dod, c["window"], c["stride"], c["tile"],
+                             options=opts)
+    na.na_sync_status()
+    got = [t.float().cpu().numpy().astype(np.float64) for t in (dq, dk, dv)]
+    ref = oracle.backward(q, k, v, do, c["grid"], c["window"], c["stride"], dtype=c["dtype"],
+                          mode=c["mode"])
+    return got, ref
+
+
+def _assert_close(c, got, ref, label):
+    for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+        assert np.isfinite(g).all(), f"{label} {name}: non-finite"
+        err = np.abs(g - r)
+        if c["dtype"] == "f32":
+            tmax, tmean = 1e-4 * max(1.0, np.abs(r).max()), 1e-5
+        else:
+            tmax = 2.0 ** -8 * np.abs(r).max() + 2e-3
+            tmean = 2.0 ** -10 * np.abs(r).mean() + 2e-4
+        assert err.max() <= tmax, f"{label} {name}: max|err|={err.max():.3e} > {tmax:.3e}"
+        assert err.mean() <= tmean, f"{label} {name}: mean|err|={err.mean():.3e} > {tmean:.3e}"
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_backward_parity(name):
+    c = CASES[name]
+    got, ref = _run(c, seed=zlib.crc32(name.encode()) % 100000)
+    _assert_close(c, got, ref, name)
+
+
+def test_backward_deterministic():
+    c = CASES["gna2d_strided"]
+    a, _ = _run(c, seed=31)
+    b, _ = _run(c, seed=31)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_backward_refuses_tensor_core_selector():
+    c = CASES["na2d_d128"]
+    q = torch.zeros((1, 1, *c["grid"], 128), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(q.shape[:-1], dtype=torch.float32, device="cuda")
+    with pytest.raises(na.NaError) as e:
+        na.backward(q, q, q, q, lse, q, c["window"], options=na.make_options(kernel=na.NA_KERNEL_TC))
+    assert e.value.status == na.NA_ERR_UNSUPPORTED
