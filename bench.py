@@ -259,6 +259,88 @@ def whole_job_tflops(flops_per_rank_step, steps, world, max_ms):
 
 
 # ---------------------------------------------------------------- GPU side --
+FP32_FMA_PER_CLK_SM = 128      # fp32 FMA lanes per SM per clock (B200)
+NUM_SM = 148
+
+
+def run_backward(args, rank, world, local_rank):
+    """The backward pass (na_backward: dq, dk, dv) on the selected workload:
+    one step = one call (three CUDA-core kernels); the forward's out and lse
+    are produced once before timing.  Effective TFLOP/s counts 10 * d FLOPs
+    per attended (query, key) pair (five products of 2 d: scores, dP, dV, dQ,
+    dK), against the fp32 FMA peak of the CUDA cores at the sampled clock."""
+    import torch
+    import torch.distributed as dist
+    import neighborhood_attention_b200 as na
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOAD
+    qkv_host = host_qkv()
+    if w["dtype"] == "bf16":
+        tensors = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) for a in qkv_host]
+    else:
+        tensors = [torch.from_numpy(a) for a in qkv_host]
+    q, k, v = (t.to(dev) for t in tensors)
+    g = torch.Generator(device=dev).manual_seed(SEED + 11)
+    dout = torch.randn(q.shape, generator=g, device=dev, dtype=torch.float32).to(q.dtype)
+    stream = torch.cuda.current_stream(dev)
+    out, lse = na.forward(q, k, v, w["window"], w["stride"], w["tile"], stream=stream)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    delta = torch.empty(lse.shape, dtype=torch.float32, device=dev)
+
+    def step():
+        na.na_backward(q, k, v, out, dout, lse, dq, dk, dv, delta, w["window"], w["stride"],
+                       w["tile"], stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    na.na_sync_status(stream)
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(1.0)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    w0 = time.time()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    w1 = time.time()
+    clocks = sampler.stop(windows=[(w0, w1)])
+    if world > 1:
+        dist.barrier()
+    na.na_sync_status(stream)
+    (total_ms,) = max_over_ranks([e0.elapsed_time(e1)], world, dev)
+    plan = na.na_plan(w["grid"], w["window"], w["stride"], w["tile"], w["head_dim"],
+                      {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32}[w["dtype"]])
+    flops = 10.0 * w["head_dim"] * w["B"] * w["heads"] * plan["useful_pairs"]
+    value = flops * args.steps * world / (total_ms / 1e3) / 1e12
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
+    peak = 2.0 * FP32_FMA_PER_CLK_SM * NUM_SM * mhz * 1e6 / 1e12
+    achieved = value / world
+    if rank != 0:
+        return 0
+    line = {
+        "metric": f"effective TFLOP/s, backward (dq, dk, dv), {w['workload']}",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
+        "config": dict(w, direction="backward", kernels="CUDA-core (fp32 FMA)"),
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_kind": "derived: 148 SM x 128 fp32 FMA/clk x 2 FLOP x sampled SM clock"},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -440,6 +522,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (na_backward) instead of the forward")
     ap.add_argument("--no-speedup", action="store_true",
                     help="skip timing dense attention for the measured speedup")
     ap.add_argument("--config", type=int, default=4, choices=sorted(WORKLOADS),
@@ -480,6 +564,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.backward:
+            return run_backward(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
