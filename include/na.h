@@ -145,8 +145,11 @@ na_status na_forward_ex(const void* q, const void* k, const void* v, void* out, 
  *                     no atomics, deterministic).
  *   delta             device float32 [B, heads, X1..Xn] workspace (written: D_i).
  * Other arguments, options (scale, window_mode) and errors as na_forward_ex.
- * Runs CUDA-core kernels (fp32 arithmetic); opt->kernel = NA_KERNEL_TC is
- * NA_ERR_UNSUPPORTED.
+ * Kernels: D_i and dk / dv on the CUDA cores (fp32 arithmetic); dq on the
+ * tensor cores (tcgen05, fp32 accumulation) for bf16 / f16 with head_dim 64 or
+ * 128 unless opt->kernel = NA_KERNEL_SIMT, else on the CUDA cores.
+ * opt->kernel = NA_KERNEL_TC for other inputs is NA_ERR_UNSUPPORTED.  A bounded
+ * in-kernel wait that expires is reported by na_sync_status.
  */
 na_status na_backward(const void* q, const void* k, const void* v, const void* out,
                       const void* dout, const float* lse, void* dq, void* dk, void* dv,

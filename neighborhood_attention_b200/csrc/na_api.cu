@@ -453,11 +453,22 @@ na_status na_backward(const void* q, const void* k, const void* v, const void* o
     if (!aligned(p, 16)) return fail(NA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
   if (!aligned(lse, 4) || !aligned(delta, 4))
     return fail(NA_ERR_INVALID_ARG, "lse and delta must be 4-byte aligned");
-  if (P.opt.kernel == NA_KERNEL_TC)
-    return fail(NA_ERR_UNSUPPORTED, "the backward pass runs on the CUDA-core kernels");
   const long long BH = (long long)B * heads;
   if (BH > (1LL << 30)) return fail(NA_ERR_UNSUPPORTED, "B*heads too large");
+  const bool tc_ok = (P.dtype == NA_BF16 || P.dtype == NA_F16) && (P.D == 64 || P.D == 128);
+  if (P.opt.kernel == NA_KERNEL_TC && !tc_ok)
+    return fail(NA_ERR_UNSUPPORTED, "the tensor-core backward takes bf16 / f16, head_dim 64 or 128");
+  const bool use_tc = tc_ok && P.opt.kernel != NA_KERNEL_SIMT;
+  Plan tc_plan;
+  if (use_tc) {
+    Problem Pt = P;
+    Pt.opt.kernel = NA_KERNEL_TC;
+    st = make_plan(Pt, tc_plan);
+    if (st != NA_OK) return st;
+  }
   P.opt.kernel = NA_KERNEL_SIMT;
+  P.opt.qblock[0] = P.opt.qblock[1] = P.opt.qblock[2] = 0;   // shapes of the TC plan do not fit
+  P.opt.kvchunk[0] = P.opt.kvchunk[1] = P.opt.kvchunk[2] = 0;
   Plan plan;
   st = make_plan(P, plan);
   if (st != NA_OK) return st;
@@ -474,9 +485,37 @@ na_status na_backward(const void* q, const void* k, const void* v, const void* o
   L.scale_log2 = scale * 1.4426950408889634f;
   L.q = q; L.k = k; L.v = v; L.out = out; L.dout = dout; L.lse = lse; L.delta = delta;
   L.dq = dq; L.dk = dk; L.dv = dv;
-  cudaError_t e = launch_bwd_simt(L, reinterpret_cast<cudaStream_t>(stream));
-  if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "backward: shape");
-  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!use_tc) {
+    cudaError_t e = launch_bwd_simt(L, s);
+    if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "backward: shape");
+    if (e != cudaSuccess) return fail(NA_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
+    return NA_OK;
+  }
+  int* status = nullptr;
+  st = status_word(&status);
+  if (st != NA_OK) return st;
+  cudaError_t e = launch_bwd_simt_delta(L, s);
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "backward delta: %s", cudaGetErrorString(e));
+  TcBwdLaunch T;
+  T.g = P.g;
+  T.t = tc_plan.t;
+  for (int d = 0; d < 3; ++d) T.kb[d] = tc_plan.kb[d];
+  T.BH = (int)BH;
+  T.N = L.N;
+  T.D = P.D;
+  T.f16 = P.dtype == NA_F16;
+  T.scale = scale;
+  T.scale_log2 = L.scale_log2;
+  T.q = q; T.k = k; T.v = v; T.dout = dout; T.lse = lse; T.delta = delta; T.dq = dq;
+  T.status = status;
+  T.timeout_ns = P.opt.wait_timeout_ns > 0 ? P.opt.wait_timeout_ns : default_timeout_ns();
+  char msg[256] = "";
+  e = launch_tc_bwd_dq(T, s, msg, sizeof msg);
+  if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "tensor-core dq: shape");
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "tensor-core dq: %s %s", cudaGetErrorString(e), msg);
+  e = launch_bwd_simt_dkdv(L, s);
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "backward dk/dv: %s", cudaGetErrorString(e));
   return NA_OK;
 }
 

@@ -324,25 +324,37 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_dkdv_kernel(const BwdLaunch P
   }
 }
 
+// Which kernels a launch runs.
+enum : int { RUN_DELTA = 1, RUN_DQ = 2, RUN_DKDV = 4 };
+
 template <int D, int T>
-cudaError_t launch_dt(const BwdLaunch& L, cudaStream_t stream) {
+cudaError_t launch_dt(const BwdLaunch& L, cudaStream_t stream, int which) {
   const long long rows = (long long)L.BH * L.N;
   const long long dblocks = (rows + 7) / 8;
   const long long blocks = (long long)L.BH * L.t.nblocks;
   if (blocks <= 0 || blocks > 0x7fffffffLL || dblocks > 0x7fffffffLL)
     return cudaErrorInvalidConfiguration;
-  row_delta_kernel<T><<<(unsigned)dblocks, 256, 0, stream>>>(L);
-  bwd_dq_kernel<D, T><<<(unsigned)blocks, BWD_THREADS, 0, stream>>>(L);
-  bwd_dkdv_kernel<D, T><<<(unsigned)blocks, BWD_THREADS, 0, stream>>>(L);
+  if (which & RUN_DELTA) row_delta_kernel<T><<<(unsigned)dblocks, 256, 0, stream>>>(L);
+  if (which & RUN_DQ) bwd_dq_kernel<D, T><<<(unsigned)blocks, BWD_THREADS, 0, stream>>>(L);
+  if (which & RUN_DKDV) bwd_dkdv_kernel<D, T><<<(unsigned)blocks, BWD_THREADS, 0, stream>>>(L);
   return cudaGetLastError();
 }
 
 template <int D>
-cudaError_t launch_d(const BwdLaunch& L, cudaStream_t stream) {
+cudaError_t launch_d(const BwdLaunch& L, cudaStream_t stream, int which) {
   switch (L.dtype) {
-    case ELEM_F32: return launch_dt<D, ELEM_F32>(L, stream);
-    case ELEM_BF16: return launch_dt<D, ELEM_BF16>(L, stream);
-    case ELEM_F16: return launch_dt<D, ELEM_F16>(L, stream);
+    case ELEM_F32: return launch_dt<D, ELEM_F32>(L, stream, which);
+    case ELEM_BF16: return launch_dt<D, ELEM_BF16>(L, stream, which);
+    case ELEM_F16: return launch_dt<D, ELEM_F16>(L, stream, which);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+cudaError_t launch_which(const BwdLaunch& L, cudaStream_t stream, int which) {
+  switch (L.D) {
+    case 32: return launch_d<32>(L, stream, which);
+    case 64: return launch_d<64>(L, stream, which);
+    case 128: return launch_d<128>(L, stream, which);
     default: return cudaErrorNotSupported;
   }
 }
@@ -350,12 +362,13 @@ cudaError_t launch_d(const BwdLaunch& L, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_bwd_simt(const BwdLaunch& L, cudaStream_t stream) {
-  switch (L.D) {
-    case 32: return launch_d<32>(L, stream);
-    case 64: return launch_d<64>(L, stream);
-    case 128: return launch_d<128>(L, stream);
-    default: return cudaErrorNotSupported;
-  }
+  return launch_which(L, stream, RUN_DELTA | RUN_DQ | RUN_DKDV);
+}
+cudaError_t launch_bwd_simt_delta(const BwdLaunch& L, cudaStream_t stream) {
+  return launch_which(L, stream, RUN_DELTA);
+}
+cudaError_t launch_bwd_simt_dkdv(const BwdLaunch& L, cudaStream_t stream) {
+  return launch_which(L, stream, RUN_DKDV);
 }
 
 }  // namespace na

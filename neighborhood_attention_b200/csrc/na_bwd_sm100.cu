@@ -1,0 +1,431 @@
+// Tensor-core backward kernel for sm_100a, dQ part (bf16 or f16 in, fp32
+// accumulate): for one 128-query block per CTA and every key chunk of the
+// block's windows,
+//   S  = Q K^T,  dP = dO V^T                  (tcgen05.mma, both operands in
+//                                              shared memory, fp32 in TMEM)
+//   P  = exp(scale S - lse),  dS = P (dP - delta)   (softmax warps, per row;
+//                                              delta_i = <dO_i, out_i>)
+//   dQ += dS K                                (tcgen05.mma, dS read from TMEM)
+// and dq = scale dQ in the epilogue -- the dQ part of the vector-Jacobian
+// product of the restricted softmax attention of "pi-Attention", section 3.1
+// eqs. (1)-(3) with section 3.2's neighbourhood.  The backward needs no running
+// maximum (lse is known), so each chunk's rows are split by keys between two
+// warps per row quarter with no exchange between them.
+//
+// Roles (12 warps): warp 0 TMA producer (Q and dO once, then K / V chunks
+// through a ring), warp 1 TMEM allocation and the single MMA issuer, warps
+// 4-7 and 8-11 the element-wise part (warp 4+q keys 0-63, warp 8+q keys
+// 64-127 of every chunk, rows 32q..32q+31).  Every wait is bounded (see
+// na_ptx.cuh); the chunk stream ends with a marker in the next K slot.
+//
+// TMEM columns: S [0, 128), dP [128, 256) -- after the element-wise pass
+// dS of keys 64h..64h+63 sits as packed 16-bit pairs in [128 + 64h, 160 + 64h),
+// inside the half of dP that warp h itself read -- and dQ [256, 256 + D).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <stdio.h>
+
+#include "na_internal.h"
+#include "na_ptx.cuh"
+
+namespace na {
+namespace {
+
+constexpr int BT_THREADS = 384;
+constexpr int BT_M = 128;                // query rows per block
+constexpr int BT_N = 128;                // keys per chunk
+constexpr int BT_HALF_BYTES = 128 * 128; // one 128-row x 64-element 16-bit box
+constexpr int BT_REGS_LOADER = 56;
+constexpr int BT_REGS_WORK = 216;
+constexpr int BT_REGS_NEEDED = 128 * BT_REGS_LOADER + 256 * BT_REGS_WORK;
+constexpr uint32_t BT_INFO_END = 0xFFFFu;
+constexpr float BT_LOG2E = 1.4426950408889634f;
+
+template <int D, bool F16>
+struct BtCfg {
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int NS = (D == 128) ? 4 : 8;   // ring slots (K and V chunks)
+  static constexpr int HALVES = D / 64;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int S_COL0 = 0;
+  static constexpr int DP_COL0 = 128;
+  static constexpr int DQ_COL0 = 256;
+  static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(BT_M, BT_N, false, false, F16);
+  static constexpr uint32_t IDESC_DQ = ptx::idesc_bf16_f32(BT_M, D, false, true, F16);
+};
+
+template <int NS>
+struct BtBars {
+  uint64_t q_full;           // Q and dO tiles
+  uint64_t full[NS];
+  uint64_t empty[NS];
+  uint64_t s_full;           // S and dP of the current chunk
+  uint64_t p_ready;          // dS stored (256 arrivals)
+  uint64_t o_done;
+  uint32_t tmem_base;
+  int abort;
+  volatile uint32_t info[NS];
+  BlockInfo bi;
+  ChunkGrid cg;
+};
+
+template <int D>
+constexpr size_t bt_smem_bytes() {
+  return 1024 + (size_t)(2 + BtCfg<D, false>::NS) * BtCfg<D, false>::TILE_BYTES +
+         sizeof(BtBars<BtCfg<D, false>::NS>);
+}
+
+template <int D, bool F16>
+__global__ void __launch_bounds__(BT_THREADS, 1)
+    tc_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const TcBwdLaunch P) {
+  using C = BtCfg<D, F16>;
+  constexpr int NS = C::NS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = base;
+  uint8_t* sDO = base + C::TILE_BYTES;
+  uint8_t* ring = base + 2 * C::TILE_BYTES;
+  BtBars<NS>* bars = reinterpret_cast<BtBars<NS>*>(ring + NS * C::TILE_BYTES);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const QTiling& t = P.t;
+  const int bh = blockIdx.x / t.nblocks;
+  const int blk = blockIdx.x % t.nblocks;
+  const BlockInfo& B = bars->bi;
+  const ChunkGrid& cg = bars->cg;
+
+  if (threadIdx.x == 0) {
+    block_info(P.g, t, blk, bars->bi);
+    chunk_grid_for(&bars->bi, 1, P.kb, bars->cg);
+    ptx::mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      ptx::mbar_init(&bars->full[s], 1);
+      ptx::mbar_init(&bars->empty[s], 1);
+    }
+    ptx::mbar_init(&bars->s_full, 1);
+    ptx::mbar_init(&bars->p_ready, 2 * BT_M);
+    ptx::mbar_init(&bars->o_done, 1);
+    bars->abort = *reinterpret_cast<volatile int*>(P.status) != 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  ptx::WaitCtl ctl;
+  ctl.abort = &bars->abort;
+  ctl.status = P.status;
+  ctl.timeout_ns = (uint64_t)P.timeout_ns;
+
+  if (warp < 4) {
+    ptx::regs_dec<BT_REGS_LOADER>();
+    if (warp == 0 && lane == 0 && B.exists) {
+      // ========================= TMA producer =========================
+      ptx::mbar_expect_tx(&bars->q_full, 2 * C::TILE_BYTES);
+      for (int h = 0; h < C::HALVES; ++h) {
+        ptx::tma_load_5d(sQ + h * BT_HALF_BYTES, &tm_q, &bars->q_full, h * 64, B.o[2], B.o[1],
+                         B.o[0], bh);
+        ptx::tma_load_5d(sDO + h * BT_HALF_BYTES, &tm_do, &bars->q_full, h * 64, B.o[2], B.o[1],
+                         B.o[0], bh);
+      }
+      int seq = 0;
+      int issued[NS];
+#pragma unroll
+      for (int s = 0; s < NS; ++s) issued[s] = 0;
+      ChunkIter it;
+      iter_begin(cg, it);
+      bool ok = true;
+      for (seek_block(cg, P.kb, B, it); ok && it.idx < cg.total;
+           iter_next(cg, P.kb, it), seek_block(cg, P.kb, B, it)) {
+        for (int kv = 0; kv < 2 && ok; ++kv) {
+          const int slot = seq % NS;
+          if (seq >= NS) ok = ptx::wait(&bars->empty[slot], ((seq / NS) - 1) & 1, ctl);
+          if (!ok) break;
+          if (kv == 0) bars->info[slot] = 0;
+          ptx::mbar_expect_tx(&bars->full[slot], C::TILE_BYTES);
+          for (int h = 0; h < C::HALVES; ++h)
+            ptx::tma_load_5d(ring + slot * C::TILE_BYTES + h * BT_HALF_BYTES, kv ? &tm_v : &tm_k,
+                             &bars->full[slot], h * 64, it.a[2], it.a[1], it.a[0], bh);
+          ++issued[slot];
+          ++seq;
+        }
+      }
+      if (ok) {
+        const int slot = seq % NS;
+        if (seq >= NS) ok = ptx::wait(&bars->empty[slot], ((seq / NS) - 1) & 1, ctl);
+        if (ok) {
+          bars->info[slot] = BT_INFO_END;
+          ptx::mbar_arrive(&bars->full[slot]);
+          ++issued[slot];
+        }
+      }
+      for (int s = 0; s < NS; ++s)
+        if (issued[s]) ptx::wait_drain(&bars->full[s], (issued[s] - 1) & 1, ctl);
+      ptx::wait_drain(&bars->q_full, 0, ctl);
+    } else if (warp == 1 && lane == 0) {
+      // =========================== MMA issuer ===========================
+      const uint32_t sQa = ptx::smem_u32(sQ), sDOa = ptx::smem_u32(sDO);
+      const uint32_t ringa = ptx::smem_u32(ring);
+      // S = Q K^T into [S_COL0, +128) and dP = dO V^T into [DP_COL0, +128):
+      // both B operands are [keys x d] tiles read K-major.
+      auto issue_sdp = [&](int kslot, int vslot) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
+          ptx::mma_ss(tmem + C::S_COL0, ptx::desc_sw128(sQa + off, 16, 1024),
+                      ptx::desc_sw128(ringa + kslot * C::TILE_BYTES + off, 16, 1024), C::IDESC_S,
+                      kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
+          ptx::mma_ss(tmem + C::DP_COL0, ptx::desc_sw128(sDOa + off, 16, 1024),
+                      ptx::desc_sw128(ringa + vslot * C::TILE_BYTES + off, 16, 1024), C::IDESC_S,
+                      kk > 0 ? 1u : 0u);
+        }
+      };
+      // dQ += dS K: dS (16-bit pairs) of keys 64h.. in [DP_COL0 + 64h, +32),
+      // K read MN-major (its rows are the reduction dimension here).
+      auto issue_dq = [&](int kslot, bool accumulate) {
+#pragma unroll
+        for (int kk = 0; kk < BT_N / 16; ++kk) {
+          const uint32_t a_t = tmem + C::DP_COL0 + (kk >> 2) * 64 + (kk & 3) * 8;
+          const uint64_t bd =
+              ptx::desc_sw128(ringa + kslot * C::TILE_BYTES + kk * 2048, BT_HALF_BYTES, 1024);
+          ptx::mma_ts(tmem + C::DQ_COL0, a_t, bd, C::IDESC_DQ, (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = B.exists;
+      if (ok) ok = ptx::wait(&bars->q_full, 0, ctl);
+      for (int j = 0; ok; ++j) {
+        const int ks = 2 * j, vs = 2 * j + 1;
+        ok = ptx::wait(&bars->full[ks % NS], (ks / NS) & 1, ctl);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        if (bars->info[ks % NS] == BT_INFO_END) break;
+        ok = ptx::wait(&bars->full[vs % NS], (vs / NS) & 1, ctl);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        issue_sdp(ks % NS, vs % NS);
+        ptx::tc_commit(&bars->s_full);
+        ptx::tc_commit(&bars->empty[vs % NS]);
+        ok = ptx::wait(&bars->p_ready, j & 1, ctl);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        issue_dq(ks % NS, j > 0);
+        ptx::tc_commit(&bars->empty[ks % NS]);
+      }
+      ptx::tc_commit(&bars->o_done);
+      ptx::wait_drain(&bars->o_done, 0, ctl);
+    }
+  } else {
+    // ======================= element-wise warps =======================
+    ptx::regs_inc<BT_REGS_WORK>();
+    const int quarter = warp & 3;
+    const int h = (warp >> 3) & 1;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + C::S_COL0 + 64 * h;
+    const uint32_t tDP = tmem + lane_base + C::DP_COL0 + 64 * h;
+    const BlockInfo Bl = B;
+    const ChunkGrid cgl = cg;
+    const int kb[3] = {P.kb[0], P.kb[1], P.kb[2]};
+    auto query_coord = [&](int rr, int gc[3]) {
+      gc[2] = Bl.o[2] + rr % t.qb[2];
+      gc[1] = Bl.o[1] + (rr / t.qb[2]) % t.qb[1];
+      gc[0] = Bl.o[0] + rr / (t.qb[2] * t.qb[1]);
+    };
+    int wlo[3], whi[3];
+    float lse2 = 0.f, Di = 0.f;
+    {
+      int gc[3];
+      query_coord(row, gc);
+      for (int d = 0; d < 3; ++d)
+        window_range(P.g.L[d], P.g.w[d], P.g.s[d], P.g.m[d], imin(gc[d], P.g.L[d] - 1), wlo[d],
+                     whi[d]);
+      const bool valid = gc[0] < P.g.L[0] && gc[1] < P.g.L[1] && gc[2] < P.g.L[2];
+      if (Bl.exists && valid) {
+        const long long token = ((long long)gc[0] * P.g.L[1] + gc[1]) * P.g.L[2] + gc[2];
+        lse2 = P.lse[(size_t)bh * P.N + token] * BT_LOG2E;
+        Di = P.delta[(size_t)bh * P.N + token];
+      }
+    }
+    const float sl2 = P.scale_log2;
+    bool ok = Bl.exists;
+    int j = 0;
+    if (ok) {
+      ChunkIter it;
+      iter_begin(cgl, it);
+      for (int st = seek_block(cgl, kb, Bl, it); it.idx < cgl.total;
+           iter_next(cgl, kb, it), st = seek_block(cgl, kb, Bl, it)) {
+        bool got = ptx::wait(&bars->s_full, j & 1, ctl);
+        got = __all_sync(0xffffffffu, got);
+        if (!got) { ok = false; break; }
+        ptx::tc_fence_after();
+        uint32_t s[64], dp[64];
+        {
+          uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
+          uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
+          uint32_t (&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[0]);
+          uint32_t (&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[32]);
+          ptx::tmem_ld32(tS, s0);
+          ptx::tmem_ld32(tS + 32, s1);
+          ptx::tmem_ld32(tDP, d0);
+          ptx::tmem_ld32(tDP + 32, d1);
+          ptx::tmem_ld_wait();
+          ptx::reg_fence(s0);
+          ptx::reg_fence(s1);
+          ptx::reg_fence(d0);
+          ptx::reg_fence(d1);
+        }
+        if (st == CHUNK_PARTIAL) {
+          uint32_t mk[4];
+          chunk_key_mask(it.a, wlo, whi, kb, P.kb_log2, mk);
+          const uint32_t w0 = h ? mk[2] : mk[0], w1 = h ? mk[3] : mk[1];
+#pragma unroll
+          for (int q = 0; q < 64; ++q)
+            if (!(((q < 32 ? w0 : w1) >> (q & 31)) & 1u)) s[q] = __float_as_uint(-INFINITY);
+        }
+        const uint64_t scale2 = ptx::f2(sl2, sl2);
+        const uint64_t neg2 = ptx::f2(-lse2, -lse2);
+        const uint64_t negd2 = ptx::f2(-Di, -Di);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const uint64_t x = ptx::f2_fma(
+              ptx::f2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), scale2, neg2);
+          float x0, x1;
+          ptx::f2_split(x, x0, x1);
+          const uint64_t p = ptx::f2(ptx::ex2(x0), ptx::ex2(x1));
+          const uint64_t g = ptx::f2_add(
+              ptx::f2(__uint_as_float(dp[2 * q]), __uint_as_float(dp[2 * q + 1])), negd2);
+          float z0, z1;
+          ptx::f2_split(ptx::f2_mul(p, g), z0, z1);
+          s[q] = ptx::pack_half2<F16>(z0, z1);
+        }
+        {
+          uint32_t (&ds)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
+          ptx::tmem_st32(tDP, ds);
+        }
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->p_ready);
+        ++j;
+      }
+    }
+    // --------------------------- epilogue: dq ---------------------------
+    if (ok && j > 0) {
+      bool got = ptx::wait(&bars->o_done, 0, ctl);
+      got = __all_sync(0xffffffffu, got);
+      if (got) {
+        ptx::tc_fence_after();
+        int rr = row;
+        asm volatile("" : "+r"(rr));
+        int gc[3];
+        query_coord(rr, gc);
+        const bool valid = gc[0] < P.g.L[0] && gc[1] < P.g.L[1] && gc[2] < P.g.L[2];
+        const long long token = ((long long)gc[0] * P.g.L[1] + gc[1]) * P.g.L[2] + gc[2];
+        const size_t rbase = ((size_t)bh * P.N + (size_t)(valid ? token : 0)) * D + h * (D / 2);
+        uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(P.dq) + rbase);
+        const float sc = P.scale;
+#pragma unroll
+        for (int cc = 0; cc < D / 64; ++cc) {
+          uint32_t o[32];
+          ptx::tmem_ld32(tmem + lane_base + C::DQ_COL0 + h * (D / 2) + cc * 32, o);
+          ptx::tmem_ld_wait();
+          ptx::reg_fence(o);
+          if (valid) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+              pk[q] = ptx::pack_half2<F16>(__uint_as_float(o[2 * q]) * sc,
+                                           __uint_as_float(o[2 * q + 1]) * sc);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              orow[cc * 4 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+      }
+    } else if (ok && j == 0 && Bl.exists) {
+      // a block with no chunk cannot occur (every query sees >= 1 key)
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D, bool F16>
+cudaError_t launch_dq_d(const TcBwdLaunch& L, cudaStream_t stream, char* err, int errlen) {
+  CUtensorMap mq, mdo, mk, mv;
+  if (!encode_grid_map(&mq, L.q, L.f16, L.D, L.g.L, L.BH, L.N, L.t.qb) ||
+      !encode_grid_map(&mdo, L.dout, L.f16, L.D, L.g.L, L.BH, L.N, L.t.qb) ||
+      !encode_grid_map(&mk, L.k, L.f16, L.D, L.g.L, L.BH, L.N, L.kb) ||
+      !encode_grid_map(&mv, L.v, L.f16, L.D, L.g.L, L.BH, L.N, L.kb)) {
+    snprintf(err, errlen, "cuTensorMapEncodeTiled failed (pointer alignment or shape)");
+    return cudaErrorInvalidValue;
+  }
+  const size_t smem = bt_smem_bytes<D>();
+  static int attr_done[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, tc_bwd_dq_kernel<D, F16>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * BT_THREADS < BT_REGS_NEEDED) {
+      snprintf(err, errlen, "kernel compiled with %d registers/thread; the register split needs %d",
+               fa.numRegs, (BT_REGS_NEEDED + BT_THREADS - 1) / BT_THREADS);
+      return cudaErrorInvalidConfiguration;
+    }
+    e = cudaFuncSetAttribute(tc_bwd_dq_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = 1;
+  }
+  const long long grid = (long long)L.t.nblocks * L.BH;
+  if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  tc_bwd_dq_kernel<D, F16><<<(unsigned)grid, BT_THREADS, smem, stream>>>(mq, mdo, mk, mv, L);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_tc_bwd_dq(const TcBwdLaunch& L0, cudaStream_t stream, char* err, int errlen) {
+  TcBwdLaunch L = L0;
+  for (int d = 0; d < 3; ++d) {
+    if (L.t.qb[d] > 256 || L.kb[d] > 256) return cudaErrorNotSupported;
+    if (L.kb[d] & (L.kb[d] - 1)) return cudaErrorNotSupported;
+    int lg = 0;
+    while ((1 << lg) < L.kb[d]) ++lg;
+    L.kb_log2[d] = lg;
+  }
+  if (L.t.qb[0] * L.t.qb[1] * L.t.qb[2] != BT_M || L.kb[0] * L.kb[1] * L.kb[2] != BT_N)
+    return cudaErrorNotSupported;
+  switch (L.D) {
+    case 64:
+      return L.f16 ? launch_dq_d<64, true>(L, stream, err, errlen)
+                   : launch_dq_d<64, false>(L, stream, err, errlen);
+    case 128:
+      return L.f16 ? launch_dq_d<128, true>(L, stream, err, errlen)
+                   : launch_dq_d<128, false>(L, stream, err, errlen);
+    default:
+      return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace na

@@ -111,51 +111,6 @@ __device__ __forceinline__ void seek_pair(const ChunkGrid& cg, const int* kb, co
   st0 = st1 = CHUNK_EMPTY;
 }
 
-// Bits i of 32-bit word w that mark keys j = 32w + i with (j mod period) in
-// [a, b): one grid dimension's window range laid over a chunk's key order.
-__device__ __forceinline__ uint32_t periodic_range_word(int w, int period, int a, int b) {
-  uint32_t m = 0;
-  const int base = 32 * w;
-  for (int p0 = base - base % period; p0 < base + 32; p0 += period) {
-    const int lo = imax(p0 + a, base) - base;
-    const int hi = imin(p0 + b, base + 32) - base;
-    if (lo < hi) m |= (hi - lo == 32 ? 0xffffffffu : ((1u << (hi - lo)) - 1u) << lo);
-  }
-  return m;
-}
-
-// Validity of the 128 keys of a chunk for one query: key j (chunk-local
-// coordinates (j >> sh0, (j >> sh1) & (kb1-1), j & (kb2-1))) is inside the
-// query's window [wlo_d, whi_d) in every dimension.
-__device__ __forceinline__ void chunk_key_mask(const int a[3], const int wlo[3], const int whi[3],
-                                               const int kb[3], const int kbl[3], uint32_t (&mk)[4]) {
-  int lo[3], hi[3], stride[3];
-  stride[2] = 1;
-  stride[1] = 1 << kbl[2];
-  stride[0] = 1 << (kbl[1] + kbl[2]);
-  for (int d = 0; d < 3; ++d) {
-    lo[d] = imin(imax(wlo[d] - a[d], 0), kb[d]);
-    hi[d] = imin(imax(whi[d] - a[d], 0), kb[d]);
-  }
-#pragma unroll
-  for (int wd = 0; wd < 4; ++wd) {
-    uint32_t m = 0xffffffffu;
-    for (int d = 0; d < 3; ++d)
-      m &= periodic_range_word(wd, kb[d] * stride[d], lo[d] * stride[d], hi[d] * stride[d]);
-    mk[wd] = m;
-  }
-}
-
-// Same for one block: the status of the chunk found (CHUNK_EMPTY at the end).
-__device__ __forceinline__ int seek_block(const ChunkGrid& cg, const int* kb, const BlockInfo& b,
-                                          ChunkIter& it) {
-  for (; it.idx < cg.total; iter_next(cg, kb, it)) {
-    const int st = chunk_status(b, it.a, kb);
-    if (st != CHUNK_EMPTY) return st;
-  }
-  return CHUNK_EMPTY;
-}
-
 template <int D, bool F16>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -584,38 +539,8 @@ __global__ void exp2_poly_selftest_kernel(const float* x, float* y, int n) {
 }
 
 // ------------------------------------------------------------ host side --
-PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// [BH, X1, X2, X3, D] bf16 / f16 as a 5-d tensor (D, X3, X2, X1, BH),
-// 64-element inner box with 128-byte swizzle.
 bool encode_map(CUtensorMap* m, const void* ptr, const TcLaunch& L, const int box[3]) {
-  auto enc = get_encoder();
-  if (!enc) return false;
-  const cuuint64_t es = 2;
-  cuuint64_t dims[5] = {(cuuint64_t)L.D, (cuuint64_t)L.g.L[2], (cuuint64_t)L.g.L[1],
-                        (cuuint64_t)L.g.L[0], (cuuint64_t)L.BH};
-  cuuint64_t strides[4] = {(cuuint64_t)L.D * es, (cuuint64_t)L.g.L[2] * L.D * es,
-                           (cuuint64_t)L.g.L[1] * L.g.L[2] * L.D * es,
-                           (cuuint64_t)L.N * L.D * es};
-  cuuint32_t boxd[5] = {64, (cuuint32_t)box[2], (cuuint32_t)box[1], (cuuint32_t)box[0], 1};
-  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = enc(m, L.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                   5, const_cast<void*>(ptr), dims, strides,
-                   boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return encode_grid_map(m, ptr, L.f16, L.D, L.g.L, L.BH, L.N, box);
 }
 
 template <int D, bool F16>
@@ -654,6 +579,35 @@ cudaError_t launch_d(const TcLaunch& L, cudaStream_t stream, char* err, int errl
 }
 
 }  // namespace
+
+// [BH, X1, X2, X3, D] bf16 / f16 as a 5-d tensor (D, X3, X2, X1, BH),
+// 64-element inner box with 128-byte swizzle.
+bool encode_grid_map(CUtensorMap* m, const void* ptr, int f16, int D, const int L[3], int BH,
+                     int N, const int box[3]) {
+  static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  if (!enc) return false;
+  const cuuint64_t es = 2;
+  cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)L[2], (cuuint64_t)L[1], (cuuint64_t)L[0],
+                        (cuuint64_t)BH};
+  cuuint64_t strides[4] = {(cuuint64_t)D * es, (cuuint64_t)L[2] * D * es,
+                           (cuuint64_t)L[1] * L[2] * D * es, (cuuint64_t)N * D * es};
+  cuuint32_t boxd[5] = {64, (cuuint32_t)box[2], (cuuint32_t)box[1], (cuuint32_t)box[0], 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
+                   const_cast<void*>(ptr), dims, strides, boxd, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t stream) {
   if (n <= 0) return cudaSuccess;

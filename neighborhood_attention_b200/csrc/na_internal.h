@@ -1,6 +1,7 @@
 // Internal interface between the C-ABI layer (na_api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -54,8 +55,35 @@ struct BwdLaunch {
   void *dq, *dk, *dv;
 };
 
+// Tensor-core backward, dQ part: per query block, S = Q K^T and dP = dO V^T
+// into tensor memory, dS = P (dP - delta) written back as 16-bit, dQ += dS K.
+struct TcBwdLaunch {
+  Geom g;
+  QTiling t;             // query blocks (128 tokens)
+  int kb[3];             // key chunks (128 tokens)
+  int kb_log2[3];        // filled by the launcher
+  int BH, N, D;
+  int f16;               // 1: f16, 0: bf16
+  float scale, scale_log2;
+  const void *q, *k, *v, *dout;
+  const float* lse;
+  const float* delta;    // <dout_i, out_i>, written by the row-delta kernel first
+  void* dq;
+  int* status;           // device status word
+  long long timeout_ns;  // bound on every in-kernel wait
+};
+
+// 5-d TMA descriptor of a [BH, X1, X2, X3, D] bf16 / f16 tensor, 64-element
+// inner box of `box` tokens, 128-byte swizzle.
+bool encode_grid_map(CUtensorMap* m, const void* ptr, int f16, int D, const int L[3], int BH,
+                     int N, const int box[3]);
+
 cudaError_t launch_simt(const SimtLaunch& L, cudaStream_t stream);
 cudaError_t launch_bwd_simt(const BwdLaunch& L, cudaStream_t stream);
+// The row-delta and dK/dV CUDA-core kernels alone (the dQ kernel left out).
+cudaError_t launch_bwd_simt_delta(const BwdLaunch& L, cudaStream_t stream);
+cudaError_t launch_bwd_simt_dkdv(const BwdLaunch& L, cudaStream_t stream);
+cudaError_t launch_tc_bwd_dq(const TcBwdLaunch& L, cudaStream_t stream, char* err, int errlen);
 
 // y[i] = the tensor-core kernel's FMA-pipe 2^x applied to x[i] (self-test).
 cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t stream);

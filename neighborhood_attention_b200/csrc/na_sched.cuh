@@ -201,4 +201,49 @@ NA_HD int make_tiling(const Geom& g, const int qb[3], const int tl[3], QTiling& 
   return 0;
 }
 
+// Bits i of 32-bit word w that mark keys j = 32w + i with (j mod period) in
+// [a, b): one grid dimension's window range laid over a chunk's key order.
+NA_HD uint32_t periodic_range_word(int w, int period, int a, int b) {
+  uint32_t m = 0;
+  const int base = 32 * w;
+  for (int p0 = base - base % period; p0 < base + 32; p0 += period) {
+    const int lo = imax(p0 + a, base) - base;
+    const int hi = imin(p0 + b, base + 32) - base;
+    if (lo < hi) m |= (hi - lo == 32 ? 0xffffffffu : ((1u << (hi - lo)) - 1u) << lo);
+  }
+  return m;
+}
+
+// Validity of the 128 keys of a chunk for one query: key j (chunk-local
+// coordinates (j >> sh0, (j >> sh1) & (kb1-1), j & (kb2-1))) is inside the
+// query's window [wlo_d, whi_d) in every dimension.
+NA_HD void chunk_key_mask(const int a[3], const int wlo[3], const int whi[3],
+                                               const int kb[3], const int kbl[3], uint32_t (&mk)[4]) {
+  int lo[3], hi[3], stride[3];
+  stride[2] = 1;
+  stride[1] = 1 << kbl[2];
+  stride[0] = 1 << (kbl[1] + kbl[2]);
+  for (int d = 0; d < 3; ++d) {
+    lo[d] = imin(imax(wlo[d] - a[d], 0), kb[d]);
+    hi[d] = imin(imax(whi[d] - a[d], 0), kb[d]);
+  }
+#pragma unroll
+  for (int wd = 0; wd < 4; ++wd) {
+    uint32_t m = 0xffffffffu;
+    for (int d = 0; d < 3; ++d)
+      m &= periodic_range_word(wd, kb[d] * stride[d], lo[d] * stride[d], hi[d] * stride[d]);
+    mk[wd] = m;
+  }
+}
+
+// Same for one block: the status of the chunk found (CHUNK_EMPTY at the end).
+NA_HD int seek_block(const ChunkGrid& cg, const int* kb, const BlockInfo& b,
+                                          ChunkIter& it) {
+  for (; it.idx < cg.total; iter_next(cg, kb, it)) {
+    const int st = chunk_status(b, it.a, kb);
+    if (st != CHUNK_EMPTY) return st;
+  }
+  return CHUNK_EMPTY;
+}
+
 }  // namespace na

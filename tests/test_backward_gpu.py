@@ -3,10 +3,13 @@ the C ABI, after the CUDA forward produced out and lse) against the fp64
 oracle's gradients on identical seeded inputs, element by element.
 
 Bar, from the arithmetic: 16-bit gradients are rounded once to the input
-type (half an ulp, 2^-9 relative for bf16, 2^-12 for f16), and the forward's
-16-bit out enters D_i = <dO_i, out_i>; fp32 accumulation adds far less.  So
-max |g - oracle| <= 2^-8 max|oracle| + 2e-3 and mean <= 2^-10 mean|oracle| + 2e-4
-for bf16 / f16; fp32 inputs: max <= 1e-4 max(1, max|oracle|), mean <= 1e-5."""
+type (half an ulp, 2^-9 relative for bf16, 2^-12 for f16); on the tensor-core
+path dS is also rounded to the input type as the operand of dq's product (as
+P is in the forward), each of the window's terms carrying that relative
+error; and the forward's 16-bit out enters D_i = <dO_i, out_i>.  fp32
+accumulation adds far less.  So for bf16 / f16
+max |g - oracle| <= 2^-7 max|oracle| + 4e-3 and mean <= 2^-8 mean|oracle| + 2e-4;
+fp32 inputs (CUDA cores only): max <= 1e-4 max(1, max|oracle|), mean <= 1e-5."""
 import zlib
 
 import numpy as np
@@ -45,7 +48,7 @@ CASES = {
 }
 
 
-def _run(c, seed):
+def _run(c, seed, kernel=None):
     shape = (c["B"], c["heads"], *c["grid"], c["d"])
     q, k, v = seeded_inputs.qkv(seed, c["B"], c["heads"], c["grid"], c["d"], c["dtype"])
     gen = {"f32": seeded_inputs.normal_f32, "bf16": seeded_inputs.normal_bf16_bits,
@@ -54,8 +57,10 @@ def _run(c, seed):
     qd, kd, vd, dod = (to_device(a, c["dtype"]) for a in (q, k, v, do))
     opts = na.make_options(window_mode=c["mode"], ndim=len(c["grid"])) if c["mode"] else None
     out, lse = na.forward(qd, kd, vd, c["window"], c["stride"], c["tile"], options=opts)
+    bopts = na.make_options(window_mode=c["mode"], ndim=len(c["grid"]),
+                            kernel=kernel if kernel is not None else na.NA_KERNEL_AUTO)
     dq, dk, dv = na.backward(qd, kd, vd, out, lse, dod, c["window"], c["stride"], c["tile"],
-                             options=opts)
+                             options=bopts)
     na.na_sync_status()
     got = [t.float().cpu().numpy().astype(np.float64) for t in (dq, dk, dv)]
     ref = oracle.backward(q, k, v, do, c["grid"], c["window"], c["stride"], dtype=c["dtype"],
@@ -70,17 +75,27 @@ def _assert_close(c, got, ref, label):
         if c["dtype"] == "f32":
             tmax, tmean = 1e-4 * max(1.0, np.abs(r).max()), 1e-5
         else:
-            tmax = 2.0 ** -8 * np.abs(r).max() + 2e-3
-            tmean = 2.0 ** -10 * np.abs(r).mean() + 2e-4
+            tmax = 2.0 ** -7 * np.abs(r).max() + 4e-3
+            tmean = 2.0 ** -8 * np.abs(r).mean() + 2e-4
         assert err.max() <= tmax, f"{label} {name}: max|err|={err.max():.3e} > {tmax:.3e}"
         assert err.mean() <= tmean, f"{label} {name}: mean|err|={err.mean():.3e} > {tmean:.3e}"
 
 
 @pytest.mark.parametrize("name", sorted(CASES))
 def test_backward_parity(name):
+    """The default path: tensor-core dQ for bf16 / f16 with head_dim 64 or 128,
+    CUDA-core kernels otherwise."""
     c = CASES[name]
     got, ref = _run(c, seed=zlib.crc32(name.encode()) % 100000)
     _assert_close(c, got, ref, name)
+
+
+@pytest.mark.parametrize("name", ["na2d_ragged_d64", "causal1d", "sta3d_small", "f16_d64"])
+def test_backward_parity_cuda_cores(name):
+    """The same cases with every backward kernel on the CUDA cores."""
+    c = CASES[name]
+    got, ref = _run(c, seed=zlib.crc32(name.encode()) % 100000, kernel=na.NA_KERNEL_SIMT)
+    _assert_close(c, got, ref, name + "/simt")
 
 
 def test_backward_deterministic():
@@ -91,9 +106,9 @@ def test_backward_deterministic():
         assert np.array_equal(x, y)
 
 
-def test_backward_refuses_tensor_core_selector():
-    c = CASES["na2d_d128"]
-    q = torch.zeros((1, 1, *c["grid"], 128), dtype=torch.bfloat16, device="cuda")
+def test_backward_tensor_core_selector_needs_16_bit():
+    c = CASES["fp32_d32"]
+    q = torch.zeros((1, 1, *c["grid"], 64), dtype=torch.float32, device="cuda")
     lse = torch.zeros(q.shape[:-1], dtype=torch.float32, device="cuda")
     with pytest.raises(na.NaError) as e:
         na.backward(q, q, q, q, lse, q, c["window"], options=na.make_options(kernel=na.NA_KERNEL_TC))
