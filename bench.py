@@ -265,10 +265,13 @@ NUM_SM = 148
 
 def run_backward(args, rank, world, local_rank):
     """The backward pass (na_backward: dq, dk, dv) on the selected workload:
-    one step = one call (three CUDA-core kernels); the forward's out and lse
-    are produced once before timing.  Effective TFLOP/s counts 10 * d FLOPs
-    per attended (query, key) pair (five products of 2 d: scores, dP, dV, dQ,
-    dK), against the fp32 FMA peak of the CUDA cores at the sampled clock."""
+    one step = one call (row delta, then the dq and dk / dv kernels -- on the
+    tensor cores for bf16 / f16 with head_dim 64 or 128); the forward's out
+    and lse are produced once before timing.  Effective TFLOP/s counts 10 * d
+    FLOPs per attended (query, key) pair (five products of 2 d: scores, dP, dV,
+    dQ, dK; the two kernels each recompute scores and dP, which is not
+    counted), against the measured dense bf16 peak -- or, when the CUDA-core
+    kernels run, the fp32 FMA peak at the sampled clock."""
     import torch
     import torch.distributed as dist
     import neighborhood_attention_b200 as na
@@ -320,8 +323,15 @@ def run_backward(args, rank, world, local_rank):
                       {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32}[w["dtype"]])
     flops = 10.0 * w["head_dim"] * w["B"] * w["heads"] * plan["useful_pairs"]
     value = flops * args.steps * world / (total_ms / 1e3) / 1e12
-    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
-    peak = 2.0 * FP32_FMA_PER_CLK_SM * NUM_SM * mhz * 1e6 / 1e12
+    tensor = w["dtype"] in ("bf16", "f16") and w["head_dim"] in (64, 128)
+    if tensor:
+        peak, _, peak_kind = read_peaks()
+        peak_kind = (f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                     else "fallback")
+    else:
+        mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
+        peak = 2.0 * FP32_FMA_PER_CLK_SM * NUM_SM * mhz * 1e6 / 1e12
+        peak_kind = "derived: 148 SM x 128 fp32 FMA/clk x 2 FLOP x sampled SM clock"
     achieved = value / world
     if rank != 0:
         return 0
@@ -330,10 +340,11 @@ def run_backward(args, rank, world, local_rank):
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
-        "config": dict(w, direction="backward", kernels="CUDA-core (fp32 FMA)"),
-        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
-                     "peak_kind": "derived: 148 SM x 128 fp32 FMA/clk x 2 FLOP x sampled SM clock"},
+        "config": dict(w, direction="backward",
+                       kernels="tcgen05 dq and dk/dv" if tensor else "CUDA-core (fp32 FMA)"),
+        "roofline": {"bound": "tensor" if tensor else "alu", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "peak_kind": peak_kind},
         "gpu_launches": 3 * args.steps,
         "clocks": clocks,
     }

@@ -507,15 +507,18 @@ na_status na_backward(const void* q, const void* k, const void* v, const void* o
   T.f16 = P.dtype == NA_F16;
   T.scale = scale;
   T.scale_log2 = L.scale_log2;
-  T.q = q; T.k = k; T.v = v; T.dout = dout; T.lse = lse; T.delta = delta; T.dq = dq;
+  T.q = q; T.k = k; T.v = v; T.dout = dout; T.lse = lse; T.delta = delta;
+  T.dq = dq; T.dk = dk; T.dv = dv;
   T.status = status;
   T.timeout_ns = P.opt.wait_timeout_ns > 0 ? P.opt.wait_timeout_ns : default_timeout_ns();
   char msg[256] = "";
   e = launch_tc_bwd_dq(T, s, msg, sizeof msg);
   if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "tensor-core dq: shape");
   if (e != cudaSuccess) return fail(NA_ERR_CUDA, "tensor-core dq: %s %s", cudaGetErrorString(e), msg);
-  e = launch_bwd_simt_dkdv(L, s);
-  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "backward dk/dv: %s", cudaGetErrorString(e));
+  e = launch_tc_bwd_dkdv(T, s, msg, sizeof msg);
+  if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "tensor-core dk/dv: shape");
+  if (e != cudaSuccess)
+    return fail(NA_ERR_CUDA, "tensor-core dk/dv: %s %s", cudaGetErrorString(e), msg);
   return NA_OK;
 }
 

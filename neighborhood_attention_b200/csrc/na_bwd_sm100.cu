@@ -18,7 +18,17 @@
 // 64-127 of every chunk, rows 32q..32q+31).  Every wait is bounded (see
 // na_ptx.cuh); the chunk stream ends with a marker in the next K slot.
 //
-// TMEM columns: S [0, 128), dP [128, 256) -- after the element-wise pass
+// The dK / dV part (tc_bwd_dkdv_kernel) is key-stationary: for one 128-key
+// block per CTA (K and V resident in shared memory) and every chunk of the
+// queries whose windows hold some of its keys,
+//   S^T = K Q^T,  dP^T = V dO^T,  P^T = exp(scale S^T - lse),
+//   dS^T = P^T (dP^T - delta),  dV += P^T dO,  dK += dS^T Q,
+// with dk = scale dK.  The queries that see a key form a box per dimension
+// (both window ends are monotone in the query coordinate), found by binary
+// search, so the same chunk walk and full / partial / empty labels as the
+// forward apply with the key block's inverse windows in place of windows.
+//
+// TMEM columns (dQ kernel): S [0, 128), dP [128, 256) -- after the element-wise pass
 // dS of keys 64h..64h+63 sits as packed 16-bit pairs in [128 + 64h, 160 + 64h),
 // inside the half of dP that warp h itself read -- and dQ [256, 256 + D).
 #include <cuda.h>
@@ -369,6 +379,462 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
   }
 }
 
+// ----------------------------------------------------------------- dK dV --
+// First i in [0, L) whose window satisfies pred (false then true as i grows).
+template <class F>
+__device__ __forceinline__ int first_query(int L, F pred) {
+  int lo = 0, hi = L;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (pred(mid)) hi = mid; else lo = mid + 1;
+  }
+  return lo;
+}
+
+// Queries whose window holds key j in one dimension: [*i0, *i1).
+__device__ __forceinline__ void inverse_range(int L, int w, int s, int m, int j, int& i0, int& i1) {
+  i0 = first_query(L, [&](int i) { int lo, hi; window_range(L, w, s, m, i, lo, hi); return hi > j; });
+  i1 = first_query(L, [&](int i) { int lo, hi; window_range(L, w, s, m, i, lo, hi); return lo > j; });
+}
+
+template <int D, bool F16>
+struct BkCfg {
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int NQ = (D == 128) ? 2 : 4;   // query-chunk stages (Q and dO each)
+  static constexpr int HALVES = D / 64;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int S_COL0 = 0;                 // S^T, then P^T
+  static constexpr int DP_COL0 = 128;              // dP^T, then dS^T
+  static constexpr int DV_COL0 = 256;
+  static constexpr int DK_COL0 = 256 + D;
+  static constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(BT_M, BT_N, false, false, F16);
+  static constexpr uint32_t IDESC_ACC = ptx::idesc_bf16_f32(BT_M, D, false, true, F16);
+};
+
+template <int NQ>
+struct BkBars {
+  uint64_t kv_full;          // K and V tiles of the key block
+  uint64_t full[NQ];         // query chunk stage loaded (TMA bytes + 32 producer lanes)
+  uint64_t empty[NQ];
+  uint64_t s_full;           // S^T and dP^T of the current chunk
+  uint64_t p_ready;          // P^T and dS^T stored (256 arrivals)
+  uint64_t o_done;
+  uint32_t tmem_base;
+  int abort;
+  volatile uint32_t info[NQ];
+  float lse2[NQ][BT_N];      // log2(e) * lse of the stage's queries
+  float dlt[NQ][BT_N];       // delta of the stage's queries
+  BlockInfo kb;              // the key block (origin, extent)
+  BlockInfo ib;              // its inverse windows: lo/hi = union, ilo/ihi = intersection
+  ChunkGrid cg;              // query chunks over ib
+};
+
+template <int D>
+constexpr size_t bk_smem_bytes() {
+  return 1024 + (size_t)(2 + 2 * BkCfg<D, false>::NQ) * BkCfg<D, false>::TILE_BYTES +
+         sizeof(BkBars<BkCfg<D, false>::NQ>);
+}
+
+template <int D, bool F16>
+__global__ void __launch_bounds__(BT_THREADS, 1)
+    tc_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                       const TcBwdLaunch P) {
+  using C = BkCfg<D, F16>;
+  constexpr int NQ = C::NQ;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = base;
+  uint8_t* sV = base + C::TILE_BYTES;
+  uint8_t* stages = base + 2 * C::TILE_BYTES;      // stage s: Q at 2s, dO at 2s+1
+  BkBars<NQ>* bars = reinterpret_cast<BkBars<NQ>*>(stages + 2 * NQ * C::TILE_BYTES);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const QTiling& t = P.t;                           // key blocks use the query tiling
+  const int bh = blockIdx.x / t.nblocks;
+  const int blk = blockIdx.x % t.nblocks;
+  const BlockInfo& KB = bars->kb;
+  const BlockInfo& IB = bars->ib;
+  const ChunkGrid& cg = bars->cg;
+
+  if (threadIdx.x == 0) {
+    block_info(P.g, t, blk, bars->kb);
+    BlockInfo& ib = bars->ib;
+    ib.exists = bars->kb.exists;
+    for (int d = 0; d < 3; ++d) {
+      ib.o[d] = 0;
+      ib.n[d] = P.g.L[d];
+      if (!ib.exists) continue;
+      const int L = P.g.L[d], w = P.g.w[d], s = P.g.s[d], m = P.g.m[d];
+      const int k0 = bars->kb.o[d], k1 = bars->kb.o[d] + bars->kb.n[d] - 1;
+      int a0, a1, b0, b1;
+      inverse_range(L, w, s, m, k0, a0, a1);
+      inverse_range(L, w, s, m, k1, b0, b1);
+      ib.lo[d] = a0;     // union of the keys' query ranges: [I0(k0), I1(k1))
+      ib.hi[d] = b1;
+      ib.ilo[d] = b0;    // intersection: [I0(k1), I1(k0))
+      ib.ihi[d] = a1;
+    }
+    chunk_grid_for(&bars->ib, 1, P.kb, bars->cg);
+    ptx::mbar_init(&bars->kv_full, 1);
+    for (int s = 0; s < NQ; ++s) {
+      ptx::mbar_init(&bars->full[s], 32);
+      ptx::mbar_init(&bars->empty[s], 1);
+    }
+    ptx::mbar_init(&bars->s_full, 1);
+    ptx::mbar_init(&bars->p_ready, 2 * BT_M);
+    ptx::mbar_init(&bars->o_done, 1);
+    bars->abort = *reinterpret_cast<volatile int*>(P.status) != 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  ptx::WaitCtl ctl;
+  ctl.abort = &bars->abort;
+  ctl.status = P.status;
+  ctl.timeout_ns = (uint64_t)P.timeout_ns;
+
+  if (warp < 4) {
+    ptx::regs_dec<BT_REGS_LOADER>();
+    if (warp == 0 && KB.exists) {
+      // ====================== producer (whole warp) ======================
+      // Lane 0 issues the TMA copies; every lane stages lse / delta of four
+      // of the chunk's queries and arrives on the stage's barrier.
+      if (lane == 0) {
+        ptx::mbar_expect_tx(&bars->kv_full, 2 * C::TILE_BYTES);
+        for (int h = 0; h < C::HALVES; ++h) {
+          ptx::tma_load_5d(sK + h * BT_HALF_BYTES, &tm_k, &bars->kv_full, h * 64, KB.o[2], KB.o[1],
+                           KB.o[0], bh);
+          ptx::tma_load_5d(sV + h * BT_HALF_BYTES, &tm_v, &bars->kv_full, h * 64, KB.o[2], KB.o[1],
+                           KB.o[0], bh);
+        }
+      }
+      int issued[NQ];
+#pragma unroll
+      for (int s = 0; s < NQ; ++s) issued[s] = 0;
+      int seq = 0;
+      ChunkIter it;
+      iter_begin(cg, it);
+      bool ok = true;
+      for (seek_block(cg, P.kb, IB, it); ok && it.idx < cg.total;
+           iter_next(cg, P.kb, it), seek_block(cg, P.kb, IB, it), ++seq) {
+        const int st = seq % NQ;
+        if (seq >= NQ) ok = ptx::wait(&bars->empty[st], ((seq / NQ) - 1) & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        for (int e = lane; e < BT_N; e += 32) {
+          const int q2 = e % P.kb[2], q1 = (e / P.kb[2]) % P.kb[1], q0 = e / (P.kb[2] * P.kb[1]);
+          const int x0 = it.a[0] + q0, x1 = it.a[1] + q1, x2 = it.a[2] + q2;
+          float l2 = 0.f, dl = 0.f;
+          if (x0 < P.g.L[0] && x1 < P.g.L[1] && x2 < P.g.L[2]) {
+            const size_t tok = ((size_t)x0 * P.g.L[1] + x1) * P.g.L[2] + x2;
+            l2 = P.lse[(size_t)bh * P.N + tok] * BT_LOG2E;
+            dl = P.delta[(size_t)bh * P.N + tok];
+          }
+          bars->lse2[st][e] = l2;
+          bars->dlt[st][e] = dl;
+        }
+        if (lane == 0) {
+          bars->info[st] = 0;
+          ptx::mbar_expect_tx(&bars->full[st], 2 * C::TILE_BYTES);
+          for (int h = 0; h < C::HALVES; ++h) {
+            ptx::tma_load_5d(stages + (2 * st) * C::TILE_BYTES + h * BT_HALF_BYTES, &tm_q,
+                             &bars->full[st], h * 64, it.a[2], it.a[1], it.a[0], bh);
+            ptx::tma_load_5d(stages + (2 * st + 1) * C::TILE_BYTES + h * BT_HALF_BYTES, &tm_do,
+                             &bars->full[st], h * 64, it.a[2], it.a[1], it.a[0], bh);
+          }
+        } else {
+          ptx::mbar_arrive(&bars->full[st]);
+        }
+        ++issued[st];
+      }
+      if (ok) {
+        const int st = seq % NQ;
+        if (seq >= NQ) ok = ptx::wait(&bars->empty[st], ((seq / NQ) - 1) & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          if (lane == 0) bars->info[st] = BT_INFO_END;
+          __syncwarp();
+          ptx::mbar_arrive(&bars->full[st]);
+          ++issued[st];
+        }
+      }
+      if (lane == 0) {
+        for (int s = 0; s < NQ; ++s)
+          if (issued[s]) ptx::wait_drain(&bars->full[s], (issued[s] - 1) & 1, ctl);
+        ptx::wait_drain(&bars->kv_full, 0, ctl);
+      }
+    } else if (warp == 1 && lane == 0) {
+      // =========================== MMA issuer ===========================
+      const uint32_t sKa = ptx::smem_u32(sK), sVa = ptx::smem_u32(sV);
+      const uint32_t sta = ptx::smem_u32(stages);
+      auto issue_s = [&](int st) {
+        const uint32_t qa = sta + (2 * st) * C::TILE_BYTES, da = qa + C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
+          ptx::mma_ss(tmem + C::S_COL0, ptx::desc_sw128(sKa + off, 16, 1024),
+                      ptx::desc_sw128(qa + off, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
+          ptx::mma_ss(tmem + C::DP_COL0, ptx::desc_sw128(sVa + off, 16, 1024),
+                      ptx::desc_sw128(da + off, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      // dV += P^T dO and dK += dS^T Q: the stage's tiles read MN-major (their
+      // rows, the chunk's queries, are the reduction dimension).
+      auto issue_acc = [&](int st, bool accumulate) {
+        const uint32_t qa = sta + (2 * st) * C::TILE_BYTES, da = qa + C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BT_N / 16; ++kk) {
+          const uint32_t col = (kk >> 2) * 64 + (kk & 3) * 8;
+          ptx::mma_ts(tmem + C::DV_COL0, tmem + C::S_COL0 + col,
+                      ptx::desc_sw128(da + kk * 2048, BT_HALF_BYTES, 1024), C::IDESC_ACC,
+                      (accumulate || kk > 0) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < BT_N / 16; ++kk) {
+          const uint32_t col = (kk >> 2) * 64 + (kk & 3) * 8;
+          ptx::mma_ts(tmem + C::DK_COL0, tmem + C::DP_COL0 + col,
+                      ptx::desc_sw128(qa + kk * 2048, BT_HALF_BYTES, 1024), C::IDESC_ACC,
+                      (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = KB.exists;
+      if (ok) ok = ptx::wait(&bars->kv_full, 0, ctl);
+      for (int j = 0; ok; ++j) {
+        const int st = j % NQ;
+        ok = ptx::wait(&bars->full[st], (j / NQ) & 1, ctl);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        if (bars->info[st] == BT_INFO_END) break;
+        issue_s(st);
+        ptx::tc_commit(&bars->s_full);
+        ok = ptx::wait(&bars->p_ready, j & 1, ctl);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        issue_acc(st, j > 0);
+        ptx::tc_commit(&bars->empty[st]);
+      }
+      ptx::tc_commit(&bars->o_done);
+      ptx::wait_drain(&bars->o_done, 0, ctl);
+    }
+  } else {
+    // ======================= element-wise warps =======================
+    ptx::regs_inc<BT_REGS_WORK>();
+    const int quarter = warp & 3;
+    const int h = (warp >> 3) & 1;              // query half of every chunk
+    const int row = quarter * 32 + lane;        // key row of the block
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_base + C::S_COL0 + 64 * h;
+    const uint32_t tDP = tmem + lane_base + C::DP_COL0 + 64 * h;
+    const BlockInfo Kl = KB;
+    const BlockInfo Il = IB;
+    const ChunkGrid cgl = cg;
+    const int qc[3] = {P.kb[0], P.kb[1], P.kb[2]};
+    auto key_coord = [&](int rr, int gc[3]) {
+      gc[2] = Kl.o[2] + rr % t.qb[2];
+      gc[1] = Kl.o[1] + (rr / t.qb[2]) % t.qb[1];
+      gc[0] = Kl.o[0] + rr / (t.qb[2] * t.qb[1]);
+    };
+    int ilo[3], ihi[3];    // queries whose window holds this key, per dimension
+    {
+      int gc[3];
+      key_coord(row, gc);
+      const bool kvalid = gc[0] < P.g.L[0] && gc[1] < P.g.L[1] && gc[2] < P.g.L[2];
+      for (int d = 0; d < 3; ++d) {
+        if (Kl.exists && kvalid) {
+          inverse_range(P.g.L[d], P.g.w[d], P.g.s[d], P.g.m[d], gc[d], ilo[d], ihi[d]);
+        } else {
+          ilo[d] = 0;
+          ihi[d] = 0;     // a key outside the grid is in no window
+        }
+      }
+    }
+    const float sl2 = P.scale_log2;
+    bool ok = Kl.exists;
+    int j = 0;
+    if (ok) {
+      ChunkIter it;
+      iter_begin(cgl, it);
+      for (int stc = seek_block(cgl, qc, Il, it); it.idx < cgl.total;
+           iter_next(cgl, qc, it), stc = seek_block(cgl, qc, Il, it)) {
+        const int st = j % NQ;
+        bool got = ptx::wait(&bars->s_full, j & 1, ctl);
+        got = __all_sync(0xffffffffu, got);
+        if (!got) { ok = false; break; }
+        ptx::tc_fence_after();
+        uint32_t s[64], dp[64];
+        {
+          uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
+          uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
+          uint32_t (&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[0]);
+          uint32_t (&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[32]);
+          ptx::tmem_ld32(tS, s0);
+          ptx::tmem_ld32(tS + 32, s1);
+          ptx::tmem_ld32(tDP, d0);
+          ptx::tmem_ld32(tDP + 32, d1);
+          ptx::tmem_ld_wait();
+          ptx::reg_fence(s0);
+          ptx::reg_fence(s1);
+          ptx::reg_fence(d0);
+          ptx::reg_fence(d1);
+        }
+        // Mask (partial chunks): query c of the chunk sees this key iff its
+        // coordinates lie in the key's inverse ranges; padded keys see none.
+        if (stc == CHUNK_PARTIAL || ihi[0] == 0) {
+          uint32_t mk[4];
+          chunk_key_mask(it.a, ilo, ihi, qc, P.kb_log2, mk);
+          const uint32_t w0 = h ? mk[2] : mk[0], w1 = h ? mk[3] : mk[1];
+#pragma unroll
+          for (int q = 0; q < 64; ++q)
+            if (!(((q < 32 ? w0 : w1) >> (q & 31)) & 1u)) s[q] = __float_as_uint(-INFINITY);
+        }
+        const uint64_t scale2 = ptx::f2(sl2, sl2);
+        const float* l2p = &bars->lse2[st][64 * h];
+        const float* dlp = &bars->dlt[st][64 * h];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const float2 l2 = *reinterpret_cast<const float2*>(l2p + 2 * q);
+          const float2 dl = *reinterpret_cast<const float2*>(dlp + 2 * q);
+          const uint64_t x = ptx::f2_fma(
+              ptx::f2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), scale2,
+              ptx::f2(-l2.x, -l2.y));
+          float x0, x1;
+          ptx::f2_split(x, x0, x1);
+          const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
+          const uint64_t g = ptx::f2_add(
+              ptx::f2(__uint_as_float(dp[2 * q]), __uint_as_float(dp[2 * q + 1])),
+              ptx::f2(-dl.x, -dl.y));
+          float z0, z1;
+          ptx::f2_split(ptx::f2_mul(ptx::f2(p0, p1), g), z0, z1);
+          s[q] = ptx::pack_half2<F16>(p0, p1);
+          dp[q] = ptx::pack_half2<F16>(z0, z1);
+        }
+        {
+          uint32_t (&pw)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
+          uint32_t (&dw)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[0]);
+          ptx::tmem_st32(tS, pw);
+          ptx::tmem_st32(tDP, dw);
+        }
+        ptx::tmem_st_wait();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->p_ready);
+        ++j;
+      }
+    }
+    // ------------------------ epilogue: dk, dv ------------------------
+    if (ok && j > 0) {
+      bool got = ptx::wait(&bars->o_done, 0, ctl);
+      got = __all_sync(0xffffffffu, got);
+      if (got) {
+        ptx::tc_fence_after();
+        int rr = row;
+        asm volatile("" : "+r"(rr));
+        int gc[3];
+        key_coord(rr, gc);
+        const bool valid = gc[0] < P.g.L[0] && gc[1] < P.g.L[1] && gc[2] < P.g.L[2];
+        const long long token = ((long long)gc[0] * P.g.L[1] + gc[1]) * P.g.L[2] + gc[2];
+        const size_t rbase = ((size_t)bh * P.N + (size_t)(valid ? token : 0)) * D + h * (D / 2);
+        for (int which = 0; which < 2; ++which) {
+          uint4* orow = reinterpret_cast<uint4*>(
+              reinterpret_cast<uint16_t*>(which ? P.dk : P.dv) + rbase);
+          const float sc = which ? P.scale : 1.f;
+          const int col0 = (which ? C::DK_COL0 : C::DV_COL0) + h * (D / 2);
+#pragma unroll
+          for (int cc = 0; cc < D / 64; ++cc) {
+            uint32_t o[32];
+            ptx::tmem_ld32(tmem + lane_base + col0 + cc * 32, o);
+            ptx::tmem_ld_wait();
+            ptx::reg_fence(o);
+            if (valid) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int q = 0; q < 16; ++q)
+                pk[q] = ptx::pack_half2<F16>(__uint_as_float(o[2 * q]) * sc,
+                                             __uint_as_float(o[2 * q + 1]) * sc);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                orow[cc * 4 + v] =
+                    make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            }
+          }
+        }
+      }
+    } else if (ok && j == 0) {
+      // No query sees any key of this block (possible: keys outside every
+      // window, e.g. the last keys under causal windows with stride 1 never
+      // are -- but a ragged grid can leave keys unseen): their gradients are
+      // zero.
+      int rr = row;
+      int gc[3];
+      key_coord(rr, gc);
+      const bool valid = gc[0] < P.g.L[0] && gc[1] < P.g.L[1] && gc[2] < P.g.L[2];
+      if (valid) {
+        const long long token = ((long long)gc[0] * P.g.L[1] + gc[1]) * P.g.L[2] + gc[2];
+        const size_t rbase = ((size_t)bh * P.N + (size_t)token) * D + h * (D / 2);
+        for (int which = 0; which < 2; ++which) {
+          uint4* orow = reinterpret_cast<uint4*>(
+              reinterpret_cast<uint16_t*>(which ? P.dk : P.dv) + rbase);
+          for (int v = 0; v < D / 16; ++v) orow[v] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int D, bool F16>
+cudaError_t launch_dkdv_d(const TcBwdLaunch& L, cudaStream_t stream, char* err, int errlen) {
+  CUtensorMap mk, mv, mq, mdo;
+  if (!encode_grid_map(&mk, L.k, L.f16, L.D, L.g.L, L.BH, L.N, L.t.qb) ||
+      !encode_grid_map(&mv, L.v, L.f16, L.D, L.g.L, L.BH, L.N, L.t.qb) ||
+      !encode_grid_map(&mq, L.q, L.f16, L.D, L.g.L, L.BH, L.N, L.kb) ||
+      !encode_grid_map(&mdo, L.dout, L.f16, L.D, L.g.L, L.BH, L.N, L.kb)) {
+    snprintf(err, errlen, "cuTensorMapEncodeTiled failed (pointer alignment or shape)");
+    return cudaErrorInvalidValue;
+  }
+  const size_t smem = bk_smem_bytes<D>();
+  static int attr_done[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, tc_bwd_dkdv_kernel<D, F16>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs * BT_THREADS < BT_REGS_NEEDED) {
+      snprintf(err, errlen, "kernel compiled with %d registers/thread; the register split needs %d",
+               fa.numRegs, (BT_REGS_NEEDED + BT_THREADS - 1) / BT_THREADS);
+      return cudaErrorInvalidConfiguration;
+    }
+    e = cudaFuncSetAttribute(tc_bwd_dkdv_kernel<D, F16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = 1;
+  }
+  const long long grid = (long long)L.t.nblocks * L.BH;
+  if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  tc_bwd_dkdv_kernel<D, F16><<<(unsigned)grid, BT_THREADS, smem, stream>>>(mk, mv, mq, mdo, L);
+  return cudaGetLastError();
+}
+
 template <int D, bool F16>
 cudaError_t launch_dq_d(const TcBwdLaunch& L, cudaStream_t stream, char* err, int errlen) {
   CUtensorMap mq, mdo, mk, mv;
@@ -404,6 +870,29 @@ cudaError_t launch_dq_d(const TcBwdLaunch& L, cudaStream_t stream, char* err, in
 }
 
 }  // namespace
+
+cudaError_t launch_tc_bwd_dkdv(const TcBwdLaunch& L0, cudaStream_t stream, char* err, int errlen) {
+  TcBwdLaunch L = L0;
+  for (int d = 0; d < 3; ++d) {
+    if (L.t.qb[d] > 256 || L.kb[d] > 256) return cudaErrorNotSupported;
+    if (L.kb[d] & (L.kb[d] - 1)) return cudaErrorNotSupported;
+    int lg = 0;
+    while ((1 << lg) < L.kb[d]) ++lg;
+    L.kb_log2[d] = lg;
+  }
+  if (L.t.qb[0] * L.t.qb[1] * L.t.qb[2] != BT_M || L.kb[0] * L.kb[1] * L.kb[2] != BT_N)
+    return cudaErrorNotSupported;
+  switch (L.D) {
+    case 64:
+      return L.f16 ? launch_dkdv_d<64, true>(L, stream, err, errlen)
+                   : launch_dkdv_d<64, false>(L, stream, err, errlen);
+    case 128:
+      return L.f16 ? launch_dkdv_d<128, true>(L, stream, err, errlen)
+                   : launch_dkdv_d<128, false>(L, stream, err, errlen);
+    default:
+      return cudaErrorNotSupported;
+  }
+}
 
 cudaError_t launch_tc_bwd_dq(const TcBwdLaunch& L0, cudaStream_t stream, char* err, int errlen) {
   TcBwdLaunch L = L0;

@@ -68,7 +68,7 @@ struct TcBwdLaunch {
   const void *q, *k, *v, *dout;
   const float* lse;
   const float* delta;    // <dout_i, out_i>, written by the row-delta kernel first
-  void* dq;
+  void *dq, *dk, *dv;
   int* status;           // device status word
   long long timeout_ns;  // bound on every in-kernel wait
 };
@@ -84,6 +84,7 @@ cudaError_t launch_bwd_simt(const BwdLaunch& L, cudaStream_t stream);
 cudaError_t launch_bwd_simt_delta(const BwdLaunch& L, cudaStream_t stream);
 cudaError_t launch_bwd_simt_dkdv(const BwdLaunch& L, cudaStream_t stream);
 cudaError_t launch_tc_bwd_dq(const TcBwdLaunch& L, cudaStream_t stream, char* err, int errlen);
+cudaError_t launch_tc_bwd_dkdv(const TcBwdLaunch& L, cudaStream_t stream, char* err, int errlen);
 
 // y[i] = the tensor-core kernel's FMA-pipe 2^x applied to x[i] (self-test).
 cudaError_t launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t stream);
