@@ -72,6 +72,12 @@ class OracleLib:
             ctypes.c_longlong, ctypes.c_int, i32p, i32p, i32p, i32p, ctypes.c_int, ctypes.c_double,
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
         lib.na_oracle_backward.restype = ctypes.c_int
+        lib.na_oracle_backward_sampled.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+            ctypes.c_longlong, ctypes.c_longlong, ctypes.c_int, i32p, i32p, i32p, i32p,
+            ctypes.c_int, ctypes.c_double, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p,
+            ctypes.c_longlong, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        lib.na_oracle_backward_sampled.restype = ctypes.c_int
         lib.na_oracle_f16_value.argtypes = [ctypes.c_uint16]
         lib.na_oracle_f16_value.restype = ctypes.c_double
         self.lib = lib
@@ -193,6 +199,37 @@ class OracleLib:
             raise RuntimeError(f"na_oracle_backward failed with code {rc}")
         return tuple(outs)
 
+    def backward_sampled(self, q, k, v, dout, grid, window, stride, bh: int, qrows, krows, *,
+                         dtype: str, scale: float = 0.0, threads: int | None = None, mode=None):
+        """Exact gradients of one (batch, head) slice ``bh`` (flat index) on
+        sampled rows: (dq [len(qrows), d], dk [len(krows), d], dv [len(krows), d])
+        in fp64; qrows / krows are token indices within the slice."""
+        grid, window, stride = _geom(grid, window, stride)
+        codes = {"f32": (np.float32, 0), "bf16": (np.uint16, 1), "f16": (np.float16, 2)}
+        want, code = codes[dtype]
+        arrs = [np.ascontiguousarray(a) for a in (q, k, v, dout)]
+        for a in arrs:
+            if a.dtype != want or a.shape != arrs[0].shape:
+                raise TypeError(f"oracle expects four {want} arrays of one shape")
+        shape = arrs[0].shape
+        nd = len(grid)
+        BH = shape[0] * shape[1]
+        d = shape[-1]
+        qr = np.ascontiguousarray(np.asarray(qrows, dtype=np.int64))
+        kr = np.ascontiguousarray(np.asarray(krows, dtype=np.int64))
+        dq = np.empty((qr.size, d), dtype=np.float64)
+        dk = np.empty((kr.size, d), dtype=np.float64)
+        dv = np.empty((kr.size, d), dtype=np.float64)
+        rc = self.lib.na_oracle_backward_sampled(
+            arrs[0].ctypes.data, arrs[1].ctypes.data, arrs[2].ctypes.data, arrs[3].ctypes.data,
+            code, BH, int(bh), nd, self._ivec(grid), self._ivec(window), self._ivec(stride),
+            self._ivec(_modes(mode, nd)), d, float(scale), qr.ctypes.data, qr.size,
+            kr.ctypes.data, kr.size, dq.ctypes.data, dk.ctypes.data, dv.ctypes.data,
+            int(threads or os.cpu_count() or 1))
+        if rc:
+            raise RuntimeError(f"na_oracle_backward_sampled failed with code {rc}")
+        return dq, dk, dv
+
     def f16_value(self, bits: int) -> float:
         """The oracle's decoding of one binary16 bit pattern."""
         return float(self.lib.na_oracle_f16_value(int(bits)))
@@ -262,6 +299,10 @@ def forward(q, k, v, grid, window, stride, **kw):
 
 def backward(q, k, v, dout, grid, window, stride, **kw):
     return load().backward(q, k, v, dout, grid, window, stride, **kw)
+
+
+def backward_sampled(q, k, v, dout, grid, window, stride, bh, qrows, krows, **kw):
+    return load().backward_sampled(q, k, v, dout, grid, window, stride, bh, qrows, krows, **kw)
 
 
 def block_counts(grid, window, stride, block, mode=None):

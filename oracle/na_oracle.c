@@ -447,6 +447,177 @@ int na_oracle_backward(const void* q, const void* k, const void* v, const void* 
     return 0;
 }
 
+/*
+ * Gradients on sampled rows of one (batch, head) slice bh, for parity checks
+ * at sizes where the full backward is too slow: first lse_t and
+ * D_t = <dO_t, out_t> for every query t of the slice (threads split the
+ * queries), then dq for the query rows `qrows` and dk, dv for the key rows
+ * `krows` (token indices within the slice), each summed over the queries
+ * whose window holds the key.  Outputs [nq, d] and [nk, d] fp64.  Same
+ * definitions as na_oracle_backward, which it equals on every row.
+ */
+typedef struct {
+    const void *q, *k, *v, *dout;
+    int dtype, ndim, d;
+    const int *L, *w, *s, *mode;
+    long long N, W, bh;
+    double scale;
+    long long t_begin, t_end;
+    double *lse, *delta;
+    int status;
+} stat_job;
+
+static void* stat_worker(void* arg) {
+    stat_job* J = (stat_job*)arg;
+    const int d = J->d;
+    const size_t hoff = (size_t)J->bh * (size_t)J->N * (size_t)d;
+    double* z = (double*)malloc(sizeof(double) * (size_t)J->W);
+    long long* idx = (long long*)malloc(sizeof(long long) * (size_t)J->W);
+    uint8_t* mask = (uint8_t*)malloc((size_t)J->N);
+    if (!z || !idx || !mask) { J->status = -2; goto done; }
+    for (long long t = J->t_begin; t < J->t_end; ++t) {
+        na_oracle_mask_row(J->ndim, J->L, J->w, J->s, J->mode, t, mask);
+        const size_t qoff = hoff + (size_t)t * (size_t)d;
+        long long cnt = 0;
+        for (long long j = 0; j < J->N; ++j) {
+            if (!mask[j]) continue;
+            if (cnt >= J->W) { J->status = -3; goto done; }
+            const size_t koff = hoff + (size_t)j * (size_t)d;
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c)
+                dot += load_in(J->q, J->dtype, qoff + c) * load_in(J->k, J->dtype, koff + (size_t)c);
+            z[cnt] = dot * J->scale;
+            idx[cnt++] = j;
+        }
+        double m = -INFINITY, l = 0.0;
+        for (long long e = 0; e < cnt; ++e) if (z[e] > m) m = z[e];
+        for (long long e = 0; e < cnt; ++e) l += exp(z[e] - m);
+        const double lse = m + log(l);
+        double D = 0.0;
+        for (long long e = 0; e < cnt; ++e) {
+            const size_t voff = hoff + (size_t)idx[e] * (size_t)d;
+            double dv = 0.0;
+            for (int c = 0; c < d; ++c)
+                dv += load_in(J->dout, J->dtype, qoff + c) * load_in(J->v, J->dtype, voff + c);
+            D += exp(z[e] - lse) * dv;
+        }
+        J->lse[t] = lse;
+        J->delta[t] = D;
+    }
+done:
+    free(z); free(idx); free(mask);
+    return NULL;
+}
+
+int na_oracle_backward_sampled(const void* q, const void* k, const void* v, const void* dout,
+                               int in_dtype, long long BH, long long bh, int ndim, const int* L,
+                               const int* w, const int* s, const int* mode, int d, double scale,
+                               const long long* qrows, long long nq, const long long* krows,
+                               long long nk, double* dq, double* dk, double* dv, int nthreads) {
+    long long N;
+    if (!q || !k || !v || !dout || BH < 1 || bh < 0 || bh >= BH || d < 1) return -1;
+    if ((nq && (!qrows || !dq)) || (nk && (!krows || !dk || !dv))) return -1;
+    if (in_dtype != IN_F32 && in_dtype != IN_BF16 && in_dtype != IN_F16) return -1;
+    if (check_geometry(ndim, L, w, s, mode, &N)) return -1;
+    long long W = 1;
+    for (int a = 0; a < ndim; ++a) W *= w[a];
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+    double* lse = (double*)malloc(sizeof(double) * (size_t)N);
+    double* delta = (double*)malloc(sizeof(double) * (size_t)N);
+    if (!lse || !delta) { free(lse); free(delta); return -2; }
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    stat_job jobs[256];
+    pthread_t th[256];
+    const long long per = (N + nthreads - 1) / nthreads;
+    for (int t = 0; t < nthreads; ++t) {
+        stat_job* J = &jobs[t];
+        J->q = q; J->k = k; J->v = v; J->dout = dout;
+        J->dtype = in_dtype; J->ndim = ndim; J->d = d;
+        J->L = L; J->w = w; J->s = s; J->mode = mode;
+        J->N = N; J->W = W; J->bh = bh; J->scale = scale;
+        J->t_begin = per * t < N ? per * t : N;
+        J->t_end = per * (t + 1) < N ? per * (t + 1) : N;
+        J->lse = lse; J->delta = delta;
+        J->status = 0;
+    }
+    for (int t = 1; t < nthreads; ++t)
+        if (pthread_create(&th[t], NULL, stat_worker, &jobs[t]) != 0) {
+            stat_worker(&jobs[t]);
+            th[t] = 0;
+        }
+    stat_worker(&jobs[0]);
+    for (int t = 1; t < nthreads; ++t)
+        if (th[t]) pthread_join(th[t], NULL);
+    int rc = 0;
+    for (int t = 0; t < nthreads; ++t)
+        if (jobs[t].status) rc = jobs[t].status;
+    const size_t hoff = (size_t)bh * (size_t)N * (size_t)d;
+    uint8_t* mask = (uint8_t*)malloc((size_t)N);
+    if (!mask) rc = -2;
+    /* dq of the sampled query rows */
+    for (long long r = 0; !rc && r < nq; ++r) {
+        const long long t = qrows[r];
+        if (t < 0 || t >= N) { rc = -1; break; }
+        na_oracle_mask_row(ndim, L, w, s, mode, t, mask);
+        const size_t qoff = hoff + (size_t)t * (size_t)d;
+        for (int c = 0; c < d; ++c) dq[(size_t)r * d + c] = 0.0;
+        for (long long j = 0; j < N; ++j) {
+            if (!mask[j]) continue;
+            const size_t koff = hoff + (size_t)j * (size_t)d;
+            double zq = 0.0, dp = 0.0;
+            for (int c = 0; c < d; ++c) {
+                zq += load_in(q, in_dtype, qoff + c) * load_in(k, in_dtype, koff + c);
+                dp += load_in(dout, in_dtype, qoff + c) * load_in(v, in_dtype, koff + c);
+            }
+            const double p = exp(scale * zq - lse[t]);
+            const double dz = p * (dp - delta[t]);
+            for (int c = 0; c < d; ++c)
+                dq[(size_t)r * d + c] += scale * dz * load_in(k, in_dtype, koff + c);
+        }
+    }
+    /* dk, dv of the sampled key rows: over every query whose window holds the key */
+    for (long long r = 0; !rc && r < nk; ++r) {
+        const long long j = krows[r];
+        if (j < 0 || j >= N) { rc = -1; break; }
+        const size_t koff = hoff + (size_t)j * (size_t)d;
+        for (int c = 0; c < d; ++c) { dk[(size_t)r * d + c] = 0.0; dv[(size_t)r * d + c] = 0.0; }
+        int kj[NA_ORACLE_MAXDIM];
+        unflatten(j, ndim, L, kj);
+        int qi[NA_ORACLE_MAXDIM];
+        for (int a = 0; a < ndim; ++a) qi[a] = 0;
+        for (long long t = 0; t < N; ++t) {
+            int in = 1;
+            for (int a = 0; a < ndim && in; ++a) {
+                int lo, hi;
+                const int ma = mode ? mode[a] : 0;
+                na_oracle_window(L[a], w[a], s[a], ma, qi[a], &lo, &hi);
+                if (kj[a] < lo || kj[a] >= hi) in = 0;
+            }
+            if (in) {
+                const size_t qoff = hoff + (size_t)t * (size_t)d;
+                double zq = 0.0, dp = 0.0;
+                for (int c = 0; c < d; ++c) {
+                    zq += load_in(q, in_dtype, qoff + c) * load_in(k, in_dtype, koff + c);
+                    dp += load_in(dout, in_dtype, qoff + c) * load_in(v, in_dtype, koff + c);
+                }
+                const double p = exp(scale * zq - lse[t]);
+                const double dz = p * (dp - delta[t]);
+                for (int c = 0; c < d; ++c) {
+                    dk[(size_t)r * d + c] += scale * dz * load_in(q, in_dtype, qoff + c);
+                    dv[(size_t)r * d + c] += p * load_in(dout, in_dtype, qoff + c);
+                }
+            }
+            for (int a = ndim - 1; a >= 0; --a) { /* advance the row-major query counter */
+                if (++qi[a] < L[a]) break;
+                qi[a] = 0;
+            }
+        }
+    }
+    free(mask); free(lse); free(delta);
+    return rc;
+}
+
 /* --------------------------------------------------------- block counts -- */
 
 /*

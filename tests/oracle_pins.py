@@ -555,6 +555,24 @@ def pin_backward_invariants(lib):
     np.testing.assert_allclose(dk3, 0.0, atol=1e-14, rtol=0)
 
 
+def pin_backward_sampled_rows(lib):
+    """The sampled-rows backward equals the full backward on every row it is
+    asked for (3-D, strided, mixed modes, two heads)."""
+    grid, window, stride, modes, d = [3, 5, 6], [2, 3, 4], [1, 1, 2], ["causal", "clamped",
+                                                                       "truncated"], 4
+    shape = (1, 2, *grid, d)
+    q, k, v, do = (_randn(180 + t, shape) for t in range(4))
+    dq, dk, dv = lib.backward(q, k, v, do, grid, window, stride, dtype="f32", mode=modes)
+    N = 90
+    rows = np.array([0, 7, 44, 89], dtype=np.int64)
+    for bh in (0, 1):
+        sq, sk, sv = lib.backward_sampled(q, k, v, do, grid, window, stride, bh, rows, rows[::-1],
+                                          dtype="f32", mode=modes)
+        np.testing.assert_allclose(sq, dq[0, bh].reshape(N, d)[rows], atol=1e-12, rtol=0)
+        np.testing.assert_allclose(sk, dk[0, bh].reshape(N, d)[rows[::-1]], atol=1e-12, rtol=0)
+        np.testing.assert_allclose(sv, dv[0, bh].reshape(N, d)[rows[::-1]], atol=1e-12, rtol=0)
+
+
 def _read_golden(name):
     rows = []
     with open(os.path.join(GOLDEN, name)) as f:
@@ -573,7 +591,7 @@ ALL_PINS = [
     pin_block_counts_closed_forms, pin_ena_density_golden, pin_truncated_eq5, pin_causal_eq5,
     pin_modes_strided, pin_mode_mask_bruteforce, pin_causal_full_sdpa, pin_mode_uniform_queries,
     pin_sa_empty_blocks_golden, pin_f16_decoding, pin_backward_finite_differences,
-    pin_backward_full_attention_autograd, pin_backward_invariants,
+    pin_backward_full_attention_autograd, pin_backward_invariants, pin_backward_sampled_rows,
 ]
 
 # The golden-file pins take a few seconds each; mutant runs use the fast ones.

@@ -113,3 +113,47 @@ def test_backward_tensor_core_selector_needs_16_bit():
     with pytest.raises(na.NaError) as e:
         na.backward(q, q, q, q, lse, q, c["window"], options=na.make_options(kernel=na.NA_KERNEL_TC))
     assert e.value.status == na.NA_ERR_UNSUPPORTED
+
+
+def _sample_keys(grid, n, seed):
+    """Corner and edge tokens of the grid plus uniform draws (token indices)."""
+    import itertools
+    N = int(np.prod(grid))
+    extremes = [sorted({0, 1, g // 2, g - 2, g - 1} & set(range(g))) for g in grid]
+    picks = {int(np.ravel_multi_index(c, grid)) for c in itertools.product(*extremes)}
+    rng = np.random.default_rng(seed)
+    while len(picks) < n:
+        picks.add(int(rng.integers(0, N)))
+    return np.array(sorted(picks), dtype=np.int64)
+
+
+@pytest.mark.parametrize("cfg", ["sta3d_full", "local3d_full"])
+def test_backward_full_size_sampled(cfg):
+    """The full-size workloads in the launch configuration the benchmark times
+    (3-D sliding tile: 24 heads, 30x48x80, d 128; 3-D local: 32 heads,
+    16x32x32, d 64), gradients checked on sampled query and key rows of the
+    first and last (batch, head) slice against the oracle's sampled backward."""
+    if cfg == "sta3d_full":
+        c = _case((30, 48, 80), (18, 24, 40), (6, 8, 8), 128, heads=24, tile=(6, 8, 8))
+        nrows = 48
+    else:
+        c = _case((16, 32, 32), (12, 20, 20), (4, 4, 4), 64, B=2, heads=16, tile=(4, 4, 4))
+        nrows = 96
+    seed = 9100 if cfg == "sta3d_full" else 9200
+    shape = (c["B"], c["heads"], *c["grid"], c["d"])
+    q, k, v = seeded_inputs.qkv(seed, c["B"], c["heads"], c["grid"], c["d"], c["dtype"])
+    do = seeded_inputs.normal_bf16_bits(seed + 7, shape)
+    qd, kd, vd, dod = (to_device(a, c["dtype"]) for a in (q, k, v, do))
+    out, lse = na.forward(qd, kd, vd, c["window"], c["stride"], c["tile"])
+    dq, dk, dv = na.backward(qd, kd, vd, out, lse, dod, c["window"], c["stride"], c["tile"])
+    na.na_sync_status()
+    BH = c["B"] * c["heads"]
+    N = int(np.prod(c["grid"]))
+    rows = _sample_keys(c["grid"], nrows, seed)
+    for bh in (0, BH - 1):
+        rq, rk, rv = oracle.backward_sampled(q, k, v, do, c["grid"], c["window"], c["stride"], bh,
+                                             rows, rows, dtype="bf16")
+        b, h = divmod(bh, c["heads"])
+        got = [t[b, h].reshape(N, c["d"])[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+               .astype(np.float64) for t in (dq, dk, dv)]
+        _assert_close(c, got, (rq, rk, rv), f"{cfg} bh={bh}")
