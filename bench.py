@@ -54,9 +54,15 @@ WORKLOADS = {
     5: dict(workload="3D local attention at ~30% density fwd", B=2, heads=16, head_dim=64,
             grid=[16, 32, 32], tile=[4, 4, 4], window=[12, 20, 20], stride=[4, 4, 4],
             dtype="bf16"),
+    # 1-D causal local attention over a long sequence: each token sees itself
+    # and the k = 4 before it (w = k + 1), 16 heads of 64, 32K tokens.
+    6: dict(workload="1D causal local attention, long sequence fwd", B=1, heads=16, head_dim=64,
+            grid=[32768], tile=None, window=[5], stride=[1], window_mode=["causal"],
+            dtype="bf16"),
 }
 SEED = 4000
 FALLBACK_PEAK_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["neighborhood_attention_b200/csrc/na_fwd_sm100.cu",
                   "neighborhood_attention_b200/csrc/na_ptx.cuh",
                   "neighborhood_attention_b200/csrc/na_sched.cuh"]
@@ -67,11 +73,29 @@ DENSE_STEPS = 3
 FLUSH_BYTES = 256 * 2**20
 
 
-def flops_per_step(w=None):
+def flops_per_step(useful_pairs, w=None):
+    """4 d FLOPs per attended (query, key) pair of one head, times the heads.
+    useful_pairs = N * prod(window) for clamped windows (every query sees a
+    full window); cut (truncated / causal) windows see fewer keys at the
+    borders, so the count comes from the scheduler's per-dimension sums."""
     w = WORKLOAD if w is None else w
-    N = int(np.prod(w["grid"]))
-    W = int(np.prod(w["window"]))
-    return 4.0 * w["head_dim"] * w["B"] * w["heads"] * N * W
+    return 4.0 * w["head_dim"] * w["B"] * w["heads"] * useful_pairs
+
+
+def min_hbm_bytes(w=None):
+    """Algorithmic HBM bytes of one forward: q, k, v read and out written once
+    (d elements each per token), lse written once (4 bytes per token)."""
+    w = WORKLOAD if w is None else w
+    tokens = w["B"] * w["heads"] * int(np.prod(w["grid"]))
+    elt = 4 if w["dtype"] == "f32" else 2
+    return tokens * (4 * w["head_dim"] * elt + 4)
+
+
+def options_for(na, w=None):
+    w = WORKLOAD if w is None else w
+    if not w.get("window_mode"):
+        return None
+    return na.make_options(window_mode=w["window_mode"], ndim=len(w["grid"]))
 
 
 def kernel_hash():
@@ -107,6 +131,14 @@ def read_peaks():
         return float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 0) or 0), "measured"
     except (OSError, KeyError, ValueError):
         return FALLBACK_PEAK_TFLOPS, 0.0, "fallback"
+
+
+def read_hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
 
 
 class ClockSampler:
@@ -190,10 +222,32 @@ def time_oracle(qkv, n_rows, threads):
     rows = oracle_sample_rows(n_rows)
     t0 = time.perf_counter()
     oracle.forward(*qkv, w["grid"], w["window"], w["stride"], dtype=w["dtype"], rows=rows,
-                   threads=threads)
+                   threads=threads, mode=w.get("window_mode"))
     dt = time.perf_counter() - t0
-    flops = 4.0 * w["head_dim"] * int(np.prod(w["window"])) * n_rows
+    flops = 4.0 * w["head_dim"] * sampled_pairs(rows)
     return flops / dt / 1e12, dt
+
+
+def sampled_pairs(rows):
+    """Attended (query, key) pairs of the sampled rows, from the oracle's own
+    window rule (the product over dimensions of each window's length)."""
+    import oracle
+    w = WORKLOAD
+    grid = w["grid"]
+    N = int(np.prod(grid))
+    modes = w.get("window_mode") or ["clamped"] * len(grid)
+    coords = np.unravel_index(np.asarray(rows) % N, grid)
+    lens = []
+    for d, L in enumerate(grid):
+        cache = {}
+        per = []
+        for i in coords[d].tolist():
+            if i not in cache:
+                lo, hi = oracle.window(L, w["window"][d], w["stride"][d], modes[d], i)
+                cache[i] = hi - lo
+            per.append(cache[i])
+        lens.append(np.array(per, dtype=np.int64))
+    return int(np.sum(np.prod(np.stack(lens), axis=0)))
 
 
 def cpu_baseline(qkv, target_s=15.0):
@@ -225,7 +279,7 @@ def run_reference(args, rank, world):
         v, dt = time_oracle(qkv, n, threads)
         vals.append(v)
         tot += dt
-    flops = 4.0 * WORKLOAD["head_dim"] * int(np.prod(WORKLOAD["window"])) * n * args.steps
+    flops = 4.0 * WORKLOAD["head_dim"] * sampled_pairs(oracle_sample_rows(n)) * args.steps
     value = flops / tot / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
@@ -289,13 +343,15 @@ def run_backward(args, rank, world, local_rank):
     g = torch.Generator(device=dev).manual_seed(SEED + 11)
     dout = torch.randn(q.shape, generator=g, device=dev, dtype=torch.float32).to(q.dtype)
     stream = torch.cuda.current_stream(dev)
-    out, lse = na.forward(q, k, v, w["window"], w["stride"], w["tile"], stream=stream)
+    opts = options_for(na)
+    out, lse = na.forward(q, k, v, w["window"], w["stride"], w["tile"], options=opts,
+                          stream=stream)
     dq, dk, dv = (torch.empty_like(q) for _ in range(3))
     delta = torch.empty(lse.shape, dtype=torch.float32, device=dev)
 
     def step():
         na.na_backward(q, k, v, out, dout, lse, dq, dk, dv, delta, w["window"], w["stride"],
-                       w["tile"], stream=stream)
+                       w["tile"], options=opts, stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -321,7 +377,8 @@ def run_backward(args, rank, world, local_rank):
     na.na_sync_status(stream)
     (total_ms,) = max_over_ranks([e0.elapsed_time(e1)], world, dev)
     plan = na.na_plan(w["grid"], w["window"], w["stride"], w["tile"], w["head_dim"],
-                      {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32}[w["dtype"]])
+                      {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32}[w["dtype"]],
+                      options=opts)
     flops = 10.0 * w["head_dim"] * w["B"] * w["heads"] * plan["useful_pairs"]
     value = flops * args.steps * world / (total_ms / 1e3) / 1e12
     tensor = w["dtype"] in ("bf16", "f16") and w["head_dim"] in (64, 128)
@@ -373,9 +430,11 @@ def run_ours(args, rank, world, local_rank):
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
     stream = torch.cuda.current_stream(dev)
+    opts = options_for(na)
 
     def step():
-        na.na_forward(q, k, v, out, lse, w["window"], w["stride"], w["tile"], stream=stream)
+        na.na_forward_ex(q, k, v, out, lse, w["window"], w["stride"], w["tile"], options=opts,
+                         stream=stream)
 
     # Inputs that do not clearly exceed L2 would stay cached from one step to
     # the next: then L2 is flushed (a 256 MB write) before every timed step and
@@ -459,8 +518,8 @@ def run_ours(args, rank, world, local_rank):
                 stream.wait_event(h2d_done[i])
                 if i >= 2:
                     stream.wait_event(d2h_done[i - 2])      # outputs of buffer i%2 copied out
-                na.na_forward(bq, bk, bv, bo, bl, w["window"], w["stride"], w["tile"],
-                              stream=stream)
+                na.na_forward_ex(bq, bk, bv, bo, bl, w["window"], w["stride"], w["tile"],
+                                 options=opts, stream=stream)
                 comp_done[i].record(stream)
                 with torch.cuda.stream(s_out):
                     s_out.wait_event(comp_done[i])
@@ -511,6 +570,7 @@ def run_ours(args, rank, world, local_rank):
         nd = len(w["grid"])
 
         def dense_step():
+            # full (non-causal) attention, as the scheduler's bound counts it
             na.na_forward(q, k, v, out, lse, w["grid"], [1] * nd, None, stream=stream)
 
         dense_step()
@@ -528,13 +588,35 @@ def run_ours(args, rank, world, local_rank):
     total_ms, e2e_ms, per_launch_ms, dense_ms = max_over_ranks(
         [total_ms, e2e_ms, per_launch_ms, dense_ms], world, dev)
 
-    flops = flops_per_step()
+    plan = na.na_plan(w["grid"], w["window"], w["stride"], w["tile"], w["head_dim"],
+                      {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32}[w["dtype"]],
+                      options=opts)
+    flops = flops_per_step(plan["useful_pairs"])
     value = whole_job_tflops(flops, args.steps, world, total_ms)
     e2e_value = whole_job_tflops(flops, args.steps, world, e2e_ms)
     peak, peak_sustained, peak_kind = read_peaks()
     achieved = flops / (per_launch_ms / 1e3) / 1e12
-    plan = na.na_plan(w["grid"], w["window"], w["stride"], w["tile"], w["head_dim"],
-                      {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32}[w["dtype"]])
+    # The bound: tensor cores when the workload's algorithmic intensity (FLOPs
+    # per minimum HBM byte) is above the measured ridge, else HBM bandwidth.
+    hbm_peak, hbm_kind = read_hbm_peak()
+    min_bytes = min_hbm_bytes()
+    hbm_bound = flops / min_bytes < peak * 1e12 / (hbm_peak * 1e9)
+    if hbm_bound:
+        gbs = min_bytes / (per_launch_ms / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": gbs / hbm_peak, "traffic": None,
+                    "algorithmic_bytes": min_bytes,
+                    "peak_kind": (f"{hbm_kind} copy bandwidth (MEASURED_PEAKS.json)"
+                                  if hbm_kind == "measured" else "fallback"),
+                    "intensity_flop_per_byte": flops / min_bytes}
+    else:
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak,
+                    "traffic": read_traffic() if TRAFFIC_APPLIES else None,
+                    "peak_kind": (f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)"
+                                  + (" x 1: f16 and bf16 share the nominal dense rate"
+                                     if w["dtype"] == "f16" else "")
+                                  if peak_kind == "measured" else "fallback")}
     if rank != 0:
         return 0
     base = cpu_baseline(qkv_host) if world == 1 and not args.no_cpu_baseline else None
@@ -550,13 +632,7 @@ def run_ours(args, rank, world, local_rank):
                        qblock=plan["qblock"], kvchunk=plan["kvchunk"],
                        parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
         "pct_of_peak": 100.0 * value / world / peak,
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak,
-                     "traffic": read_traffic() if TRAFFIC_APPLIES else None,
-                     "peak_kind": (f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)"
-                                   + (" x 1: f16 and bf16 share the nominal dense rate"
-                                      if w["dtype"] == "f16" else "")
-                                   if peak_kind == "measured" else "fallback")},
+        "roofline": roofline,
         "cpu_baseline": base,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
@@ -592,7 +668,7 @@ def main():
                     help="skip timing dense attention for the measured speedup")
     ap.add_argument("--config", type=int, default=4, choices=sorted(WORKLOADS),
                     help="workload: 4 (default) is the 3-D sliding tile one the metric is "
-                         "quoted on; 1, 2, 3, 5 are the other parity workloads")
+                         "quoted on; 1, 2, 3, 5, 6 are the other parity workloads")
     ap.add_argument("--dtype", choices=["bf16", "f16"], default=None,
                     help="input type of a 16-bit workload (default: the workload's own, bf16)")
     ap.add_argument("--heads", type=int, default=0,

@@ -18,9 +18,10 @@ TOL = {
     "f16": dict(out_max=4e-3, out_mean=4e-4, lse_max=1e-3),
 }
 
-# The five workloads: 2-D neighborhood attention (fp32 and bf16), 2-D strided
-# (generalized) neighborhood attention, 3-D sliding tile attention, and a 3-D
-# local window covering ~30% of the sequence.
+# The workloads: 2-D neighborhood attention (fp32 and bf16), 2-D strided
+# (generalized) neighborhood attention, 3-D sliding tile attention, a 3-D
+# local window covering ~30% of the sequence, and 1-D causal local attention
+# over a long sequence.
 CONFIGS = {
     1: dict(B=1, heads=2, grid=(16, 16), window=(5, 5), stride=(1, 1), tile=None, d=32, dtype="f32"),
     2: dict(B=4, heads=4, grid=(64, 64), window=(13, 13), stride=(1, 1), tile=None, d=64, dtype="bf16"),
@@ -30,6 +31,11 @@ CONFIGS = {
             d=128, dtype="bf16"),
     5: dict(B=2, heads=16, grid=(16, 32, 32), window=(12, 20, 20), stride=(4, 4, 4), tile=(4, 4, 4),
             d=64, dtype="bf16"),
+    # 1-D causal local attention over a long sequence ("pi-Attention" section 3.2
+    # eq. (5), causal case, k = 4 so w = k + 1 = 5 keys with the query itself):
+    # the Medium model's 16 heads of 64 at the 32K context of its longest runs.
+    6: dict(B=1, heads=16, grid=(32768,), window=(5,), stride=(1,), tile=None, d=64, dtype="bf16",
+            mode=["causal"]),
 }
 
 

@@ -67,7 +67,7 @@ def test_config2_full_parity_both_kernels():
         assert_within(c, compare(c, qkv, o, l), f"config2/{kernel}")
 
 
-@pytest.mark.parametrize("cfg,n_rows", [(3, 3000), (4, 1200), (5, 4000)])
+@pytest.mark.parametrize("cfg,n_rows", [(3, 3000), (4, 1200), (5, 4000), (6, 3000)])
 def test_full_size_sampled_parity(cfg, n_rows):
     c = CONFIGS[cfg]
     qkv = host_inputs(c, seed_for(cfg))
