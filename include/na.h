@@ -72,10 +72,21 @@ typedef enum {
 } na_window_mode;
 
 typedef enum {
-  NA_KERNEL_AUTO = 0,  /* tensor-core kernel where it applies, else the CUDA-core kernel */
-  NA_KERNEL_SIMT = 1,  /* CUDA-core kernel (fp32, bf16 and f16, head_dim 32/64/128) */
-  NA_KERNEL_TC = 2     /* tcgen05 tensor-core kernel (bf16 or f16, head_dim 64/128) */
+  NA_KERNEL_AUTO = 0,   /* the window-gather kernel for windows of at most
+                           NA_GATHER_MAX_KEYS keys (product of the window sizes),
+                           else the tensor-core kernel where it applies, else the
+                           CUDA-core tile kernel */
+  NA_KERNEL_SIMT = 1,   /* CUDA-core tile kernel (fp32, bf16 and f16, head_dim 32/64/128) */
+  NA_KERNEL_TC = 2,     /* tcgen05 tensor-core kernel (bf16 or f16, head_dim 64/128) */
+  NA_KERNEL_GATHER = 3  /* CUDA-core window-gather kernel (fp32, bf16 and f16, head_dim
+                           32/64/128): each query reads only its own window's keys, for
+                           narrow windows where the pass is bound by HBM traffic.
+                           Forward only. */
 } na_kernel;
+
+/* Largest window (keys per query, the product of the window sizes) that
+ * NA_KERNEL_AUTO sends to the window-gather kernel. */
+#define NA_GATHER_MAX_KEYS 32
 
 /*
  * na_forward -- enqueue one forward pass.
@@ -148,7 +159,8 @@ na_status na_forward_ex(const void* q, const void* k, const void* v, void* out, 
  * Kernels: D_i and dk / dv on the CUDA cores (fp32 arithmetic); dq on the
  * tensor cores (tcgen05, fp32 accumulation) for bf16 / f16 with head_dim 64 or
  * 128 unless opt->kernel = NA_KERNEL_SIMT, else on the CUDA cores.
- * opt->kernel = NA_KERNEL_TC for other inputs is NA_ERR_UNSUPPORTED.  A bounded
+ * opt->kernel = NA_KERNEL_TC for other inputs, and NA_KERNEL_GATHER (a
+ * forward-only kernel), are NA_ERR_UNSUPPORTED.  A bounded
  * in-kernel wait that expires is reported by na_sync_status.
  */
 na_status na_backward(const void* q, const void* k, const void* v, const void* out,
@@ -178,11 +190,14 @@ const char* na_last_error(void);
  */
 typedef struct {
   int kernel;               /* na_kernel actually chosen */
-  int qblock[3];            /* query block shape (3-d padded, outermost first) */
-  int kvchunk[3];           /* key chunk shape */
+  int qblock[3];            /* query block shape (3-d padded, outermost first); 1 x 1 x 1
+                               for the window-gather kernel (each query on its own) */
+  int kvchunk[3];           /* key chunk shape; 1 x 1 x 1 for the window-gather kernel
+                               (it reads exactly the window's keys) */
   int tile[3];              /* query tile shape used to order blocks */
   long long query_blocks;   /* blocks per head */
-  long long ctas;           /* CTAs per head */
+  long long ctas;           /* CTAs per head (window-gather: head's rows / rows per CTA,
+                               rounded up; its CTAs may straddle heads) */
   long long chunks_loaded;  /* key chunks staged per head */
   long long units_full;     /* (block, chunk) products with no mask */
   long long units_partial;  /* (block, chunk) products with an element mask */
@@ -255,7 +270,8 @@ na_status na_selftest_exp2(const float* x, float* y, int n, void* stream);
  * Same arguments and layouts as na_forward_ex; the caller still passes q, k,
  * v, out and lse.  It runs the tensor-core kernel only (bf16, head_dim 64 or
  * 128, or f16 with the same head dims; opt->kernel must be NA_KERNEL_AUTO or
- * NA_KERNEL_TC), else returns
+ * NA_KERNEL_TC -- AUTO means the tensor-core kernel here, whatever the
+ * window size), else returns
  * NA_ERR_UNSUPPORTED.  The kernel's scratch need (4 bytes) is checked against
  * the array's size and refused with NA_ERR_UNSUPPORTED if it ever exceeded it.
  *

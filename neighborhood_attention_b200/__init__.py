@@ -20,8 +20,10 @@ LIB_PATH = os.path.join(_PKG, "libna.so")
 
 NA_OK, NA_ERR_INVALID_ARG, NA_ERR_UNSUPPORTED, NA_ERR_CUDA, NA_ERR_TIMEOUT = range(5)
 NA_F32, NA_BF16, NA_F16 = 0, 1, 2
-NA_KERNEL_AUTO, NA_KERNEL_SIMT, NA_KERNEL_TC = 0, 1, 2
-KERNEL_NAMES = {NA_KERNEL_AUTO: "auto", NA_KERNEL_SIMT: "simt", NA_KERNEL_TC: "tc"}
+NA_KERNEL_AUTO, NA_KERNEL_SIMT, NA_KERNEL_TC, NA_KERNEL_GATHER = 0, 1, 2, 3
+NA_GATHER_MAX_KEYS = 32
+KERNEL_NAMES = {NA_KERNEL_AUTO: "auto", NA_KERNEL_SIMT: "simt", NA_KERNEL_TC: "tc",
+                NA_KERNEL_GATHER: "gather"}
 NA_WINDOW_CLAMPED, NA_WINDOW_TRUNCATED, NA_WINDOW_CAUSAL = range(3)
 WINDOW_MODES = {"clamped": NA_WINDOW_CLAMPED, "truncated": NA_WINDOW_TRUNCATED,
                 "causal": NA_WINDOW_CAUSAL}

@@ -18,7 +18,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libna.so")
-SOURCES = ["na_api.cu", "na_fwd_simt.cu", "na_fwd_sm100.cu", "na_bwd_simt.cu", "na_bwd_sm100.cu"]
+SOURCES = ["na_api.cu", "na_fwd_simt.cu", "na_fwd_gather.cu", "na_fwd_sm100.cu", "na_bwd_simt.cu",
+           "na_bwd_sm100.cu"]
 HEADERS = ["na_internal.h", "na_sched.cuh", "na_ptx.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -47,7 +47,72 @@ struct Plan {
   int kernel = NA_KERNEL_SIMT;
   QTiling t{};
   int kb[3] = {1, 1, 1};
+  // window-gather kernel: query tile staged per CTA (gq[0] == 0: direct reads),
+  // its shared memory, and the K / V rows staged per head
+  int gq[3] = {0, 0, 0};
+  int gsmem = 0;
+  long long gstaged = 0;
 };
+
+// Key-box extents along one dimension for query tiles of extent t: the
+// largest box (shared memory) and the sum over tile positions (rows staged).
+void gather_box_extent(const Geom& g, int d, int t, int& kmax, long long& sum) {
+  kmax = 0;
+  sum = 0;
+  for (int o = 0; o < g.L[d]; o += t) {
+    const int n = imin(t, g.L[d] - o);
+    int a, b, c, e;
+    window_range(g.L[d], g.w[d], g.s[d], g.m[d], o, a, b);
+    window_range(g.L[d], g.w[d], g.s[d], g.m[d], o + n - 1, c, e);
+    kmax = imax(kmax, e - a);
+    sum += e - a;
+  }
+}
+
+// Query tile of the window-gather kernel: among boxes of 2^k queries (k <= 8)
+// whose largest key box fits the shared-memory budget, the one that stages
+// the fewest K / V rows per head, counting each CTA as 32 rows of fixed cost.
+// No fitting box (a wide window): gq stays 0 and the kernel reads directly.
+void choose_gather_tile(const Problem& P, Plan& plan) {
+  const int esz = P.dtype == NA_F32 ? 4 : 2;
+  double best = 0;
+  bool found = false;
+  for (int lp = 8; lp >= 0; --lp) {
+    for (int e0 = 0; e0 <= lp; ++e0)
+      for (int e1 = 0; e0 + e1 <= lp; ++e1) {
+        const int e[3] = {e0, e1, lp - e0 - e1};
+        int t[3], km[3];
+        long long sm[3];
+        bool ok = true;
+        long long box = 1, staged = 1, tiles = 1;
+        for (int d = 0; d < 3 && ok; ++d) {
+          t[d] = 1 << e[d];
+          if (t[d] > 1 && t[d] / 2 >= P.g.L[d]) ok = false;   // no wider than needed
+          if (!ok) break;
+          gather_box_extent(P.g, d, t[d], km[d], sm[d]);
+          box *= km[d];
+          staged *= sm[d];
+          tiles *= (P.g.L[d] + t[d] - 1) / t[d];
+        }
+        if (!ok) continue;
+        const long long bytes = 2 * box * P.D * esz;
+        if (bytes > GATHER_SMEM_BUDGET) continue;
+        const double cost = (double)staged + 32.0 * (double)tiles;
+        if (!found || cost < best - 1e-9) {
+          found = true;
+          best = cost;
+          for (int d = 0; d < 3; ++d) plan.gq[d] = t[d];
+          plan.gsmem = (int)bytes;
+          plan.gstaged = staged;
+        }
+      }
+  }
+  if (!found) {
+    plan.gq[0] = plan.gq[1] = plan.gq[2] = 0;
+    plan.gsmem = 0;
+    plan.gstaged = 0;
+  }
+}
 
 na_status read_problem(const int dims[2], const int* grid, const int* window, const int* stride,
                        const int* tile, na_dtype dtype, const na_options* opt, Problem& P) {
@@ -86,7 +151,7 @@ na_status read_problem(const int dims[2], const int* grid, const int* window, co
     if (N > (1LL << 31)) return fail(NA_ERR_UNSUPPORTED, "grid has more than 2^31 tokens");
   }
   P.opt = opt ? *opt : na_default_options();
-  if (P.opt.kernel < NA_KERNEL_AUTO || P.opt.kernel > NA_KERNEL_TC)
+  if (P.opt.kernel < NA_KERNEL_AUTO || P.opt.kernel > NA_KERNEL_GATHER)
     return fail(NA_ERR_INVALID_ARG, "unknown kernel selector %d", P.opt.kernel);
   for (int i = 0; i < nd; ++i) {
     const int m = P.opt.window_mode[i];
@@ -181,6 +246,8 @@ std::map<std::vector<long long>, Plan> g_plans;
 na_status make_plan(const Problem& P, Plan& out) {
   int kernel = P.opt.kernel;
   const bool half = P.dtype == NA_BF16 || P.dtype == NA_F16;
+  const long long wkeys = (long long)P.g.w[0] * P.g.w[1] * P.g.w[2];
+  if (kernel == NA_KERNEL_AUTO && wkeys <= NA_GATHER_MAX_KEYS) kernel = NA_KERNEL_GATHER;
   if (kernel == NA_KERNEL_AUTO)
     kernel = (half && (P.D == 64 || P.D == 128)) ? NA_KERNEL_TC : NA_KERNEL_SIMT;
   if (kernel == NA_KERNEL_TC && !half)
@@ -200,6 +267,22 @@ na_status make_plan(const Problem& P, Plan& out) {
       out = it->second;
       return NA_OK;
     }
+  }
+  if (kernel == NA_KERNEL_GATHER) {
+    // No blocks or chunks: each query on its own with exactly its window's
+    // keys; the query tile staged per CTA is chosen here (and cached).
+    const int one[3] = {1, 1, 1};
+    Plan g;
+    g.kernel = NA_KERNEL_GATHER;
+    if (make_tiling(P.g, one, one, g.t) != 0)
+      return fail(NA_ERR_UNSUPPORTED, "window-gather kernel: grid too large");
+    choose_gather_tile(P, g);
+    {
+      std::lock_guard<std::mutex> lk(g_plan_mu);
+      g_plans[key] = g;
+    }
+    out = g;
+    return NA_OK;
   }
   const int qprod = kernel == NA_KERNEL_TC ? 128 : 128 / (P.D / 32);
   const int kprod = kernel == NA_KERNEL_TC ? 128 : 32;
@@ -423,6 +506,26 @@ na_status na_forward_ex(const void* q, const void* k, const void* v, void* out, 
   L.dtype = P.dtype;
   L.scale_log2 = scale * log2e;
   L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
+  if (plan.kernel == NA_KERNEL_GATHER) {
+    GatherLaunch G;
+    G.g = P.g;
+    G.BH = (int)BH;
+    G.N = (int)N;
+    G.D = P.D;
+    G.dtype = P.dtype;
+    G.scale_log2 = scale * log2e;
+    G.q = q; G.k = k; G.v = v; G.out = out; G.lse = lse;
+    for (int d = 0; d < 3; ++d) {
+      G.qt[d] = plan.gq[d];
+      G.nt[d] = plan.gq[0] > 0 ? (P.g.L[d] + plan.gq[d] - 1) / plan.gq[d] : 0;
+    }
+    G.smem_bytes = plan.gsmem;
+    cudaError_t e = launch_gather(G, s);
+    if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "window-gather kernel: shape");
+    if (e != cudaSuccess)
+      return fail(NA_ERR_CUDA, "window-gather launch: %s", cudaGetErrorString(e));
+    return NA_OK;
+  }
   cudaError_t e = launch_simt(L, s);
   if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "CUDA-core kernel: shape");
   if (e != cudaSuccess) return fail(NA_ERR_CUDA, "CUDA-core launch: %s", cudaGetErrorString(e));
@@ -456,6 +559,8 @@ na_status na_backward(const void* q, const void* k, const void* v, const void* o
   const long long BH = (long long)B * heads;
   if (BH > (1LL << 30)) return fail(NA_ERR_UNSUPPORTED, "B*heads too large");
   const bool tc_ok = (P.dtype == NA_BF16 || P.dtype == NA_F16) && (P.D == 64 || P.D == 128);
+  if (P.opt.kernel == NA_KERNEL_GATHER)
+    return fail(NA_ERR_UNSUPPORTED, "the window-gather kernel is forward only");
   if (P.opt.kernel == NA_KERNEL_TC && !tc_ok)
     return fail(NA_ERR_UNSUPPORTED, "the tensor-core backward takes bf16 / f16, head_dim 64 or 128");
   const bool use_tc = tc_ok && P.opt.kernel != NA_KERNEL_SIMT;
@@ -555,23 +660,6 @@ na_status na_plan(const int dims[2], const int* grid, const int* window, const i
   Plan plan;
   st = make_plan(P, plan);
   if (st != NA_OK) return st;
-  const int group = plan.kernel == NA_KERNEL_TC ? 2 : 1;
-  const Cost c = walk(P.g, plan.t, plan.kb, group, 0);
-  memset(info, 0, sizeof *info);
-  info->kernel = plan.kernel;
-  for (int d = 0; d < 3; ++d) {
-    info->qblock[d] = plan.t.qb[d];
-    info->kvchunk[d] = plan.kb[d];
-    info->tile[d] = plan.t.tl[d];
-  }
-  const long long rows = (long long)plan.t.qb[0] * plan.t.qb[1] * plan.t.qb[2];
-  const long long keys = (long long)plan.kb[0] * plan.kb[1] * plan.kb[2];
-  info->query_blocks = plan.t.nblocks;
-  info->ctas = (plan.t.nblocks + group - 1) / group;
-  info->chunks_loaded = c.loads;
-  info->units_full = c.full;
-  info->units_partial = c.partial;
-  info->computed_pairs = (c.full + c.partial) * rows * keys;
   // sum over queries of the window size = product over dimensions of the sum
   // over coordinates of the 1-D window length (the window is a product).
   long long useful = 1;
@@ -584,20 +672,65 @@ na_status na_plan(const int dims[2], const int* grid, const int* window, const i
     }
     useful *= sum;
   }
+  const long long N = (long long)P.g.L[0] * P.g.L[1] * P.g.L[2];
+  const bool gather = plan.kernel == NA_KERNEL_GATHER;
+  const int group = plan.kernel == NA_KERNEL_TC ? 2 : 1;
+  Cost c{};
+  if (gather) {
+    // one (query, key) pair per unit, exactly the window's keys: no walk needed;
+    // "chunks" loaded = K / V rows staged in shared memory (staged form) or
+    // read per query (direct form)
+    c.full = useful;
+    c.partial = 0;
+    c.loads = plan.gq[0] > 0 ? plan.gstaged : useful;
+  } else {
+    c = walk(P.g, plan.t, plan.kb, group, 0);
+  }
+  memset(info, 0, sizeof *info);
+  info->kernel = plan.kernel;
+  for (int d = 0; d < 3; ++d) {
+    info->qblock[d] = plan.t.qb[d];
+    info->kvchunk[d] = plan.kb[d];
+    info->tile[d] = plan.t.tl[d];
+  }
+  const long long rows = (long long)plan.t.qb[0] * plan.t.qb[1] * plan.t.qb[2];
+  const long long keys = (long long)plan.kb[0] * plan.kb[1] * plan.kb[2];
+  info->query_blocks = plan.t.nblocks;
+  info->ctas = (plan.t.nblocks + group - 1) / group;
+  if (gather) {
+    if (plan.gq[0] > 0) {
+      info->ctas = 1;
+      for (int d = 0; d < 3; ++d) {
+        info->qblock[d] = plan.gq[d];
+        info->tile[d] = plan.gq[d];
+        info->ctas *= (P.g.L[d] + plan.gq[d] - 1) / plan.gq[d];
+      }
+    } else {
+      const long long rpc = gather_rows_per_cta(P.D, P.dtype);
+      info->ctas = (plan.t.nblocks + rpc - 1) / rpc;
+    }
+  }
+  info->chunks_loaded = c.loads;
+  info->units_full = c.full;
+  info->units_partial = c.partial;
+  info->computed_pairs = (c.full + c.partial) * rows * keys;
   info->useful_pairs = useful;
   // Speedup bound: dense attention (every window the whole grid) under the
   // same block / chunk shapes computes every (block, chunk) unit; this
   // schedule computes only the non-empty ones, each at full tile cost.
-  Geom dense = P.g;
-  for (int d = 0; d < 3; ++d) {
-    dense.w[d] = dense.L[d];
-    dense.s[d] = 1;
-    dense.m[d] = WIN_CLAMPED;
-  }
-  const Cost cd = walk(dense, plan.t, plan.kb, group, 0);
-  const long long N = (long long)P.g.L[0] * P.g.L[1] * P.g.L[2];
   info->dense_pairs = N * N;
-  info->dense_units = cd.full + cd.partial;
+  if (gather) {
+    info->dense_units = N * N;
+  } else {
+    Geom dense = P.g;
+    for (int d = 0; d < 3; ++d) {
+      dense.w[d] = dense.L[d];
+      dense.s[d] = 1;
+      dense.m[d] = WIN_CLAMPED;
+    }
+    const Cost cd = walk(dense, plan.t, plan.kb, group, 0);
+    info->dense_units = cd.full + cd.partial;
+  }
   const long long units = c.full + c.partial;
   info->speedup_bound = units > 0 ? (double)info->dense_units / (double)units : 0.0;
   return NA_OK;
@@ -657,7 +790,7 @@ na_status na_forward_noalloc(const void* q, const void* k, const void* v, void* 
     return fail(NA_ERR_INVALID_ARG, "q, k, v, out must be 16-byte aligned and lse 4-byte aligned");
   const long long BH = (long long)B * heads;
   if (BH > (1LL << 30)) return fail(NA_ERR_UNSUPPORTED, "B*heads too large");
-  if (P.opt.kernel == NA_KERNEL_SIMT)
+  if (P.opt.kernel == NA_KERNEL_SIMT || P.opt.kernel == NA_KERNEL_GATHER)
     return fail(NA_ERR_UNSUPPORTED, "na_forward_noalloc runs the tensor-core kernel only");
   P.opt.kernel = NA_KERNEL_TC;
   Plan plan;

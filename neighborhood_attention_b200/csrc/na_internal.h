@@ -73,6 +73,29 @@ struct TcBwdLaunch {
   long long timeout_ns;  // bound on every in-kernel wait
 };
 
+// Window-gather kernel (CUDA cores): each query reads its own window's keys.
+// 256 threads, one 16-byte slice of the head dimension each: query rows served
+// at once per CTA.
+inline int gather_rows_per_cta(int D, int dtype) { return 256 / (D / (dtype == 0 ? 4 : 8)); }
+
+struct GatherLaunch {
+  Geom g;
+  int BH, N, D;
+  int dtype;             // na_dtype of q, k, v and out
+  float scale_log2;      // scale * log2(e)
+  const void *q, *k, *v;
+  void* out;
+  float* lse;
+  int qt[3];             // query tile per CTA (a box of the grid); qt[0] == 0: no
+                         // staging, every key read straight from global memory
+  int nt[3];             // tiles per dimension
+  int smem_bytes;        // K and V rows of the largest key box of a tile
+};
+
+// Shared memory the staged form may use per CTA (two CTAs fit on an SM).
+constexpr int GATHER_SMEM_BUDGET = 100 * 1024;
+cudaError_t launch_gather(const GatherLaunch& L, cudaStream_t stream);
+
 // 5-d TMA descriptor of a [BH, X1, X2, X3, D] bf16 / f16 tensor, 64-element
 // inner box of `box` tokens, 128-byte swizzle.
 bool encode_grid_map(CUtensorMap* m, const void* ptr, int f16, int D, const int L[3], int BH,

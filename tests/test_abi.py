@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -95,3 +96,69 @@ def test_window_mode_beyond_ndim_is_ignored():
     opts = na.make_options(window_mode=[2, 1, 77])
     p = na.na_plan([8, 8], [3, 3], None, None, 64, na.NA_BF16, options=opts)
     assert p["useful_pairs"] > 0
+
+
+@pytest.mark.parametrize("window,dtype,expect", [
+    ((5, 5), "bf16", "gather"),       # 25 keys: at most NA_GATHER_MAX_KEYS
+    ((4, 8), "f16", "gather"),        # 32 keys
+    ((6, 6), "bf16", "tc"),           # 36 keys
+    ((5, 5), "f32", "gather"),
+    ((7, 7), "f32", "simt"),
+])
+def test_auto_sends_narrow_windows_to_the_gather_kernel(window, dtype, expect):
+    import neighborhood_attention_b200 as na
+    dt = {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32}[dtype]
+    p = na.na_plan([40, 48], list(window), None, None, 64, dt)
+    assert p["kernel"] == expect
+    if expect == "gather":
+        # each query attends exactly its window's keys: nothing is masked; a
+        # CTA stages the key box of a query tile (qblock) in shared memory
+        assert p["kvchunk"] == [1, 1, 1]
+        assert p["units_partial"] == 0
+        assert p["units_full"] == p["useful_pairs"] == p["computed_pairs"]
+        g3 = [1, 40, 48]
+        assert p["ctas"] == int(np.prod([-(-g3[d] // p["qblock"][d]) for d in range(3)]))
+        # every key row is staged at least once, each tile's box at most once
+        assert 40 * 48 <= p["chunks_loaded"] <= p["ctas"] * np.prod(window) * 256
+
+
+def test_gather_selector_takes_any_window_and_cut_modes():
+    import neighborhood_attention_b200 as na
+    opts = na.make_options(kernel=na.NA_KERNEL_GATHER, window_mode=["causal", "truncated"])
+    p = na.na_plan([33, 17], [9, 7], [3, 1], None, 128, na.NA_BF16, options=opts)
+    assert p["kernel"] == "gather"
+    # causal over 33 with w 9, s 3; truncated over 17 with w 7: per-dimension sums
+    causal = sum(min(33, (i // 3 + 1) * 3) - max(0, (i // 3 + 1) * 3 - 9) for i in range(33))
+    trunc = sum(min(17, i - 3 + 7) - max(0, i - 3) for i in range(17))
+    assert p["useful_pairs"] == causal * trunc == p["units_full"]
+
+
+def _fake_call(lib, fn, kernel):
+    import neighborhood_attention_b200 as na
+    iv = lambda xs: (ctypes.c_int * len(xs))(*xs)
+    o = na.make_options(kernel=kernel)
+    p = ctypes.c_void_p(256)   # aligned and never dereferenced: the call fails on the host
+    if fn == "na_backward":
+        f = lib.na_backward
+        f.argtypes = [ctypes.c_void_p] * 10 + [ctypes.c_int, ctypes.c_int] + \
+            [ctypes.POINTER(ctypes.c_int)] * 5 + [ctypes.c_int, ctypes.POINTER(na.na_options),
+                                                  ctypes.c_void_p]
+        return f(*([p] * 10), 1, 1, iv([2, 64]), iv([8, 8]), iv([3, 3]), None, None, 1,
+                 ctypes.byref(o), None)
+    f = getattr(lib, fn)
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_int] + \
+        [ctypes.POINTER(ctypes.c_int)] * 5 + [ctypes.c_int, ctypes.POINTER(na.na_options),
+                                              ctypes.c_void_p]
+    return f(*([p] * 5), 1, 1, iv([2, 64]), iv([8, 8]), iv([3, 3]), None, None, 1,
+             ctypes.byref(o), None)
+
+
+@pytest.mark.parametrize("fn", ["na_backward", "na_forward_noalloc"])
+def test_gather_selector_is_refused_where_it_does_not_apply(fn):
+    """The window-gather kernel is forward only, and the allocation-free entry
+    point runs the tensor-core kernel only: both refuse the selector on the host."""
+    import neighborhood_attention_b200 as na
+    lib = ctypes.CDLL(na.LIB_PATH)
+    assert _fake_call(lib, fn, na.NA_KERNEL_GATHER) == na.NA_ERR_UNSUPPORTED
+    lib.na_last_error.restype = ctypes.c_char_p
+    assert lib.na_last_error().decode() != ""

@@ -115,7 +115,9 @@ def test_plan_statistics(i):
     assert p["useful_pairs"] == N * W
     assert p["computed_pairs"] >= p["useful_pairs"]
     if i == 1:
-        assert p["kernel"] == "simt"
+        # 25 keys per query: the window-gather kernel, one query per unit
+        assert p["kernel"] == "gather"
+        assert p["computed_pairs"] == p["useful_pairs"]
     else:
         assert p["kernel"] == "tc"
         assert np.prod(p["qblock"]) == 128 and np.prod(p["kvchunk"]) == 128
