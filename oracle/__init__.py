@@ -59,6 +59,16 @@ class OracleLib:
         lib.na_oracle_mask_row.argtypes = [ctypes.c_int, i32p, i32p, i32p, i32p,
                                            ctypes.c_longlong, ctypes.c_void_p]
         lib.na_oracle_mask_row.restype = ctypes.c_longlong
+        lib.na_oracle_mask_row_dil.argtypes = [ctypes.c_int, i32p, i32p, i32p, i32p, i32p,
+                                               ctypes.c_longlong, ctypes.c_void_p]
+        lib.na_oracle_mask_row_dil.restype = ctypes.c_longlong
+        lib.na_oracle_dilated_window.argtypes = [ctypes.c_int] * 6 + [i32p, i32p, i32p]
+        lib.na_oracle_dilated_window.restype = ctypes.c_int
+        lib.na_oracle_forward_dil.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong,
+            ctypes.c_int, i32p, i32p, i32p, i32p, i32p, ctypes.c_int, ctypes.c_double,
+            ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        lib.na_oracle_forward_dil.restype = ctypes.c_int
         lib.na_oracle_forward.argtypes = [
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong,
             ctypes.c_int, i32p, i32p, i32p, i32p, ctypes.c_int, ctypes.c_double,
@@ -106,20 +116,31 @@ class OracleLib:
             raise ValueError(f"invalid window arguments L={L} w={w} s={s} mode={mode} i={i}")
         return lo.value, hi.value
 
-    def mask_row(self, grid, window, stride, token: int, mode=None) -> np.ndarray:
+    def dilated_window(self, L: int, w: int, s: int, mode, dil: int, i: int):
+        """(r, lo, hi): coordinate i's keys are r + dil * t for t in [lo, hi)."""
+        r, lo, hi = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+        rc = self.lib.na_oracle_dilated_window(L, w, s, _modes([mode], 1)[0], dil, i,
+                                               ctypes.byref(r), ctypes.byref(lo), ctypes.byref(hi))
+        if rc < 0:
+            raise ValueError(f"invalid dilated window L={L} w={w} s={s} dil={dil} i={i}")
+        return r.value, lo.value, hi.value
+
+    def mask_row(self, grid, window, stride, token: int, mode=None, dilation=None) -> np.ndarray:
         grid, window, stride = _geom(grid, window, stride)
         n = int(np.prod(grid))
         out = np.zeros(n, dtype=np.uint8)
-        rc = self.lib.na_oracle_mask_row(len(grid), self._ivec(grid), self._ivec(window),
-                                         self._ivec(stride), self._ivec(_modes(mode, len(grid))),
-                                         int(token), out.ctypes.data)
+        rc = self.lib.na_oracle_mask_row_dil(len(grid), self._ivec(grid), self._ivec(window),
+                                             self._ivec(stride),
+                                             self._ivec(_modes(mode, len(grid))),
+                                             self._ivec(_dil(dilation, len(grid))), int(token),
+                                             out.ctypes.data)
         if rc < 0:
             raise ValueError("na_oracle_mask_row: invalid arguments")
         return out.astype(bool)
 
     # -- forward -----------------------------------------------------------
     def forward(self, q, k, v, grid, window, stride, *, dtype: str, rows=None,
-                scale: float = 0.0, threads: int | None = None, mode=None):
+                scale: float = 0.0, threads: int | None = None, mode=None, dilation=None):
         """Exact forward in fp64.
 
         q, k, v: arrays of shape [B, heads, *grid, d]; float32 values for
@@ -157,10 +178,11 @@ class OracleLib:
             rows_ptr = rows.ctypes.data
         out = np.empty((nrows, d), dtype=np.float64)
         lse = np.empty(nrows, dtype=np.float64)
-        rc = self.lib.na_oracle_forward(
+        rc = self.lib.na_oracle_forward_dil(
             arrs[0].ctypes.data, arrs[1].ctypes.data, arrs[2].ctypes.data,
             code, BH, nd, self._ivec(grid), self._ivec(window),
-            self._ivec(stride), self._ivec(_modes(mode, nd)), d, float(scale), rows_ptr, nrows,
+            self._ivec(stride), self._ivec(_modes(mode, nd)), self._ivec(_dil(dilation, nd)), d,
+            float(scale), rows_ptr, nrows,
             out.ctypes.data, lse.ctypes.data, int(threads or os.cpu_count() or 1))
         if rc:
             raise RuntimeError(f"na_oracle_forward failed with code {rc}")
@@ -271,6 +293,18 @@ def _modes(mode, nd):
     return out
 
 
+def _dil(dilation, nd):
+    """Per-dimension dilation as ints (None stays None: all 1)."""
+    if dilation is None:
+        return None
+    if isinstance(dilation, int):
+        dilation = [dilation] * nd
+    out = [int(x) for x in dilation]
+    if len(out) != nd:
+        raise ValueError(f"{len(out)} dilations for {nd} dimensions")
+    return out
+
+
 def load(path: str | None = None) -> OracleLib:
     """The oracle library at ``path`` (default: the real one, built on demand)."""
     with _lock:
@@ -289,8 +323,12 @@ def window(L, w, s, mode, i):
     return load().window(L, w, s, mode, i)
 
 
-def mask_row(grid, window, stride, token, mode=None):
-    return load().mask_row(grid, window, stride, token, mode)
+def mask_row(grid, window, stride, token, mode=None, dilation=None):
+    return load().mask_row(grid, window, stride, token, mode, dilation)
+
+
+def dilated_window(L, w, s, mode, dil, i):
+    return load().dilated_window(L, w, s, mode, dil, i)
 
 
 def forward(q, k, v, grid, window, stride, **kw):

@@ -56,6 +56,17 @@
  *   (truncated: the same centring as the clamped rule; causal: the group as
  *   the unit of causality) and coincide with eq. (5) at s = 1.
  *
+ * Dilation (per grid dimension, dil >= 1): the pages name dilated patterns
+ * only as related work ("pi-Attention", section 2: "strided/dilated
+ * patterns") and define none.  The reading here is the plainest one that
+ * keeps the rules above intact: coordinates split into dil interleaved
+ * sub-sequences by residue r = i mod dil; sub-sequence r holds the
+ * Lr = ceil((L - r) / dil) coordinates r, r + dil, r + 2 dil, ...; a query
+ * at i = r + dil * p takes the window [lo, hi) of position p inside its
+ * sub-sequence (any mode, stride in sub-sequence positions) and attends to
+ * the keys r + dil * t for t in [lo, hi).  dil = 1 is the undilated rule;
+ * clamped windows need w <= Lr for every r, i.e. w * dil <= L.
+ *
  * Backward (the gradients of the forward pass for an upstream gradient dO of
  * out): the pages give only the forward; the gradients here are its
  * vector-Jacobian product written out with P_ij = exp(z_ij - lse_i) over the
@@ -120,13 +131,28 @@ int na_oracle_window(int L, int w, int s, int mode, int i, int* lo, int* hi) {
     return 0;
 }
 
+/*
+ * Dilated window of coordinate i in one dimension: the keys r + dil * t for
+ * t in [*lo, *hi), with *r = i mod dil (definition above).
+ */
+int na_oracle_dilated_window(int L, int w, int s, int mode, int dil, int i, int* r, int* lo,
+                             int* hi) {
+    if (dil < 1 || L < 1 || i < 0 || i >= L || !r || !lo || !hi) return -1;
+    const int res = i % dil;
+    const int Lr = (L - res + dil - 1) / dil;      /* coordinates res, res + dil, ... below L */
+    if (w > L / dil) return -1;                    /* every sub-sequence holds the window */
+    *r = res;
+    return na_oracle_window(Lr, w, s, mode, i / dil, lo, hi);
+}
+
 static int check_geometry(int ndim, const int* L, const int* w, const int* s, const int* mode,
-                          long long* N) {
+                          const int* dil, long long* N) {
     if (ndim < 1 || ndim > NA_ORACLE_MAXDIM || !L || !w || !s) return -1;
     long long n = 1;
     for (int a = 0; a < ndim; ++a) {
         if (L[a] < 1 || w[a] < 1 || w[a] > L[a] || s[a] < 1 || s[a] > w[a]) return -1;
         if (mode && (mode[a] < WIN_CLAMPED || mode[a] > WIN_CAUSAL)) return -1;
+        if (dil && (dil[a] < 1 || (long long)w[a] * dil[a] > L[a])) return -1;
         n *= L[a];
     }
     *N = n;
@@ -142,23 +168,32 @@ static void unflatten(long long t, int ndim, const int* L, int* coord) {
 
 /*
  * Dense membership row: mask[j] = 1 iff key token j is in the window of query
- * token t.  mode: per-dimension window modes, NULL = all clamped.  Returns the
- * number of keys in the window (> 0), or -1 on invalid input.
+ * token t.  mode: per-dimension window modes, NULL = all clamped; dil:
+ * per-dimension dilation, NULL = all 1.  Returns the number of keys in the
+ * window (> 0), or -1 on invalid input.
  */
-long long na_oracle_mask_row(int ndim, const int* L, const int* w, const int* s, const int* mode,
-                             long long t, uint8_t* mask) {
+long long na_oracle_mask_row_dil(int ndim, const int* L, const int* w, const int* s,
+                                 const int* mode, const int* dil, long long t, uint8_t* mask) {
     long long N;
-    if (check_geometry(ndim, L, w, s, mode, &N) || t < 0 || t >= N || !mask) return -1;
+    if (check_geometry(ndim, L, w, s, mode, dil, &N) || t < 0 || t >= N || !mask) return -1;
     int qi[NA_ORACLE_MAXDIM], lo[NA_ORACLE_MAXDIM], hi[NA_ORACLE_MAXDIM], kj[NA_ORACLE_MAXDIM];
+    int res[NA_ORACLE_MAXDIM], step[NA_ORACLE_MAXDIM];
     unflatten(t, ndim, L, qi);
-    for (int a = 0; a < ndim; ++a)
-        na_oracle_window(L[a], w[a], s[a], mode ? mode[a] : WIN_CLAMPED, qi[a], &lo[a], &hi[a]);
+    for (int a = 0; a < ndim; ++a) {
+        step[a] = dil ? dil[a] : 1;
+        na_oracle_dilated_window(L[a], w[a], s[a], mode ? mode[a] : WIN_CLAMPED, step[a], qi[a],
+                                 &res[a], &lo[a], &hi[a]);
+    }
     for (int a = 0; a < ndim; ++a) kj[a] = 0;
     long long count = 0;
     for (long long j = 0; j < N; ++j) {
         int in = 1;
-        for (int a = 0; a < ndim; ++a)
-            if (kj[a] < lo[a] || kj[a] >= hi[a]) in = 0;
+        for (int a = 0; a < ndim; ++a) {
+            /* key coordinate kj = res + step * u with u in [lo, hi) */
+            if (kj[a] % step[a] != res[a]) in = 0;
+            const int u = kj[a] / step[a];
+            if (u < lo[a] || u >= hi[a]) in = 0;
+        }
         count += in;
         mask[j] = (uint8_t)in;
         for (int a = ndim - 1; a >= 0; --a) { /* advance the row-major key counter */
@@ -167,6 +202,11 @@ long long na_oracle_mask_row(int ndim, const int* L, const int* w, const int* s,
         }
     }
     return count;
+}
+
+long long na_oracle_mask_row(int ndim, const int* L, const int* w, const int* s, const int* mode,
+                             long long t, uint8_t* mask) {
+    return na_oracle_mask_row_dil(ndim, L, w, s, mode, NULL, t, mask);
 }
 
 /* --------------------------------------------------------------- forward -- */
@@ -206,6 +246,7 @@ typedef struct {
     const long long* rows;
     long long r_begin, r_end;
     double *out, *lse;
+    const int* dil;
     int status;
 } fwd_job;
 
@@ -225,7 +266,8 @@ static void* fwd_worker(void* arg) {
         long long row = J->rows ? J->rows[r] : r;
         if (row < 0 || row >= J->BH * N) { J->status = -1; break; }
         long long bh = row / N, t = row % N;
-        const long long inwin = na_oracle_mask_row(ndim, J->L, J->w, J->s, J->mode, t, mask);
+        const long long inwin =
+            na_oracle_mask_row_dil(ndim, J->L, J->w, J->s, J->mode, J->dil, t, mask);
         size_t qoff = (size_t)row * (size_t)d;
         long long cnt = 0;
         for (long long j = 0; j < N; ++j) {
@@ -272,15 +314,14 @@ done:
  * scale <= 0 means 1/sqrt(d).  Returns 0, or a negative code on bad input
  * (-1), allocation failure (-2) or a window whose key count is inconsistent (-3).
  */
-int na_oracle_forward(const void* q, const void* k, const void* v, int in_dtype, long long BH,
-                      int ndim, const int* L, const int* w, const int* s, const int* mode, int d,
-                      double scale,
-                      const long long* rows, long long nrows, double* out, double* lse,
-                      int nthreads) {
+int na_oracle_forward_dil(const void* q, const void* k, const void* v, int in_dtype, long long BH,
+                          int ndim, const int* L, const int* w, const int* s, const int* mode,
+                          const int* dil, int d, double scale, const long long* rows,
+                          long long nrows, double* out, double* lse, int nthreads) {
     long long N;
     if (!q || !k || !v || !out || !lse || BH < 1 || d < 1 || nrows < 0) return -1;
     if (in_dtype != IN_F32 && in_dtype != IN_BF16 && in_dtype != IN_F16) return -1;
-    if (check_geometry(ndim, L, w, s, mode, &N)) return -1;
+    if (check_geometry(ndim, L, w, s, mode, dil, &N)) return -1;
     if (!rows && nrows != BH * N) return -1;
     long long W = 1;
     for (int a = 0; a < ndim; ++a) W *= w[a];
@@ -302,6 +343,7 @@ int na_oracle_forward(const void* q, const void* k, const void* v, int in_dtype,
         J->r_begin = per * t < nrows ? per * t : nrows;
         J->r_end = per * (t + 1) < nrows ? per * (t + 1) : nrows;
         J->out = out; J->lse = lse;
+        J->dil = dil;
         J->status = 0;
     }
     for (int t = 1; t < nthreads; ++t)
@@ -315,6 +357,14 @@ int na_oracle_forward(const void* q, const void* k, const void* v, int in_dtype,
     for (int t = 0; t < nthreads; ++t)
         if (jobs[t].status) return jobs[t].status;
     return 0;
+}
+
+int na_oracle_forward(const void* q, const void* k, const void* v, int in_dtype, long long BH,
+                      int ndim, const int* L, const int* w, const int* s, const int* mode, int d,
+                      double scale, const long long* rows, long long nrows, double* out,
+                      double* lse, int nthreads) {
+    return na_oracle_forward_dil(q, k, v, in_dtype, BH, ndim, L, w, s, mode, NULL, d, scale, rows,
+                                 nrows, out, lse, nthreads);
 }
 
 /* -------------------------------------------------------------- backward -- */
@@ -410,7 +460,7 @@ int na_oracle_backward(const void* q, const void* k, const void* v, const void* 
     long long N;
     if (!q || !k || !v || !dout || !dq || !dk || !dv || BH < 1 || d < 1) return -1;
     if (in_dtype != IN_F32 && in_dtype != IN_BF16 && in_dtype != IN_F16) return -1;
-    if (check_geometry(ndim, L, w, s, mode, &N)) return -1;
+    if (check_geometry(ndim, L, w, s, mode, NULL, &N)) return -1;
     long long W = 1;
     for (int a = 0; a < ndim; ++a) W *= w[a];
     if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
@@ -518,7 +568,7 @@ int na_oracle_backward_sampled(const void* q, const void* k, const void* v, cons
     if (!q || !k || !v || !dout || BH < 1 || bh < 0 || bh >= BH || d < 1) return -1;
     if ((nq && (!qrows || !dq)) || (nk && (!krows || !dk || !dv))) return -1;
     if (in_dtype != IN_F32 && in_dtype != IN_BF16 && in_dtype != IN_F16) return -1;
-    if (check_geometry(ndim, L, w, s, mode, &N)) return -1;
+    if (check_geometry(ndim, L, w, s, mode, NULL, &N)) return -1;
     long long W = 1;
     for (int a = 0; a < ndim; ++a) W *= w[a];
     if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
@@ -628,7 +678,7 @@ int na_oracle_backward_sampled(const void* q, const void* k, const void* v, cons
 int na_oracle_block_counts(int ndim, const int* L, const int* w, const int* s, const int* mode,
                            long long blk, long long* counts) {
     long long N;
-    if (check_geometry(ndim, L, w, s, mode, &N) || blk < 1 || !counts) return -1;
+    if (check_geometry(ndim, L, w, s, mode, NULL, &N) || blk < 1 || !counts) return -1;
     long long nb = (N + blk - 1) / blk;
     long long* members = (long long*)calloc((size_t)(nb * nb), sizeof(long long));
     uint8_t* mask = (uint8_t*)malloc((size_t)N);

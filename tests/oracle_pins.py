@@ -477,6 +477,76 @@ def pin_mode_uniform_queries(lib):
             np.testing.assert_allclose(out.reshape(N, d)[t, :nd], expect, atol=1e-12, rtol=0)
 
 
+# ------------------------------------------------------------- dilation --
+# Dilation is not defined by the pages (only named as a related pattern); the
+# reading: the window rule applied inside each residue class modulo dil.  The
+# brute force below builds each residue class's coordinate list explicitly
+# and indexes into it, so it shares no arithmetic with the oracle's
+# length / position formulas.
+
+def _dilated_set(L, w, s, mode, dil, i):
+    sub = [c for c in range(L) if c % dil == i % dil]      # the residue class, in order
+    p = sub.index(i)
+    return {sub[t] for t in _mode_set(len(sub), w, s, mode, p)}
+
+
+def pin_dilated_window_bruteforce(lib):
+    """Every mode, stride, dilation and window with w * dil <= L on short
+    grids (ragged residue classes included) vs the explicit residue lists."""
+    for L in range(1, 15):
+        for dil in range(1, L + 1):
+            for w in range(1, L // dil + 1):
+                for s in range(1, w + 1):
+                    for i in range(L):
+                        for mode in ("clamped", "truncated", "causal"):
+                            r, lo, hi = lib.dilated_window(L, w, s, mode, dil, i)
+                            got = {r + dil * t for t in range(lo, hi)}
+                            assert got == _dilated_set(L, w, s, mode, dil, i), \
+                                (L, w, s, mode, dil, i)
+
+
+def pin_dilated_mask_bruteforce(lib):
+    """Dense mask rows with dilation (and modes) per dimension vs the
+    product of the brute-force 1-D sets."""
+    cases = [([11, 7], [3, 2], [1, 1], ["clamped", "causal"], [3, 2]),
+             ([9, 10], [2, 3], [2, 1], ["truncated", "clamped"], [4, 3]),
+             ([5, 6, 7], [2, 3, 3], [1, 3, 1], ["causal", "truncated", "clamped"], [2, 2, 2])]
+    for grid, window, stride, modes, dil in cases:
+        N = int(np.prod(grid))
+        keys = np.array(np.unravel_index(np.arange(N), grid))
+        for t in range(N):
+            coords = np.unravel_index(t, grid)
+            ok = np.ones(N, dtype=bool)
+            for a in range(len(grid)):
+                ok &= np.isin(keys[a], sorted(_dilated_set(grid[a], window[a], stride[a], modes[a],
+                                                           dil[a], int(coords[a]))))
+            got = lib.mask_row(grid, window, stride, t, mode=modes, dilation=dil)
+            assert np.array_equal(got, ok), (grid, dil, t)
+
+
+def pin_dilated_residue_subgrids(lib):
+    """Dilated attention is undilated attention on each residue-class
+    sub-grid: slice q, k, v with step dil, run the (undilated, separately
+    pinned) forward on the slice, compare with the dilated forward's rows for
+    those queries.  Grids whose extents dil does not divide give sub-grids of
+    different lengths."""
+    d = 8
+    for grid, window, stride, modes, dil in [([13, 10], [3, 2], [1, 2], ["clamped", "truncated"],
+                                              [3, 2]),
+                                             ([7, 9], [2, 3], [1, 1], ["causal", "causal"], [2, 3])]:
+        q, k, v = (_randn(300 + t, (1, 2, *grid, d)) for t in range(3))
+        out, lse = lib.forward(q, k, v, grid, window, stride, dtype="f32", mode=modes,
+                               dilation=dil)
+        for r0 in range(dil[0]):
+            for r1 in range(dil[1]):
+                sl = (slice(None), slice(None), slice(r0, None, dil[0]), slice(r1, None, dil[1]))
+                qs, ks, vs = (np.ascontiguousarray(a[sl]) for a in (q, k, v))
+                sub = list(qs.shape[2:4])
+                o2, l2 = lib.forward(qs, ks, vs, sub, window, stride, dtype="f32", mode=modes)
+                np.testing.assert_allclose(out[sl], o2, atol=1e-13, rtol=0)
+                np.testing.assert_allclose(lse[sl[:4]], l2, atol=1e-13, rtol=0)
+
+
 def pin_sa_empty_blocks_golden(lib):
     """The Hilbert page's empty-block ratio for row-major slide attention
     (Table 3, SA (Flex) at 96x96) reproduces from the truncated window."""
@@ -592,6 +662,7 @@ ALL_PINS = [
     pin_modes_strided, pin_mode_mask_bruteforce, pin_causal_full_sdpa, pin_mode_uniform_queries,
     pin_sa_empty_blocks_golden, pin_f16_decoding, pin_backward_finite_differences,
     pin_backward_full_attention_autograd, pin_backward_invariants, pin_backward_sampled_rows,
+    pin_dilated_window_bruteforce, pin_dilated_mask_bruteforce, pin_dilated_residue_subgrids,
 ]
 
 # The golden-file pins take a few seconds each; mutant runs use the fast ones.

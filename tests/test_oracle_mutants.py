@@ -24,7 +24,7 @@ MUTANTS = [
     ("sign_flip_exp", "double p = exp(z[e] - m) / l;", "double p = exp(m - z[e]) / l;"),
     ("column_major_tokens", "for (int a = ndim - 1; a >= 0; --a) {\n        coord[a]",
      "for (int a = 0; a < ndim; ++a) {\n        coord[a]"),
-    ("mask_upper_inclusive", "kj[a] >= hi[a]) in = 0;", "kj[a] > hi[a]) in = 0;"),
+    ("mask_upper_inclusive", "u >= hi[a]) in = 0;", "u > hi[a]) in = 0;"),
     ("full_partial_swapped", "m == ra * cb ? 2 : 1", "m == ra * cb ? 1 : 2"),
     ("causal_excludes_self", "a = (g + 1) * s - w;", "a = g * s - w;"),
     ("causal_looks_ahead", "a = (g + 1) * s - w;", "a = g * s;"),
@@ -42,6 +42,12 @@ MUTANTS = [
      "J->dv[koff + c] += load_in(J->dout, J->dtype, qoff + c);"),
     ("bwd_dq_unscaled", "g[c] += J->scale * dz * load_in(J->k, J->dtype, koff + (size_t)c);",
      "g[c] += dz * load_in(J->k, J->dtype, koff + (size_t)c);"),
+    ("dilation_floor_length", "const int Lr = (L - res + dil - 1) / dil;",
+     "const int Lr = L / dil;"),
+    ("dilation_residue_ignored", "if (kj[a] % step[a] != res[a]) in = 0;", ""),
+    ("dilation_position_undivided", "na_oracle_window(Lr, w, s, mode, i / dil, lo, hi)",
+     "na_oracle_window(Lr, w, s, mode, i / dil / dil, lo, hi)"),
+    ("dilation_step_one", "const int u = kj[a] / step[a];", "const int u = kj[a];"),
     ("bwd_delta_from_v", "Di += load_in(J->dout, J->dtype, qoff + c) * o[c];",
      "Di += load_in(J->dout, J->dtype, qoff + c) * load_in(J->v, J->dtype, qoff + c);"),
 ]
