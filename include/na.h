@@ -128,6 +128,15 @@ typedef struct {
                                na_sync_status) is exercised without any fault or hang. */
   int window_mode[3];       /* na_window_mode of grid dimension i (i < ndim, the order of
                                `window`); entries from ndim on are ignored.  0 = clamped. */
+  int dilation[3];          /* dilation of grid dimension i (i < ndim); 0 or 1 = none.  The
+                               pages define none; the reading: coordinates split into
+                               `dilation` interleaved residue classes (i mod dilation), and
+                               a query's window is taken inside its own class -- the window
+                               rule above on the class's positions, stride counted in class
+                               positions -- so it attends to keys r + dilation * t.
+                               Needs window[i] * dilation[i] <= grid[i] (else
+                               NA_ERR_INVALID_ARG).  Forward only: na_backward and
+                               na_forward_noalloc return NA_ERR_UNSUPPORTED when set. */
 } na_options;
 
 /* na_options with every field at its default (automatic) value. */
@@ -207,6 +216,8 @@ typedef struct {
   long long dense_pairs;    /* N * N: the pairs of full self attention */
   long long dense_units;    /* (block, chunk) products of full self attention under the
                                same block and chunk shapes */
+  /* With dilation the counts above are sums over the residue classes (each
+     scheduled as a grid of its own); dense_units and speedup_bound are 0. */
   double speedup_bound;     /* dense_units / (units_full + units_partial): the speedup over
                                the same kernel run densely that tile-granular skipping
                                allows at most, a partial tile costing as much as a full

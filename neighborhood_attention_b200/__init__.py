@@ -40,7 +40,7 @@ class na_options(ctypes.Structure):
     _fields_ = [("scale", ctypes.c_float), ("kernel", ctypes.c_int),
                 ("qblock", ctypes.c_int * 3), ("kvchunk", ctypes.c_int * 3),
                 ("wait_timeout_ns", ctypes.c_longlong), ("debug_flags", ctypes.c_int),
-                ("window_mode", ctypes.c_int * 3)]
+                ("window_mode", ctypes.c_int * 3), ("dilation", ctypes.c_int * 3)]
 
 
 class na_plan_info(ctypes.Structure):
@@ -155,10 +155,16 @@ def window_modes(mode, ndim: int):
 
 def make_options(kernel: int = NA_KERNEL_AUTO, scale: float = 0.0, qblock=None, kvchunk=None,
                  wait_timeout_ns: int = 0, debug_flags: int = 0, window_mode=None,
-                 ndim: int | None = None) -> na_options:
+                 ndim: int | None = None, dilation=None) -> na_options:
     """na_options from keyword values; ``window_mode`` as in window_modes()
-    (a single mode needs ``ndim``, or applies to all three slots)."""
+    (a single mode needs ``ndim``, or applies to all three slots);
+    ``dilation``: one int per grid dimension (or one for all of them)."""
     o = na_default_options()
+    if dilation is not None:
+        if isinstance(dilation, int):
+            dilation = [dilation] * (ndim if ndim is not None else 3)
+        for i, x in enumerate(dilation):
+            o.dilation[i] = int(x)
     if window_mode is not None:
         modes = window_modes(window_mode, ndim if ndim is not None else
                              (3 if isinstance(window_mode, (str, int)) else len(window_mode)))
@@ -367,15 +373,21 @@ def na_block_schedule(grid, window, stride, qblock, kvchunk, block: int, max_chu
 
 
 def forward(q, k, v, window, stride=None, tile=None, options=None, stream=None,
-            window_mode=None):
+            window_mode=None, dilation=None):
     """Allocate out / lse with torch and enqueue the forward pass; returns (out, lse).
-    ``window_mode`` (as in window_modes()) overrides options.window_mode."""
+    ``window_mode`` (as in window_modes()) and ``dilation`` (one int per grid
+    dimension) override the corresponding options fields."""
     import torch
-    if window_mode is not None:
+    if window_mode is not None or dilation is not None:
         if options is None:
             options = na_default_options()
+    if window_mode is not None:
         for i, m in enumerate(window_modes(window_mode, len(window))):
             options.window_mode[i] = m
+    if dilation is not None:
+        dl = [dilation] * len(window) if isinstance(dilation, int) else list(dilation)
+        for i, x in enumerate(dl):
+            options.dilation[i] = int(x)
     out = torch.empty_like(q)
     lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
     return na_forward_ex(q, k, v, out, lse, window, stride, tile, options, stream)

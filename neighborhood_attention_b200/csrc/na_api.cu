@@ -38,6 +38,7 @@ int* g_status[MAX_DEVICES] = {nullptr};
 struct Problem {
   int ndim = 0, D = 0;
   Geom g{};
+  int dil[3] = {1, 1, 1};    // dilation per (padded) dimension
   int tile[3] = {0, 0, 0};   // 0 = none given
   int dtype = NA_BF16;
   na_options opt{};
@@ -158,8 +159,33 @@ na_status read_problem(const int dims[2], const int* grid, const int* window, co
     if (m < NA_WINDOW_CLAMPED || m > NA_WINDOW_CAUSAL)
       return fail(NA_ERR_INVALID_ARG, "window_mode[%d]=%d is not a na_window_mode", i, m);
     P.g.m[pad + i] = m;
+    const int dl = P.opt.dilation[i] == 0 ? 1 : P.opt.dilation[i];
+    if (dl < 1)
+      return fail(NA_ERR_INVALID_ARG, "dilation[%d]=%d must be >= 1", i, P.opt.dilation[i]);
+    if ((long long)P.g.w[pad + i] * dl > P.g.L[pad + i])
+      return fail(NA_ERR_INVALID_ARG, "window[%d] * dilation[%d] = %lld exceeds grid[%d]=%d", i,
+                  i, (long long)P.g.w[pad + i] * dl, i, P.g.L[pad + i]);
+    P.dil[pad + i] = dl;
   }
   return NA_OK;
+}
+
+bool dilated(const Problem& P) { return P.dil[0] > 1 || P.dil[1] > 1 || P.dil[2] > 1; }
+
+// Residue class (r0, r1, r2) of a dilated problem as a problem of its own:
+// per dimension the ceil((L - r) / dil) coordinates r, r + dil, ...  The tile
+// hint, which describes the full grid, is dropped.
+Problem residue_problem(const Problem& P, const int r[3], DilMap& map) {
+  Problem Q = P;
+  for (int d = 0; d < 3; ++d) {
+    Q.g.L[d] = (P.g.L[d] - r[d] + P.dil[d] - 1) / P.dil[d];
+    Q.dil[d] = 1;
+    Q.tile[d] = 0;
+    map.dil[d] = P.dil[d];
+    map.res[d] = r[d];
+    map.Lf[d] = P.g.L[d];
+  }
+  return Q;
 }
 
 // Shapes of `prod` tokens (powers of two per dimension, <= 256 each), with
@@ -400,6 +426,165 @@ na_status noalloc_scratch(void** out) {
   return NA_OK;
 }
 
+// Plan and launch the forward kernel for one grid (the whole problem, or one
+// residue class of a dilated one: `map` takes its coordinates to the full
+// grid's tokens).
+na_status launch_forward(const Problem& P, const DilMap& map, long long BH, const void* q,
+                         const void* k, const void* v, void* out, float* lse, void* stream) {
+  Plan plan;
+  na_status st = make_plan(P, plan);
+  if (st != NA_OK) return st;
+  const long long N = (long long)map.Lf[0] * map.Lf[1] * map.Lf[2];   // tokens per head
+  const float scale = P.opt.scale > 0.f ? P.opt.scale : 1.0f / sqrtf((float)P.D);
+  const float log2e = 1.4426950408889634f;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  if (plan.kernel == NA_KERNEL_TC) {
+    int* status = nullptr;
+    st = status_word(&status);
+    if (st != NA_OK) return st;
+    TcLaunch L;
+    L.g = P.g;
+    L.t = plan.t;
+    for (int d = 0; d < 3; ++d) L.kb[d] = plan.kb[d];
+    L.map = map;
+    L.BH = (int)BH;
+    L.N = (int)N;
+    L.D = P.D;
+    L.f16 = P.dtype == NA_F16;
+    L.scale_log2 = scale * log2e;
+    L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
+    L.status = status;
+    L.timeout_ns = P.opt.wait_timeout_ns > 0 ? P.opt.wait_timeout_ns : default_timeout_ns();
+    L.debug_flags = P.opt.debug_flags;
+    char msg[256] = "";
+    cudaError_t e = launch_tc(L, s, msg, sizeof msg);
+    if (e == cudaErrorNotSupported)
+      return fail(NA_ERR_UNSUPPORTED, "tensor-core kernel does not take this shape");
+    if (e != cudaSuccess)
+      return fail(NA_ERR_CUDA, "tensor-core launch: %s %s", cudaGetErrorString(e), msg);
+    return NA_OK;
+  }
+  SimtLaunch L;
+  L.g = P.g;
+  L.t = plan.t;
+  for (int d = 0; d < 3; ++d) L.kb[d] = plan.kb[d];
+  L.map = map;
+  L.BH = (int)BH;
+  L.N = (int)N;
+  L.D = P.D;
+  L.dtype = P.dtype;
+  L.scale_log2 = scale * log2e;
+  L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
+  if (plan.kernel == NA_KERNEL_GATHER) {
+    GatherLaunch G;
+    G.g = P.g;
+    G.map = map;
+    G.BH = (int)BH;
+    G.N = (int)N;
+    G.D = P.D;
+    G.dtype = P.dtype;
+    G.scale_log2 = scale * log2e;
+    G.q = q; G.k = k; G.v = v; G.out = out; G.lse = lse;
+    for (int d = 0; d < 3; ++d) {
+      G.qt[d] = plan.gq[d];
+      G.nt[d] = plan.gq[0] > 0 ? (P.g.L[d] + plan.gq[d] - 1) / plan.gq[d] : 0;
+    }
+    G.smem_bytes = plan.gsmem;
+    cudaError_t e = launch_gather(G, s);
+    if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "window-gather kernel: shape");
+    if (e != cudaSuccess)
+      return fail(NA_ERR_CUDA, "window-gather launch: %s", cudaGetErrorString(e));
+    return NA_OK;
+  }
+  cudaError_t e = launch_simt(L, s);
+  if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "CUDA-core kernel: shape");
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "CUDA-core launch: %s", cudaGetErrorString(e));
+  return NA_OK;
+}
+
+// Schedule statistics of one grid (see na_plan_info).
+na_status plan_info(const Problem& P, na_plan_info* info) {
+  na_status st;
+  Plan plan;
+  st = make_plan(P, plan);
+  if (st != NA_OK) return st;
+  // sum over queries of the window size = product over dimensions of the sum
+  // over coordinates of the 1-D window length (the window is a product).
+  long long useful = 1;
+  for (int d = 0; d < 3; ++d) {
+    long long sum = 0;
+    for (int i = 0; i < P.g.L[d]; ++i) {
+      int lo, hi;
+      window_range(P.g.L[d], P.g.w[d], P.g.s[d], P.g.m[d], i, lo, hi);
+      sum += hi - lo;
+    }
+    useful *= sum;
+  }
+  const long long N = (long long)P.g.L[0] * P.g.L[1] * P.g.L[2];
+  const bool gather = plan.kernel == NA_KERNEL_GATHER;
+  const int group = plan.kernel == NA_KERNEL_TC ? 2 : 1;
+  Cost c{};
+  if (gather) {
+    // one (query, key) pair per unit, exactly the window's keys: no walk needed;
+    // "chunks" loaded = K / V rows staged in shared memory (staged form) or
+    // read per query (direct form)
+    c.full = useful;
+    c.partial = 0;
+    c.loads = plan.gq[0] > 0 ? plan.gstaged : useful;
+  } else {
+    c = walk(P.g, plan.t, plan.kb, group, 0);
+  }
+  memset(info, 0, sizeof *info);
+  info->kernel = plan.kernel;
+  for (int d = 0; d < 3; ++d) {
+    info->qblock[d] = plan.t.qb[d];
+    info->kvchunk[d] = plan.kb[d];
+    info->tile[d] = plan.t.tl[d];
+  }
+  const long long rows = (long long)plan.t.qb[0] * plan.t.qb[1] * plan.t.qb[2];
+  const long long keys = (long long)plan.kb[0] * plan.kb[1] * plan.kb[2];
+  info->query_blocks = plan.t.nblocks;
+  info->ctas = (plan.t.nblocks + group - 1) / group;
+  if (gather) {
+    if (plan.gq[0] > 0) {
+      info->ctas = 1;
+      for (int d = 0; d < 3; ++d) {
+        info->qblock[d] = plan.gq[d];
+        info->tile[d] = plan.gq[d];
+        info->ctas *= (P.g.L[d] + plan.gq[d] - 1) / plan.gq[d];
+      }
+    } else {
+      const long long rpc = gather_rows_per_cta(P.D, P.dtype);
+      info->ctas = (plan.t.nblocks + rpc - 1) / rpc;
+    }
+  }
+  info->chunks_loaded = c.loads;
+  info->units_full = c.full;
+  info->units_partial = c.partial;
+  info->computed_pairs = (c.full + c.partial) * rows * keys;
+  info->useful_pairs = useful;
+  // Speedup bound: dense attention (every window the whole grid) under the
+  // same block / chunk shapes computes every (block, chunk) unit; this
+  // schedule computes only the non-empty ones, each at full tile cost.
+  info->dense_pairs = N * N;
+  if (gather) {
+    info->dense_units = N * N;
+  } else {
+    Geom dense = P.g;
+    for (int d = 0; d < 3; ++d) {
+      dense.w[d] = dense.L[d];
+      dense.s[d] = 1;
+      dense.m[d] = WIN_CLAMPED;
+    }
+    const Cost cd = walk(dense, plan.t, plan.kb, group, 0);
+    info->dense_units = cd.full + cd.partial;
+  }
+  const long long units = c.full + c.partial;
+  info->speedup_bound = units > 0 ? (double)info->dense_units / (double)units : 0.0;
+  return NA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -463,72 +648,18 @@ na_status na_forward_ex(const void* q, const void* k, const void* v, void* out, 
     return fail(NA_ERR_INVALID_ARG, "q, k, v, out must be 16-byte aligned and lse 4-byte aligned");
   const long long BH = (long long)B * heads;
   if (BH > (1LL << 30)) return fail(NA_ERR_UNSUPPORTED, "B*heads too large");
-  Plan plan;
-  st = make_plan(P, plan);
-  if (st != NA_OK) return st;
-  const long long N = (long long)P.g.L[0] * P.g.L[1] * P.g.L[2];
-  const float scale = P.opt.scale > 0.f ? P.opt.scale : 1.0f / sqrtf((float)P.D);
-  const float log2e = 1.4426950408889634f;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-
-  if (plan.kernel == NA_KERNEL_TC) {
-    int* status = nullptr;
-    st = status_word(&status);
-    if (st != NA_OK) return st;
-    TcLaunch L;
-    L.g = P.g;
-    L.t = plan.t;
-    for (int d = 0; d < 3; ++d) L.kb[d] = plan.kb[d];
-    L.BH = (int)BH;
-    L.N = (int)N;
-    L.D = P.D;
-    L.f16 = P.dtype == NA_F16;
-    L.scale_log2 = scale * log2e;
-    L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
-    L.status = status;
-    L.timeout_ns = P.opt.wait_timeout_ns > 0 ? P.opt.wait_timeout_ns : default_timeout_ns();
-    L.debug_flags = P.opt.debug_flags;
-    char msg[256] = "";
-    cudaError_t e = launch_tc(L, s, msg, sizeof msg);
-    if (e == cudaErrorNotSupported)
-      return fail(NA_ERR_UNSUPPORTED, "tensor-core kernel does not take this shape");
-    if (e != cudaSuccess)
-      return fail(NA_ERR_CUDA, "tensor-core launch: %s %s", cudaGetErrorString(e), msg);
-    return NA_OK;
-  }
-  SimtLaunch L;
-  L.g = P.g;
-  L.t = plan.t;
-  for (int d = 0; d < 3; ++d) L.kb[d] = plan.kb[d];
-  L.BH = (int)BH;
-  L.N = (int)N;
-  L.D = P.D;
-  L.dtype = P.dtype;
-  L.scale_log2 = scale * log2e;
-  L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
-  if (plan.kernel == NA_KERNEL_GATHER) {
-    GatherLaunch G;
-    G.g = P.g;
-    G.BH = (int)BH;
-    G.N = (int)N;
-    G.D = P.D;
-    G.dtype = P.dtype;
-    G.scale_log2 = scale * log2e;
-    G.q = q; G.k = k; G.v = v; G.out = out; G.lse = lse;
-    for (int d = 0; d < 3; ++d) {
-      G.qt[d] = plan.gq[d];
-      G.nt[d] = plan.gq[0] > 0 ? (P.g.L[d] + plan.gq[d] - 1) / plan.gq[d] : 0;
-    }
-    G.smem_bytes = plan.gsmem;
-    cudaError_t e = launch_gather(G, s);
-    if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "window-gather kernel: shape");
-    if (e != cudaSuccess)
-      return fail(NA_ERR_CUDA, "window-gather launch: %s", cudaGetErrorString(e));
-    return NA_OK;
-  }
-  cudaError_t e = launch_simt(L, s);
-  if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "CUDA-core kernel: shape");
-  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "CUDA-core launch: %s", cudaGetErrorString(e));
+  if (!dilated(P)) return launch_forward(P, identity_map(P.g.L), BH, q, k, v, out, lse, stream);
+  // One launch per residue class, each a grid of its own (same stream, so
+  // they run in order; each writes only its own class's rows).
+  int r[3];
+  for (r[0] = 0; r[0] < P.dil[0]; ++r[0])
+    for (r[1] = 0; r[1] < P.dil[1]; ++r[1])
+      for (r[2] = 0; r[2] < P.dil[2]; ++r[2]) {
+        DilMap map;
+        const Problem Q = residue_problem(P, r, map);
+        st = launch_forward(Q, map, BH, q, k, v, out, lse, stream);
+        if (st != NA_OK) return st;
+      }
   return NA_OK;
 }
 
@@ -561,6 +692,7 @@ na_status na_backward(const void* q, const void* k, const void* v, const void* o
   const bool tc_ok = (P.dtype == NA_BF16 || P.dtype == NA_F16) && (P.D == 64 || P.D == 128);
   if (P.opt.kernel == NA_KERNEL_GATHER)
     return fail(NA_ERR_UNSUPPORTED, "the window-gather kernel is forward only");
+  if (dilated(P)) return fail(NA_ERR_UNSUPPORTED, "dilation is supported by the forward only");
   if (P.opt.kernel == NA_KERNEL_TC && !tc_ok)
     return fail(NA_ERR_UNSUPPORTED, "the tensor-core backward takes bf16 / f16, head_dim 64 or 128");
   const bool use_tc = tc_ok && P.opt.kernel != NA_KERNEL_SIMT;
@@ -657,82 +789,39 @@ na_status na_plan(const int dims[2], const int* grid, const int* window, const i
   Problem P;
   na_status st = read_problem(dims, grid, window, stride, tile, dtype, opt, P);
   if (st != NA_OK) return st;
-  Plan plan;
-  st = make_plan(P, plan);
-  if (st != NA_OK) return st;
-  // sum over queries of the window size = product over dimensions of the sum
-  // over coordinates of the 1-D window length (the window is a product).
-  long long useful = 1;
-  for (int d = 0; d < 3; ++d) {
-    long long sum = 0;
-    for (int i = 0; i < P.g.L[d]; ++i) {
-      int lo, hi;
-      window_range(P.g.L[d], P.g.w[d], P.g.s[d], P.g.m[d], i, lo, hi);
-      sum += hi - lo;
-    }
-    useful *= sum;
-  }
-  const long long N = (long long)P.g.L[0] * P.g.L[1] * P.g.L[2];
-  const bool gather = plan.kernel == NA_KERNEL_GATHER;
-  const int group = plan.kernel == NA_KERNEL_TC ? 2 : 1;
-  Cost c{};
-  if (gather) {
-    // one (query, key) pair per unit, exactly the window's keys: no walk needed;
-    // "chunks" loaded = K / V rows staged in shared memory (staged form) or
-    // read per query (direct form)
-    c.full = useful;
-    c.partial = 0;
-    c.loads = plan.gq[0] > 0 ? plan.gstaged : useful;
-  } else {
-    c = walk(P.g, plan.t, plan.kb, group, 0);
-  }
-  memset(info, 0, sizeof *info);
-  info->kernel = plan.kernel;
-  for (int d = 0; d < 3; ++d) {
-    info->qblock[d] = plan.t.qb[d];
-    info->kvchunk[d] = plan.kb[d];
-    info->tile[d] = plan.t.tl[d];
-  }
-  const long long rows = (long long)plan.t.qb[0] * plan.t.qb[1] * plan.t.qb[2];
-  const long long keys = (long long)plan.kb[0] * plan.kb[1] * plan.kb[2];
-  info->query_blocks = plan.t.nblocks;
-  info->ctas = (plan.t.nblocks + group - 1) / group;
-  if (gather) {
-    if (plan.gq[0] > 0) {
-      info->ctas = 1;
-      for (int d = 0; d < 3; ++d) {
-        info->qblock[d] = plan.gq[d];
-        info->tile[d] = plan.gq[d];
-        info->ctas *= (P.g.L[d] + plan.gq[d] - 1) / plan.gq[d];
+  if (!dilated(P)) return plan_info(P, info);
+  // Dilated: each residue class is scheduled as a grid of its own; the counts
+  // are summed over the classes.
+  na_plan_info sum;
+  memset(&sum, 0, sizeof sum);
+  bool first = true;
+  int r[3];
+  for (r[0] = 0; r[0] < P.dil[0]; ++r[0])
+    for (r[1] = 0; r[1] < P.dil[1]; ++r[1])
+      for (r[2] = 0; r[2] < P.dil[2]; ++r[2]) {
+        DilMap map;
+        const Problem Q = residue_problem(P, r, map);
+        na_plan_info one;
+        st = plan_info(Q, &one);
+        if (st != NA_OK) return st;
+        if (first) {
+          sum = one;
+          first = false;
+        } else {
+          sum.query_blocks += one.query_blocks;
+          sum.ctas += one.ctas;
+          sum.chunks_loaded += one.chunks_loaded;
+          sum.units_full += one.units_full;
+          sum.units_partial += one.units_partial;
+          sum.computed_pairs += one.computed_pairs;
+          sum.useful_pairs += one.useful_pairs;
+        }
       }
-    } else {
-      const long long rpc = gather_rows_per_cta(P.D, P.dtype);
-      info->ctas = (plan.t.nblocks + rpc - 1) / rpc;
-    }
-  }
-  info->chunks_loaded = c.loads;
-  info->units_full = c.full;
-  info->units_partial = c.partial;
-  info->computed_pairs = (c.full + c.partial) * rows * keys;
-  info->useful_pairs = useful;
-  // Speedup bound: dense attention (every window the whole grid) under the
-  // same block / chunk shapes computes every (block, chunk) unit; this
-  // schedule computes only the non-empty ones, each at full tile cost.
-  info->dense_pairs = N * N;
-  if (gather) {
-    info->dense_units = N * N;
-  } else {
-    Geom dense = P.g;
-    for (int d = 0; d < 3; ++d) {
-      dense.w[d] = dense.L[d];
-      dense.s[d] = 1;
-      dense.m[d] = WIN_CLAMPED;
-    }
-    const Cost cd = walk(dense, plan.t, plan.kb, group, 0);
-    info->dense_units = cd.full + cd.partial;
-  }
-  const long long units = c.full + c.partial;
-  info->speedup_bound = units > 0 ? (double)info->dense_units / (double)units : 0.0;
+  const long long N = (long long)P.g.L[0] * P.g.L[1] * P.g.L[2];
+  sum.dense_pairs = N * N;
+  sum.dense_units = 0;
+  sum.speedup_bound = 0.0;
+  *info = sum;
   return NA_OK;
 }
 
@@ -792,6 +881,8 @@ na_status na_forward_noalloc(const void* q, const void* k, const void* v, void* 
   if (BH > (1LL << 30)) return fail(NA_ERR_UNSUPPORTED, "B*heads too large");
   if (P.opt.kernel == NA_KERNEL_SIMT || P.opt.kernel == NA_KERNEL_GATHER)
     return fail(NA_ERR_UNSUPPORTED, "na_forward_noalloc runs the tensor-core kernel only");
+  if (dilated(P))
+    return fail(NA_ERR_UNSUPPORTED, "na_forward_noalloc takes no dilation (use na_forward_ex)");
   P.opt.kernel = NA_KERNEL_TC;
   Plan plan;
   st = make_plan(P, plan);
@@ -811,6 +902,7 @@ na_status na_forward_noalloc(const void* q, const void* k, const void* v, void* 
   L.g = P.g;
   L.t = plan.t;
   for (int d = 0; d < 3; ++d) L.kb[d] = plan.kb[d];
+  L.map = identity_map(P.g.L);
   L.BH = (int)BH;
   L.N = P.g.L[0] * P.g.L[1] * P.g.L[2];
   L.D = P.D;

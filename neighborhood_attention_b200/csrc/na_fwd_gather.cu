@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(GATHER_THREADS) gather_tile_kernel(const Gathe
   for (int i = threadIdx.x; i < rows * SPR; i += GATHER_THREADS) {
     const int r = i / SPR, sl = i % SPR;
     const int r2 = r % kx[2], r1 = (r / kx[2]) % kx[1], r0 = r / (kx[2] * kx[1]);
-    const size_t tok = ((size_t)(lo[0] + r0) * g.L[1] + (lo[1] + r1)) * g.L[2] + (lo[2] + r2);
+    const size_t tok = (size_t)full_token(P.map, lo[0] + r0, lo[1] + r1, lo[2] + r2);
     const size_t off = (head + tok) * D * ESZ + (size_t)sl * 16;
     const int slot = r * SPR + (sl ^ (r & (SPR - 1)));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(GATHER_THREADS) gather_tile_kernel(const Gathe
     }
     const int W = valid ? n[0] * n[1] * n[2] : 0;
     const int Wmax = __reduce_max_sync(0xffffffffu, W);   // uniform trip count for the shuffles
-    const size_t token = ((size_t)c[0] * g.L[1] + c[1]) * g.L[2] + c[2];
+    const size_t token = (size_t)full_token(P.map, c[0], c[1], c[2]);
     const size_t row_off = (head + token) * D * ESZ + (size_t)part * S * 16;
 
     uint64_t q2[E / 2], acc2[E / 2];
@@ -386,17 +386,19 @@ __global__ void __launch_bounds__(GATHER_THREADS) gather_direct_kernel(const Gat
   static_assert(G >= 4 && G <= 32 && (G & (G - 1)) == 0, "group size");
 
   const Geom& g = P.g;
-  const long long rows = (long long)P.BH * P.N;
+  const long long nsub = (long long)g.L[0] * g.L[1] * g.L[2];   // this grid's tokens per head
+  const long long rows = (long long)P.BH * nsub;
   const long long row = (long long)blockIdx.x * QPC + threadIdx.x / G;
   const int part = threadIdx.x % G;
   const bool valid = row < rows;
   const long long r = valid ? row : 0;
-  const size_t head = (size_t)(r / P.N) * (size_t)P.N;
-  const int token = (int)(r % P.N);
+  const size_t head = (size_t)(r / nsub) * (size_t)P.N;
+  const int sub = (int)(r % nsub);
   int c[3];
-  c[2] = token % g.L[2];
-  c[1] = (token / g.L[2]) % g.L[1];
-  c[0] = token / (g.L[2] * g.L[1]);
+  c[2] = sub % g.L[2];
+  c[1] = (sub / g.L[2]) % g.L[1];
+  c[0] = sub / (g.L[2] * g.L[1]);
+  const size_t token = (size_t)full_token(P.map, c[0], c[1], c[2]);
   int lo[3], n[3];
   for (int d = 0; d < 3; ++d) {
     int hi;
@@ -411,8 +413,7 @@ __global__ void __launch_bounds__(GATHER_THREADS) gather_direct_kernel(const Gat
   load_q<D, T>(P, row_off, qv);
   attend_row<D, T>(qv, W, Wmax, n,
                    [&](int j0, int j1, int j2, uint4& ku, uint4& vu) {
-                     const size_t kt =
-                         ((size_t)(lo[0] + j0) * g.L[1] + (lo[1] + j1)) * g.L[2] + (lo[2] + j2);
+                     const size_t kt = (size_t)full_token(P.map, lo[0] + j0, lo[1] + j1, lo[2] + j2);
                      const size_t off = (head + kt) * D * ESZ + slice;
                      ku = load_slice(P.k, off);
                      vu = load_slice(P.v, off);
@@ -439,7 +440,7 @@ cudaError_t launch_dt(const GatherLaunch& L, cudaStream_t stream) {
     gather_tile_kernel<D, T><<<(unsigned)blocks, GATHER_THREADS, L.smem_bytes, stream>>>(L);
   } else {
     const long long qpc = GATHER_THREADS / (D / slice_elems<T>());
-    const long long rows = (long long)L.BH * L.N;
+    const long long rows = (long long)L.BH * L.g.L[0] * L.g.L[1] * L.g.L[2];
     const long long blocks = (rows + qpc - 1) / qpc;
     if (blocks <= 0 || blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     gather_direct_kernel<D, T><<<(unsigned)blocks, GATHER_THREADS, 0, stream>>>(L);

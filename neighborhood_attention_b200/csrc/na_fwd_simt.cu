@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(SIMT_THREADS) simt_fwd_kernel(const SimtLaunch
     window_range(g.L[d], g.w[d], g.s[d], g.m[d], imin(gc[d], g.L[d] - 1), wlo[d], whi);
     wn[d] = whi - wlo[d];
   }
-  const long long token = ((long long)gc[0] * g.L[1] + gc[1]) * g.L[2] + gc[2];
+  const long long token = full_token(P.map, gc[0], gc[1], gc[2]);
   const size_t head_off = (size_t)bh * (size_t)P.N * D;
 
   float qr[32], acc[32];
@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(SIMT_THREADS) simt_fwd_kernel(const SimtLaunch
       const int x0 = a[0] + k0, x1 = a[1] + k1, x2 = a[2] + k2;
       float kv = 0.f, vv = 0.f;
       if (x0 < g.L[0] && x1 < g.L[1] && x2 < g.L[2]) {
-        const size_t off = head_off + (((size_t)x0 * g.L[1] + x1) * g.L[2] + x2) * D + ch;
+        const size_t off = head_off + (size_t)full_token(P.map, x0, x1, x2) * D + ch;
         kv = load_elem<T>(P.k, off);
         vv = load_elem<T>(P.v, off);
       }

@@ -493,7 +493,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         int g[3];
         query_coord(rr, g);
         const bool valid = B.exists && g[0] < P.g.L[0] && g[1] < P.g.L[1] && g[2] < P.g.L[2];
-        const long long token = ((long long)g[0] * P.g.L[1] + g[1]) * P.g.L[2] + g[2];
+        const long long token = full_token(P.map, g[0], g[1], g[2]);
         const size_t rbase = ((size_t)bh * P.N + (size_t)(valid ? token : 0)) * D;
         const float inv_l = 1.f / l;
         uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(P.out) + rbase);
@@ -540,7 +540,7 @@ __global__ void exp2_poly_selftest_kernel(const float* x, float* y, int n) {
 
 // ------------------------------------------------------------ host side --
 bool encode_map(CUtensorMap* m, const void* ptr, const TcLaunch& L, const int box[3]) {
-  return encode_grid_map(m, ptr, L.f16, L.D, L.g.L, L.BH, L.N, box);
+  return encode_grid_map_dil(m, ptr, L.f16, L.D, L.g.L, L.map, L.BH, L.N, box);
 }
 
 template <int D, bool F16>
@@ -584,6 +584,13 @@ cudaError_t launch_d(const TcLaunch& L, cudaStream_t stream, char* err, int errl
 // 64-element inner box with 128-byte swizzle.
 bool encode_grid_map(CUtensorMap* m, const void* ptr, int f16, int D, const int L[3], int BH,
                      int N, const int box[3]) {
+  return encode_grid_map_dil(m, ptr, f16, D, L, identity_map(L), BH, N, box);
+}
+
+// Residue class of a dilated grid: coordinate x of dimension d steps map.dil[d]
+// tokens of the full grid, and the class starts at token full_token(map, 0, 0, 0).
+bool encode_grid_map_dil(CUtensorMap* m, const void* ptr, int f16, int D, const int L[3],
+                         const DilMap& map, int BH, int N, const int box[3]) {
   static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -598,8 +605,12 @@ bool encode_grid_map(CUtensorMap* m, const void* ptr, int f16, int D, const int 
   const cuuint64_t es = 2;
   cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)L[2], (cuuint64_t)L[1], (cuuint64_t)L[0],
                         (cuuint64_t)BH};
-  cuuint64_t strides[4] = {(cuuint64_t)D * es, (cuuint64_t)L[2] * D * es,
-                           (cuuint64_t)L[1] * L[2] * D * es, (cuuint64_t)N * D * es};
+  const cuuint64_t row = (cuuint64_t)D * es;
+  cuuint64_t strides[4] = {(cuuint64_t)map.dil[2] * row,
+                           (cuuint64_t)map.dil[1] * map.Lf[2] * row,
+                           (cuuint64_t)map.dil[0] * map.Lf[1] * map.Lf[2] * row,
+                           (cuuint64_t)N * row};
+  ptr = static_cast<const char*>(ptr) + (size_t)full_token(map, 0, 0, 0) * row;
   cuuint32_t boxd[5] = {64, (cuuint32_t)box[2], (cuuint32_t)box[1], (cuuint32_t)box[0], 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,

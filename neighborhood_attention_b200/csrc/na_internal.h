@@ -16,7 +16,8 @@ struct SimtLaunch {
   Geom g;
   QTiling t;
   int kb[3];
-  int BH, N, D;
+  DilMap map;            // grid coordinates -> token of the full (undilated) grid
+  int BH, N, D;          // N: tokens per head of the full grid
   int dtype;             // na_dtype of q, k, v and out (fp32, bf16 or f16)
   float scale_log2;      // scale * log2(e)
   const void *q, *k, *v;
@@ -29,7 +30,8 @@ struct TcLaunch {
   QTiling t;
   int kb[3];
   int kb_log2[3];        // filled by launch_tc (chunk extents are powers of two)
-  int BH, N, D;
+  DilMap map;            // grid coordinates -> token of the full (undilated) grid
+  int BH, N, D;          // N: tokens per head of the full grid
   int f16;               // 1: f16 in/out, 0: bf16 in/out
   float scale_log2;
   const void *q, *k, *v;
@@ -80,7 +82,8 @@ inline int gather_rows_per_cta(int D, int dtype) { return 256 / (D / (dtype == 0
 
 struct GatherLaunch {
   Geom g;
-  int BH, N, D;
+  DilMap map;            // grid coordinates -> token of the full (undilated) grid
+  int BH, N, D;          // N: tokens per head of the full grid
   int dtype;             // na_dtype of q, k, v and out
   float scale_log2;      // scale * log2(e)
   const void *q, *k, *v;
@@ -100,6 +103,10 @@ cudaError_t launch_gather(const GatherLaunch& L, cudaStream_t stream);
 // inner box of `box` tokens, 128-byte swizzle.
 bool encode_grid_map(CUtensorMap* m, const void* ptr, int f16, int D, const int L[3], int BH,
                      int N, const int box[3]);
+// The same for a residue class of a dilated grid: the class's coordinates x
+// address token map.res + map.dil * x of the full grid (N tokens per head).
+bool encode_grid_map_dil(CUtensorMap* m, const void* ptr, int f16, int D, const int L[3],
+                         const DilMap& map, int BH, int N, const int box[3]);
 
 cudaError_t launch_simt(const SimtLaunch& L, cudaStream_t stream);
 cudaError_t launch_bwd_simt(const BwdLaunch& L, cudaStream_t stream);

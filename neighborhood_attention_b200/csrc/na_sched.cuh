@@ -67,6 +67,30 @@ struct Geom {
   int m[3];  // WindowMode per dimension
 };
 
+// A dilated problem runs as one grid per residue class: class (r0, r1, r2)
+// holds the coordinates r + dil * x of the full grid (extents Lf), seen as a
+// grid of its own with coordinates x.  full_token maps x back to the full
+// grid's row-major token index.  Undilated: dil 1, res 0, Lf = the grid.
+struct DilMap {
+  int dil[3], res[3], Lf[3];
+};
+
+NA_HD long long full_token(const DilMap& m, int x0, int x1, int x2) {
+  return ((long long)(m.res[0] + m.dil[0] * x0) * m.Lf[1] + (m.res[1] + m.dil[1] * x1)) *
+             m.Lf[2] +
+         (m.res[2] + m.dil[2] * x2);
+}
+
+NA_HD DilMap identity_map(const int L[3]) {
+  DilMap m;
+  for (int d = 0; d < 3; ++d) {
+    m.dil[d] = 1;
+    m.res[d] = 0;
+    m.Lf[d] = L[d];
+  }
+  return m;
+}
+
 // Tiling of the queries: tiles of tl tokens per dim, each split into blocks
 // of qb tokens (qb divides tl).  Blocks are numbered tile by tile, row-major
 // over the tile grid and row-major over the blocks inside a tile, so that

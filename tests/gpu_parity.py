@@ -61,7 +61,7 @@ def run_gpu(c, qkv_host, kernel=0, tile="cfg", qblock=None, kvchunk=None, stream
     import neighborhood_attention_b200 as na
     q, k, v = (to_device(a, c["dtype"]) for a in qkv_host)
     opts = na.make_options(kernel=kernel, qblock=qblock, kvchunk=kvchunk,
-                           window_mode=c.get("mode"), ndim=len(c["grid"]))
+                           window_mode=c.get("mode"), ndim=len(c["grid"]), dilation=c.get("dil"))
     out, lse = na.forward(q, k, v, c["window"], c["stride"], c["tile"] if tile == "cfg" else tile,
                           options=opts, stream=stream)
     na.na_sync_status(stream)
@@ -94,14 +94,14 @@ def compare(c, qkv_host, out_gpu, lse_gpu, rows=None):
     d = c["d"]
     if rows is None:
         ref_o, ref_l = oracle.forward(q, k, v, c["grid"], c["window"], c["stride"], dtype=c["dtype"],
-                                      mode=c.get("mode"))
+                                      mode=c.get("mode"), dilation=c.get("dil"))
         go = out_gpu
         gl = lse_gpu
         ref_o = ref_o.reshape(go.shape)
         ref_l = ref_l.reshape(gl.shape)
     else:
         ref_o, ref_l = oracle.forward(q, k, v, c["grid"], c["window"], c["stride"], dtype=c["dtype"],
-                                      rows=rows, mode=c.get("mode"))
+                                      rows=rows, mode=c.get("mode"), dilation=c.get("dil"))
         go = out_gpu.reshape(-1, d)[rows]
         gl = lse_gpu.reshape(-1)[rows]
     do = np.abs(go - ref_o)

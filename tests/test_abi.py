@@ -162,3 +162,38 @@ def test_gather_selector_is_refused_where_it_does_not_apply(fn):
     assert _fake_call(lib, fn, na.NA_KERNEL_GATHER) == na.NA_ERR_UNSUPPORTED
     lib.na_last_error.restype = ctypes.c_char_p
     assert lib.na_last_error().decode() != ""
+
+
+@pytest.mark.parametrize("dilation,detail", [([0, -1], "dilation[1]"), ([3, 1], "exceeds grid[0]")])
+def test_bad_dilation_is_refused(dilation, detail):
+    import neighborhood_attention_b200 as na
+    opts = na.make_options(dilation=dilation)
+    with pytest.raises(na.NaError) as e:
+        na.na_plan([8, 8], [3, 3], None, None, 64, na.NA_BF16, options=opts)
+    assert e.value.status == na.NA_ERR_INVALID_ARG
+    assert detail in e.value.detail
+
+
+@pytest.mark.parametrize("fn", ["na_backward", "na_forward_noalloc"])
+def test_dilation_is_forward_only(fn):
+    """Dilation runs through na_forward / na_forward_ex only: the backward and
+    the allocation-free entry point refuse it on the host."""
+    import neighborhood_attention_b200 as na
+    lib = ctypes.CDLL(na.LIB_PATH)
+    iv = lambda xs: (ctypes.c_int * len(xs))(*xs)
+    o = na.make_options(dilation=[2, 2])
+    p = ctypes.c_void_p(256)
+    f = getattr(lib, fn)
+    if fn == "na_backward":
+        f.argtypes = [ctypes.c_void_p] * 10 + [ctypes.c_int, ctypes.c_int] + \
+            [ctypes.POINTER(ctypes.c_int)] * 5 + [ctypes.c_int, ctypes.POINTER(na.na_options),
+                                                  ctypes.c_void_p]
+        st = f(*([p] * 10), 1, 1, iv([2, 64]), iv([8, 8]), iv([3, 3]), None, None, 1,
+               ctypes.byref(o), None)
+    else:
+        f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_int] + \
+            [ctypes.POINTER(ctypes.c_int)] * 5 + [ctypes.c_int, ctypes.POINTER(na.na_options),
+                                                  ctypes.c_void_p]
+        st = f(*([p] * 5), 1, 1, iv([2, 64]), iv([8, 8]), iv([3, 3]), None, None, 1,
+               ctypes.byref(o), None)
+    assert st == na.NA_ERR_UNSUPPORTED

@@ -162,3 +162,25 @@ def test_speedup_bound_simulator(oracle_lib):
     assert p["dense_units"] == e + part + full == 64
     assert p["units_full"] + p["units_partial"] == part + full == 8
     assert p["speedup_bound"] == pytest.approx(8.0)
+
+
+@pytest.mark.parametrize("grid,window,stride,modes,dil", [
+    ([13, 10], [3, 2], [1, 2], ["clamped", "truncated"], [3, 2]),
+    ([50], [5], [1], ["causal"], [4]),
+    ([7, 9, 11], [2, 3, 3], [1, 1, 3], None, [2, 3, 2]),
+])
+@pytest.mark.parametrize("kernel", ["auto", "tc", "simt", "gather"])
+def test_plan_with_dilation_counts_the_oracles_pairs(grid, window, stride, modes, dil, kernel,
+                                                     oracle_lib):
+    """A dilated problem is scheduled one residue class at a time; the summed
+    useful pairs equal the pairs of the oracle's dilated masks."""
+    sel = {"auto": na.NA_KERNEL_AUTO, "tc": na.NA_KERNEL_TC, "simt": na.NA_KERNEL_SIMT,
+           "gather": na.NA_KERNEL_GATHER}[kernel]
+    opts = na.make_options(kernel=sel, window_mode=modes, ndim=len(grid), dilation=dil)
+    p = na.na_plan(grid, window, stride, None, 64, na.NA_BF16, options=opts)
+    N = int(np.prod(grid))
+    expect = sum(int(oracle_lib.mask_row(grid, window, stride, t, mode=modes, dilation=dil).sum())
+                 for t in range(N))
+    assert p["useful_pairs"] == expect
+    assert p["computed_pairs"] >= expect
+    assert p["speedup_bound"] == 0.0 and p["dense_pairs"] == N * N
