@@ -82,6 +82,11 @@ class OracleLib:
             ctypes.c_longlong, ctypes.c_int, i32p, i32p, i32p, i32p, ctypes.c_int, ctypes.c_double,
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
         lib.na_oracle_backward.restype = ctypes.c_int
+        lib.na_oracle_backward_dil.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+            ctypes.c_longlong, ctypes.c_int, i32p, i32p, i32p, i32p, i32p, ctypes.c_int,
+            ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        lib.na_oracle_backward_dil.restype = ctypes.c_int
         lib.na_oracle_backward_sampled.argtypes = [
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
             ctypes.c_longlong, ctypes.c_longlong, ctypes.c_int, i32p, i32p, i32p, i32p,
@@ -191,7 +196,7 @@ class OracleLib:
         return out, lse
 
     def backward(self, q, k, v, dout, grid, window, stride, *, dtype: str, scale: float = 0.0,
-                 threads: int | None = None, mode=None):
+                 threads: int | None = None, mode=None, dilation=None):
         """Exact gradients (dq, dk, dv) in fp64 for upstream gradient dout.
 
         q, k, v, dout: arrays of shape [B, heads, *grid, d] in the encoding of
@@ -212,10 +217,11 @@ class OracleLib:
         BH = shape[0] * shape[1]
         d = shape[-1]
         outs = [np.empty(shape, dtype=np.float64) for _ in range(3)]
-        rc = self.lib.na_oracle_backward(
+        rc = self.lib.na_oracle_backward_dil(
             arrs[0].ctypes.data, arrs[1].ctypes.data, arrs[2].ctypes.data, arrs[3].ctypes.data,
             code, BH, nd, self._ivec(grid), self._ivec(window), self._ivec(stride),
-            self._ivec(_modes(mode, nd)), d, float(scale), outs[0].ctypes.data,
+            self._ivec(_modes(mode, nd)), self._ivec(_dil(dilation, nd)), d, float(scale),
+            outs[0].ctypes.data,
             outs[1].ctypes.data, outs[2].ctypes.data, int(threads or os.cpu_count() or 1))
         if rc:
             raise RuntimeError(f"na_oracle_backward failed with code {rc}")

@@ -377,6 +377,7 @@ typedef struct {
     double scale;
     long long bh_begin, bh_end;
     double *dq, *dk, *dv;
+    const int* dil;
     int status;
 } bwd_job;
 
@@ -393,7 +394,8 @@ static void* bwd_worker(void* arg) {
     for (long long bh = J->bh_begin; bh < J->bh_end; ++bh) {
         const size_t hoff = (size_t)bh * (size_t)N * (size_t)d;
         for (long long t = 0; t < N; ++t) {
-            const long long inwin = na_oracle_mask_row(J->ndim, J->L, J->w, J->s, J->mode, t, mask);
+            const long long inwin =
+                na_oracle_mask_row_dil(J->ndim, J->L, J->w, J->s, J->mode, J->dil, t, mask);
             const size_t qoff = hoff + (size_t)t * (size_t)d;
             long long cnt = 0;
             for (long long j = 0; j < N; ++j) {
@@ -449,18 +451,19 @@ done:
 /*
  * Gradients of the forward pass for upstream gradient dout (same layout and
  * dtype as q): dq, dk, dv are [BH, N, d] fp64 (written).  mode: per-dimension
- * window modes or NULL (all clamped).  scale <= 0 means 1/sqrt(d).  Threads
- * split the BH (batch, head) slices, so dk and dv need no reduction across
- * threads.  Returns 0 or a negative code as na_oracle_forward.
+ * window modes or NULL (all clamped); dil: per-dimension dilation or NULL.
+ * scale <= 0 means 1/sqrt(d).  Threads split the BH (batch, head) slices, so
+ * dk and dv need no reduction across threads.  Returns 0 or a negative code
+ * as na_oracle_forward.
  */
-int na_oracle_backward(const void* q, const void* k, const void* v, const void* dout, int in_dtype,
-                       long long BH, int ndim, const int* L, const int* w, const int* s,
-                       const int* mode, int d, double scale, double* dq, double* dk, double* dv,
-                       int nthreads) {
+int na_oracle_backward_dil(const void* q, const void* k, const void* v, const void* dout,
+                           int in_dtype, long long BH, int ndim, const int* L, const int* w,
+                           const int* s, const int* mode, const int* dil, int d, double scale,
+                           double* dq, double* dk, double* dv, int nthreads) {
     long long N;
     if (!q || !k || !v || !dout || !dq || !dk || !dv || BH < 1 || d < 1) return -1;
     if (in_dtype != IN_F32 && in_dtype != IN_BF16 && in_dtype != IN_F16) return -1;
-    if (check_geometry(ndim, L, w, s, mode, NULL, &N)) return -1;
+    if (check_geometry(ndim, L, w, s, mode, dil, &N)) return -1;
     long long W = 1;
     for (int a = 0; a < ndim; ++a) W *= w[a];
     if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
@@ -482,6 +485,7 @@ int na_oracle_backward(const void* q, const void* k, const void* v, const void* 
         J->bh_begin = per * t < BH ? per * t : BH;
         J->bh_end = per * (t + 1) < BH ? per * (t + 1) : BH;
         J->dq = dq; J->dk = dk; J->dv = dv;
+        J->dil = dil;
         J->status = 0;
     }
     for (int t = 1; t < nthreads; ++t)
@@ -495,6 +499,14 @@ int na_oracle_backward(const void* q, const void* k, const void* v, const void* 
     for (int t = 0; t < nthreads; ++t)
         if (jobs[t].status) return jobs[t].status;
     return 0;
+}
+
+int na_oracle_backward(const void* q, const void* k, const void* v, const void* dout, int in_dtype,
+                       long long BH, int ndim, const int* L, const int* w, const int* s,
+                       const int* mode, int d, double scale, double* dq, double* dk, double* dv,
+                       int nthreads) {
+    return na_oracle_backward_dil(q, k, v, dout, in_dtype, BH, ndim, L, w, s, mode, NULL, d, scale,
+                                  dq, dk, dv, nthreads);
 }
 
 /*

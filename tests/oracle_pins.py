@@ -547,6 +547,24 @@ def pin_dilated_residue_subgrids(lib):
                 np.testing.assert_allclose(lse[sl[:4]], l2, atol=1e-13, rtol=0)
 
 
+def pin_dilated_backward_subgrids(lib):
+    """The gradients of dilated attention are those of undilated attention on
+    each residue-class sub-grid (the sub-grids do not interact)."""
+    d = 6
+    grid, window, stride, modes, dil = [11, 9], [3, 2], [1, 1], ["truncated", "causal"], [2, 3]
+    q, k, v, do = (_randn(330 + t, (1, 2, *grid, d)) for t in range(4))
+    dq, dk, dv = lib.backward(q, k, v, do, grid, window, stride, dtype="f32", mode=modes,
+                              dilation=dil)
+    for r0 in range(dil[0]):
+        for r1 in range(dil[1]):
+            sl = (slice(None), slice(None), slice(r0, None, dil[0]), slice(r1, None, dil[1]))
+            qs, ks, vs, ds = (np.ascontiguousarray(a[sl]) for a in (q, k, v, do))
+            g2 = lib.backward(qs, ks, vs, ds, list(qs.shape[2:4]), window, stride, dtype="f32",
+                              mode=modes)
+            for a, b in zip((dq, dk, dv), g2):
+                np.testing.assert_allclose(a[sl], b, atol=1e-12, rtol=0)
+
+
 def pin_sa_empty_blocks_golden(lib):
     """The Hilbert page's empty-block ratio for row-major slide attention
     (Table 3, SA (Flex) at 96x96) reproduces from the truncated window."""
@@ -663,6 +681,7 @@ ALL_PINS = [
     pin_sa_empty_blocks_golden, pin_f16_decoding, pin_backward_finite_differences,
     pin_backward_full_attention_autograd, pin_backward_invariants, pin_backward_sampled_rows,
     pin_dilated_window_bruteforce, pin_dilated_mask_bruteforce, pin_dilated_residue_subgrids,
+    pin_dilated_backward_subgrids,
 ]
 
 # The golden-file pins take a few seconds each; mutant runs use the fast ones.

@@ -48,6 +48,8 @@ MUTANTS = [
     ("dilation_position_undivided", "na_oracle_window(Lr, w, s, mode, i / dil, lo, hi)",
      "na_oracle_window(Lr, w, s, mode, i / dil / dil, lo, hi)"),
     ("dilation_step_one", "const int u = kj[a] / step[a];", "const int u = kj[a];"),
+    ("bwd_dilation_ignored", "J->mode, J->dil, t, mask);\n            const size_t qoff",
+     "J->mode, NULL, t, mask);\n            const size_t qoff"),
     ("bwd_delta_from_v", "Di += load_in(J->dout, J->dtype, qoff + c) * o[c];",
      "Di += load_in(J->dout, J->dtype, qoff + c) * load_in(J->v, J->dtype, qoff + c);"),
 ]
