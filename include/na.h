@@ -135,8 +135,9 @@ typedef struct {
                                rule above on the class's positions, stride counted in class
                                positions -- so it attends to keys r + dilation * t.
                                Needs window[i] * dilation[i] <= grid[i] (else
-                               NA_ERR_INVALID_ARG).  Forward only: na_backward and
-                               na_forward_noalloc return NA_ERR_UNSUPPORTED when set. */
+                               NA_ERR_INVALID_ARG).  na_forward_ex and na_backward run one
+                               launch per residue class; na_forward_noalloc returns
+                               NA_ERR_UNSUPPORTED when it is set. */
 } na_options;
 
 /* na_options with every field at its default (automatic) value. */

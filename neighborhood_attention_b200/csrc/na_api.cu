@@ -692,70 +692,105 @@ na_status na_backward(const void* q, const void* k, const void* v, const void* o
   const bool tc_ok = (P.dtype == NA_BF16 || P.dtype == NA_F16) && (P.D == 64 || P.D == 128);
   if (P.opt.kernel == NA_KERNEL_GATHER)
     return fail(NA_ERR_UNSUPPORTED, "the window-gather kernel is forward only");
-  if (dilated(P)) return fail(NA_ERR_UNSUPPORTED, "dilation is supported by the forward only");
   if (P.opt.kernel == NA_KERNEL_TC && !tc_ok)
     return fail(NA_ERR_UNSUPPORTED, "the tensor-core backward takes bf16 / f16, head_dim 64 or 128");
   const bool use_tc = tc_ok && P.opt.kernel != NA_KERNEL_SIMT;
-  Plan tc_plan;
+  const float scale = P.opt.scale > 0.f ? P.opt.scale : 1.0f / sqrtf((float)P.D);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* status = nullptr;
   if (use_tc) {
-    Problem Pt = P;
-    Pt.opt.kernel = NA_KERNEL_TC;
-    st = make_plan(Pt, tc_plan);
+    st = status_word(&status);
     if (st != NA_OK) return st;
   }
-  P.opt.kernel = NA_KERNEL_SIMT;
-  P.opt.qblock[0] = P.opt.qblock[1] = P.opt.qblock[2] = 0;   // shapes of the TC plan do not fit
-  P.opt.kvchunk[0] = P.opt.kvchunk[1] = P.opt.kvchunk[2] = 0;
-  Plan plan;
-  st = make_plan(P, plan);
-  if (st != NA_OK) return st;
-  const float scale = P.opt.scale > 0.f ? P.opt.scale : 1.0f / sqrtf((float)P.D);
-  BwdLaunch L;
-  L.g = P.g;
-  L.t = plan.t;
-  for (int d = 0; d < 3; ++d) L.kb[d] = plan.kb[d];
-  L.BH = (int)BH;
-  L.N = P.g.L[0] * P.g.L[1] * P.g.L[2];
-  L.D = P.D;
-  L.dtype = P.dtype;
-  L.scale = scale;
-  L.scale_log2 = scale * 1.4426950408889634f;
-  L.q = q; L.k = k; L.v = v; L.out = out; L.dout = dout; L.lse = lse; L.delta = delta;
-  L.dq = dq; L.dk = dk; L.dv = dv;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (!use_tc) {
-    cudaError_t e = launch_bwd_simt(L, s);
-    if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "backward: shape");
-    if (e != cudaSuccess) return fail(NA_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
+  // One grid (a dilated problem: each residue class as a grid of its own,
+  // `map` taking its coordinates to full-grid tokens) -> its launch structs.
+  auto simt_launch = [&](const Problem& Q, const DilMap& map, BwdLaunch& L) -> na_status {
+    Problem Qs = Q;
+    Qs.opt.kernel = NA_KERNEL_SIMT;
+    Qs.opt.qblock[0] = Qs.opt.qblock[1] = Qs.opt.qblock[2] = 0;   // a TC plan's shapes do not fit
+    Qs.opt.kvchunk[0] = Qs.opt.kvchunk[1] = Qs.opt.kvchunk[2] = 0;
+    Plan plan;
+    const na_status r = make_plan(Qs, plan);
+    if (r != NA_OK) return r;
+    L.g = Q.g;
+    L.t = plan.t;
+    for (int d = 0; d < 3; ++d) L.kb[d] = plan.kb[d];
+    L.map = map;
+    L.BH = (int)BH;
+    L.N = map.Lf[0] * map.Lf[1] * map.Lf[2];
+    L.D = Q.D;
+    L.dtype = Q.dtype;
+    L.scale = scale;
+    L.scale_log2 = scale * 1.4426950408889634f;
+    L.q = q; L.k = k; L.v = v; L.out = out; L.dout = dout; L.lse = lse; L.delta = delta;
+    L.dq = dq; L.dk = dk; L.dv = dv;
     return NA_OK;
+  };
+  auto grads = [&](const Problem& Q, const DilMap& map) -> na_status {
+    BwdLaunch L;
+    na_status r = simt_launch(Q, map, L);
+    if (r != NA_OK) return r;
+    if (!use_tc) {
+      const cudaError_t e = launch_bwd_simt_grads(L, s);
+      if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "backward: shape");
+      if (e != cudaSuccess) return fail(NA_ERR_CUDA, "backward launch: %s", cudaGetErrorString(e));
+      return NA_OK;
+    }
+    Problem Qt = Q;
+    Qt.opt.kernel = NA_KERNEL_TC;
+    Plan tc_plan;
+    r = make_plan(Qt, tc_plan);
+    if (r != NA_OK) return r;
+    TcBwdLaunch T;
+    T.g = Q.g;
+    T.t = tc_plan.t;
+    for (int d = 0; d < 3; ++d) T.kb[d] = tc_plan.kb[d];
+    T.map = map;
+    T.BH = (int)BH;
+    T.N = L.N;
+    T.D = Q.D;
+    T.f16 = Q.dtype == NA_F16;
+    T.scale = scale;
+    T.scale_log2 = L.scale_log2;
+    T.q = q; T.k = k; T.v = v; T.dout = dout; T.lse = lse; T.delta = delta;
+    T.dq = dq; T.dk = dk; T.dv = dv;
+    T.status = status;
+    T.timeout_ns = Q.opt.wait_timeout_ns > 0 ? Q.opt.wait_timeout_ns : default_timeout_ns();
+    char msg[256] = "";
+    cudaError_t e = launch_tc_bwd_dq(T, s, msg, sizeof msg);
+    if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "tensor-core dq: shape");
+    if (e != cudaSuccess)
+      return fail(NA_ERR_CUDA, "tensor-core dq: %s %s", cudaGetErrorString(e), msg);
+    e = launch_tc_bwd_dkdv(T, s, msg, sizeof msg);
+    if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "tensor-core dk/dv: shape");
+    if (e != cudaSuccess)
+      return fail(NA_ERR_CUDA, "tensor-core dk/dv: %s %s", cudaGetErrorString(e), msg);
+    return NA_OK;
+  };
+
+  // D_i = <dout_i, out_i> for every row of the full grid, once.
+  {
+    Problem Pu = P;
+    for (int d = 0; d < 3; ++d) {
+      Pu.dil[d] = 1;
+      Pu.tile[d] = dilated(P) ? 0 : P.tile[d];
+    }
+    BwdLaunch L;
+    st = simt_launch(Pu, identity_map(P.g.L), L);
+    if (st != NA_OK) return st;
+    const cudaError_t e = launch_bwd_simt_delta(L, s);
+    if (e != cudaSuccess) return fail(NA_ERR_CUDA, "backward delta: %s", cudaGetErrorString(e));
   }
-  int* status = nullptr;
-  st = status_word(&status);
-  if (st != NA_OK) return st;
-  cudaError_t e = launch_bwd_simt_delta(L, s);
-  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "backward delta: %s", cudaGetErrorString(e));
-  TcBwdLaunch T;
-  T.g = P.g;
-  T.t = tc_plan.t;
-  for (int d = 0; d < 3; ++d) T.kb[d] = tc_plan.kb[d];
-  T.BH = (int)BH;
-  T.N = L.N;
-  T.D = P.D;
-  T.f16 = P.dtype == NA_F16;
-  T.scale = scale;
-  T.scale_log2 = L.scale_log2;
-  T.q = q; T.k = k; T.v = v; T.dout = dout; T.lse = lse; T.delta = delta;
-  T.dq = dq; T.dk = dk; T.dv = dv;
-  T.status = status;
-  T.timeout_ns = P.opt.wait_timeout_ns > 0 ? P.opt.wait_timeout_ns : default_timeout_ns();
-  char msg[256] = "";
-  e = launch_tc_bwd_dq(T, s, msg, sizeof msg);
-  if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "tensor-core dq: shape");
-  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "tensor-core dq: %s %s", cudaGetErrorString(e), msg);
-  e = launch_tc_bwd_dkdv(T, s, msg, sizeof msg);
-  if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "tensor-core dk/dv: shape");
-  if (e != cudaSuccess)
-    return fail(NA_ERR_CUDA, "tensor-core dk/dv: %s %s", cudaGetErrorString(e), msg);
+  if (!dilated(P)) return grads(P, identity_map(P.g.L));
+  int r[3];
+  for (r[0] = 0; r[0] < P.dil[0]; ++r[0])
+    for (r[1] = 0; r[1] < P.dil[1]; ++r[1])
+      for (r[2] = 0; r[2] < P.dil[2]; ++r[2]) {
+        DilMap map;
+        const Problem Q = residue_problem(P, r, map);
+        st = grads(Q, map);
+        if (st != NA_OK) return st;
+      }
   return NA_OK;
 }
 

@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_dq_kernel(const BwdLaunch P) 
     window_range(g.L[d], g.w[d], g.s[d], g.m[d], imin(r[d], g.L[d] - 1), wlo[d], whi);
     wn[d] = whi - wlo[d];
   }
-  const long long token = ((long long)r[0] * g.L[1] + r[1]) * g.L[2] + r[2];
+  const long long token = full_token(P.map, r[0], r[1], r[2]);
   const size_t head = (size_t)bh * (size_t)P.N * D;
   const size_t rowoff = head + (size_t)(valid ? token : 0) * D + gg * 32;
   float qr[32], dor[32], dq[32];
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_dq_kernel(const BwdLaunch P) 
       const int x0 = a[0] + k0, x1 = a[1] + k1, x2 = a[2] + k2;
       float kv = 0.f, vv = 0.f;
       if (x0 < g.L[0] && x1 < g.L[1] && x2 < g.L[2]) {
-        const size_t off = head + (((size_t)x0 * g.L[1] + x1) * g.L[2] + x2) * D + ch;
+        const size_t off = head + (size_t)full_token(P.map, x0, x1, x2) * D + ch;
         kv = ld<T>(P.k, off);
         vv = ld<T>(P.v, off);
       }
@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_dkdv_kernel(const BwdLaunch P
   bool kvalid = ki < KPB;
   for (int d = 0; d < 3; ++d)
     if (kx[d] >= g.L[d]) kvalid = false;
-  const long long ktok = ((long long)kx[0] * g.L[1] + kx[1]) * g.L[2] + kx[2];
+  const long long ktok = full_token(P.map, kx[0], kx[1], kx[2]);
   const size_t head = (size_t)bh * (size_t)P.N * D;
   const size_t koff = head + (size_t)(kvalid ? ktok : 0) * D + gg * 32;
   float kr[32], vr[32], dk[32], dv[32];
@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(BWD_THREADS) bwd_dkdv_kernel(const BwdLaunch P
       const int x0 = a[0] + q0, x1 = a[1] + q1, x2 = a[2] + q2;
       float qv = 0.f, ov = 0.f;
       const bool in = x0 < g.L[0] && x1 < g.L[1] && x2 < g.L[2];
-      const long long qt = ((long long)x0 * g.L[1] + x1) * g.L[2] + x2;
+      const long long qt = full_token(P.map, x0, x1, x2);
       if (in) {
         const size_t off = head + (size_t)qt * D + ch;
         qv = ld<T>(P.q, off);
@@ -369,6 +369,9 @@ cudaError_t launch_bwd_simt_delta(const BwdLaunch& L, cudaStream_t stream) {
 }
 cudaError_t launch_bwd_simt_dkdv(const BwdLaunch& L, cudaStream_t stream) {
   return launch_which(L, stream, RUN_DKDV);
+}
+cudaError_t launch_bwd_simt_grads(const BwdLaunch& L, cudaStream_t stream) {
+  return launch_which(L, stream, RUN_DQ | RUN_DKDV);
 }
 
 }  // namespace na

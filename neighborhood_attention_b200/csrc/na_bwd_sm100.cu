@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
                      whi[d]);
       const bool valid = gc[0] < P.g.L[0] && gc[1] < P.g.L[1] && gc[2] < P.g.L[2];
       if (Bl.exists && valid) {
-        const long long token = ((long long)gc[0] * P.g.L[1] + gc[1]) * P.g.L[2] + gc[2];
+        const long long token = full_token(P.map, gc[0], gc[1], gc[2]);
         lse2 = P.lse[(size_t)bh * P.N + token] * BT_LOG2E;
         Di = P.delta[(size_t)bh * P.N + token];
       }
@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
         int gc[3];
         query_coord(rr, gc);
         const bool valid = gc[0] < P.g.L[0] && gc[1] < P.g.L[1] && gc[2] < P.g.L[2];
-        const long long token = ((long long)gc[0] * P.g.L[1] + gc[1]) * P.g.L[2] + gc[2];
+        const long long token = full_token(P.map, gc[0], gc[1], gc[2]);
         const size_t rbase = ((size_t)bh * P.N + (size_t)(valid ? token : 0)) * D + h * (D / 2);
         uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(P.dq) + rbase);
         const float sc = P.scale;
@@ -536,7 +536,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
           const int x0 = it.a[0] + q0, x1 = it.a[1] + q1, x2 = it.a[2] + q2;
           float l2 = 0.f, dl = 0.f;
           if (x0 < P.g.L[0] && x1 < P.g.L[1] && x2 < P.g.L[2]) {
-            const size_t tok = ((size_t)x0 * P.g.L[1] + x1) * P.g.L[2] + x2;
+            const size_t tok = (size_t)full_token(P.map, x0, x1, x2);
             l2 = P.lse[(size_t)bh * P.N + tok] * BT_LOG2E;
             dl = P.delta[(size_t)bh * P.N + tok];
           }
@@ -745,7 +745,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
         int gc[3];
         key_coord(rr, gc);
         const bool valid = gc[0] < P.g.L[0] && gc[1] < P.g.L[1] && gc[2] < P.g.L[2];
-        const long long token = ((long long)gc[0] * P.g.L[1] + gc[1]) * P.g.L[2] + gc[2];
+        const long long token = full_token(P.map, gc[0], gc[1], gc[2]);
         const size_t rbase = ((size_t)bh * P.N + (size_t)(valid ? token : 0)) * D + h * (D / 2);
         for (int which = 0; which < 2; ++which) {
           uint4* orow = reinterpret_cast<uint4*>(
@@ -782,7 +782,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       key_coord(rr, gc);
       const bool valid = gc[0] < P.g.L[0] && gc[1] < P.g.L[1] && gc[2] < P.g.L[2];
       if (valid) {
-        const long long token = ((long long)gc[0] * P.g.L[1] + gc[1]) * P.g.L[2] + gc[2];
+        const long long token = full_token(P.map, gc[0], gc[1], gc[2]);
         const size_t rbase = ((size_t)bh * P.N + (size_t)token) * D + h * (D / 2);
         for (int which = 0; which < 2; ++which) {
           uint4* orow = reinterpret_cast<uint4*>(
@@ -804,10 +804,10 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
 template <int D, bool F16>
 cudaError_t launch_dkdv_d(const TcBwdLaunch& L, cudaStream_t stream, char* err, int errlen) {
   CUtensorMap mk, mv, mq, mdo;
-  if (!encode_grid_map(&mk, L.k, L.f16, L.D, L.g.L, L.BH, L.N, L.t.qb) ||
-      !encode_grid_map(&mv, L.v, L.f16, L.D, L.g.L, L.BH, L.N, L.t.qb) ||
-      !encode_grid_map(&mq, L.q, L.f16, L.D, L.g.L, L.BH, L.N, L.kb) ||
-      !encode_grid_map(&mdo, L.dout, L.f16, L.D, L.g.L, L.BH, L.N, L.kb)) {
+  if (!encode_grid_map_dil(&mk, L.k, L.f16, L.D, L.g.L, L.map, L.BH, L.N, L.t.qb) ||
+      !encode_grid_map_dil(&mv, L.v, L.f16, L.D, L.g.L, L.map, L.BH, L.N, L.t.qb) ||
+      !encode_grid_map_dil(&mq, L.q, L.f16, L.D, L.g.L, L.map, L.BH, L.N, L.kb) ||
+      !encode_grid_map_dil(&mdo, L.dout, L.f16, L.D, L.g.L, L.map, L.BH, L.N, L.kb)) {
     snprintf(err, errlen, "cuTensorMapEncodeTiled failed (pointer alignment or shape)");
     return cudaErrorInvalidValue;
   }
@@ -838,10 +838,10 @@ cudaError_t launch_dkdv_d(const TcBwdLaunch& L, cudaStream_t stream, char* err, 
 template <int D, bool F16>
 cudaError_t launch_dq_d(const TcBwdLaunch& L, cudaStream_t stream, char* err, int errlen) {
   CUtensorMap mq, mdo, mk, mv;
-  if (!encode_grid_map(&mq, L.q, L.f16, L.D, L.g.L, L.BH, L.N, L.t.qb) ||
-      !encode_grid_map(&mdo, L.dout, L.f16, L.D, L.g.L, L.BH, L.N, L.t.qb) ||
-      !encode_grid_map(&mk, L.k, L.f16, L.D, L.g.L, L.BH, L.N, L.kb) ||
-      !encode_grid_map(&mv, L.v, L.f16, L.D, L.g.L, L.BH, L.N, L.kb)) {
+  if (!encode_grid_map_dil(&mq, L.q, L.f16, L.D, L.g.L, L.map, L.BH, L.N, L.t.qb) ||
+      !encode_grid_map_dil(&mdo, L.dout, L.f16, L.D, L.g.L, L.map, L.BH, L.N, L.t.qb) ||
+      !encode_grid_map_dil(&mk, L.k, L.f16, L.D, L.g.L, L.map, L.BH, L.N, L.kb) ||
+      !encode_grid_map_dil(&mv, L.v, L.f16, L.D, L.g.L, L.map, L.BH, L.N, L.kb)) {
     snprintf(err, errlen, "cuTensorMapEncodeTiled failed (pointer alignment or shape)");
     return cudaErrorInvalidValue;
   }

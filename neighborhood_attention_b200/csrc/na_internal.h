@@ -47,7 +47,8 @@ struct BwdLaunch {
   Geom g;
   QTiling t;             // query blocks (dQ) and key blocks (dK, dV)
   int kb[3];             // key chunks (dQ) and query chunks (dK, dV), 32 tokens
-  int BH, N, D;
+  DilMap map;            // grid coordinates -> token of the full (undilated) grid
+  int BH, N, D;          // N: tokens per head of the full grid
   int dtype;             // na_dtype of q, k, v, out, dout and the gradients
   float scale;           // softmax scale
   float scale_log2;      // scale * log2(e)
@@ -64,7 +65,8 @@ struct TcBwdLaunch {
   QTiling t;             // query blocks (128 tokens)
   int kb[3];             // key chunks (128 tokens)
   int kb_log2[3];        // filled by the launcher
-  int BH, N, D;
+  DilMap map;            // grid coordinates -> token of the full (undilated) grid
+  int BH, N, D;          // N: tokens per head of the full grid
   int f16;               // 1: f16, 0: bf16
   float scale, scale_log2;
   const void *q, *k, *v, *dout;
@@ -113,6 +115,7 @@ cudaError_t launch_bwd_simt(const BwdLaunch& L, cudaStream_t stream);
 // The row-delta and dK/dV CUDA-core kernels alone (the dQ kernel left out).
 cudaError_t launch_bwd_simt_delta(const BwdLaunch& L, cudaStream_t stream);
 cudaError_t launch_bwd_simt_dkdv(const BwdLaunch& L, cudaStream_t stream);
+cudaError_t launch_bwd_simt_grads(const BwdLaunch& L, cudaStream_t stream);   // dq, dk, dv
 cudaError_t launch_tc_bwd_dq(const TcBwdLaunch& L, cudaStream_t stream, char* err, int errlen);
 cudaError_t launch_tc_bwd_dkdv(const TcBwdLaunch& L, cudaStream_t stream, char* err, int errlen);
 

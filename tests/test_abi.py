@@ -174,26 +174,18 @@ def test_bad_dilation_is_refused(dilation, detail):
     assert detail in e.value.detail
 
 
-@pytest.mark.parametrize("fn", ["na_backward", "na_forward_noalloc"])
-def test_dilation_is_forward_only(fn):
-    """Dilation runs through na_forward / na_forward_ex only: the backward and
-    the allocation-free entry point refuse it on the host."""
+def test_allocation_free_entry_refuses_dilation():
+    """na_forward_noalloc runs one tensor-core launch; dilation (one launch per
+    residue class) is refused on the host."""
     import neighborhood_attention_b200 as na
     lib = ctypes.CDLL(na.LIB_PATH)
     iv = lambda xs: (ctypes.c_int * len(xs))(*xs)
     o = na.make_options(dilation=[2, 2])
-    p = ctypes.c_void_p(256)
-    f = getattr(lib, fn)
-    if fn == "na_backward":
-        f.argtypes = [ctypes.c_void_p] * 10 + [ctypes.c_int, ctypes.c_int] + \
-            [ctypes.POINTER(ctypes.c_int)] * 5 + [ctypes.c_int, ctypes.POINTER(na.na_options),
-                                                  ctypes.c_void_p]
-        st = f(*([p] * 10), 1, 1, iv([2, 64]), iv([8, 8]), iv([3, 3]), None, None, 1,
-               ctypes.byref(o), None)
-    else:
-        f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_int] + \
-            [ctypes.POINTER(ctypes.c_int)] * 5 + [ctypes.c_int, ctypes.POINTER(na.na_options),
-                                                  ctypes.c_void_p]
-        st = f(*([p] * 5), 1, 1, iv([2, 64]), iv([8, 8]), iv([3, 3]), None, None, 1,
-               ctypes.byref(o), None)
+    p = ctypes.c_void_p(256)   # aligned and never dereferenced: the call fails on the host
+    f = lib.na_forward_noalloc
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_int] + \
+        [ctypes.POINTER(ctypes.c_int)] * 5 + [ctypes.c_int, ctypes.POINTER(na.na_options),
+                                              ctypes.c_void_p]
+    st = f(*([p] * 5), 1, 1, iv([2, 64]), iv([8, 8]), iv([3, 3]), None, None, 1, ctypes.byref(o),
+           None)
     assert st == na.NA_ERR_UNSUPPORTED

@@ -27,9 +27,9 @@ import seeded_inputs  # noqa: E402
 from gpu_parity import to_device  # noqa: E402
 
 
-def _case(grid, window, stride, d, dtype="bf16", B=1, heads=2, mode=None, tile=None):
+def _case(grid, window, stride, d, dtype="bf16", B=1, heads=2, mode=None, tile=None, dil=None):
     return dict(B=B, heads=heads, grid=tuple(grid), window=tuple(window), stride=tuple(stride),
-                d=d, dtype=dtype, mode=mode, tile=tile)
+                d=d, dtype=dtype, mode=mode, tile=tile, dil=dil)
 
 
 CASES = {
@@ -45,6 +45,11 @@ CASES = {
     "fp32_d32": _case((16, 16), (5, 5), (1, 1), 32, dtype="f32", heads=3),
     "f16_d64": _case((18, 22), (7, 9), (2, 1), 64, dtype="f16"),
     "sta3d_medium_d128": _case((6, 16, 40), (6, 12, 24), (2, 4, 8), 128, tile=(2, 4, 8)),
+    # dilated windows (residue classes of different lengths)
+    "dilated2d_d64": _case((23, 17), (5, 4), (1, 2), 64, dil=(3, 2),
+                           mode=["clamped", "truncated"]),
+    "dilated1d_causal_d128": _case((401,), (33,), (1,), 128, dil=(4,), mode=["causal"]),
+    "dilated3d_f32": _case((6, 9, 10), (3, 3, 4), (1, 1, 2), 32, dtype="f32", dil=(2, 3, 2)),
 }
 
 
@@ -55,16 +60,16 @@ def _run(c, seed, kernel=None):
            "f16": seeded_inputs.normal_f16}[c["dtype"]]
     do = gen(seed + 7, shape, threads=1)
     qd, kd, vd, dod = (to_device(a, c["dtype"]) for a in (q, k, v, do))
-    opts = na.make_options(window_mode=c["mode"], ndim=len(c["grid"])) if c["mode"] else None
+    opts = na.make_options(window_mode=c["mode"], ndim=len(c["grid"]), dilation=c["dil"])
     out, lse = na.forward(qd, kd, vd, c["window"], c["stride"], c["tile"], options=opts)
-    bopts = na.make_options(window_mode=c["mode"], ndim=len(c["grid"]),
+    bopts = na.make_options(window_mode=c["mode"], ndim=len(c["grid"]), dilation=c["dil"],
                             kernel=kernel if kernel is not None else na.NA_KERNEL_AUTO)
     dq, dk, dv = na.backward(qd, kd, vd, out, lse, dod, c["window"], c["stride"], c["tile"],
                              options=bopts)
     na.na_sync_status()
     got = [t.float().cpu().numpy().astype(np.float64) for t in (dq, dk, dv)]
     ref = oracle.backward(q, k, v, do, c["grid"], c["window"], c["stride"], dtype=c["dtype"],
-                          mode=c["mode"])
+                          mode=c["mode"], dilation=c["dil"])
     return got, ref
 
 
@@ -90,7 +95,8 @@ def test_backward_parity(name):
     _assert_close(c, got, ref, name)
 
 
-@pytest.mark.parametrize("name", ["na2d_ragged_d64", "causal1d", "sta3d_small", "f16_d64"])
+@pytest.mark.parametrize("name", ["na2d_ragged_d64", "causal1d", "sta3d_small", "f16_d64",
+                                  "dilated2d_d64"])
 def test_backward_parity_cuda_cores(name):
     """The same cases with every backward kernel on the CUDA cores."""
     c = CASES[name]
