@@ -225,17 +225,32 @@ NA_HD int make_tiling(const Geom& g, const int qb[3], const int tl[3], QTiling& 
   return 0;
 }
 
-// Bits i of 32-bit word w that mark keys j = 32w + i with (j mod period) in
-// [a, b): one grid dimension's window range laid over a chunk's key order.
-NA_HD uint32_t periodic_range_word(int w, int period, int a, int b) {
-  uint32_t m = 0;
-  const int base = 32 * w;
-  for (int p0 = base - base % period; p0 < base + 32; p0 += period) {
-    const int lo = imax(p0 + a, base) - base;
-    const int hi = imin(p0 + b, base + 32) - base;
-    if (lo < hi) m |= (hi - lo == 32 ? 0xffffffffu : ((1u << (hi - lo)) - 1u) << lo);
+// Bits [a, b) of a 32-bit word (0 <= a <= b <= 32).
+NA_HD uint32_t range_bits(int a, int b) {
+  if (b - a >= 32) return 0xffffffffu;
+  return ((1u << (b - a)) - 1u) << a;
+}
+
+// Bits i of 32-bit word w marking keys j = 32w + i whose coordinate along one
+// dimension, (j >> sh) & (kb - 1) (kb a power of two), lies in [lo, hi).
+// Along that dimension the key order repeats with period P = kb << sh: a
+// period of at most 32 bits is one range of bits, copied across the word by
+// at most five doubling shifts; a longer period puts one range of
+// coordinates, or a single coordinate, in the word.  No division and no
+// per-period loop: this runs on the softmax's critical path for every
+// partial chunk.
+NA_HD uint32_t dim_word_mask(int w, int sh, int kb, int lo, int hi) {
+  if (lo >= hi) return 0u;
+  const int P = kb << sh;
+  if (P <= 32) {
+    uint32_t v = range_bits(lo << sh, hi << sh);
+    for (int step = P; step < 32; step <<= 1) v |= v << step;
+    return v;
   }
-  return m;
+  const int xs = ((32 * w) >> sh) & (kb - 1);   // first coordinate in this word
+  if (sh >= 5) return (xs >= lo && xs < hi) ? 0xffffffffu : 0u;
+  const int a = imax(lo, xs), b = imin(hi, xs + (32 >> sh));
+  return a < b ? range_bits((a - xs) << sh, (b - xs) << sh) : 0u;
 }
 
 // Validity of the 128 keys of a chunk for one query: key j (chunk-local
@@ -243,10 +258,8 @@ NA_HD uint32_t periodic_range_word(int w, int period, int a, int b) {
 // query's window [wlo_d, whi_d) in every dimension.
 NA_HD void chunk_key_mask(const int a[3], const int wlo[3], const int whi[3],
                                                const int kb[3], const int kbl[3], uint32_t (&mk)[4]) {
-  int lo[3], hi[3], stride[3];
-  stride[2] = 1;
-  stride[1] = 1 << kbl[2];
-  stride[0] = 1 << (kbl[1] + kbl[2]);
+  int lo[3], hi[3];
+  const int sh[3] = {kbl[1] + kbl[2], kbl[2], 0};
   for (int d = 0; d < 3; ++d) {
     lo[d] = imin(imax(wlo[d] - a[d], 0), kb[d]);
     hi[d] = imin(imax(whi[d] - a[d], 0), kb[d]);
@@ -254,8 +267,8 @@ NA_HD void chunk_key_mask(const int a[3], const int wlo[3], const int whi[3],
 #pragma unroll
   for (int wd = 0; wd < 4; ++wd) {
     uint32_t m = 0xffffffffu;
-    for (int d = 0; d < 3; ++d)
-      m &= periodic_range_word(wd, kb[d] * stride[d], lo[d] * stride[d], hi[d] * stride[d]);
+#pragma unroll
+    for (int d = 0; d < 3; ++d) m &= dim_word_mask(wd, sh[d], kb[d], lo[d], hi[d]);
     mk[wd] = m;
   }
 }
