@@ -72,6 +72,7 @@ struct BtBars {
   uint64_t full[NS];
   uint64_t empty[NS];
   uint64_t s_full;           // S and dP of the current chunk
+  uint64_t s_loaded;         // S and dP read into registers (one arrival per element-wise warp)
   uint64_t p_ready;          // dS stored (256 arrivals)
   uint64_t o_done;
   uint32_t tmem_base;
@@ -119,6 +120,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       ptx::mbar_init(&bars->empty[s], 1);
     }
     ptx::mbar_init(&bars->s_full, 1);
+    ptx::mbar_init(&bars->s_loaded, 8);
     ptx::mbar_init(&bars->p_ready, 2 * BT_M);
     ptx::mbar_init(&bars->o_done, 1);
     bars->abort = *reinterpret_cast<volatile int*>(P.status) != 0;
@@ -189,7 +191,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       const uint32_t ringa = ptx::smem_u32(ring);
       // S = Q K^T into [S_COL0, +128) and dP = dO V^T into [DP_COL0, +128):
       // both B operands are [keys x d] tiles read K-major.
-      auto issue_sdp = [&](int kslot, int vslot) {
+      auto issue_s = [&](int kslot) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
@@ -197,6 +199,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
                       ptx::desc_sw128(ringa + kslot * C::TILE_BYTES + off, 16, 1024), C::IDESC_S,
                       kk > 0 ? 1u : 0u);
         }
+      };
+      auto issue_dp = [&](int vslot) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
@@ -216,25 +220,50 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
           ptx::mma_ts(tmem + C::DQ_COL0, a_t, bd, C::IDESC_DQ, (accumulate || kk > 0) ? 1u : 0u);
         }
       };
+      // Pipelined by one chunk: S of chunk j + 1 is issued as soon as the
+      // element-wise warps have read S and dP of chunk j into registers (S's
+      // columns are then free; dS goes to dP's columns), so it runs during
+      // their pass; dP of chunk j + 1 follows dQ of chunk j, which reads dS
+      // from dP's columns (the tensor pipe executes in issue order).
       bool ok = B.exists;
+      bool more = false;
       if (ok) ok = ptx::wait(&bars->q_full, 0, ctl);
-      for (int j = 0; ok; ++j) {
-        const int ks = 2 * j, vs = 2 * j + 1;
-        ok = ptx::wait(&bars->full[ks % NS], (ks / NS) & 1, ctl);
+      if (ok) ok = ptx::wait(&bars->full[0], 0, ctl);
+      if (ok) {
+        ptx::tc_fence_after();
+        more = bars->info[0] != BT_INFO_END;
+        if (more) {
+          ok = ptx::wait(&bars->full[1 % NS], (1 / NS) & 1, ctl);
+          if (ok) {
+            ptx::tc_fence_after();
+            issue_s(0);
+            issue_dp(1 % NS);
+            ptx::tc_commit(&bars->s_full);
+            ptx::tc_commit(&bars->empty[1 % NS]);
+          }
+        }
+      }
+      for (int j = 0; ok && more; ++j) {
+        const int ks = 2 * j, nks = 2 * j + 2, nvs = 2 * j + 3;
+        ok = ptx::wait(&bars->s_loaded, j & 1, ctl);
+        if (!ok) break;
+        ok = ptx::wait(&bars->full[nks % NS], (nks / NS) & 1, ctl);
         if (!ok) break;
         ptx::tc_fence_after();
-        if (bars->info[ks % NS] == BT_INFO_END) break;
-        ok = ptx::wait(&bars->full[vs % NS], (vs / NS) & 1, ctl);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        issue_sdp(ks % NS, vs % NS);
-        ptx::tc_commit(&bars->s_full);
-        ptx::tc_commit(&bars->empty[vs % NS]);
+        more = bars->info[nks % NS] != BT_INFO_END;
+        if (more) issue_s(nks % NS);
         ok = ptx::wait(&bars->p_ready, j & 1, ctl);
         if (!ok) break;
         ptx::tc_fence_after();
         issue_dq(ks % NS, j > 0);
         ptx::tc_commit(&bars->empty[ks % NS]);
+        if (!more) break;
+        ok = ptx::wait(&bars->full[nvs % NS], (nvs / NS) & 1, ctl);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        issue_dp(nvs % NS);
+        ptx::tc_commit(&bars->s_full);
+        ptx::tc_commit(&bars->empty[nvs % NS]);
       }
       ptx::tc_commit(&bars->o_done);
       ptx::wait_drain(&bars->o_done, 0, ctl);
@@ -299,6 +328,10 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
           ptx::reg_fence(d0);
           ptx::reg_fence(d1);
         }
+        // S's columns may now take the next chunk's scores.
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->s_loaded);
         if (st == CHUNK_PARTIAL) {
           uint32_t mk[4];
           chunk_key_mask(it.a, wlo, whi, kb, P.kb_log2, mk);
