@@ -381,7 +381,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           ptx::reg_fence(s3);
           if (st == CHUNK_PARTIAL) {
             uint32_t mk[4];
-            chunk_key_mask(it.a, wlo, whi, P.kb, P.kb_log2, mk);
+            if constexpr (D == 128)
+              chunk_key_mask_compact(it.a, wlo, whi, P.kb, P.kb_log2, mk);
+            else
+              chunk_key_mask(it.a, wlo, whi, P.kb, P.kb_log2, mk);
 #pragma unroll
             for (int j = 0; j < 128; ++j)
               if (!((mk[j >> 5] >> (j & 31)) & 1u)) s[j] = __float_as_uint(-INFINITY);

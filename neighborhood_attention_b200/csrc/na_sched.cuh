@@ -273,6 +273,41 @@ NA_HD void chunk_key_mask(const int a[3], const int wlo[3], const int whi[3],
   }
 }
 
+// The same mask from a loop over the periods of each dimension: slower on
+// partial chunks, but its code is a fraction of the straight-line form's.
+// The forward kernel at head_dim 128 uses it: there the straight-line form,
+// inlined in the softmax loop, slowed the full-chunk path by about 5 %
+// (measured on the sliding-tile workload, which has no partial chunks).
+NA_HD uint32_t periodic_range_word(int w, int period, int a, int b) {
+  uint32_t m = 0;
+  const int base = 32 * w;
+  for (int p0 = base - base % period; p0 < base + 32; p0 += period) {
+    const int lo = imax(p0 + a, base) - base;
+    const int hi = imin(p0 + b, base + 32) - base;
+    if (lo < hi) m |= range_bits(lo, hi);
+  }
+  return m;
+}
+
+NA_HD void chunk_key_mask_compact(const int a[3], const int wlo[3], const int whi[3],
+                                  const int kb[3], const int kbl[3], uint32_t (&mk)[4]) {
+  int lo[3], hi[3], stride[3];
+  stride[2] = 1;
+  stride[1] = 1 << kbl[2];
+  stride[0] = 1 << (kbl[1] + kbl[2]);
+  for (int d = 0; d < 3; ++d) {
+    lo[d] = imin(imax(wlo[d] - a[d], 0), kb[d]);
+    hi[d] = imin(imax(whi[d] - a[d], 0), kb[d]);
+  }
+#pragma unroll
+  for (int wd = 0; wd < 4; ++wd) {
+    uint32_t m = 0xffffffffu;
+    for (int d = 0; d < 3; ++d)
+      m &= periodic_range_word(wd, kb[d] * stride[d], lo[d] * stride[d], hi[d] * stride[d]);
+    mk[wd] = m;
+  }
+}
+
 // Same for one block: the status of the chunk found (CHUNK_EMPTY at the end).
 NA_HD int seek_block(const ChunkGrid& cg, const int* kb, const BlockInfo& b,
                                           ChunkIter& it) {

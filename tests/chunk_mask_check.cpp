@@ -1,5 +1,6 @@
-// Host check of the chunk key mask (chunk_key_mask in na_sched.cuh, used on
-// the softmax's critical path of every partial chunk): for every chunk shape
+// Host check of the chunk key mask (chunk_key_mask and chunk_key_mask_compact
+// in na_sched.cuh, used on the softmax's critical path of every partial
+// chunk): for every chunk shape
 // of 128 keys (powers of two per dimension) and pseudo-random chunk origins
 // and windows, every bit against a direct per-key range test.  Built and run
 // by tests/test_chunk_mask.py; exit status 0 when every bit matches.
@@ -20,8 +21,11 @@ int main() {
         x = x * 1103515245u + 12345u; wlo[d] = a[d] - kb[d] + (int)((x >> 8) % (3 * kb[d] + 2));
         x = x * 1103515245u + 12345u; whi[d] = wlo[d] + (int)((x >> 8) % (2 * kb[d] + 3));
       }
-      uint32_t mk[4];
+      uint32_t mk[4], mc[4];
       chunk_key_mask(a, wlo, whi, kb, kbl, mk);
+      chunk_key_mask_compact(a, wlo, whi, kb, kbl, mc);
+      for (int w = 0; w < 4; ++w)
+        if (mk[w] != mc[w]) ++bad;   // the two forms agree word for word
       for (int j = 0; j < 128; ++j) {
         const int x0 = j >> (e1 + e2), x1 = (j >> e2) & (kb[1] - 1), x2 = j & (kb[2] - 1);
         const bool in = a[0] + x0 >= wlo[0] && a[0] + x0 < whi[0] && a[1] + x1 >= wlo[1] &&
