@@ -585,8 +585,32 @@ def run_ours(args, rank, world, local_rank):
         na.na_sync_status(stream)
         dense_ms = float(np.mean([a.elapsed_time(b) for a, b in d_ev]))
 
-    total_ms, e2e_ms, per_launch_ms, dense_ms = max_over_ranks(
-        [total_ms, e2e_ms, per_launch_ms, dense_ms], world, dev)
+    # Context only: the same dense attention through torch's fused
+    # scaled_dot_product_attention (a library kernel, never on the measured
+    # path), over the flattened token sequence.
+    sdpa_ms = 0.0
+    if not args.no_speedup and w["dtype"] in ("bf16", "f16"):
+        import torch.nn.functional as F
+        BH_ = w["B"] * w["heads"]
+        N_ = int(np.prod(w["grid"]))
+        qs, ks, vs = (t.view(w["B"], w["heads"], N_, w["head_dim"]) for t in (q, k, v))
+        try:
+            F.scaled_dot_product_attention(qs, ks, vs)
+            s_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(DENSE_STEPS)]
+            for i in range(DENSE_STEPS):
+                flush_l2(i)
+                s_ev[i][0].record(stream)
+                F.scaled_dot_product_attention(qs, ks, vs)
+                s_ev[i][1].record(stream)
+            torch.cuda.synchronize()
+            sdpa_ms = float(np.mean([a.elapsed_time(b) for a, b in s_ev]))
+        except RuntimeError:
+            sdpa_ms = 0.0
+        del BH_
+
+    total_ms, e2e_ms, per_launch_ms, dense_ms, sdpa_ms = max_over_ranks(
+        [total_ms, e2e_ms, per_launch_ms, dense_ms, sdpa_ms], world, dev)
 
     plan = na.na_plan(w["grid"], w["window"], w["stride"], w["tile"], w["head_dim"],
                       {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32}[w["dtype"]],
@@ -645,8 +669,12 @@ def run_ours(args, rank, world, local_rank):
             "bound": plan["speedup_bound"], "measured": dense_ms / per_launch_ms,
             "ideal": plan["dense_pairs"] / plan["useful_pairs"], "dense_ms": dense_ms,
             "kernel_ms": per_launch_ms,
+            "vs_torch_sdpa": (sdpa_ms / per_launch_ms) if sdpa_ms > 0 else None,
+            "torch_sdpa_dense_ms": sdpa_ms if sdpa_ms > 0 else None,
             "note": "dense = the same kernel with the window set to the whole grid, timed "
-                    "after the timed region; bound = dense tile units / computed tile units"},
+                    "after the timed region; bound = dense tile units / computed tile units; "
+                    "vs_torch_sdpa = torch scaled_dot_product_attention on the same tensors "
+                    "as one dense sequence (context only)"},
         "gpu_launches": args.steps,
         "clocks": clocks,
         "kernel_ms": per_launch_ms,
