@@ -301,15 +301,21 @@ def na_backward(q, k, v, out, dout, lse, dq, dk, dv, delta, window, stride=None,
 
 
 def backward(q, k, v, out, lse, dout, window, stride=None, tile=None, options=None, stream=None,
-             window_mode=None):
+             window_mode=None, dilation=None):
     """Allocate dq, dk, dv (and the delta workspace) with torch and enqueue the
-    backward pass; returns (dq, dk, dv)."""
+    backward pass; returns (dq, dk, dv).  ``window_mode`` and ``dilation``
+    as in forward() (they must match the forward's)."""
     import torch
-    if window_mode is not None:
+    if window_mode is not None or dilation is not None:
         if options is None:
             options = na_default_options()
+    if window_mode is not None:
         for i, m in enumerate(window_modes(window_mode, len(window))):
             options.window_mode[i] = m
+    if dilation is not None:
+        dl = [dilation] * len(window) if isinstance(dilation, int) else list(dilation)
+        for i, x in enumerate(dl):
+            options.dilation[i] = int(x)
     dq, dk, dv = (torch.empty_like(q) for _ in range(3))
     delta = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
     return na_backward(q, k, v, out, dout, lse, dq, dk, dv, delta, window, stride, tile, options,
