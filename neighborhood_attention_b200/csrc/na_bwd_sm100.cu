@@ -449,8 +449,10 @@ struct BkBars {
   uint64_t kv_full;          // K and V tiles of the key block
   uint64_t full[NQ];         // query chunk stage loaded (TMA bytes + 32 producer lanes)
   uint64_t empty[NQ];
-  uint64_t s_full;           // S^T and dP^T of the current chunk
-  uint64_t p_ready;          // P^T and dS^T stored (256 arrivals)
+  uint64_t s_full;           // S^T of the current chunk
+  uint64_t dp_full;          // dP^T of the current chunk
+  uint64_t p_ready;          // P^T stored over S^T (256 arrivals)
+  uint64_t ds_ready;         // dS^T stored over dP^T (256 arrivals)
   uint64_t o_done;
   uint32_t tmem_base;
   int abort;
@@ -517,7 +519,9 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       ptx::mbar_init(&bars->empty[s], 1);
     }
     ptx::mbar_init(&bars->s_full, 1);
+    ptx::mbar_init(&bars->dp_full, 1);
     ptx::mbar_init(&bars->p_ready, 2 * BT_M);
+    ptx::mbar_init(&bars->ds_ready, 2 * BT_M);
     ptx::mbar_init(&bars->o_done, 1);
     bars->abort = *reinterpret_cast<volatile int*>(P.status) != 0;
     ptx::fence_mbar_init();
@@ -610,14 +614,17 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       // =========================== MMA issuer ===========================
       const uint32_t sKa = ptx::smem_u32(sK), sVa = ptx::smem_u32(sV);
       const uint32_t sta = ptx::smem_u32(stages);
-      auto issue_s = [&](int st) {
-        const uint32_t qa = sta + (2 * st) * C::TILE_BYTES, da = qa + C::TILE_BYTES;
+      auto issue_st = [&](int st) {        // S^T = K Q^T
+        const uint32_t qa = sta + (2 * st) * C::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
           ptx::mma_ss(tmem + C::S_COL0, ptx::desc_sw128(sKa + off, 16, 1024),
                       ptx::desc_sw128(qa + off, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
         }
+      };
+      auto issue_dpt = [&](int st) {       // dP^T = V dO^T
+        const uint32_t da = sta + (2 * st + 1) * C::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
@@ -627,8 +634,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       };
       // dV += P^T dO and dK += dS^T Q: the stage's tiles read MN-major (their
       // rows, the chunk's queries, are the reduction dimension).
-      auto issue_acc = [&](int st, bool accumulate) {
-        const uint32_t qa = sta + (2 * st) * C::TILE_BYTES, da = qa + C::TILE_BYTES;
+      auto issue_dv = [&](int st, bool accumulate) {   // dV += P^T dO
+        const uint32_t da = sta + (2 * st + 1) * C::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BT_N / 16; ++kk) {
           const uint32_t col = (kk >> 2) * 64 + (kk & 3) * 8;
@@ -636,6 +643,9 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
                       ptx::desc_sw128(da + kk * 2048, BT_HALF_BYTES, 1024), C::IDESC_ACC,
                       (accumulate || kk > 0) ? 1u : 0u);
         }
+      };
+      auto issue_dk = [&](int st, bool accumulate) {   // dK += dS^T Q
+        const uint32_t qa = sta + (2 * st) * C::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BT_N / 16; ++kk) {
           const uint32_t col = (kk >> 2) * 64 + (kk & 3) * 8;
@@ -644,21 +654,62 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
                       (accumulate || kk > 0) ? 1u : 0u);
         }
       };
+      // The element-wise pass stores P^T first and dS^T second, so dV of
+      // chunk j runs while dS^T is formed.  With four or more stages, S^T of
+      // chunk j + 1 is issued right behind dV (into the columns dV just
+      // read), ahead of dK, so the next chunk's exponentials overlap dK and
+      // dP^T; with two stages the next chunk's Q is then rarely loaded yet,
+      // so dK goes first.  The tensor pipe runs in issue order, which keeps
+      // every overwrite of a TMEM operand behind its reader.
+      constexpr bool EARLY_S = NQ >= 3;
       bool ok = KB.exists;
+      bool more = false;
       if (ok) ok = ptx::wait(&bars->kv_full, 0, ctl);
-      for (int j = 0; ok; ++j) {
-        const int st = j % NQ;
-        ok = ptx::wait(&bars->full[st], (j / NQ) & 1, ctl);
-        if (!ok) break;
+      if (ok) ok = ptx::wait(&bars->full[0], 0, ctl);
+      if (ok) {
         ptx::tc_fence_after();
-        if (bars->info[st] == BT_INFO_END) break;
-        issue_s(st);
-        ptx::tc_commit(&bars->s_full);
+        more = bars->info[0] != BT_INFO_END;
+        if (more) {
+          issue_st(0);
+          ptx::tc_commit(&bars->s_full);
+          issue_dpt(0);
+          ptx::tc_commit(&bars->dp_full);
+        }
+      }
+      for (int j = 0; ok && more; ++j) {
+        const int st = j % NQ, nst = (j + 1) % NQ;
         ok = ptx::wait(&bars->p_ready, j & 1, ctl);
         if (!ok) break;
         ptx::tc_fence_after();
-        issue_acc(st, j > 0);
+        issue_dv(st, j > 0);
+        if constexpr (EARLY_S) {
+          ok = ptx::wait(&bars->full[nst], ((j + 1) / NQ) & 1, ctl);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          more = bars->info[nst] != BT_INFO_END;
+          if (more) {
+            issue_st(nst);
+            ptx::tc_commit(&bars->s_full);
+          }
+        }
+        ok = ptx::wait(&bars->ds_ready, j & 1, ctl);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        issue_dk(st, j > 0);
         ptx::tc_commit(&bars->empty[st]);
+        if constexpr (!EARLY_S) {
+          ok = ptx::wait(&bars->full[nst], ((j + 1) / NQ) & 1, ctl);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          more = bars->info[nst] != BT_INFO_END;
+          if (more) {
+            issue_st(nst);
+            ptx::tc_commit(&bars->s_full);
+          }
+        }
+        if (!more) break;
+        issue_dpt(nst);
+        ptx::tc_commit(&bars->dp_full);
       }
       ptx::tc_commit(&bars->o_done);
       ptx::wait_drain(&bars->o_done, 0, ctl);
@@ -708,21 +759,17 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
         got = __all_sync(0xffffffffu, got);
         if (!got) { ok = false; break; }
         ptx::tc_fence_after();
-        uint32_t s[64], dp[64];
+        // Phase 1: P^T = exp(scale S^T - lse) from S^T alone, stored over S^T
+        // so that dV can start; P stays in registers (fp32) for phase 2.
+        uint32_t s[64];
         {
           uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
           uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
-          uint32_t (&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[0]);
-          uint32_t (&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[32]);
           ptx::tmem_ld32(tS, s0);
           ptx::tmem_ld32(tS + 32, s1);
-          ptx::tmem_ld32(tDP, d0);
-          ptx::tmem_ld32(tDP + 32, d1);
           ptx::tmem_ld_wait();
           ptx::reg_fence(s0);
           ptx::reg_fence(s1);
-          ptx::reg_fence(d0);
-          ptx::reg_fence(d1);
         }
         // Mask (partial chunks): query c of the chunk sees this key iff its
         // coordinates lie in the key's inverse ranges; padded keys see none.
@@ -737,33 +784,59 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
         const uint64_t scale2 = ptx::f2(sl2, sl2);
         const float* l2p = &bars->lse2[st][64 * h];
         const float* dlp = &bars->dlt[st][64 * h];
+        {
+          uint32_t pw[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            const float2 l2 = *reinterpret_cast<const float2*>(l2p + 2 * q);
+            const uint64_t x = ptx::f2_fma(
+                ptx::f2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), scale2,
+                ptx::f2(-l2.x, -l2.y));
+            float x0, x1;
+            ptx::f2_split(x, x0, x1);
+            const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
+            s[2 * q] = __float_as_uint(p0);       // P kept in fp32 for dS
+            s[2 * q + 1] = __float_as_uint(p1);
+            pw[q] = ptx::pack_half2<F16>(p0, p1);
+          }
+          ptx::tmem_st32(tS, pw);
+          ptx::tmem_st_wait();
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->p_ready);
+        // Phase 2: dS^T = P^T (dP^T - delta), stored over dP^T for dK.
+        got = ptx::wait(&bars->dp_full, j & 1, ctl);
+        got = __all_sync(0xffffffffu, got);
+        if (!got) { ok = false; break; }
+        ptx::tc_fence_after();
+        uint32_t dp[64];
+        {
+          uint32_t (&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[0]);
+          uint32_t (&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[32]);
+          ptx::tmem_ld32(tDP, d0);
+          ptx::tmem_ld32(tDP + 32, d1);
+          ptx::tmem_ld_wait();
+          ptx::reg_fence(d0);
+          ptx::reg_fence(d1);
+        }
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
-          const float2 l2 = *reinterpret_cast<const float2*>(l2p + 2 * q);
           const float2 dl = *reinterpret_cast<const float2*>(dlp + 2 * q);
-          const uint64_t x = ptx::f2_fma(
-              ptx::f2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), scale2,
-              ptx::f2(-l2.x, -l2.y));
-          float x0, x1;
-          ptx::f2_split(x, x0, x1);
-          const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
           const uint64_t g = ptx::f2_add(
               ptx::f2(__uint_as_float(dp[2 * q]), __uint_as_float(dp[2 * q + 1])),
               ptx::f2(-dl.x, -dl.y));
           float z0, z1;
-          ptx::f2_split(ptx::f2_mul(ptx::f2(p0, p1), g), z0, z1);
-          s[q] = ptx::pack_half2<F16>(p0, p1);
+          ptx::f2_split(ptx::f2_mul(ptx::f2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), g),
+                        z0, z1);
           dp[q] = ptx::pack_half2<F16>(z0, z1);
         }
         {
-          uint32_t (&pw)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
           uint32_t (&dw)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[0]);
-          ptx::tmem_st32(tS, pw);
           ptx::tmem_st32(tDP, dw);
         }
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
-        ptx::mbar_arrive(&bars->p_ready);
+        ptx::mbar_arrive(&bars->ds_ready);
         ++j;
       }
     }
