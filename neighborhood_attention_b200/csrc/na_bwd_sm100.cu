@@ -71,8 +71,9 @@ struct BtBars {
   uint64_t q_full;           // Q and dO tiles
   uint64_t full[NS];
   uint64_t empty[NS];
-  uint64_t s_full;           // S and dP of the current chunk
-  uint64_t s_loaded;         // S and dP read into registers (one arrival per element-wise warp)
+  uint64_t s_full;           // S of the current chunk
+  uint64_t dp_full;          // dP of the current chunk
+  uint64_t s_loaded;         // S read into registers (one arrival per element-wise warp)
   uint64_t p_ready;          // dS stored (256 arrivals)
   uint64_t o_done;
   uint32_t tmem_base;
@@ -120,6 +121,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       ptx::mbar_init(&bars->empty[s], 1);
     }
     ptx::mbar_init(&bars->s_full, 1);
+    ptx::mbar_init(&bars->dp_full, 1);
     ptx::mbar_init(&bars->s_loaded, 8);
     ptx::mbar_init(&bars->p_ready, 2 * BT_M);
     ptx::mbar_init(&bars->o_done, 1);
@@ -221,10 +223,11 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
         }
       };
       // Pipelined by one chunk: S of chunk j + 1 is issued as soon as the
-      // element-wise warps have read S and dP of chunk j into registers (S's
+      // element-wise warps have read S of chunk j into registers (S's
       // columns are then free; dS goes to dP's columns), so it runs during
-      // their pass; dP of chunk j + 1 follows dQ of chunk j, which reads dS
-      // from dP's columns (the tensor pipe executes in issue order).
+      // their pass, and they exponentiate it while dQ of chunk j and dP of
+      // chunk j + 1 run; dP of chunk j + 1 follows dQ of chunk j, which
+      // reads dS from dP's columns (the tensor pipe executes in issue order).
       bool ok = B.exists;
       bool more = false;
       if (ok) ok = ptx::wait(&bars->q_full, 0, ctl);
@@ -237,8 +240,9 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
           if (ok) {
             ptx::tc_fence_after();
             issue_s(0);
-            issue_dp(1 % NS);
             ptx::tc_commit(&bars->s_full);
+            issue_dp(1 % NS);
+            ptx::tc_commit(&bars->dp_full);
             ptx::tc_commit(&bars->empty[1 % NS]);
           }
         }
@@ -251,7 +255,10 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
         if (!ok) break;
         ptx::tc_fence_after();
         more = bars->info[nks % NS] != BT_INFO_END;
-        if (more) issue_s(nks % NS);
+        if (more) {
+          issue_s(nks % NS);
+          ptx::tc_commit(&bars->s_full);
+        }
         ok = ptx::wait(&bars->p_ready, j & 1, ctl);
         if (!ok) break;
         ptx::tc_fence_after();
@@ -262,7 +269,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
         if (!ok) break;
         ptx::tc_fence_after();
         issue_dp(nvs % NS);
-        ptx::tc_commit(&bars->s_full);
+        ptx::tc_commit(&bars->dp_full);
         ptx::tc_commit(&bars->empty[nvs % NS]);
       }
       ptx::tc_commit(&bars->o_done);
@@ -312,21 +319,15 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
         got = __all_sync(0xffffffffu, got);
         if (!got) { ok = false; break; }
         ptx::tc_fence_after();
-        uint32_t s[64], dp[64];
+        uint32_t s[64];
         {
           uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
           uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
-          uint32_t (&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[0]);
-          uint32_t (&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[32]);
           ptx::tmem_ld32(tS, s0);
           ptx::tmem_ld32(tS + 32, s1);
-          ptx::tmem_ld32(tDP, d0);
-          ptx::tmem_ld32(tDP + 32, d1);
           ptx::tmem_ld_wait();
           ptx::reg_fence(s0);
           ptx::reg_fence(s1);
-          ptx::reg_fence(d0);
-          ptx::reg_fence(d1);
         }
         // S's columns may now take the next chunk's scores.
         ptx::tc_fence_before();
@@ -340,6 +341,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
           for (int q = 0; q < 64; ++q)
             if (!(((q < 32 ? w0 : w1) >> (q & 31)) & 1u)) s[q] = __float_as_uint(-INFINITY);
         }
+        // P = exp(scale S - lse) in fp32, while dQ of the previous chunk and
+        // dP of this one run.
         const uint64_t scale2 = ptx::f2(sl2, sl2);
         const uint64_t neg2 = ptx::f2(-lse2, -lse2);
         const uint64_t negd2 = ptx::f2(-Di, -Di);
@@ -349,15 +352,35 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
               ptx::f2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), scale2, neg2);
           float x0, x1;
           ptx::f2_split(x, x0, x1);
-          const uint64_t p = ptx::f2(ptx::ex2(x0), ptx::ex2(x1));
+          s[2 * q] = __float_as_uint(ptx::ex2(x0));
+          s[2 * q + 1] = __float_as_uint(ptx::ex2(x1));
+        }
+        got = ptx::wait(&bars->dp_full, j & 1, ctl);
+        got = __all_sync(0xffffffffu, got);
+        if (!got) { ok = false; break; }
+        ptx::tc_fence_after();
+        uint32_t dp[64];
+        {
+          uint32_t (&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[0]);
+          uint32_t (&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[32]);
+          ptx::tmem_ld32(tDP, d0);
+          ptx::tmem_ld32(tDP + 32, d1);
+          ptx::tmem_ld_wait();
+          ptx::reg_fence(d0);
+          ptx::reg_fence(d1);
+        }
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
           const uint64_t g = ptx::f2_add(
               ptx::f2(__uint_as_float(dp[2 * q]), __uint_as_float(dp[2 * q + 1])), negd2);
           float z0, z1;
-          ptx::f2_split(ptx::f2_mul(p, g), z0, z1);
-          s[q] = ptx::pack_half2<F16>(z0, z1);
+          ptx::f2_split(
+              ptx::f2_mul(ptx::f2(__uint_as_float(s[2 * q]), __uint_as_float(s[2 * q + 1])), g),
+              z0, z1);
+          dp[q] = ptx::pack_half2<F16>(z0, z1);
         }
         {
-          uint32_t (&ds)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
+          uint32_t (&ds)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[0]);
           ptx::tmem_st32(tDP, ds);
         }
         ptx::tmem_st_wait();
