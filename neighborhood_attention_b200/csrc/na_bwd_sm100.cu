@@ -470,8 +470,8 @@ struct BkCfg {
 template <int NQ>
 struct BkBars {
   uint64_t kv_full;          // K and V tiles of the key block
-  uint64_t full[NQ];         // query chunk stage loaded (TMA bytes + 32 producer lanes)
-  uint64_t empty[NQ];
+  uint64_t full[2 * NQ];     // tile slot loaded (TMA bytes + 32 producer lanes)
+  uint64_t empty[2 * NQ];    // tile slot read by its last MMA
   uint64_t s_full;           // S^T of the current chunk
   uint64_t dp_full;          // dP^T of the current chunk
   uint64_t p_ready;          // P^T stored over S^T (256 arrivals)
@@ -479,13 +479,22 @@ struct BkBars {
   uint64_t o_done;
   uint32_t tmem_base;
   int abort;
-  volatile uint32_t info[NQ];
+  volatile uint32_t info[NQ];  // stage's chunk or end marker (with its Q slot)
   float lse2[NQ][BT_N];      // log2(e) * lse of the stage's queries
   float dlt[NQ][BT_N];       // delta of the stage's queries
   BlockInfo kb;              // the key block (origin, extent)
   BlockInfo ib;              // its inverse windows: lo/hi = union, ilo/ihi = intersection
   ChunkGrid cg;              // query chunks over ib
 };
+
+// Stage st = j % NQ of chunk j owns tile slots 2 st and 2 st + 1; which of
+// them holds Q and which dO alternates with the round j / NQ.  dO of chunk j
+// is last read by dV (j), before dK (j) reads Q, so Q of chunk j + NQ goes
+// into the slot that dO of chunk j frees first.
+template <int NQ>
+__device__ __forceinline__ int q_slot(int j) { return 2 * (j % NQ) + ((j / NQ) & 1); }
+template <int NQ>
+__device__ __forceinline__ int do_slot(int j) { return 2 * (j % NQ) + 1 - ((j / NQ) & 1); }
 
 template <int D>
 constexpr size_t bk_smem_bytes() {
@@ -505,7 +514,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sK = base;
   uint8_t* sV = base + C::TILE_BYTES;
-  uint8_t* stages = base + 2 * C::TILE_BYTES;      // stage s: Q at 2s, dO at 2s+1
+  uint8_t* stages = base + 2 * C::TILE_BYTES;      // tile slots (q_slot / do_slot)
   BkBars<NQ>* bars = reinterpret_cast<BkBars<NQ>*>(stages + 2 * NQ * C::TILE_BYTES);
 
   const int warp = threadIdx.x >> 5;
@@ -537,7 +546,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
     }
     chunk_grid_for(&bars->ib, 1, P.kb, bars->cg);
     ptx::mbar_init(&bars->kv_full, 1);
-    for (int s = 0; s < NQ; ++s) {
+    for (int s = 0; s < 2 * NQ; ++s) {
       ptx::mbar_init(&bars->full[s], 32);
       ptx::mbar_init(&bars->empty[s], 1);
     }
@@ -578,58 +587,81 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
                            KB.o[0], bh);
         }
       }
-      int issued[NQ];
+      int issued[2 * NQ];
 #pragma unroll
-      for (int s = 0; s < NQ; ++s) issued[s] = 0;
+      for (int s = 0; s < 2 * NQ; ++s) issued[s] = 0;
       int seq = 0;
       ChunkIter it;
       iter_begin(cg, it);
       bool ok = true;
+      // Stage a chunk's per-query scalars, then load one of its tiles into
+      // slot sl once the slot's previous tile has been read (fill number
+      // seq / NQ of the slot).
+      auto wait_slot = [&](int sl) {
+        bool w = true;
+        if (seq >= NQ) w = ptx::wait(&bars->empty[sl], ((seq / NQ) - 1) & 1, ctl);
+        return __all_sync(0xffffffffu, w);
+      };
       for (seek_block(cg, P.kb, IB, it); ok && it.idx < cg.total;
            iter_next(cg, P.kb, it), seek_block(cg, P.kb, IB, it), ++seq) {
         const int st = seq % NQ;
-        if (seq >= NQ) ok = ptx::wait(&bars->empty[st], ((seq / NQ) - 1) & 1, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        for (int e = lane; e < BT_N; e += 32) {
+        const int qs = q_slot<NQ>(seq), ds = do_slot<NQ>(seq);
+        float l2[BT_N / 32], dl[BT_N / 32];
+#pragma unroll
+        for (int r = 0; r < BT_N / 32; ++r) {
+          const int e = lane + 32 * r;
           const int q2 = e % P.kb[2], q1 = (e / P.kb[2]) % P.kb[1], q0 = e / (P.kb[2] * P.kb[1]);
           const int x0 = it.a[0] + q0, x1 = it.a[1] + q1, x2 = it.a[2] + q2;
-          float l2 = 0.f, dl = 0.f;
+          l2[r] = 0.f;
+          dl[r] = 0.f;
           if (x0 < P.g.L[0] && x1 < P.g.L[1] && x2 < P.g.L[2]) {
             const size_t tok = (size_t)full_token(P.map, x0, x1, x2);
-            l2 = P.lse[(size_t)bh * P.N + tok] * BT_LOG2E;
-            dl = P.delta[(size_t)bh * P.N + tok];
+            l2[r] = P.lse[(size_t)bh * P.N + tok] * BT_LOG2E;
+            dl[r] = P.delta[(size_t)bh * P.N + tok];
           }
-          bars->lse2[st][e] = l2;
-          bars->dlt[st][e] = dl;
         }
+        // Q (with lse and the chunk's marker): its slot was last read by dV.
+        ok = wait_slot(qs);
+        if (!ok) break;
+#pragma unroll
+        for (int r = 0; r < BT_N / 32; ++r) bars->lse2[st][lane + 32 * r] = l2[r];
         if (lane == 0) {
           bars->info[st] = 0;
-          ptx::mbar_expect_tx(&bars->full[st], 2 * C::TILE_BYTES);
-          for (int h = 0; h < C::HALVES; ++h) {
-            ptx::tma_load_5d(stages + (2 * st) * C::TILE_BYTES + h * BT_HALF_BYTES, &tm_q,
-                             &bars->full[st], h * 64, it.a[2], it.a[1], it.a[0], bh);
-            ptx::tma_load_5d(stages + (2 * st + 1) * C::TILE_BYTES + h * BT_HALF_BYTES, &tm_do,
-                             &bars->full[st], h * 64, it.a[2], it.a[1], it.a[0], bh);
-          }
+          ptx::mbar_expect_tx(&bars->full[qs], C::TILE_BYTES);
+          for (int h = 0; h < C::HALVES; ++h)
+            ptx::tma_load_5d(stages + qs * C::TILE_BYTES + h * BT_HALF_BYTES, &tm_q,
+                             &bars->full[qs], h * 64, it.a[2], it.a[1], it.a[0], bh);
         } else {
-          ptx::mbar_arrive(&bars->full[st]);
+          ptx::mbar_arrive(&bars->full[qs]);
         }
-        ++issued[st];
+        ++issued[qs];
+        // dO (with delta): its slot was last read by dK.
+        ok = wait_slot(ds);
+        if (!ok) break;
+#pragma unroll
+        for (int r = 0; r < BT_N / 32; ++r) bars->dlt[st][lane + 32 * r] = dl[r];
+        if (lane == 0) {
+          ptx::mbar_expect_tx(&bars->full[ds], C::TILE_BYTES);
+          for (int h = 0; h < C::HALVES; ++h)
+            ptx::tma_load_5d(stages + ds * C::TILE_BYTES + h * BT_HALF_BYTES, &tm_do,
+                             &bars->full[ds], h * 64, it.a[2], it.a[1], it.a[0], bh);
+        } else {
+          ptx::mbar_arrive(&bars->full[ds]);
+        }
+        ++issued[ds];
       }
       if (ok) {
-        const int st = seq % NQ;
-        if (seq >= NQ) ok = ptx::wait(&bars->empty[st], ((seq / NQ) - 1) & 1, ctl);
-        ok = __all_sync(0xffffffffu, ok);
+        const int qs = q_slot<NQ>(seq);
+        ok = wait_slot(qs);
         if (ok) {
-          if (lane == 0) bars->info[st] = BT_INFO_END;
+          if (lane == 0) bars->info[seq % NQ] = BT_INFO_END;
           __syncwarp();
-          ptx::mbar_arrive(&bars->full[st]);
-          ++issued[st];
+          ptx::mbar_arrive(&bars->full[qs]);
+          ++issued[qs];
         }
       }
       if (lane == 0) {
-        for (int s = 0; s < NQ; ++s)
+        for (int s = 0; s < 2 * NQ; ++s)
           if (issued[s]) ptx::wait_drain(&bars->full[s], (issued[s] - 1) & 1, ctl);
         ptx::wait_drain(&bars->kv_full, 0, ctl);
       }
@@ -637,8 +669,9 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       // =========================== MMA issuer ===========================
       const uint32_t sKa = ptx::smem_u32(sK), sVa = ptx::smem_u32(sV);
       const uint32_t sta = ptx::smem_u32(stages);
-      auto issue_st = [&](int st) {        // S^T = K Q^T
-        const uint32_t qa = sta + (2 * st) * C::TILE_BYTES;
+      auto slot_addr = [&](int sl) { return sta + (uint32_t)(sl * C::TILE_BYTES); };
+      auto issue_st = [&](int qs) {        // S^T = K Q^T
+        const uint32_t qa = slot_addr(qs);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
@@ -646,8 +679,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
                       ptx::desc_sw128(qa + off, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_dpt = [&](int st) {       // dP^T = V dO^T
-        const uint32_t da = sta + (2 * st + 1) * C::TILE_BYTES;
+      auto issue_dpt = [&](int ds) {       // dP^T = V dO^T
+        const uint32_t da = slot_addr(ds);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
@@ -655,10 +688,10 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
                       ptx::desc_sw128(da + off, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
-      // dV += P^T dO and dK += dS^T Q: the stage's tiles read MN-major (their
+      // dV += P^T dO and dK += dS^T Q: the chunk's tiles read MN-major (their
       // rows, the chunk's queries, are the reduction dimension).
-      auto issue_dv = [&](int st, bool accumulate) {   // dV += P^T dO
-        const uint32_t da = sta + (2 * st + 1) * C::TILE_BYTES;
+      auto issue_dv = [&](int ds, bool accumulate) {   // dV += P^T dO
+        const uint32_t da = slot_addr(ds);
 #pragma unroll
         for (int kk = 0; kk < BT_N / 16; ++kk) {
           const uint32_t col = (kk >> 2) * 64 + (kk & 3) * 8;
@@ -667,8 +700,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
                       (accumulate || kk > 0) ? 1u : 0u);
         }
       };
-      auto issue_dk = [&](int st, bool accumulate) {   // dK += dS^T Q
-        const uint32_t qa = sta + (2 * st) * C::TILE_BYTES;
+      auto issue_dk = [&](int qs, bool accumulate) {   // dK += dS^T Q
+        const uint32_t qa = slot_addr(qs);
 #pragma unroll
         for (int kk = 0; kk < BT_N / 16; ++kk) {
           const uint32_t col = (kk >> 2) * 64 + (kk & 3) * 8;
@@ -678,60 +711,58 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
         }
       };
       // The element-wise pass stores P^T first and dS^T second, so dV of
-      // chunk j runs while dS^T is formed.  With four or more stages, S^T of
-      // chunk j + 1 is issued right behind dV (into the columns dV just
-      // read), ahead of dK, so the next chunk's exponentials overlap dK and
-      // dP^T; with two stages the next chunk's Q is then rarely loaded yet,
-      // so dK goes first.  The tensor pipe runs in issue order, which keeps
-      // every overwrite of a TMEM operand behind its reader.
-      constexpr bool EARLY_S = NQ >= 3;
+      // chunk j runs while dS^T is formed.  S^T of chunk j + 1 is issued
+      // right behind that dV (into the columns dV just read), ahead of dK,
+      // so the next chunk's exponentials overlap dK and dP^T; its Q sits in
+      // the slot that dO of chunk j + 1 - NQ left when its dV completed.  The
+      // tensor pipe runs in issue order, which keeps every overwrite of a
+      // TMEM operand behind its reader.  A slot is released by the commit
+      // behind its last reader: dV for dO, dK for Q.
       bool ok = KB.exists;
       bool more = false;
       if (ok) ok = ptx::wait(&bars->kv_full, 0, ctl);
-      if (ok) ok = ptx::wait(&bars->full[0], 0, ctl);
+      if (ok) ok = ptx::wait(&bars->full[q_slot<NQ>(0)], 0, ctl);
       if (ok) {
         ptx::tc_fence_after();
         more = bars->info[0] != BT_INFO_END;
         if (more) {
-          issue_st(0);
+          issue_st(q_slot<NQ>(0));
           ptx::tc_commit(&bars->s_full);
-          issue_dpt(0);
-          ptx::tc_commit(&bars->dp_full);
+          ok = ptx::wait(&bars->full[do_slot<NQ>(0)], 0, ctl);
+          if (ok) {
+            ptx::tc_fence_after();
+            issue_dpt(do_slot<NQ>(0));
+            ptx::tc_commit(&bars->dp_full);
+          }
         }
       }
       for (int j = 0; ok && more; ++j) {
-        const int st = j % NQ, nst = (j + 1) % NQ;
+        const int qs = q_slot<NQ>(j), ds = do_slot<NQ>(j);
+        const int nqs = q_slot<NQ>(j + 1), nds = do_slot<NQ>(j + 1);
+        const uint32_t nph = ((j + 1) / NQ) & 1;
         ok = ptx::wait(&bars->p_ready, j & 1, ctl);
         if (!ok) break;
         ptx::tc_fence_after();
-        issue_dv(st, j > 0);
-        if constexpr (EARLY_S) {
-          ok = ptx::wait(&bars->full[nst], ((j + 1) / NQ) & 1, ctl);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          more = bars->info[nst] != BT_INFO_END;
-          if (more) {
-            issue_st(nst);
-            ptx::tc_commit(&bars->s_full);
-          }
+        issue_dv(ds, j > 0);
+        ptx::tc_commit(&bars->empty[ds]);
+        ok = ptx::wait(&bars->full[nqs], nph, ctl);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        more = bars->info[(j + 1) % NQ] != BT_INFO_END;
+        if (more) {
+          issue_st(nqs);
+          ptx::tc_commit(&bars->s_full);
         }
         ok = ptx::wait(&bars->ds_ready, j & 1, ctl);
         if (!ok) break;
         ptx::tc_fence_after();
-        issue_dk(st, j > 0);
-        ptx::tc_commit(&bars->empty[st]);
-        if constexpr (!EARLY_S) {
-          ok = ptx::wait(&bars->full[nst], ((j + 1) / NQ) & 1, ctl);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          more = bars->info[nst] != BT_INFO_END;
-          if (more) {
-            issue_st(nst);
-            ptx::tc_commit(&bars->s_full);
-          }
-        }
+        issue_dk(qs, j > 0);
+        ptx::tc_commit(&bars->empty[qs]);
         if (!more) break;
-        issue_dpt(nst);
+        ok = ptx::wait(&bars->full[nds], nph, ctl);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        issue_dpt(nds);
         ptx::tc_commit(&bars->dp_full);
       }
       ptx::tc_commit(&bars->o_done);
