@@ -56,7 +56,7 @@ constexpr float BT_LOG2E = 1.4426950408889634f;
 template <int D, bool F16>
 struct BtCfg {
   static constexpr int TILE_BYTES = 128 * D * 2;
-  static constexpr int NS = (D == 128) ? 4 : 8;   // ring slots (K and V chunks)
+  static constexpr int NS = (D == 128) ? 4 : 8;   // tile slots (K and V of NS / 2 chunks)
   static constexpr int HALVES = D / 64;
   static constexpr int TMEM_COLS = 512;
   static constexpr int S_COL0 = 0;
@@ -82,6 +82,17 @@ struct BtBars {
   BlockInfo bi;
   ChunkGrid cg;
 };
+
+// Stage st = j % NST of chunk j owns tile slots 2 st and 2 st + 1; which of
+// them holds the first tile and which the second alternates with the round
+// j / NST, so that the first tile of chunk j + NST goes into the slot that
+// the second tile of chunk j frees (the dK / dV kernel: Q into dO's slot,
+// freed by dV before dK reads Q; the dQ kernel: K into V's slot, freed by dP
+// before dQ reads K).
+template <int NST>
+__device__ __forceinline__ int first_slot(int j) { return 2 * (j % NST) + ((j / NST) & 1); }
+template <int NST>
+__device__ __forceinline__ int second_slot(int j) { return 2 * (j % NST) + 1 - ((j / NST) & 1); }
 
 template <int D>
 constexpr size_t bt_smem_bytes() {
@@ -153,7 +164,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
         ptx::tma_load_5d(sDO + h * BT_HALF_BYTES, &tm_do, &bars->q_full, h * 64, B.o[2], B.o[1],
                          B.o[0], bh);
       }
-      int seq = 0;
+      constexpr int NST = NS / 2;
+      int c = 0;                 // chunk number
       int issued[NS];
 #pragma unroll
       for (int s = 0; s < NS; ++s) issued[s] = 0;
@@ -161,10 +173,11 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       iter_begin(cg, it);
       bool ok = true;
       for (seek_block(cg, P.kb, B, it); ok && it.idx < cg.total;
-           iter_next(cg, P.kb, it), seek_block(cg, P.kb, B, it)) {
+           iter_next(cg, P.kb, it), seek_block(cg, P.kb, B, it), ++c) {
         for (int kv = 0; kv < 2 && ok; ++kv) {
-          const int slot = seq % NS;
-          if (seq >= NS) ok = ptx::wait(&bars->empty[slot], ((seq / NS) - 1) & 1, ctl);
+          // K's slot was last read by dP, V's by dQ (fill number c / NST).
+          const int slot = kv ? second_slot<NST>(c) : first_slot<NST>(c);
+          if (c >= NST) ok = ptx::wait(&bars->empty[slot], ((c / NST) - 1) & 1, ctl);
           if (!ok) break;
           if (kv == 0) bars->info[slot] = 0;
           ptx::mbar_expect_tx(&bars->full[slot], C::TILE_BYTES);
@@ -172,12 +185,11 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
             ptx::tma_load_5d(ring + slot * C::TILE_BYTES + h * BT_HALF_BYTES, kv ? &tm_v : &tm_k,
                              &bars->full[slot], h * 64, it.a[2], it.a[1], it.a[0], bh);
           ++issued[slot];
-          ++seq;
         }
       }
       if (ok) {
-        const int slot = seq % NS;
-        if (seq >= NS) ok = ptx::wait(&bars->empty[slot], ((seq / NS) - 1) & 1, ctl);
+        const int slot = first_slot<NST>(c);
+        if (c >= NST) ok = ptx::wait(&bars->empty[slot], ((c / NST) - 1) & 1, ctl);
         if (ok) {
           bars->info[slot] = BT_INFO_END;
           ptx::mbar_arrive(&bars->full[slot]);
@@ -228,49 +240,54 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       // their pass, and they exponentiate it while dQ of chunk j and dP of
       // chunk j + 1 run; dP of chunk j + 1 follows dQ of chunk j, which
       // reads dS from dP's columns (the tensor pipe executes in issue order).
+      // K of chunk j sits in first_slot (j), V in second_slot (j); a slot is
+      // released by the commit behind its last reader (dQ for K, dP for V).
+      constexpr int NST = NS / 2;
       bool ok = B.exists;
       bool more = false;
       if (ok) ok = ptx::wait(&bars->q_full, 0, ctl);
-      if (ok) ok = ptx::wait(&bars->full[0], 0, ctl);
+      if (ok) ok = ptx::wait(&bars->full[first_slot<NST>(0)], 0, ctl);
       if (ok) {
         ptx::tc_fence_after();
-        more = bars->info[0] != BT_INFO_END;
+        more = bars->info[first_slot<NST>(0)] != BT_INFO_END;
         if (more) {
-          ok = ptx::wait(&bars->full[1 % NS], (1 / NS) & 1, ctl);
+          ok = ptx::wait(&bars->full[second_slot<NST>(0)], 0, ctl);
           if (ok) {
             ptx::tc_fence_after();
-            issue_s(0);
+            issue_s(first_slot<NST>(0));
             ptx::tc_commit(&bars->s_full);
-            issue_dp(1 % NS);
+            issue_dp(second_slot<NST>(0));
             ptx::tc_commit(&bars->dp_full);
-            ptx::tc_commit(&bars->empty[1 % NS]);
+            ptx::tc_commit(&bars->empty[second_slot<NST>(0)]);
           }
         }
       }
       for (int j = 0; ok && more; ++j) {
-        const int ks = 2 * j, nks = 2 * j + 2, nvs = 2 * j + 3;
+        const int ks = first_slot<NST>(j);
+        const int nks = first_slot<NST>(j + 1), nvs = second_slot<NST>(j + 1);
+        const uint32_t nph = ((j + 1) / NST) & 1;
         ok = ptx::wait(&bars->s_loaded, j & 1, ctl);
         if (!ok) break;
-        ok = ptx::wait(&bars->full[nks % NS], (nks / NS) & 1, ctl);
+        ok = ptx::wait(&bars->full[nks], nph, ctl);
         if (!ok) break;
         ptx::tc_fence_after();
-        more = bars->info[nks % NS] != BT_INFO_END;
+        more = bars->info[nks] != BT_INFO_END;
         if (more) {
-          issue_s(nks % NS);
+          issue_s(nks);
           ptx::tc_commit(&bars->s_full);
         }
         ok = ptx::wait(&bars->p_ready, j & 1, ctl);
         if (!ok) break;
         ptx::tc_fence_after();
-        issue_dq(ks % NS, j > 0);
-        ptx::tc_commit(&bars->empty[ks % NS]);
+        issue_dq(ks, j > 0);
+        ptx::tc_commit(&bars->empty[ks]);
         if (!more) break;
-        ok = ptx::wait(&bars->full[nvs % NS], (nvs / NS) & 1, ctl);
+        ok = ptx::wait(&bars->full[nvs], nph, ctl);
         if (!ok) break;
         ptx::tc_fence_after();
-        issue_dp(nvs % NS);
+        issue_dp(nvs);
         ptx::tc_commit(&bars->dp_full);
-        ptx::tc_commit(&bars->empty[nvs % NS]);
+        ptx::tc_commit(&bars->empty[nvs]);
       }
       ptx::tc_commit(&bars->o_done);
       ptx::wait_drain(&bars->o_done, 0, ctl);
@@ -487,14 +504,10 @@ struct BkBars {
   ChunkGrid cg;              // query chunks over ib
 };
 
-// Stage st = j % NQ of chunk j owns tile slots 2 st and 2 st + 1; which of
-// them holds Q and which dO alternates with the round j / NQ.  dO of chunk j
-// is last read by dV (j), before dK (j) reads Q, so Q of chunk j + NQ goes
-// into the slot that dO of chunk j frees first.
 template <int NQ>
-__device__ __forceinline__ int q_slot(int j) { return 2 * (j % NQ) + ((j / NQ) & 1); }
+__device__ __forceinline__ int q_slot(int j) { return first_slot<NQ>(j); }
 template <int NQ>
-__device__ __forceinline__ int do_slot(int j) { return 2 * (j % NQ) + 1 - ((j / NQ) & 1); }
+__device__ __forceinline__ int do_slot(int j) { return second_slot<NQ>(j); }
 
 template <int D>
 constexpr size_t bk_smem_bytes() {
