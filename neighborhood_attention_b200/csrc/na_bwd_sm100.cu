@@ -199,8 +199,20 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       for (int s = 0; s < NS; ++s)
         if (issued[s]) ptx::wait_drain(&bars->full[s], (issued[s] - 1) & 1, ctl);
       ptx::wait_drain(&bars->q_full, 0, ctl);
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
       // =========================== MMA issuer ===========================
+      // The whole warp issues: every lane sleeps in the hinted barrier wait
+      // and elect.sync picks the lane that issues each MMA and commit.
+      auto wait_i = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, ptx::wait_sleep(bar, parity, ctl));
+      };
+      auto commit_i = [&](uint64_t* bar) { ptx::tc_commit_warp(bar); };
+      auto mma_ss_i = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+        ptx::mma_ss_warp(d, a, b, id, acc);
+      };
+      auto mma_ts_i = [&](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
+        ptx::mma_ts_warp(d, a, b, id, acc);
+      };
       const uint32_t sQa = ptx::smem_u32(sQ), sDOa = ptx::smem_u32(sDO);
       const uint32_t ringa = ptx::smem_u32(ring);
       // S = Q K^T into [S_COL0, +128) and dP = dO V^T into [DP_COL0, +128):
@@ -209,18 +221,18 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
-          ptx::mma_ss(tmem + C::S_COL0, ptx::desc_sw128(sQa + off, 16, 1024),
-                      ptx::desc_sw128(ringa + kslot * C::TILE_BYTES + off, 16, 1024), C::IDESC_S,
-                      kk > 0 ? 1u : 0u);
+          mma_ss_i(tmem + C::S_COL0, ptx::desc_sw128(sQa + off, 16, 1024),
+                   ptx::desc_sw128(ringa + kslot * C::TILE_BYTES + off, 16, 1024), C::IDESC_S,
+                   kk > 0 ? 1u : 0u);
         }
       };
       auto issue_dp = [&](int vslot) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
-          ptx::mma_ss(tmem + C::DP_COL0, ptx::desc_sw128(sDOa + off, 16, 1024),
-                      ptx::desc_sw128(ringa + vslot * C::TILE_BYTES + off, 16, 1024), C::IDESC_S,
-                      kk > 0 ? 1u : 0u);
+          mma_ss_i(tmem + C::DP_COL0, ptx::desc_sw128(sDOa + off, 16, 1024),
+                   ptx::desc_sw128(ringa + vslot * C::TILE_BYTES + off, 16, 1024), C::IDESC_S,
+                   kk > 0 ? 1u : 0u);
         }
       };
       // dQ += dS K: dS (16-bit pairs) of keys 64h.. in [DP_COL0 + 64h, +32),
@@ -231,7 +243,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
           const uint32_t a_t = tmem + C::DP_COL0 + (kk >> 2) * 64 + (kk & 3) * 8;
           const uint64_t bd =
               ptx::desc_sw128(ringa + kslot * C::TILE_BYTES + kk * 2048, BT_HALF_BYTES, 1024);
-          ptx::mma_ts(tmem + C::DQ_COL0, a_t, bd, C::IDESC_DQ, (accumulate || kk > 0) ? 1u : 0u);
+          mma_ts_i(tmem + C::DQ_COL0, a_t, bd, C::IDESC_DQ, (accumulate || kk > 0) ? 1u : 0u);
         }
       };
       // Pipelined by one chunk: S of chunk j + 1 is issued as soon as the
@@ -245,20 +257,20 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       constexpr int NST = NS / 2;
       bool ok = B.exists;
       bool more = false;
-      if (ok) ok = ptx::wait(&bars->q_full, 0, ctl);
-      if (ok) ok = ptx::wait(&bars->full[first_slot<NST>(0)], 0, ctl);
+      if (ok) ok = wait_i(&bars->q_full, 0);
+      if (ok) ok = wait_i(&bars->full[first_slot<NST>(0)], 0);
       if (ok) {
         ptx::tc_fence_after();
         more = bars->info[first_slot<NST>(0)] != BT_INFO_END;
         if (more) {
-          ok = ptx::wait(&bars->full[second_slot<NST>(0)], 0, ctl);
+          ok = wait_i(&bars->full[second_slot<NST>(0)], 0);
           if (ok) {
             ptx::tc_fence_after();
             issue_s(first_slot<NST>(0));
-            ptx::tc_commit(&bars->s_full);
+            commit_i(&bars->s_full);
             issue_dp(second_slot<NST>(0));
-            ptx::tc_commit(&bars->dp_full);
-            ptx::tc_commit(&bars->empty[second_slot<NST>(0)]);
+            commit_i(&bars->dp_full);
+            commit_i(&bars->empty[second_slot<NST>(0)]);
           }
         }
       }
@@ -266,30 +278,30 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
         const int ks = first_slot<NST>(j);
         const int nks = first_slot<NST>(j + 1), nvs = second_slot<NST>(j + 1);
         const uint32_t nph = ((j + 1) / NST) & 1;
-        ok = ptx::wait(&bars->s_loaded, j & 1, ctl);
+        ok = wait_i(&bars->s_loaded, j & 1);
         if (!ok) break;
-        ok = ptx::wait(&bars->full[nks], nph, ctl);
+        ok = wait_i(&bars->full[nks], nph);
         if (!ok) break;
         ptx::tc_fence_after();
         more = bars->info[nks] != BT_INFO_END;
         if (more) {
           issue_s(nks);
-          ptx::tc_commit(&bars->s_full);
+          commit_i(&bars->s_full);
         }
-        ok = ptx::wait(&bars->p_ready, j & 1, ctl);
+        ok = wait_i(&bars->p_ready, j & 1);
         if (!ok) break;
         ptx::tc_fence_after();
         issue_dq(ks, j > 0);
-        ptx::tc_commit(&bars->empty[ks]);
+        commit_i(&bars->empty[ks]);
         if (!more) break;
-        ok = ptx::wait(&bars->full[nvs], nph, ctl);
+        ok = wait_i(&bars->full[nvs], nph);
         if (!ok) break;
         ptx::tc_fence_after();
         issue_dp(nvs);
-        ptx::tc_commit(&bars->dp_full);
-        ptx::tc_commit(&bars->empty[nvs]);
+        commit_i(&bars->dp_full);
+        commit_i(&bars->empty[nvs]);
       }
-      ptx::tc_commit(&bars->o_done);
+      commit_i(&bars->o_done);
       ptx::wait_drain(&bars->o_done, 0, ctl);
     }
   } else {
@@ -678,8 +690,20 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
           if (issued[s]) ptx::wait_drain(&bars->full[s], (issued[s] - 1) & 1, ctl);
         ptx::wait_drain(&bars->kv_full, 0, ctl);
       }
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
       // =========================== MMA issuer ===========================
+      // The whole warp issues: every lane sleeps in the hinted barrier wait
+      // and elect.sync picks the lane that issues each MMA and commit.
+      auto wait_i = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, ptx::wait_sleep(bar, parity, ctl));
+      };
+      auto commit_i = [&](uint64_t* bar) { ptx::tc_commit_warp(bar); };
+      auto mma_ss_i = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
+        ptx::mma_ss_warp(d, a, b, id, acc);
+      };
+      auto mma_ts_i = [&](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
+        ptx::mma_ts_warp(d, a, b, id, acc);
+      };
       const uint32_t sKa = ptx::smem_u32(sK), sVa = ptx::smem_u32(sV);
       const uint32_t sta = ptx::smem_u32(stages);
       auto slot_addr = [&](int sl) { return sta + (uint32_t)(sl * C::TILE_BYTES); };
@@ -688,8 +712,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
-          ptx::mma_ss(tmem + C::S_COL0, ptx::desc_sw128(sKa + off, 16, 1024),
-                      ptx::desc_sw128(qa + off, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss_i(tmem + C::S_COL0, ptx::desc_sw128(sKa + off, 16, 1024),
+                   ptx::desc_sw128(qa + off, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_dpt = [&](int ds) {       // dP^T = V dO^T
@@ -697,8 +721,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * BT_HALF_BYTES + (kk & 3) * 32;
-          ptx::mma_ss(tmem + C::DP_COL0, ptx::desc_sw128(sVa + off, 16, 1024),
-                      ptx::desc_sw128(da + off, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss_i(tmem + C::DP_COL0, ptx::desc_sw128(sVa + off, 16, 1024),
+                   ptx::desc_sw128(da + off, 16, 1024), C::IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
       // dV += P^T dO and dK += dS^T Q: the chunk's tiles read MN-major (their
@@ -708,9 +732,9 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < BT_N / 16; ++kk) {
           const uint32_t col = (kk >> 2) * 64 + (kk & 3) * 8;
-          ptx::mma_ts(tmem + C::DV_COL0, tmem + C::S_COL0 + col,
-                      ptx::desc_sw128(da + kk * 2048, BT_HALF_BYTES, 1024), C::IDESC_ACC,
-                      (accumulate || kk > 0) ? 1u : 0u);
+          mma_ts_i(tmem + C::DV_COL0, tmem + C::S_COL0 + col,
+                   ptx::desc_sw128(da + kk * 2048, BT_HALF_BYTES, 1024), C::IDESC_ACC,
+                   (accumulate || kk > 0) ? 1u : 0u);
         }
       };
       auto issue_dk = [&](int qs, bool accumulate) {   // dK += dS^T Q
@@ -718,9 +742,9 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < BT_N / 16; ++kk) {
           const uint32_t col = (kk >> 2) * 64 + (kk & 3) * 8;
-          ptx::mma_ts(tmem + C::DK_COL0, tmem + C::DP_COL0 + col,
-                      ptx::desc_sw128(qa + kk * 2048, BT_HALF_BYTES, 1024), C::IDESC_ACC,
-                      (accumulate || kk > 0) ? 1u : 0u);
+          mma_ts_i(tmem + C::DK_COL0, tmem + C::DP_COL0 + col,
+                   ptx::desc_sw128(qa + kk * 2048, BT_HALF_BYTES, 1024), C::IDESC_ACC,
+                   (accumulate || kk > 0) ? 1u : 0u);
         }
       };
       // The element-wise pass stores P^T first and dS^T second, so dV of
@@ -733,19 +757,19 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
       // behind its last reader: dV for dO, dK for Q.
       bool ok = KB.exists;
       bool more = false;
-      if (ok) ok = ptx::wait(&bars->kv_full, 0, ctl);
-      if (ok) ok = ptx::wait(&bars->full[q_slot<NQ>(0)], 0, ctl);
+      if (ok) ok = wait_i(&bars->kv_full, 0);
+      if (ok) ok = wait_i(&bars->full[q_slot<NQ>(0)], 0);
       if (ok) {
         ptx::tc_fence_after();
         more = bars->info[0] != BT_INFO_END;
         if (more) {
           issue_st(q_slot<NQ>(0));
-          ptx::tc_commit(&bars->s_full);
-          ok = ptx::wait(&bars->full[do_slot<NQ>(0)], 0, ctl);
+          commit_i(&bars->s_full);
+          ok = wait_i(&bars->full[do_slot<NQ>(0)], 0);
           if (ok) {
             ptx::tc_fence_after();
             issue_dpt(do_slot<NQ>(0));
-            ptx::tc_commit(&bars->dp_full);
+            commit_i(&bars->dp_full);
           }
         }
       }
@@ -753,32 +777,32 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
         const int qs = q_slot<NQ>(j), ds = do_slot<NQ>(j);
         const int nqs = q_slot<NQ>(j + 1), nds = do_slot<NQ>(j + 1);
         const uint32_t nph = ((j + 1) / NQ) & 1;
-        ok = ptx::wait(&bars->p_ready, j & 1, ctl);
+        ok = wait_i(&bars->p_ready, j & 1);
         if (!ok) break;
         ptx::tc_fence_after();
         issue_dv(ds, j > 0);
-        ptx::tc_commit(&bars->empty[ds]);
-        ok = ptx::wait(&bars->full[nqs], nph, ctl);
+        commit_i(&bars->empty[ds]);
+        ok = wait_i(&bars->full[nqs], nph);
         if (!ok) break;
         ptx::tc_fence_after();
         more = bars->info[(j + 1) % NQ] != BT_INFO_END;
         if (more) {
           issue_st(nqs);
-          ptx::tc_commit(&bars->s_full);
+          commit_i(&bars->s_full);
         }
-        ok = ptx::wait(&bars->ds_ready, j & 1, ctl);
+        ok = wait_i(&bars->ds_ready, j & 1);
         if (!ok) break;
         ptx::tc_fence_after();
         issue_dk(qs, j > 0);
-        ptx::tc_commit(&bars->empty[qs]);
+        commit_i(&bars->empty[qs]);
         if (!more) break;
-        ok = ptx::wait(&bars->full[nds], nph, ctl);
+        ok = wait_i(&bars->full[nds], nph);
         if (!ok) break;
         ptx::tc_fence_after();
         issue_dpt(nds);
-        ptx::tc_commit(&bars->dp_full);
+        commit_i(&bars->dp_full);
       }
-      ptx::tc_commit(&bars->o_done);
+      commit_i(&bars->o_done);
       ptx::wait_drain(&bars->o_done, 0, ctl);
     }
   } else {
