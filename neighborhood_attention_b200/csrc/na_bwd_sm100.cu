@@ -83,17 +83,6 @@ struct BtBars {
   ChunkGrid cg;
 };
 
-// Stage st = j % NST of chunk j owns tile slots 2 st and 2 st + 1; which of
-// them holds the first tile and which the second alternates with the round
-// j / NST, so that the first tile of chunk j + NST goes into the slot that
-// the second tile of chunk j frees (the dK / dV kernel: Q into dO's slot,
-// freed by dV before dK reads Q; the dQ kernel: K into V's slot, freed by dP
-// before dQ reads K).
-template <int NST>
-__device__ __forceinline__ int first_slot(int j) { return 2 * (j % NST) + ((j / NST) & 1); }
-template <int NST>
-__device__ __forceinline__ int second_slot(int j) { return 2 * (j % NST) + 1 - ((j / NST) & 1); }
-
 template <int D>
 constexpr size_t bt_smem_bytes() {
   return 1024 + (size_t)(2 + BtCfg<D, false>::NS) * BtCfg<D, false>::TILE_BYTES +
