@@ -13,10 +13,15 @@
 // warps per row quarter with no exchange between them.
 //
 // Roles (12 warps): warp 0 TMA producer (Q and dO once, then K / V chunks
-// through a ring), warp 1 TMEM allocation and the single MMA issuer, warps
-// 4-7 and 8-11 the element-wise part (warp 4+q keys 0-63, warp 8+q keys
-// 64-127 of every chunk, rows 32q..32q+31).  Every wait is bounded (see
+// into two-tile stages whose slots swap roles every round, see first_slot
+// in na_sched.cuh), warp 1 TMEM allocation and the MMA issuer (the whole
+// warp, elect.sync choosing the issuing lane), warps 4-7 and 8-11 the
+// element-wise part (warp 4+q keys 0-63, warp 8+q keys 64-127 of every
+// chunk, rows 32q..32q+31), which exponentiates S as soon as it is in
+// registers and waits for dP only to form dS.  Every wait is bounded (see
 // na_ptx.cuh); the chunk stream ends with a marker in the next K slot.
+// In both kernels S (S^T) of the next chunk is issued while the element-wise
+// warps still work on the current one.
 //
 // The dK / dV part (tc_bwd_dkdv_kernel) is key-stationary: for one 128-key
 // block per CTA (K and V resident in shared memory) and every chunk of the
@@ -27,6 +32,8 @@
 // (both window ends are monotone in the query coordinate), found by binary
 // search, so the same chunk walk and full / partial / empty labels as the
 // forward apply with the key block's inverse windows in place of windows.
+// Its element-wise pass stores P^T (over S^T) before it forms dS^T (over
+// dP^T), so dV of a chunk runs during the dS pass.
 //
 // TMEM columns (dQ kernel): S [0, 128), dP [128, 256) -- after the element-wise pass
 // dS of keys 64h..64h+63 sits as packed 16-bit pairs in [128 + 64h, 160 + 64h),
@@ -47,8 +54,8 @@ constexpr int BT_THREADS = 384;
 constexpr int BT_M = 128;                // query rows per block
 constexpr int BT_N = 128;                // keys per chunk
 constexpr int BT_HALF_BYTES = 128 * 128; // one 128-row x 64-element 16-bit box
-constexpr int BT_REGS_LOADER = 56;
-constexpr int BT_REGS_WORK = 216;
+constexpr int BT_REGS_LOADER = 64;
+constexpr int BT_REGS_WORK = 208;
 constexpr int BT_REGS_NEEDED = 128 * BT_REGS_LOADER + 256 * BT_REGS_WORK;
 constexpr uint32_t BT_INFO_END = 0xFFFFu;
 constexpr float BT_LOG2E = 1.4426950408889634f;
