@@ -45,6 +45,9 @@ CASES = {
     "fp32_d32": _case((16, 16), (5, 5), (1, 1), 32, dtype="f32", heads=3),
     "f16_d64": _case((18, 22), (7, 9), (2, 1), 64, dtype="f16"),
     "sta3d_medium_d128": _case((6, 16, 40), (6, 12, 24), (2, 4, 8), 128, tile=(2, 4, 8)),
+    # about ten chunks per block at head_dim 64: the four-stage slots of both
+    # gradient kernels go through several rounds
+    "sta3d_medium_d64": _case((6, 16, 40), (6, 12, 24), (2, 4, 8), 64, tile=(2, 4, 8)),
     # dilated windows (residue classes of different lengths)
     "dilated2d_d64": _case((23, 17), (5, 4), (1, 2), 64, dil=(3, 2),
                            mode=["clamped", "truncated"]),
