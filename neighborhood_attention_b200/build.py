@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libna.so")
 SOURCES = ["na_api.cu", "na_fwd_simt.cu", "na_fwd_gather.cu", "na_fwd_sm100.cu", "na_bwd_simt.cu",
            "na_bwd_sm100.cu"]
-HEADERS = ["na_internal.h", "na_sched.cuh", "na_ptx.cuh"]
+HEADERS = ["na_internal.h", "na_sched.cuh", "na_stages.cuh", "na_ptx.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

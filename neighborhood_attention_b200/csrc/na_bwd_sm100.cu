@@ -14,7 +14,7 @@
 //
 // Roles (12 warps): warp 0 TMA producer (Q and dO once, then K / V chunks
 // into two-tile stages whose slots swap roles every round, see first_slot
-// in na_sched.cuh), warp 1 TMEM allocation and the MMA issuer (the whole
+// in na_stages.cuh), warp 1 TMEM allocation and the MMA issuer (the whole
 // warp, elect.sync choosing the issuing lane), warps 4-7 and 8-11 the
 // element-wise part (warp 4+q keys 0-63, warp 8+q keys 64-127 of every
 // chunk, rows 32q..32q+31), which exponentiates S as soon as it is in
@@ -46,6 +46,7 @@
 
 #include "na_internal.h"
 #include "na_ptx.cuh"
+#include "na_stages.cuh"
 
 namespace na {
 namespace {

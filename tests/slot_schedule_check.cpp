@@ -1,5 +1,5 @@
 // Host check of the backward's two-tile stage slots (first_slot and
-// second_slot in na_sched.cuh): for 2, 3 and 4 stages and the first 1000
+// second_slot in na_stages.cuh): for 2, 3 and 4 stages and the first 1000
 // chunks, the two tiles of a chunk take the two slots of its stage; the
 // first tile of chunk j + NST takes the slot the second tile of chunk j
 // leaves and vice versa; and replaying the chunks in order, every slot is
@@ -8,7 +8,7 @@
 // Built and run by tests/test_slot_schedule.py; exit status 0 when all hold.
 #include <cstdint>
 #include <cstdio>
-#include "na_sched.cuh"
+#include "na_stages.cuh"
 using namespace na;
 
 template <int NST>
