@@ -189,3 +189,51 @@ def test_allocation_free_entry_refuses_dilation():
     st = f(*([p] * 5), 1, 1, iv([2, 64]), iv([8, 8]), iv([3, 3]), None, None, 1, ctypes.byref(o),
            None)
     assert st == na.NA_ERR_UNSUPPORTED
+
+
+_BWD_PTRS = ("q", "k", "v", "out", "dout", "lse", "dq", "dk", "dv", "delta")
+
+
+def _backward_call(lib, ptr_over=None, B=1, heads=1, dims=(2, 64), grid=(8, 8), window=(3, 3),
+                   stride=None, dtype=1, kernel=0):
+    import neighborhood_attention_b200 as na
+    iv = lambda xs: None if xs is None else (ctypes.c_int * len(xs))(*xs)
+    ptrs = {n: 256 for n in _BWD_PTRS}      # aligned, never dereferenced
+    ptrs.update(ptr_over or {})
+    f = lib.na_backward
+    f.argtypes = [ctypes.c_void_p] * 10 + [ctypes.c_int, ctypes.c_int] + \
+        [ctypes.POINTER(ctypes.c_int)] * 5 + [ctypes.c_int, ctypes.POINTER(na.na_options),
+                                              ctypes.c_void_p]
+    o = na.make_options(kernel=kernel)
+    return f(*[ctypes.c_void_p(ptrs[n]) if ptrs[n] else None for n in _BWD_PTRS], B, heads,
+             iv(dims), iv(grid), iv(window), iv(stride), None, dtype, ctypes.byref(o), None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    *[(dict(ptr_over={n: 0}), 1) for n in _BWD_PTRS],          # each pointer NULL
+    (dict(ptr_over={"q": 8}), 1),                              # 16-byte alignment
+    (dict(ptr_over={"dv": 264}), 1),
+    (dict(ptr_over={"lse": 258}), 1),                          # 4-byte alignment
+    (dict(ptr_over={"delta": 2}), 1),
+    (dict(B=0), 1),
+    (dict(heads=0), 1),
+    (dict(dims=(4, 64)), 1),
+    (dict(dims=(2, 48)), 2),
+    (dict(window=(9, 3)), 1),
+    (dict(stride=(4, 1)), 1),
+    (dict(dtype=0, kernel="tc"), 2),                           # tensor cores with fp32
+])
+def test_backward_argument_errors_need_no_device(kw, expect):
+    """na_backward refuses every malformed call on the host, before any device
+    work.  Fake pointers stand in for tensors, so this runs only where no
+    CUDA device is visible."""
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("host refusal test with fake pointers: CPU machines only")
+    import neighborhood_attention_b200 as na
+    if kw.get("kernel") == "tc":
+        kw = dict(kw, kernel=na.NA_KERNEL_TC)
+    lib = ctypes.CDLL(na.LIB_PATH)
+    assert _backward_call(lib, **kw) == expect
+    lib.na_last_error.restype = ctypes.c_char_p
+    assert lib.na_last_error().decode() != ""
