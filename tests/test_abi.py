@@ -80,6 +80,31 @@ def test_binding_refuses_cpu_tensors():
         na.na_forward(q, q, q, q.clone(), lse, window=(3, 3))
 
 
+@pytest.mark.parametrize("bad,match", [("cpu", "CUDA tensor"), ("shape", "v must match q"),
+                                       ("dtype", "dout must match q"),
+                                       ("lse_dtype", "lse must be float32"),
+                                       ("ndim", "expected")])
+def test_backward_binding_refuses_mismatched_tensors(bad, match):
+    """na.backward checks shapes, dtypes and devices before the library is
+    called; CPU tensors (all this test has) are refused last."""
+    import torch
+    import neighborhood_attention_b200 as na
+    q = torch.zeros(1, 1, 8, 8, 64, dtype=torch.bfloat16)
+    t = {n: q.clone() for n in ("k", "v", "out", "dout")}
+    lse = torch.zeros(1, 1, 8, 8)
+    window = (3, 3)
+    if bad == "shape":
+        t["v"] = torch.zeros(1, 1, 8, 4, 64, dtype=torch.bfloat16)
+    elif bad == "dtype":
+        t["dout"] = torch.zeros(1, 1, 8, 8, 64, dtype=torch.float16)
+    elif bad == "lse_dtype":
+        lse = torch.zeros(1, 1, 8, 8, dtype=torch.float64)
+    elif bad == "ndim":
+        window = (3, 3, 3)
+    with pytest.raises(ValueError, match=match):
+        na.backward(q, t["k"], t["v"], t["out"], lse, t["dout"], window=window)
+
+
 @pytest.mark.parametrize("mode", [3, -1, 100])
 def test_bad_window_mode_is_refused(mode):
     """An unknown na_window_mode is NA_ERR_INVALID_ARG, found on the host."""
