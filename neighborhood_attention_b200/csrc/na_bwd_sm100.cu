@@ -462,23 +462,6 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
 }
 
 // ----------------------------------------------------------------- dK dV --
-// First i in [0, L) whose window satisfies pred (false then true as i grows).
-template <class F>
-__device__ __forceinline__ int first_query(int L, F pred) {
-  int lo = 0, hi = L;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (pred(mid)) hi = mid; else lo = mid + 1;
-  }
-  return lo;
-}
-
-// Queries whose window holds key j in one dimension: [*i0, *i1).
-__device__ __forceinline__ void inverse_range(int L, int w, int s, int m, int j, int& i0, int& i1) {
-  i0 = first_query(L, [&](int i) { int lo, hi; window_range(L, w, s, m, i, lo, hi); return hi > j; });
-  i1 = first_query(L, [&](int i) { int lo, hi; window_range(L, w, s, m, i, lo, hi); return lo > j; });
-}
-
 template <int D, bool F16>
 struct BkCfg {
   static constexpr int TILE_BYTES = 128 * D * 2;

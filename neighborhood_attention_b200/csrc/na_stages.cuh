@@ -1,11 +1,31 @@
-// Tile-slot schedule of the backward kernels' two-tile stages, shared by the
-// device code and host checks (the same __host__ __device__ convention as
-// na_sched.cuh).
+// Schedule helpers of the backward kernels, shared by the device code and
+// host checks (the same __host__ __device__ convention as na_sched.cuh): the
+// inverse windows of the key-stationary dK / dV kernel and the tile-slot
+// schedule of both gradient kernels' two-tile stages.
 #pragma once
 
 #include "na_sched.cuh"
 
 namespace na {
+
+// First i in [0, L) whose window satisfies pred (false then true as i grows).
+template <class F>
+NA_HD int first_query(int L, F pred) {
+  int lo = 0, hi = L;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (pred(mid)) hi = mid; else lo = mid + 1;
+  }
+  return lo;
+}
+
+// Queries whose window holds key j in one dimension: [i0, i1).  Both window
+// ends are non-decreasing in the query coordinate (every mode), so the set is
+// an interval, found by two binary searches.
+NA_HD void inverse_range(int L, int w, int s, int m, int j, int& i0, int& i1) {
+  i0 = first_query(L, [&](int i) { int lo, hi; window_range(L, w, s, m, i, lo, hi); return hi > j; });
+  i1 = first_query(L, [&](int i) { int lo, hi; window_range(L, w, s, m, i, lo, hi); return lo > j; });
+}
 
 // Two-tile stages of the backward's pipelines: stage st = j % NST of chunk j
 // owns tile slots 2 st and 2 st + 1; which of them holds the chunk's first
