@@ -203,11 +203,20 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- CPU side --
+def workload_rows(w=None):
+    """Query rows of a workload: B * heads * grid tokens."""
+    w = WORKLOAD if w is None else w
+    return int(w["B"] * w["heads"] * np.prod(w["grid"]))
+
+
 def oracle_sample_rows(n_rows, seed=1):
-    w = WORKLOAD
-    N = int(np.prod(w["grid"]))
+    """n_rows distinct query rows drawn uniformly (sorted); every row when the
+    workload has no more than n_rows."""
+    total = workload_rows()
+    if n_rows >= total:
+        return np.arange(total, dtype=np.int64)
     rng = np.random.default_rng(seed)
-    return np.sort(rng.choice(w["B"] * w["heads"] * N, size=n_rows, replace=False)).astype(np.int64)
+    return np.sort(rng.choice(total, size=n_rows, replace=False)).astype(np.int64)
 
 
 def host_qkv():
@@ -254,11 +263,10 @@ def cpu_baseline(qkv, target_s=15.0):
     threads = os.cpu_count() or 1
     probe = max(64, threads * 8)
     _, dt = time_oracle(qkv, probe, threads)
-    n = int(min(200000, max(probe, probe * target_s / max(dt, 1e-3))))
+    n = min(workload_rows(), int(min(200000, max(probe, probe * target_s / max(dt, 1e-3)))))
     val, dt = time_oracle(qkv, n, threads)
     return {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"{n} query rows drawn uniformly from the workload's "
-                      f"{int(np.prod(WORKLOAD['grid'])) * WORKLOAD['heads'] * WORKLOAD['B']} "
+            "sample": f"{n} query rows drawn uniformly from the workload's {workload_rows()} "
                       f"(fp64 dense-mask oracle, {dt:.1f} s)"}
 
 
@@ -271,13 +279,12 @@ def run_reference(args, rank, world):
     _, dt = time_oracle(qkv, probe, threads)
     # each step a bounded sample sized so that warm-up + timed steps end within minutes
     budget = 120.0 / max(1, args.steps + args.warmup)
-    n = int(max(probe, probe * min(budget, 20.0) / max(dt, 1e-3)))
+    n = min(workload_rows(), int(max(probe, probe * min(budget, 20.0) / max(dt, 1e-3))))
     for _ in range(args.warmup):
         time_oracle(qkv, n, threads)
-    vals, tot = [], 0.0
+    tot = 0.0
     for _ in range(args.steps):
-        v, dt = time_oracle(qkv, n, threads)
-        vals.append(v)
+        _, dt = time_oracle(qkv, n, threads)
         tot += dt
     flops = 4.0 * WORKLOAD["head_dim"] * sampled_pairs(oracle_sample_rows(n)) * args.steps
     value = flops / tot / 1e12
