@@ -533,22 +533,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1)
 
   if (threadIdx.x == 0) {
     block_info(P.g, t, blk, bars->kb);
-    BlockInfo& ib = bars->ib;
-    ib.exists = bars->kb.exists;
-    for (int d = 0; d < 3; ++d) {
-      ib.o[d] = 0;
-      ib.n[d] = P.g.L[d];
-      if (!ib.exists) continue;
-      const int L = P.g.L[d], w = P.g.w[d], s = P.g.s[d], m = P.g.m[d];
-      const int k0 = bars->kb.o[d], k1 = bars->kb.o[d] + bars->kb.n[d] - 1;
-      int a0, a1, b0, b1;
-      inverse_range(L, w, s, m, k0, a0, a1);
-      inverse_range(L, w, s, m, k1, b0, b1);
-      ib.lo[d] = a0;     // union of the keys' query ranges: [I0(k0), I1(k1))
-      ib.hi[d] = b1;
-      ib.ilo[d] = b0;    // intersection: [I0(k1), I1(k0))
-      ib.ihi[d] = a1;
-    }
+    key_block_query_box(P.g, bars->kb, bars->ib);
     chunk_grid_for(&bars->ib, 1, P.kb, bars->cg);
     ptx::mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < 2 * NQ; ++s) {

@@ -27,6 +27,30 @@ NA_HD void inverse_range(int L, int w, int s, int m, int j, int& i0, int& i1) {
   i1 = first_query(L, [&](int i) { int lo, hi; window_range(L, w, s, m, i, lo, hi); return lo > j; });
 }
 
+// Query side of one key block kb (the dK / dV kernel's work item), as a
+// BlockInfo over the whole grid so that chunk_grid_for / chunk_status walk
+// query chunks the way the forward walks key chunks.  Per dimension, with k0
+// and k1 the block's first and last keys inside the grid: [lo, hi) =
+// [I0(k0), I1(k1)), the queries whose window meets the block, and
+// [ilo, ihi) = [I0(k1), I1(k0)), those whose window holds all of it.
+NA_HD void key_block_query_box(const Geom& g, const BlockInfo& kb, BlockInfo& ib) {
+  ib.exists = kb.exists;
+  for (int d = 0; d < 3; ++d) {
+    ib.o[d] = 0;
+    ib.n[d] = g.L[d];
+    if (!ib.exists) continue;
+    const int L = g.L[d], w = g.w[d], s = g.s[d], m = g.m[d];
+    const int k0 = kb.o[d], k1 = kb.o[d] + kb.n[d] - 1;
+    int a0, a1, b0, b1;
+    inverse_range(L, w, s, m, k0, a0, a1);
+    inverse_range(L, w, s, m, k1, b0, b1);
+    ib.lo[d] = a0;
+    ib.hi[d] = b1;
+    ib.ilo[d] = b0;
+    ib.ihi[d] = a1;
+  }
+}
+
 // Two-tile stages of the backward's pipelines: stage st = j % NST of chunk j
 // owns tile slots 2 st and 2 st + 1; which of them holds the chunk's first
 // tile and which its second alternates with the round j / NST, so that the
