@@ -7,8 +7,9 @@
 // the block and every query of the grid checks that:
 //  - every query that attends some key of the block lies in a visited chunk;
 //  - every visited chunk holds at least one such query;
-//  - in a FULL chunk every query inside the grid attends every key of the block.
-// Built and run by tests/test_inverse_window.py; exit status 0 when all hold.
+//  - a FULL chunk lies inside the grid and every query of it attends every
+//    key of the block.
+// Built and run by tests/test_schedule_walks.py; exit status 0 when all hold.
 #include <cstdint>
 #include <cstdio>
 #include <vector>
@@ -77,6 +78,9 @@ int main() {
         const int st = chunk_status(ib, it.a, qc);
         if (st == CHUNK_EMPTY) continue;
         ++chunks;
+        bool inside = true;
+        for (int d = 0; d < 3; ++d) inside = inside && it.a[d] >= 0 && it.a[d] + qc[d] <= g.L[d];
+        if (st == CHUNK_FULL && !inside) ++bad;
         bool holds_one = false;
         for (int y0 = it.a[0]; y0 < it.a[0] + qc[0] && y0 < g.L[0]; ++y0)
           for (int y1 = it.a[1]; y1 < it.a[1] + qc[1] && y1 < g.L[1]; ++y1)

@@ -23,17 +23,3 @@ def test_inverse_range_is_the_set_of_queries_that_see_the_key(tmp_path):
     assert out.returncode == 0, out.stdout + out.stderr
     assert out.stdout.count(" 0 wrong") == 2, out.stdout
 
-
-@pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
-def test_key_block_walk_covers_every_attending_query(tmp_path):
-    """The dK / dV kernel's walk over query chunks (key_block_query_box,
-    chunk_grid_for, chunk_status) on random 1-D, 2-D and 3-D problems in
-    every window mode: every query that attends a key of the block lies in a
-    visited chunk, every visited chunk holds one, and FULL chunks need no mask."""
-    exe = tmp_path / "key_block_walk_check"
-    subprocess.check_call(["g++", "-O2", "-std=c++17", "-I",
-                           os.path.join(ROOT, "neighborhood_attention_b200", "csrc"),
-                           "-o", str(exe), os.path.join(ROOT, "tests", "key_block_walk_check.cpp")])
-    out = subprocess.run([str(exe)], capture_output=True, text=True)
-    assert out.returncode == 0, out.stdout + out.stderr
-    assert " 0 wrong" in out.stdout
