@@ -62,6 +62,8 @@ def _call(lib, q=16, dims=(2, 64), grid=(8, 8), window=(3, 3), stride=None, tile
     (dict(stride=(0, 1)), 1),
     (dict(tile=(0, 4)), 1),
     (dict(dtype=7), 1),
+    (dict(B=1 << 16, heads=1 << 15), 2),            # B * heads = 2^31 > 2^30
+    (dict(dims=(3, 64), grid=(2048, 2048, 1024), window=(3, 3, 3)), 2),   # 2^32 tokens
 ])
 def test_argument_errors_need_no_device(kw, expect):
     import neighborhood_attention_b200 as na
@@ -247,6 +249,8 @@ def _backward_call(lib, ptr_over=None, B=1, heads=1, dims=(2, 64), grid=(8, 8), 
     (dict(window=(9, 3)), 1),
     (dict(stride=(4, 1)), 1),
     (dict(dtype=0, kernel="tc"), 2),                           # tensor cores with fp32
+    (dict(B=1 << 16, heads=1 << 15), 2),                       # B * heads = 2^31 > 2^30
+    (dict(dims=(3, 64), grid=(2048, 2048, 1024), window=(3, 3, 3)), 2),   # 2^32 tokens
 ])
 def test_backward_argument_errors_need_no_device(kw, expect):
     """na_backward refuses every malformed call on the host, before any device
