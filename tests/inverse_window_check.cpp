@@ -1,6 +1,9 @@
 // Host check of the dK / dV kernel's inverse windows (inverse_range in
 // na_stages.cuh), for every 1-D grid length up to 40, window, stride and
 // window mode:
+//  - both ends of the window (window_range) never decrease as the query
+//    coordinate grows: the premise of the query-block key boxes, of the
+//    window-gather kernel's staged key box and of the inverse windows;
 //  - for every key j, the queries whose window (window_range) holds j are
 //    exactly [i0, i1), and i0, i1 never decrease as j grows;
 //  - for every key block [k0, k1] (grid lengths up to 24, all blocks), the
@@ -22,7 +25,10 @@ int main() {
       for (int s = 1; s <= w; ++s)
         for (int m = WIN_CLAMPED; m <= WIN_CAUSAL; ++m) {
           std::vector<int> lo(L), hi(L), i0(L), i1(L);
-          for (int i = 0; i < L; ++i) window_range(L, w, s, m, i, lo[i], hi[i]);
+          for (int i = 0; i < L; ++i) {
+            window_range(L, w, s, m, i, lo[i], hi[i]);
+            if (i > 0 && (lo[i] < lo[i - 1] || hi[i] < hi[i - 1])) ++bad;
+          }
           for (int j = 0; j < L; ++j) {
             inverse_range(L, w, s, m, j, i0[j], i1[j]);
             if (j > 0 && (i0[j] < i0[j - 1] || i1[j] < i1[j - 1])) ++bad;
