@@ -4,6 +4,7 @@ that never exceeds the workload's own query rows, and, under a two-process
 launch, a line from rank 0 only while the other rank exits 0 without work."""
 import json
 import os
+import socket
 import subprocess
 import sys
 
@@ -51,10 +52,16 @@ def test_reference_arm_prints_one_contract_line():
     assert line["config"]["sample_rows_per_step"] == 512
 
 
+def _free_port():
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
 def test_reference_arm_two_ranks_only_rank0_prints():
     env = dict(os.environ, MASTER_ADDR="127.0.0.1")
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
-           "--master-addr", "127.0.0.1", "--master-port", "29631", "bench.py", "--impl",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--impl",
            "reference", "--gpus", "2", "--config", "1", "--steps", "1", "--warmup", "3"]
     out = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stderr[-2000:]
