@@ -122,10 +122,11 @@ typedef struct {
   int kvchunk[3];           /* 0s: automatic; else the key chunk shape (product 128 for TC,
                                32 for SIMT) */
   long long wait_timeout_ns;/* bound on each in-kernel wait; <= 0: 4 s (or env NA_WAIT_TIMEOUT_MS) */
-  int debug_flags;          /* testing hook, 0 in normal use.  1: the tensor-core kernel's
-                               loader withholds the first key chunk, so the consumer's bounded
-                               wait expires and the timeout path (NA_ERR_TIMEOUT from
-                               na_sync_status) is exercised without any fault or hang. */
+  int debug_flags;          /* TESTING HOOK, not a supported option: leave it 0.  1: the
+                               tensor-core forward kernel's loader withholds the first key
+                               chunk, so the consumer's bounded wait expires and the timeout
+                               path (NA_ERR_TIMEOUT from na_sync_status) is exercised without
+                               any fault or hang; the outputs of such a call are undefined. */
   int window_mode[3];       /* na_window_mode of grid dimension i (i < ndim, the order of
                                `window`); entries from ndim on are ignored.  0 = clamped. */
   int dilation[3];          /* dilation of grid dimension i (i < ndim); 0 or 1 = none.  The
@@ -166,9 +167,11 @@ na_status na_forward_ex(const void* q, const void* k, const void* v, void* out, 
  *                     no atomics, deterministic).
  *   delta             device float32 [B, heads, X1..Xn] workspace (written: D_i).
  * Other arguments, options (scale, window_mode) and errors as na_forward_ex.
- * Kernels: D_i and dk / dv on the CUDA cores (fp32 arithmetic); dq on the
- * tensor cores (tcgen05, fp32 accumulation) for bf16 / f16 with head_dim 64 or
- * 128 unless opt->kernel = NA_KERNEL_SIMT, else on the CUDA cores.
+ * Kernels: the row delta D_i on the CUDA cores (fp32 arithmetic); for bf16 /
+ * f16 with head_dim 64 or 128, dq (one kernel per query block) and dk / dv
+ * (one kernel per key block, over the queries whose windows hold it) on the
+ * tensor cores (tcgen05, fp32 accumulation in tensor memory) unless
+ * opt->kernel = NA_KERNEL_SIMT; every other input on the CUDA cores.
  * opt->kernel = NA_KERNEL_TC for other inputs, and NA_KERNEL_GATHER (a
  * forward-only kernel), are NA_ERR_UNSUPPORTED.  A bounded
  * in-kernel wait that expires is reported by na_sync_status.
@@ -256,11 +259,12 @@ na_status na_block_schedule(const int dims[2], const int* grid, const int* windo
 int na_version(void);
 
 /*
- * na_selftest_exp2 -- y[i] = 2^x[i] computed by the FMA-pipe polynomial the
- * tensor-core kernel uses for part of its softmax exponentials (degree-3
- * minimax fit of 2^f on [-1/2, 1/2], relative error <= 1.02e-4 for
- * -125 <= x <= 8).  x and y are device float arrays of n elements; enqueued on
- * `stream`.  For tests: it checks the device arithmetic against exact values.
+ * na_selftest_exp2 -- TESTING HOOK, not part of the attention interface.
+ * y[i] = 2^x[i] computed by the FMA-pipe polynomial that the tensor-core
+ * kernels can use for a share of their softmax exponentials (degree-3 minimax
+ * fit of 2^f on [-1/2, 1/2], relative error <= 1.02e-4 for -125 <= x <= 8).
+ * x and y are device float arrays of n elements; enqueued on `stream`.  It
+ * lets the tests check that device arithmetic against exact values.
  */
 na_status na_selftest_exp2(const float* x, float* y, int n, void* stream);
 
@@ -291,17 +295,33 @@ na_status na_selftest_exp2(const float* x, float* y, int n, void* stream);
  * (cudaGetSymbolAddress) with that device current; make that first call before
  * any stream capture.
  *
+ * The looked-up address belongs to the device's current context: after a
+ * cudaDeviceReset (or anything else that destroys the primary context) the
+ * library's cached address is stale, so do not reset a device between calls.
+ *
  * Sharing: all calls on a device use the same array, which keeps the last
  * call's contents.  Each call clears the status word on `stream` before its
  * kernel, so calls whose kernels overlap on the GPU (different streams, no
  * ordering between them) race on it.  A bounded in-kernel wait that expires
- * leaves out/lse undefined and is not reported here (na_sync_status reads only
- * na_forward's status word); use na_forward when that report is needed.
+ * leaves out/lse undefined; na_noalloc_status reports it (na_sync_status
+ * reads only na_forward's status word).
  */
 na_status na_forward_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
                              int B, int heads, const int dims[2], const int* grid,
                              const int* window, const int* stride, const int* tile,
                              na_dtype dtype, const na_options* opt, void* stream);
+
+/*
+ * na_noalloc_status -- na_sync_status for na_forward_noalloc: synchronise
+ * `stream`, then read this device's status word in the static array (copied
+ * into a host int, so no device memory is allocated) and clear it if set.
+ * NA_ERR_TIMEOUT if a na_forward_noalloc kernel since the last clear gave up on
+ * a bounded wait (its out / lse are then undefined); NA_ERR_CUDA if a copy or
+ * the synchronisation failed; NA_OK otherwise, also when na_forward_noalloc was
+ * never called on this device.  Like the calls it reports on, it shares the
+ * array with every other caller on the device.
+ */
+na_status na_noalloc_status(void* stream);
 
 #ifdef __cplusplus
 }

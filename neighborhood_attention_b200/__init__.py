@@ -7,8 +7,8 @@ no fallback of any kind.
 
 Functions keep the C-ABI names (``include/na.h``): ``na_forward``,
 ``na_forward_ex``, ``na_sync_status``, ``na_plan``, ``na_window_start``,
-``na_window_range``, ``na_block_schedule``, ``na_backward``, ``na_status_string``,
-``na_last_error``.
+``na_window_range``, ``na_block_schedule``, ``na_backward``, ``na_forward_noalloc``,
+``na_noalloc_status``, ``na_status_string``, ``na_last_error``.
 """
 from __future__ import annotations
 
@@ -96,6 +96,8 @@ def _load():
     lib.na_version.restype = ctypes.c_int
     lib.na_forward_noalloc.argtypes = lib.na_forward_ex.argtypes
     lib.na_forward_noalloc.restype = ctypes.c_int
+    lib.na_noalloc_status.argtypes = [vp]
+    lib.na_noalloc_status.restype = ctypes.c_int
     lib.na_backward.argtypes = [vp] * 10 + [ctypes.c_int, ctypes.c_int, i32p, i32p, i32p, i32p,
                                             i32p, ctypes.c_int, ctypes.POINTER(na_options), vp]
     lib.na_backward.restype = ctypes.c_int
@@ -334,6 +336,12 @@ def na_selftest_exp2(x, y, stream=None):
 def na_sync_status(stream=None):
     """Synchronise the stream and raise NaError if a kernel's bounded wait expired."""
     _check(_lib.na_sync_status(_stream_ptr(stream)))
+
+
+def na_noalloc_status(stream=None):
+    """Synchronise the stream and raise NaError if a na_forward_noalloc kernel's
+    bounded wait expired (read from the library's static array; no allocation)."""
+    _check(_lib.na_noalloc_status(_stream_ptr(stream)))
 
 
 def na_plan(grid, window, stride=None, tile=None, head_dim=128, dtype=NA_BF16, options=None):

@@ -149,7 +149,8 @@ na_status read_problem(const int dims[2], const int* grid, const int* window, co
     P.g.s[pad + i] = s;
     if (tile) P.tile[pad + i] = tile[i];
     N *= L;
-    if (N > (1LL << 31)) return fail(NA_ERR_UNSUPPORTED, "grid has more than 2^31 tokens");
+    // Token counts travel to the kernels as int: 2^31 tokens or more are refused.
+    if (N >= (1LL << 31)) return fail(NA_ERR_UNSUPPORTED, "grid has 2^31 tokens or more");
   }
   P.opt = opt ? *opt : na_default_options();
   if (P.opt.kernel < NA_KERNEL_AUTO || P.opt.kernel > NA_KERNEL_GATHER)
@@ -899,6 +900,33 @@ na_status na_block_schedule(const int dims[2], const int* grid, const int* windo
   return NA_OK;
 }
 
+na_status na_noalloc_status(void* stream) {
+  g_err[0] = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return NA_OK;
+  void* p = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    p = g_noalloc_ptr[dev];
+  }
+  if (!p) return NA_OK;   // no na_forward_noalloc call on this device yet
+  // A plain host int as the destination: the copy needs no device memory.
+  int h = 0;
+  e = cudaMemcpyAsync(&h, p, sizeof h, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return fail(NA_ERR_CUDA, "reading the scratch status: %s", cudaGetErrorString(e));
+  if (h != DEV_OK) {
+    e = cudaMemsetAsync(p, 0, sizeof(int), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return fail(NA_ERR_CUDA, "clearing the scratch status: %s", cudaGetErrorString(e));
+    return fail(NA_ERR_TIMEOUT, "a bounded in-kernel wait expired (code %d)", h);
+  }
+  return NA_OK;
+}
+
 na_status na_forward_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
                              int B, int heads, const int dims[2], const int* grid,
                              const int* window, const int* stride, const int* tile,
@@ -939,7 +967,7 @@ na_status na_forward_noalloc(const void* q, const void* k, const void* v, void* 
   for (int d = 0; d < 3; ++d) L.kb[d] = plan.kb[d];
   L.map = identity_map(P.g.L);
   L.BH = (int)BH;
-  L.N = P.g.L[0] * P.g.L[1] * P.g.L[2];
+  L.N = (int)((long long)P.g.L[0] * P.g.L[1] * P.g.L[2]);   // < 2^31 (read_problem)
   L.D = P.D;
   L.f16 = P.dtype == NA_F16;
   L.scale_log2 = scale * 1.4426950408889634f;

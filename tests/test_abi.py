@@ -64,6 +64,7 @@ def _call(lib, q=16, dims=(2, 64), grid=(8, 8), window=(3, 3), stride=None, tile
     (dict(dtype=7), 1),
     (dict(B=1 << 16, heads=1 << 15), 2),            # B * heads = 2^31 > 2^30
     (dict(dims=(3, 64), grid=(2048, 2048, 1024), window=(3, 3, 3)), 2),   # 2^32 tokens
+    (dict(dims=(3, 64), grid=(2048, 1024, 1024), window=(3, 3, 3)), 2),   # exactly 2^31 tokens
 ])
 def test_argument_errors_need_no_device(kw, expect):
     import neighborhood_attention_b200 as na
@@ -251,6 +252,7 @@ def _backward_call(lib, ptr_over=None, B=1, heads=1, dims=(2, 64), grid=(8, 8), 
     (dict(dtype=0, kernel="tc"), 2),                           # tensor cores with fp32
     (dict(B=1 << 16, heads=1 << 15), 2),                       # B * heads = 2^31 > 2^30
     (dict(dims=(3, 64), grid=(2048, 2048, 1024), window=(3, 3, 3)), 2),   # 2^32 tokens
+    (dict(dims=(3, 64), grid=(2048, 1024, 1024), window=(3, 3, 3)), 2),   # exactly 2^31 tokens
 ])
 def test_backward_argument_errors_need_no_device(kw, expect):
     """na_backward refuses every malformed call on the host, before any device
@@ -266,3 +268,21 @@ def test_backward_argument_errors_need_no_device(kw, expect):
     assert _backward_call(lib, **kw) == expect
     lib.na_last_error.restype = ctypes.c_char_p
     assert lib.na_last_error().decode() != ""
+
+
+@pytest.mark.parametrize("grid,expect", [((2048, 1024, 1024), 2),     # exactly 2^31 tokens
+                                         ((2048, 2048, 1024), 2)])    # 2^32 tokens
+def test_noalloc_refuses_token_counts_an_int_cannot_hold(grid, expect):
+    """The allocation-free entry point shares the forward's host checks: a grid
+    of 2^31 tokens or more is refused before any device work (fake pointers)."""
+    import neighborhood_attention_b200 as na
+    lib = ctypes.CDLL(na.LIB_PATH)
+    iv = lambda xs: (ctypes.c_int * len(xs))(*xs)
+    f = lib.na_forward_noalloc
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_int] + \
+        [ctypes.POINTER(ctypes.c_int)] * 5 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
+    p = ctypes.c_void_p(16)
+    assert f(p, p, p, p, p, 1, 1, iv((3, 64)), iv(grid), iv((3, 3, 3)), None, None, 1, None,
+             None) == expect
+    lib.na_last_error.restype = ctypes.c_char_p
+    assert "2^31" in lib.na_last_error().decode()

@@ -10,6 +10,10 @@ last so that a failure here never hides the other tests in a run that stops at
 the first failure, and it passes both alone and after the rest of the suite.
 """
 import ctypes
+import json
+import os
+import subprocess
+import sys
 
 import numpy as np
 import pytest
@@ -82,3 +86,81 @@ def test_noalloc_rejects_what_it_cannot_run():
     st = _noalloc_c_abi(q, k, v, out, lse, (8, 8), (3, 3), (1, 1), (8, 8))
     assert st == na.NA_ERR_UNSUPPORTED
     assert na.na_last_error()
+
+
+def test_noalloc_reports_an_expired_wait():
+    """A bounded in-kernel wait that runs out inside na_forward_noalloc (the
+    testing hook withholds one key chunk; wait limit 50 ms) is reported by
+    na_noalloc_status, which reads the static array without allocating; the
+    report is cleared and the next call is correct."""
+    grid, window, stride, tile, d = CASES[0]
+    q, k, v = _inputs(913, grid, d)
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
+    opts = na.make_options(kernel=na.NA_KERNEL_TC, wait_timeout_ns=50_000_000, debug_flags=1)
+    na.na_forward_noalloc(q, k, v, out, lse, window, stride, tile, options=opts)
+    with pytest.raises(na.NaError) as ei:
+        na.na_noalloc_status()
+    assert ei.value.status == na.NA_ERR_TIMEOUT
+    na.na_noalloc_status()          # cleared by the report
+    na.na_sync_status()             # na_forward's own status word saw nothing
+    na.na_forward_noalloc(q, k, v, out, lse, window, stride, tile)
+    na.na_noalloc_status()
+    ref_o, ref_l = na.forward(q, k, v, window, stride, tile)
+    na.na_sync_status()
+    assert (out.float() - ref_o.float()).abs().max().item() <= TOL["out_max"]
+    assert (lse - ref_l).abs().max().item() <= TOL["lse_max"]
+
+
+_FRESH = r"""
+import ctypes, json, sys
+import numpy as np
+import torch
+sys.path.insert(0, sys.argv[1])
+import neighborhood_attention_b200 as na
+import seeded_inputs
+grid, window, stride, tile, d = (8, 16, 16), (4, 8, 8), (2, 4, 4), (2, 4, 4), 64
+arrs = seeded_inputs.qkv(914, 1, 3, grid, d, "bf16")
+q, k, v = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda() for a in arrs]
+outs = [torch.empty_like(q) for _ in range(3)]
+lses = [torch.empty(q.shape[:-1], dtype=torch.float32, device="cuda") for _ in range(3)]
+torch.cuda.synchronize()
+na.na_sync_status()      # the library's runtime is up; na_forward has not run, so no status word
+free = [torch.cuda.mem_get_info()[0]]
+for i in range(2):       # the first na_forward_noalloc calls of this process
+    na.na_forward_noalloc(q, k, v, outs[i], lses[i], window, stride, tile)
+    na.na_noalloc_status()
+    free.append(torch.cuda.mem_get_info()[0])
+# Control: na_forward's first call allocates its status word with cudaMalloc.
+lib = ctypes.CDLL(na.LIB_PATH)
+iv = lambda xs: (ctypes.c_int * len(xs))(*[int(x) for x in xs])
+lib.na_forward.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int, ctypes.c_int] +     [ctypes.POINTER(ctypes.c_int)] * 5 + [ctypes.c_int, ctypes.c_void_p]
+st = lib.na_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), outs[2].data_ptr(),
+                    lses[2].data_ptr(), 1, 3, iv([3, d]), iv(grid), iv(window), iv(stride),
+                    iv(tile), na.NA_BF16, None)
+assert st == 0
+na.na_sync_status()
+free.append(torch.cuda.mem_get_info()[0])
+err = max((outs[i].float() - outs[2].float()).abs().max().item() for i in range(2))
+print(json.dumps({"free": free, "err": err}))
+"""
+
+
+def test_noalloc_first_calls_in_a_fresh_process_take_no_device_memory():
+    """In a process where na_forward has never run, the first two
+    na_forward_noalloc calls leave the device's free memory unchanged
+    (cudaMemGetInfo), while na_forward's first call -- which allocates its
+    4-byte status word with cudaMalloc -- lowers it: the measurement sees an
+    allocation of that size, and this entry point makes none.  Modules load
+    eagerly in the child so that loading the library's code is not mistaken
+    for an allocation."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, CUDA_MODULE_LOADING="EAGER")
+    r = subprocess.run([sys.executable, "-c", _FRESH, root], env=env, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-3000:]
+    res = json.loads(r.stdout.strip().splitlines()[-1])
+    free = res["free"]
+    assert free[1] == free[0] and free[2] == free[0], f"free bytes changed: {free}"
+    assert free[3] < free[2], f"control allocation not visible: {free}"
+    assert res["err"] <= TOL["out_max"]
