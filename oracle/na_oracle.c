@@ -512,11 +512,13 @@ int na_oracle_backward(const void* q, const void* k, const void* v, const void* 
 /*
  * Gradients on sampled rows of one (batch, head) slice bh, for parity checks
  * at sizes where the full backward is too slow: first lse_t and
- * D_t = <dO_t, out_t> for every query t of the slice (threads split the
- * queries), then dq for the query rows `qrows` and dk, dv for the key rows
- * `krows` (token indices within the slice), each summed over the queries
- * whose window holds the key.  Outputs [nq, d] and [nk, d] fp64.  Same
- * definitions as na_oracle_backward, which it equals on every row.
+ * D_t = <dO_t, out_t> for the queries t the sampled rows depend on -- the
+ * query rows `qrows` themselves and every query whose window holds one of the
+ * key rows `krows` (token indices within the slice) -- then dq for the query
+ * rows and dk, dv for the key rows, each summed over the queries whose window
+ * holds the key.  Threads split the queries of the first step and the rows of
+ * the second.  Outputs [nq, d] and [nk, d] fp64.  Same definitions as
+ * na_oracle_backward, which it equals on every row.
  */
 typedef struct {
     const void *q, *k, *v, *dout;
@@ -524,7 +526,8 @@ typedef struct {
     const int *L, *w, *s, *mode;
     long long N, W, bh;
     double scale;
-    long long t_begin, t_end;
+    const long long* list;          /* the queries whose lse_t, D_t are needed */
+    long long i_begin, i_end;       /* this thread's share of `list` */
     double *lse, *delta;
     int status;
 } stat_job;
@@ -537,7 +540,8 @@ static void* stat_worker(void* arg) {
     long long* idx = (long long*)malloc(sizeof(long long) * (size_t)J->W);
     uint8_t* mask = (uint8_t*)malloc((size_t)J->N);
     if (!z || !idx || !mask) { J->status = -2; goto done; }
-    for (long long t = J->t_begin; t < J->t_end; ++t) {
+    for (long long i = J->i_begin; i < J->i_end; ++i) {
+        const long long t = J->list[i];
         na_oracle_mask_row(J->ndim, J->L, J->w, J->s, J->mode, t, mask);
         const size_t qoff = hoff + (size_t)t * (size_t)d;
         long long cnt = 0;
@@ -571,6 +575,93 @@ done:
     return NULL;
 }
 
+/* Does the window of query t (grid coordinates qi) hold key kj? */
+static int window_holds(int ndim, const int* L, const int* w, const int* s, const int* mode,
+                        const int* qi, const int* kj) {
+    for (int a = 0; a < ndim; ++a) {
+        int lo, hi;
+        na_oracle_window(L[a], w[a], s[a], mode ? mode[a] : 0, qi[a], &lo, &hi);
+        if (kj[a] < lo || kj[a] >= hi) return 0;
+    }
+    return 1;
+}
+
+typedef struct {
+    const void *q, *k, *v, *dout;
+    int dtype, ndim, d;
+    const int *L, *w, *s, *mode;
+    long long N, bh;
+    double scale;
+    const double *lse, *delta;
+    const long long *qrows, *krows;
+    long long q_begin, q_end, k_begin, k_end;   /* this thread's sampled rows */
+    double *dq, *dk, *dv;
+    int status;
+} grad_job;
+
+static void* grad_worker(void* arg) {
+    grad_job* J = (grad_job*)arg;
+    const int d = J->d, ndim = J->ndim, dt = J->dtype;
+    const void *Q = J->q, *K = J->k, *V = J->v, *DO = J->dout;
+    const size_t hoff = (size_t)J->bh * (size_t)J->N * (size_t)d;
+    uint8_t* mask = (uint8_t*)malloc((size_t)J->N);
+    if (!mask) { J->status = -2; return NULL; }
+    /* dq of the sampled query rows */
+    for (long long r = J->q_begin; r < J->q_end; ++r) {
+        const long long t = J->qrows[r];
+        na_oracle_mask_row(ndim, J->L, J->w, J->s, J->mode, t, mask);
+        const size_t qoff = hoff + (size_t)t * (size_t)d;
+        double* g = J->dq + (size_t)r * d;
+        for (int c = 0; c < d; ++c) g[c] = 0.0;
+        for (long long j = 0; j < J->N; ++j) {
+            if (!mask[j]) continue;
+            const size_t koff = hoff + (size_t)j * (size_t)d;
+            double zq = 0.0, dp = 0.0;
+            for (int c = 0; c < d; ++c) {
+                zq += load_in(Q, dt, qoff + c) * load_in(K, dt, koff + c);
+                dp += load_in(DO, dt, qoff + c) * load_in(V, dt, koff + c);
+            }
+            const double p = exp(J->scale * zq - J->lse[t]);
+            const double dz = p * (dp - J->delta[t]);
+            for (int c = 0; c < d; ++c) g[c] += J->scale * dz * load_in(K, dt, koff + c);
+        }
+    }
+    /* dk, dv of the sampled key rows: over every query whose window holds the key */
+    for (long long r = J->k_begin; r < J->k_end; ++r) {
+        const long long j = J->krows[r];
+        const size_t koff = hoff + (size_t)j * (size_t)d;
+        double* gk = J->dk + (size_t)r * d;
+        double* gv = J->dv + (size_t)r * d;
+        for (int c = 0; c < d; ++c) { gk[c] = 0.0; gv[c] = 0.0; }
+        int kj[NA_ORACLE_MAXDIM];
+        unflatten(j, ndim, J->L, kj);
+        int qi[NA_ORACLE_MAXDIM];
+        for (int a = 0; a < ndim; ++a) qi[a] = 0;
+        for (long long t = 0; t < J->N; ++t) {
+            if (window_holds(ndim, J->L, J->w, J->s, J->mode, qi, kj)) {
+                const size_t qoff = hoff + (size_t)t * (size_t)d;
+                double zq = 0.0, dp = 0.0;
+                for (int c = 0; c < d; ++c) {
+                    zq += load_in(Q, dt, qoff + c) * load_in(K, dt, koff + c);
+                    dp += load_in(DO, dt, qoff + c) * load_in(V, dt, koff + c);
+                }
+                const double p = exp(J->scale * zq - J->lse[t]);
+                const double dz = p * (dp - J->delta[t]);
+                for (int c = 0; c < d; ++c) {
+                    gk[c] += J->scale * dz * load_in(Q, dt, qoff + c);
+                    gv[c] += p * load_in(DO, dt, qoff + c);
+                }
+            }
+            for (int a = ndim - 1; a >= 0; --a) { /* advance the row-major query counter */
+                if (++qi[a] < J->L[a]) break;
+                qi[a] = 0;
+            }
+        }
+    }
+    free(mask);
+    return NULL;
+}
+
 int na_oracle_backward_sampled(const void* q, const void* k, const void* v, const void* dout,
                                int in_dtype, long long BH, long long bh, int ndim, const int* L,
                                const int* w, const int* s, const int* mode, int d, double scale,
@@ -581,25 +672,52 @@ int na_oracle_backward_sampled(const void* q, const void* k, const void* v, cons
     if ((nq && (!qrows || !dq)) || (nk && (!krows || !dk || !dv))) return -1;
     if (in_dtype != IN_F32 && in_dtype != IN_BF16 && in_dtype != IN_F16) return -1;
     if (check_geometry(ndim, L, w, s, mode, NULL, &N)) return -1;
+    for (long long r = 0; r < nq; ++r) if (qrows[r] < 0 || qrows[r] >= N) return -1;
+    for (long long r = 0; r < nk; ++r) if (krows[r] < 0 || krows[r] >= N) return -1;
     long long W = 1;
     for (int a = 0; a < ndim; ++a) W *= w[a];
     if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
     double* lse = (double*)malloc(sizeof(double) * (size_t)N);
     double* delta = (double*)malloc(sizeof(double) * (size_t)N);
-    if (!lse || !delta) { free(lse); free(delta); return -2; }
+    uint8_t* needed = (uint8_t*)calloc((size_t)N, 1);
+    long long* list = (long long*)malloc(sizeof(long long) * (size_t)N);
+    if (!lse || !delta || !needed || !list) {
+        free(lse); free(delta); free(needed); free(list);
+        return -2;
+    }
+    /* the queries whose statistics the sampled rows read */
+    for (long long r = 0; r < nq; ++r) needed[qrows[r]] = 1;
+    if (nk) {
+        int qi[NA_ORACLE_MAXDIM];
+        for (int a = 0; a < ndim; ++a) qi[a] = 0;
+        for (long long t = 0; t < N; ++t) {
+            for (long long r = 0; r < nk && !needed[t]; ++r) {
+                int kj[NA_ORACLE_MAXDIM];
+                unflatten(krows[r], ndim, L, kj);
+                if (window_holds(ndim, L, w, s, mode, qi, kj)) needed[t] = 1;
+            }
+            for (int a = ndim - 1; a >= 0; --a) {
+                if (++qi[a] < L[a]) break;
+                qi[a] = 0;
+            }
+        }
+    }
+    long long nlist = 0;
+    for (long long t = 0; t < N; ++t) if (needed[t]) list[nlist++] = t;
     if (nthreads < 1) nthreads = 1;
     if (nthreads > 256) nthreads = 256;
-    stat_job jobs[256];
     pthread_t th[256];
-    const long long per = (N + nthreads - 1) / nthreads;
+    stat_job jobs[256];
+    const long long per = (nlist + nthreads - 1) / nthreads;
     for (int t = 0; t < nthreads; ++t) {
         stat_job* J = &jobs[t];
         J->q = q; J->k = k; J->v = v; J->dout = dout;
         J->dtype = in_dtype; J->ndim = ndim; J->d = d;
         J->L = L; J->w = w; J->s = s; J->mode = mode;
         J->N = N; J->W = W; J->bh = bh; J->scale = scale;
-        J->t_begin = per * t < N ? per * t : N;
-        J->t_end = per * (t + 1) < N ? per * (t + 1) : N;
+        J->list = list;
+        J->i_begin = per * t < nlist ? per * t : nlist;
+        J->i_end = per * (t + 1) < nlist ? per * (t + 1) : nlist;
         J->lse = lse; J->delta = delta;
         J->status = 0;
     }
@@ -614,69 +732,36 @@ int na_oracle_backward_sampled(const void* q, const void* k, const void* v, cons
     int rc = 0;
     for (int t = 0; t < nthreads; ++t)
         if (jobs[t].status) rc = jobs[t].status;
-    const size_t hoff = (size_t)bh * (size_t)N * (size_t)d;
-    uint8_t* mask = (uint8_t*)malloc((size_t)N);
-    if (!mask) rc = -2;
-    /* dq of the sampled query rows */
-    for (long long r = 0; !rc && r < nq; ++r) {
-        const long long t = qrows[r];
-        if (t < 0 || t >= N) { rc = -1; break; }
-        na_oracle_mask_row(ndim, L, w, s, mode, t, mask);
-        const size_t qoff = hoff + (size_t)t * (size_t)d;
-        for (int c = 0; c < d; ++c) dq[(size_t)r * d + c] = 0.0;
-        for (long long j = 0; j < N; ++j) {
-            if (!mask[j]) continue;
-            const size_t koff = hoff + (size_t)j * (size_t)d;
-            double zq = 0.0, dp = 0.0;
-            for (int c = 0; c < d; ++c) {
-                zq += load_in(q, in_dtype, qoff + c) * load_in(k, in_dtype, koff + c);
-                dp += load_in(dout, in_dtype, qoff + c) * load_in(v, in_dtype, koff + c);
-            }
-            const double p = exp(scale * zq - lse[t]);
-            const double dz = p * (dp - delta[t]);
-            for (int c = 0; c < d; ++c)
-                dq[(size_t)r * d + c] += scale * dz * load_in(k, in_dtype, koff + c);
+    if (!rc) {
+        grad_job gj[256];
+        const long long pq = (nq + nthreads - 1) / nthreads, pk = (nk + nthreads - 1) / nthreads;
+        for (int t = 0; t < nthreads; ++t) {
+            grad_job* J = &gj[t];
+            J->q = q; J->k = k; J->v = v; J->dout = dout;
+            J->dtype = in_dtype; J->ndim = ndim; J->d = d;
+            J->L = L; J->w = w; J->s = s; J->mode = mode;
+            J->N = N; J->bh = bh; J->scale = scale;
+            J->lse = lse; J->delta = delta;
+            J->qrows = qrows; J->krows = krows;
+            J->q_begin = pq * t < nq ? pq * t : nq;
+            J->q_end = pq * (t + 1) < nq ? pq * (t + 1) : nq;
+            J->k_begin = pk * t < nk ? pk * t : nk;
+            J->k_end = pk * (t + 1) < nk ? pk * (t + 1) : nk;
+            J->dq = dq; J->dk = dk; J->dv = dv;
+            J->status = 0;
         }
+        for (int t = 1; t < nthreads; ++t)
+            if (pthread_create(&th[t], NULL, grad_worker, &gj[t]) != 0) {
+                grad_worker(&gj[t]);
+                th[t] = 0;
+            }
+        grad_worker(&gj[0]);
+        for (int t = 1; t < nthreads; ++t)
+            if (th[t]) pthread_join(th[t], NULL);
+        for (int t = 0; t < nthreads; ++t)
+            if (gj[t].status) rc = gj[t].status;
     }
-    /* dk, dv of the sampled key rows: over every query whose window holds the key */
-    for (long long r = 0; !rc && r < nk; ++r) {
-        const long long j = krows[r];
-        if (j < 0 || j >= N) { rc = -1; break; }
-        const size_t koff = hoff + (size_t)j * (size_t)d;
-        for (int c = 0; c < d; ++c) { dk[(size_t)r * d + c] = 0.0; dv[(size_t)r * d + c] = 0.0; }
-        int kj[NA_ORACLE_MAXDIM];
-        unflatten(j, ndim, L, kj);
-        int qi[NA_ORACLE_MAXDIM];
-        for (int a = 0; a < ndim; ++a) qi[a] = 0;
-        for (long long t = 0; t < N; ++t) {
-            int in = 1;
-            for (int a = 0; a < ndim && in; ++a) {
-                int lo, hi;
-                const int ma = mode ? mode[a] : 0;
-                na_oracle_window(L[a], w[a], s[a], ma, qi[a], &lo, &hi);
-                if (kj[a] < lo || kj[a] >= hi) in = 0;
-            }
-            if (in) {
-                const size_t qoff = hoff + (size_t)t * (size_t)d;
-                double zq = 0.0, dp = 0.0;
-                for (int c = 0; c < d; ++c) {
-                    zq += load_in(q, in_dtype, qoff + c) * load_in(k, in_dtype, koff + c);
-                    dp += load_in(dout, in_dtype, qoff + c) * load_in(v, in_dtype, koff + c);
-                }
-                const double p = exp(scale * zq - lse[t]);
-                const double dz = p * (dp - delta[t]);
-                for (int c = 0; c < d; ++c) {
-                    dk[(size_t)r * d + c] += scale * dz * load_in(q, in_dtype, qoff + c);
-                    dv[(size_t)r * d + c] += p * load_in(dout, in_dtype, qoff + c);
-                }
-            }
-            for (int a = ndim - 1; a >= 0; --a) { /* advance the row-major query counter */
-                if (++qi[a] < L[a]) break;
-                qi[a] = 0;
-            }
-        }
-    }
-    free(mask); free(lse); free(delta);
+    free(lse); free(delta); free(needed); free(list);
     return rc;
 }
 

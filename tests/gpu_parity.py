@@ -88,6 +88,28 @@ def sample_rows(c, n_rows, seed=0):
     return np.array(sorted(picks), dtype=np.int64)
 
 
+def tile_tokens(grid, tile, tcoord):
+    """Token indices (row-major) of the query tile at tile coordinate `tcoord`."""
+    import itertools
+    ranges = [range(tcoord[i] * tile[i], min((tcoord[i] + 1) * tile[i], grid[i]))
+              for i in range(len(grid))]
+    return np.array([np.ravel_multi_index(p, grid) for p in itertools.product(*ranges)],
+                    dtype=np.int64)
+
+
+def survey_tiles(grid, tile):
+    """Tile coordinates of a 3-D tile grid sampled at its 8 corner tiles, 4 tiles
+    on its edges (two coordinates at a border, one inside) and 4 interior
+    tiles: the places where clamped windows differ most, and the bulk."""
+    T = [grid[i] // tile[i] for i in range(3)]
+    corners = [(a, b, c) for a in (0, T[0] - 1) for b in (0, T[1] - 1) for c in (0, T[2] - 1)]
+    edges = [(0, 0, T[2] // 2), (T[0] - 1, T[1] - 1, T[2] // 2 - 1), (0, T[1] // 2, T[2] - 1),
+             (T[0] // 2, 0, 0)]
+    interior = [(T[0] // 2, T[1] // 2, T[2] // 2), (1, 1, 1), (T[0] - 2, T[1] - 2, T[2] - 2),
+                (T[0] // 2, 1, T[2] - 3)]
+    return corners, edges, interior
+
+
 def compare(c, qkv_host, out_gpu, lse_gpu, rows=None):
     """Oracle on the same host buffers; returns (max|dout|, mean|dout|, max|dlse|)."""
     q, k, v = qkv_host

@@ -659,6 +659,19 @@ def pin_backward_sampled_rows(lib):
         np.testing.assert_allclose(sq, dq[0, bh].reshape(N, d)[rows], atol=1e-12, rtol=0)
         np.testing.assert_allclose(sk, dk[0, bh].reshape(N, d)[rows[::-1]], atol=1e-12, rtol=0)
         np.testing.assert_allclose(sv, dv[0, bh].reshape(N, d)[rows[::-1]], atol=1e-12, rtol=0)
+    # Only the statistics of the queries the sampled rows read are computed:
+    # key rows alone (their queries, none asked for as rows), query rows
+    # alone, every row, and more threads than rows.
+    every = np.arange(N, dtype=np.int64)
+    none = np.zeros(0, dtype=np.int64)
+    for qr, kr, th in ((none, np.array([3, 61], dtype=np.int64), 3),
+                       (np.array([88, 2], dtype=np.int64), none, 5),
+                       (every, every, 4), (rows, rows, 64)):
+        sq, sk, sv = lib.backward_sampled(q, k, v, do, grid, window, stride, 1, qr, kr,
+                                          dtype="f32", mode=modes, threads=th)
+        np.testing.assert_allclose(sq, dq[0, 1].reshape(N, d)[qr], atol=1e-12, rtol=0)
+        np.testing.assert_allclose(sk, dk[0, 1].reshape(N, d)[kr], atol=1e-12, rtol=0)
+        np.testing.assert_allclose(sv, dv[0, 1].reshape(N, d)[kr], atol=1e-12, rtol=0)
 
 
 def _read_golden(name):

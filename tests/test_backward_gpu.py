@@ -76,8 +76,8 @@ def _run(c, seed, kernel=None):
     return got, ref
 
 
-def _assert_close(c, got, ref, label):
-    for name, g, r in zip(("dq", "dk", "dv"), got, ref):
+def _assert_close(c, got, ref, label, names=("dq", "dk", "dv")):
+    for name, g, r in zip(names, got, ref):
         assert np.isfinite(g).all(), f"{label} {name}: non-finite"
         err = np.abs(g - r)
         if c["dtype"] == "f32":
@@ -136,19 +136,7 @@ def _sample_keys(grid, n, seed):
     return np.array(sorted(picks), dtype=np.int64)
 
 
-@pytest.mark.parametrize("cfg", ["sta3d_full", "local3d_full"])
-def test_backward_full_size_sampled(cfg):
-    """The full-size workloads in the launch configuration the benchmark times
-    (3-D sliding tile: 24 heads, 30x48x80, d 128; 3-D local: 32 heads,
-    16x32x32, d 64), gradients checked on sampled query and key rows of the
-    first and last (batch, head) slice against the oracle's sampled backward."""
-    if cfg == "sta3d_full":
-        c = _case((30, 48, 80), (18, 24, 40), (6, 8, 8), 128, heads=24, tile=(6, 8, 8))
-        nrows = 48
-    else:
-        c = _case((16, 32, 32), (12, 20, 20), (4, 4, 4), 64, B=2, heads=16, tile=(4, 4, 4))
-        nrows = 96
-    seed = 9100 if cfg == "sta3d_full" else 9200
+def _full_size_grads(c, seed):
     shape = (c["B"], c["heads"], *c["grid"], c["d"])
     q, k, v = seeded_inputs.qkv(seed, c["B"], c["heads"], c["grid"], c["d"], c["dtype"])
     do = seeded_inputs.normal_bf16_bits(seed + 7, shape)
@@ -156,13 +144,70 @@ def test_backward_full_size_sampled(cfg):
     out, lse = na.forward(qd, kd, vd, c["window"], c["stride"], c["tile"])
     dq, dk, dv = na.backward(qd, kd, vd, out, lse, dod, c["window"], c["stride"], c["tile"])
     na.na_sync_status()
+    return (q, k, v, do), (dq, dk, dv), dod
+
+
+def _rows_of(t, b, h, N, d, rows):
+    return (t[b, h].reshape(N, d)[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+            .astype(np.float64))
+
+
+def test_backward_sliding_tile_full_size_tiles_of_every_head():
+    """The 3-D sliding tile workload (24 heads, 30 x 48 x 80, tile 6 x 8 x 8,
+    window 18 x 24 x 40, d 128) in the benchmark's launch configuration.
+    In every head: dq of 8 rows from each of the 8 corner, 4 edge and 4
+    interior tiles, and dk, dv of every key of one whole tile (heads 0-7 the
+    8 corner tiles, 8-11 the edge tiles, 12-13 two interior tiles, 14-23 the
+    corner tiles again), against the oracle's sampled backward, which computes
+    the softmax statistics of exactly the queries those rows read.  Every head
+    also keeps sum_j dv_j = sum_i dO_i (each row of P sums to one) over all
+    115,200 keys; its bar is 8 times the root-sum-square of the two rounding
+    steps that perturb it: dv_j to bf16 (2^-9 |dv_j|) and, per query, the
+    window's P rounded to bf16 as the operand of dV (2^-9 P_ij per key,
+    averaging over the W keys of the window)."""
+    c = _case((30, 48, 80), (18, 24, 40), (6, 8, 8), 128, heads=24, tile=(6, 8, 8))
+    from gpu_parity import survey_tiles, tile_tokens
+    host, (dq, dk, dv), dod = _full_size_grads(c, 9100)
+    q, k, v, do = host
+    N = int(np.prod(c["grid"]))
+    W = int(np.prod(c["window"]))
+    corners, edges, interior = survey_tiles(c["grid"], c["tile"])
+    qrows = np.concatenate([tile_tokens(c["grid"], c["tile"], t)[::48]
+                            for t in corners + edges + interior])
+    key_tiles = corners + edges + interior[:2] + corners[::-1] + edges[:2]
+    assert len(key_tiles) == c["heads"]
+    # sum over keys of dv, per head, in fp64 on the device
+    sum_dv = dv.double().reshape(c["heads"], N, c["d"]).sum(dim=1)
+    sum_do = dod.double().reshape(c["heads"], N, c["d"]).sum(dim=1)
+    rss = torch.sqrt((dv.double() ** 2).reshape(c["heads"], N, c["d"]).sum(dim=1)
+                     + (dod.double() ** 2).reshape(c["heads"], N, c["d"]).sum(dim=1) / W)
+    assert ((sum_dv - sum_do).abs() <= 8 * 2.0 ** -9 * rss).all(), \
+        float(((sum_dv - sum_do).abs() / rss).max())
+    for h in range(c["heads"]):
+        krows = tile_tokens(c["grid"], c["tile"], key_tiles[h])
+        rq, rk, rv = oracle.backward_sampled(q, k, v, do, c["grid"], c["window"], c["stride"], h,
+                                             qrows, krows, dtype="bf16")
+        got_q = _rows_of(dq, 0, h, N, c["d"], qrows)
+        got_k, got_v = (_rows_of(t, 0, h, N, c["d"], krows) for t in (dk, dv))
+        _assert_close(c, [got_q], [rq], f"head {h}", names=("dq",))
+        _assert_close(c, [got_k, got_v], [rk, rv], f"head {h} tile {key_tiles[h]}",
+                      names=("dk", "dv"))
+
+
+def test_backward_local3d_full_size_sampled():
+    """The 3-D local workload (32 heads, 16 x 32 x 32, window 12 x 20 x 20,
+    stride 4, d 64) in the benchmark's launch configuration: dq, dk, dv of
+    sampled rows (grid corners, edges and uniform draws) of the first and last
+    (batch, head) slice against the oracle's sampled backward."""
+    c = _case((16, 32, 32), (12, 20, 20), (4, 4, 4), 64, B=2, heads=16, tile=(4, 4, 4))
+    host, (dq, dk, dv), _ = _full_size_grads(c, 9200)
+    q, k, v, do = host
     BH = c["B"] * c["heads"]
     N = int(np.prod(c["grid"]))
-    rows = _sample_keys(c["grid"], nrows, seed)
+    rows = _sample_keys(c["grid"], 96, 9200)
     for bh in (0, BH - 1):
         rq, rk, rv = oracle.backward_sampled(q, k, v, do, c["grid"], c["window"], c["stride"], bh,
                                              rows, rows, dtype="bf16")
         b, h = divmod(bh, c["heads"])
-        got = [t[b, h].reshape(N, c["d"])[torch.from_numpy(rows).cuda()].float().cpu().numpy()
-               .astype(np.float64) for t in (dq, dk, dv)]
-        _assert_close(c, got, (rq, rk, rv), f"{cfg} bh={bh}")
+        got = [_rows_of(t, b, h, N, c["d"], rows) for t in (dq, dk, dv)]
+        _assert_close(c, got, (rq, rk, rv), f"local3d bh={bh}")

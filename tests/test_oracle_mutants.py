@@ -52,6 +52,9 @@ MUTANTS = [
      "J->mode, NULL, t, mask);\n            const size_t qoff"),
     ("bwd_delta_from_v", "Di += load_in(J->dout, J->dtype, qoff + c) * o[c];",
      "Di += load_in(J->dout, J->dtype, qoff + c) * load_in(J->v, J->dtype, qoff + c);"),
+    # the sampled backward forgets the queries that only its key rows read
+    ("sampled_stats_miss_key_queries",
+     "if (window_holds(ndim, L, w, s, mode, qi, kj)) needed[t] = 1;", ""),
 ]
 
 

@@ -1,8 +1,9 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
 identical seeded inputs.  Small cases are compared element by element over
-every output; the five full-size workloads in the launch configuration the
-benchmark times are compared on sampled rows that include every grid corner
-and edge."""
+every output; the full-size workloads in the launch configuration the
+benchmark times are compared on every element where the oracle takes
+seconds, and on whole corner, edge and interior tiles of every head for the
+3-D sliding tile workload."""
 import zlib
 
 import numpy as np
@@ -16,7 +17,7 @@ if not torch.cuda.is_available():  # pragma: no cover - CPU machines skip the mo
 
 import neighborhood_attention_b200 as na  # noqa: E402
 from gpu_parity import (CONFIGS, assert_within, compare, host_inputs, run_gpu,  # noqa: E402
-                        sample_rows, seed_for)
+                        sample_rows, seed_for, survey_tiles, tile_tokens)
 
 SIMT, TC = na.NA_KERNEL_SIMT, na.NA_KERNEL_TC
 
@@ -67,8 +68,38 @@ def test_config2_full_parity_both_kernels():
         assert_within(c, compare(c, qkv, o, l), f"config2/{kernel}")
 
 
-@pytest.mark.parametrize("cfg,n_rows", [(3, 3000), (4, 1200), (5, 4000), (6, 3000)])
+@pytest.mark.parametrize("cfg", [3, 5, 6])
+def test_full_size_full_parity(cfg):
+    """2-D strided (16 x 128 x 128, w 32, s 8), 3-D local (32 x 16 x 32 x 32,
+    w 12 x 20 x 20) and 1-D causal (16 x 32768, w 5) workloads, in the launch
+    configuration the benchmark times, compared with the oracle on every
+    output element."""
+    c = CONFIGS[cfg]
+    qkv = host_inputs(c, seed_for(cfg))
+    o, l = run_gpu(c, qkv)
+    assert_within(c, compare(c, qkv, o, l), f"config{cfg}")
+
+
+def test_sliding_tile_full_size_tiles_of_every_head():
+    """3-D sliding tile workload (24 heads, 30 x 48 x 80, tile 6 x 8 x 8, window
+    18 x 24 x 40, d 128) in the benchmark's launch configuration: every row of
+    its 8 corner tiles, 4 edge tiles and 4 interior tiles, in all 24 heads
+    (147,456 rows), compared with the oracle element by element."""
+    c = CONFIGS[4]
+    qkv = host_inputs(c, seed_for(4))
+    N = int(np.prod(c["grid"]))
+    corners, edges, interior = survey_tiles(c["grid"], c["tile"])
+    toks = np.concatenate([tile_tokens(c["grid"], c["tile"], t)
+                           for t in corners + edges + interior])
+    BH = c["B"] * c["heads"]
+    rows = (np.arange(BH, dtype=np.int64)[:, None] * N + toks[None, :]).ravel()
+    o, l = run_gpu(c, qkv)
+    assert_within(c, compare(c, qkv, o, l, rows=rows), "config4 tiles")
+
+
+@pytest.mark.parametrize("cfg,n_rows", [(4, 1200)])
 def test_full_size_sampled_parity(cfg, n_rows):
+    """Uniformly drawn rows of the sliding tile workload, on top of its tiles."""
     c = CONFIGS[cfg]
     qkv = host_inputs(c, seed_for(cfg))
     rows = sample_rows(c, n_rows, seed=cfg)
