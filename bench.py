@@ -72,6 +72,7 @@ L2_BYTES = 126 * 10**6
 DENSE_STEPS = 3
 FLUSH_BYTES = 256 * 2**20
 RUNS = 10                 # repeated runs for the median / min
+FP8_PER_BF16 = 2.0        # nominal dense tensor rate of 8-bit vs 16-bit operands
 REPEAT_BUDGET_S = 8.0     # launches per run sized to about this much kernel time in all
 
 
@@ -89,6 +90,8 @@ def min_hbm_bytes(w=None):
     (d elements each per token), lse written once (4 bytes per token)."""
     w = WORKLOAD if w is None else w
     tokens = w["B"] * w["heads"] * int(np.prod(w["grid"]))
+    if w["dtype"] == "e4m3":      # 1-byte q, k, v; bf16 out
+        return tokens * ((3 * 1 + 2) * w["head_dim"] + 4)
     elt = 4 if w["dtype"] == "f32" else 2
     return tokens * (4 * w["head_dim"] * elt + 4)
 
@@ -386,7 +389,8 @@ def run_backward(args, rank, world, local_rank):
     na.na_sync_status(stream)
     (total_ms,) = max_over_ranks([e0.elapsed_time(e1)], world, dev)
     plan = na.na_plan(w["grid"], w["window"], w["stride"], w["tile"], w["head_dim"],
-                      {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32}[w["dtype"]],
+                      {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32,
+                       "e4m3": na.NA_E4M3}[w["dtype"]],
                       options=opts)
     flops = 10.0 * w["head_dim"] * w["B"] * w["heads"] * plan["useful_pairs"]
     value = flops * args.steps * world / (total_ms / 1e3) / 1e12
@@ -431,10 +435,12 @@ def run_ours(args, rank, world, local_rank):
     if w["dtype"] == "bf16":
         pinned = [torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).pin_memory()
                   for a in qkv_host]
+    elif w["dtype"] == "e4m3":
+        pinned = [torch.from_numpy(a).view(torch.float8_e4m3fn).pin_memory() for a in qkv_host]
     else:
         pinned = [torch.from_numpy(a).pin_memory() for a in qkv_host]
     q, k, v = (t.to(dev) for t in pinned)
-    out = torch.empty_like(q)
+    out = torch.empty(q.shape, dtype=na.out_dtype(q), device=dev)
     lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=dev)
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
@@ -631,7 +637,7 @@ def run_ours(args, rank, world, local_rank):
     # scaled_dot_product_attention (a library kernel, never on the measured
     # path), over the flattened token sequence.
     sdpa_ms = 0.0
-    if not args.no_speedup and w["dtype"] in ("bf16", "f16"):
+    if not args.no_speedup and w["dtype"] in ("bf16", "f16"):   # (torch has no E4M3 attention)
         import torch.nn.functional as F
         BH_ = w["B"] * w["heads"]
         N_ = int(np.prod(w["grid"]))
@@ -655,12 +661,17 @@ def run_ours(args, rank, world, local_rank):
         [total_ms, e2e_ms, per_launch_ms, dense_ms, sdpa_ms, runs_med, runs_min], world, dev)
 
     plan = na.na_plan(w["grid"], w["window"], w["stride"], w["tile"], w["head_dim"],
-                      {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32}[w["dtype"]],
+                      {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32,
+                       "e4m3": na.NA_E4M3}[w["dtype"]],
                       options=opts)
     flops = flops_per_step(plan["useful_pairs"])
     value = whole_job_tflops(flops, args.steps, world, total_ms)
     e2e_value = whole_job_tflops(flops, args.steps, world, e2e_ms)
     peak, peak_sustained, peak_kind = read_peaks()
+    if w["dtype"] == "e4m3":
+        # 8-bit products: the measured bf16 rate times the nominal dense
+        # fp8 : bf16 ratio (4.5 : 2.25 PFLOP/s)
+        peak *= FP8_PER_BF16
     achieved = flops / (per_launch_ms / 1e3) / 1e12
     # The bound: tensor cores when the workload's algorithmic intensity (FLOPs
     # per minimum HBM byte) is above the measured ridge, else HBM bandwidth.
@@ -682,6 +693,8 @@ def run_ours(args, rank, world, local_rank):
                     "peak_kind": (f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)"
                                   + (" x 1: f16 and bf16 share the nominal dense rate"
                                      if w["dtype"] == "f16" else "")
+                                  + (" x 2: the nominal dense fp8 : bf16 ratio (4.5 : 2.25 "
+                                     "PFLOP/s)" if w["dtype"] == "e4m3" else "")
                                   if peak_kind == "measured" else "fallback")}
     if rank != 0:
         return 0
@@ -753,14 +766,17 @@ def main():
     ap.add_argument("--config", type=int, default=4, choices=sorted(WORKLOADS),
                     help="workload: 4 (default) is the 3-D sliding tile one the metric is "
                          "quoted on; 1, 2, 3, 5, 6 are the other parity workloads")
-    ap.add_argument("--dtype", choices=["bf16", "f16"], default=None,
-                    help="input type of a 16-bit workload (default: the workload's own, bf16)")
+    ap.add_argument("--dtype", choices=["bf16", "f16", "e4m3"], default=None,
+                    help="input type of a 16-bit workload (default: the workload's own, bf16); "
+                         "e4m3: OFP8 E4M3 q, k, v with bf16 out")
     ap.add_argument("--heads", type=int, default=0,
                     help="profiling only: run the workload with this many heads instead of 24 "
                          "(the JSON line then reports that smaller workload)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.backward and args.dtype == "e4m3":
+        ap.error("the backward takes fp32, bf16 or f16 inputs (not e4m3)")
     global WORKLOAD, METRIC, TRAFFIC_APPLIES
     if args.config != 4:
         WORKLOAD = WORKLOADS[args.config]

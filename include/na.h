@@ -62,7 +62,12 @@ typedef enum {
   NA_ERR_TIMEOUT = 4       /* a bounded in-kernel wait expired (reported by na_sync_status) */
 } na_status;
 
-typedef enum { NA_F32 = 0, NA_BF16 = 1, NA_F16 = 2 } na_dtype;
+/* Input types.  NA_E4M3: q, k and v in the OFP8 E4M3 format (one byte per
+ * element; finite range +-448, no infinities); out is then written as bf16
+ * (two bytes per element), lse as fp32.  E4M3 runs on the tensor-core kernel
+ * only (head_dim 64 or 128, forward only); the softmax weights fed to the
+ * second product are rounded to E4M3 as well (see na_forward). */
+typedef enum { NA_F32 = 0, NA_BF16 = 1, NA_F16 = 2, NA_E4M3 = 3 } na_dtype;
 
 /* Per-dimension window rule (see the top of this file). */
 typedef enum {
@@ -105,7 +110,12 @@ typedef enum {
  *   dtype     NA_F32 (CUDA-core kernel), NA_BF16 or NA_F16 (tensor-core kernel
  *             when head_dim is 64 or 128; out is written in the input type and
  *             P, the softmax weights fed to the second product, are rounded to
- *             it as well).
+ *             it as well), or NA_E4M3 (tensor-core kernel, head_dim 64 or 128:
+ *             both products take 8-bit operands with fp32 accumulation, P is
+ *             rounded to E4M3 -- formed at up to 2^4 times the row's running
+ *             maximum weight so that typical weights stay in the format's
+ *             normal range, with the reference moved before any weight could
+ *             pass 256 -- and out is bf16 [B, heads, X1..Xn, d]).
  *   stream    cudaStream_t.
  * Returns NA_OK once the work is queued, NA_ERR_INVALID_ARG / NA_ERR_UNSUPPORTED
  * without touching the device, or NA_ERR_CUDA.  Scale is 1/sqrt(head_dim).
@@ -166,7 +176,8 @@ na_status na_forward_ex(const void* q, const void* k, const void* v, void* out, 
  *   dq, dk, dv        device, same shape / dtype as q (written; every row once,
  *                     no atomics, deterministic).
  *   delta             device float32 [B, heads, X1..Xn] workspace (written: D_i).
- * Other arguments, options (scale, window_mode) and errors as na_forward_ex.
+ * Other arguments, options (scale, window_mode) and errors as na_forward_ex;
+ * dtype NA_E4M3 is NA_ERR_UNSUPPORTED (the backward is not built for 8-bit inputs).
  * Kernels: the row delta D_i on the CUDA cores (fp32 arithmetic); for bf16 /
  * f16 with head_dim 64 or 128, dq (one kernel per query block) and dk / dv
  * (one kernel per key block, over the queries whose windows hold it) on the
@@ -284,8 +295,8 @@ na_status na_selftest_exp2(const float* x, float* y, int n, void* stream);
  * device-allocating routine.  Host-side planning may still use the C++ heap.
  *
  * Same arguments and layouts as na_forward_ex; the caller still passes q, k,
- * v, out and lse.  It runs the tensor-core kernel only (bf16, head_dim 64 or
- * 128, or f16 with the same head dims; opt->kernel must be NA_KERNEL_AUTO or
+ * v, out and lse.  It runs the tensor-core kernel only (bf16, f16 or E4M3,
+ * head_dim 64 or 128; opt->kernel must be NA_KERNEL_AUTO or
  * NA_KERNEL_TC -- AUTO means the tensor-core kernel here, whatever the
  * window size), else returns
  * NA_ERR_UNSUPPORTED.  The kernel's scratch need (4 bytes) is checked against

@@ -19,7 +19,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libna.so")
 
 NA_OK, NA_ERR_INVALID_ARG, NA_ERR_UNSUPPORTED, NA_ERR_CUDA, NA_ERR_TIMEOUT = range(5)
-NA_F32, NA_BF16, NA_F16 = 0, 1, 2
+NA_F32, NA_BF16, NA_F16, NA_E4M3 = 0, 1, 2, 3
 NA_KERNEL_AUTO, NA_KERNEL_SIMT, NA_KERNEL_TC, NA_KERNEL_GATHER = 0, 1, 2, 3
 NA_GATHER_MAX_KEYS = 32
 KERNEL_NAMES = {NA_KERNEL_AUTO: "auto", NA_KERNEL_SIMT: "simt", NA_KERNEL_TC: "tc",
@@ -193,8 +193,17 @@ def _dtype_of(t) -> int:
         return NA_F16
     if t.dtype == torch.float32:
         return NA_F32
-    raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16, torch.float16 or "
-                    "torch.float32")
+    if t.dtype == torch.float8_e4m3fn:
+        return NA_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16, torch.float16, "
+                    "torch.float32 or torch.float8_e4m3fn")
+
+
+def out_dtype(t):
+    """torch dtype of `out` for inputs like `t`: the input type, except bf16
+    for E4M3 inputs."""
+    import torch
+    return torch.bfloat16 if t.dtype == torch.float8_e4m3fn else t.dtype
 
 
 def _stream_ptr(stream) -> int:
@@ -217,9 +226,11 @@ def na_forward_ex(q, k, v, out, lse, window, stride=None, tile=None, options=Non
     shape = tuple(q.shape)
     if len(shape) != nd + 3:
         raise ValueError(f"q has shape {shape}; expected [B, heads, {nd} grid dims, d]")
-    for name, t in (("k", k), ("v", v), ("out", out)):
+    for name, t in (("k", k), ("v", v)):
         if tuple(t.shape) != shape or t.dtype != q.dtype:
             raise ValueError(f"{name} must match q in shape and dtype")
+    if tuple(out.shape) != shape or out.dtype != out_dtype(q):
+        raise ValueError(f"out must have q's shape and dtype {out_dtype(q)}")
     import torch
     if tuple(lse.shape) != shape[:-1] or lse.dtype != torch.float32:
         raise ValueError("lse must be float32 with q's shape minus head_dim")
@@ -252,9 +263,11 @@ def na_forward_noalloc(q, k, v, out, lse, window, stride=None, tile=None, option
     shape = tuple(q.shape)
     if len(shape) != nd + 3:
         raise ValueError(f"q has shape {shape}; expected [B, heads, {nd} grid dims, d]")
-    for name, t in (("k", k), ("v", v), ("out", out)):
+    for name, t in (("k", k), ("v", v)):
         if tuple(t.shape) != shape or t.dtype != q.dtype:
             raise ValueError(f"{name} must match q in shape and dtype")
+    if tuple(out.shape) != shape or out.dtype != out_dtype(q):
+        raise ValueError(f"out must have q's shape and dtype {out_dtype(q)}")
     if tuple(lse.shape) != shape[:-1] or lse.dtype != torch.float32:
         raise ValueError("lse must be float32 with q's shape minus head_dim")
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("lse", lse)):
@@ -402,6 +415,6 @@ def forward(q, k, v, window, stride=None, tile=None, options=None, stream=None,
         dl = [dilation] * len(window) if isinstance(dilation, int) else list(dilation)
         for i, x in enumerate(dl):
             options.dilation[i] = int(x)
-    out = torch.empty_like(q)
+    out = torch.empty(q.shape, dtype=out_dtype(q), device=q.device)
     lse = torch.empty(q.shape[:-1], dtype=torch.float32, device=q.device)
     return na_forward_ex(q, k, v, out, lse, window, stride, tile, options, stream)

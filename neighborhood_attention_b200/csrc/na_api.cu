@@ -124,7 +124,7 @@ na_status read_problem(const int dims[2], const int* grid, const int* window, co
   if (D != 32 && D != 64 && D != 128)
     return fail(NA_ERR_UNSUPPORTED, "head_dim=%d not in {32, 64, 128}", D);
   if (!grid || !window) return fail(NA_ERR_INVALID_ARG, "grid or window is NULL");
-  if (dtype != NA_F32 && dtype != NA_BF16 && dtype != NA_F16)
+  if (dtype != NA_F32 && dtype != NA_BF16 && dtype != NA_F16 && dtype != NA_E4M3)
     return fail(NA_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
   P.ndim = nd;
   P.D = D;
@@ -274,11 +274,19 @@ na_status make_plan(const Problem& P, Plan& out) {
   int kernel = P.opt.kernel;
   const bool half = P.dtype == NA_BF16 || P.dtype == NA_F16;
   const long long wkeys = (long long)P.g.w[0] * P.g.w[1] * P.g.w[2];
+  if (P.dtype == NA_E4M3) {
+    // 8-bit inputs run on the tensor cores only (kind::f8f6f4 products).
+    if (kernel == NA_KERNEL_SIMT || kernel == NA_KERNEL_GATHER)
+      return fail(NA_ERR_UNSUPPORTED, "E4M3 inputs run on the tensor-core kernel only");
+    kernel = NA_KERNEL_TC;
+    if (P.D != 64 && P.D != 128)
+      return fail(NA_ERR_UNSUPPORTED, "E4M3 inputs need head_dim 64 or 128");
+  }
   if (kernel == NA_KERNEL_AUTO && wkeys <= NA_GATHER_MAX_KEYS) kernel = NA_KERNEL_GATHER;
   if (kernel == NA_KERNEL_AUTO)
     kernel = (half && (P.D == 64 || P.D == 128)) ? NA_KERNEL_TC : NA_KERNEL_SIMT;
-  if (kernel == NA_KERNEL_TC && !half)
-    return fail(NA_ERR_UNSUPPORTED, "the tensor-core kernel takes bf16 or f16 only");
+  if (kernel == NA_KERNEL_TC && !half && P.dtype != NA_E4M3)
+    return fail(NA_ERR_UNSUPPORTED, "the tensor-core kernel takes bf16, f16 or E4M3 only");
   if (kernel == NA_KERNEL_TC && P.D != 64 && P.D != 128)
     return fail(NA_ERR_UNSUPPORTED, "the tensor-core kernel takes head_dim 64 or 128");
 
@@ -395,6 +403,9 @@ na_status status_word(int** out) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// The tensor-core kernel's input-type code of a na_dtype (0 bf16, 1 f16, 2 E4M3).
+int tc_dtype(int d) { return d == NA_F16 ? 1 : (d == NA_E4M3 ? 2 : 0); }
+
 // ---------------------------------------------- allocation-free variant --
 // Device scratch of na_forward_noalloc: a fixed array in the library's own
 // device image instead of memory from cudaMalloc.  Every GPU that loads the
@@ -452,7 +463,7 @@ na_status launch_forward(const Problem& P, const DilMap& map, long long BH, cons
     L.BH = (int)BH;
     L.N = (int)N;
     L.D = P.D;
-    L.f16 = P.dtype == NA_F16;
+    L.dt = tc_dtype(P.dtype);
     L.scale_log2 = scale * log2e;
     L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
     L.status = status;
@@ -690,6 +701,8 @@ na_status na_backward(const void* q, const void* k, const void* v, const void* o
     return fail(NA_ERR_INVALID_ARG, "lse and delta must be 4-byte aligned");
   const long long BH = (long long)B * heads;
   if (BH > (1LL << 30)) return fail(NA_ERR_UNSUPPORTED, "B*heads too large");
+  if (P.dtype == NA_E4M3)
+    return fail(NA_ERR_UNSUPPORTED, "the backward takes fp32, bf16 or f16 inputs (not E4M3)");
   const bool tc_ok = (P.dtype == NA_BF16 || P.dtype == NA_F16) && (P.D == 64 || P.D == 128);
   if (P.opt.kernel == NA_KERNEL_GATHER)
     return fail(NA_ERR_UNSUPPORTED, "the window-gather kernel is forward only");
@@ -969,7 +982,7 @@ na_status na_forward_noalloc(const void* q, const void* k, const void* v, void* 
   L.BH = (int)BH;
   L.N = (int)((long long)P.g.L[0] * P.g.L[1] * P.g.L[2]);   // < 2^31 (read_problem)
   L.D = P.D;
-  L.f16 = P.dtype == NA_F16;
+  L.dt = tc_dtype(P.dtype);
   L.scale_log2 = scale * 1.4426950408889634f;
   L.q = q; L.k = k; L.v = v; L.out = out; L.lse = lse;
   L.status = static_cast<int*>(scratch);

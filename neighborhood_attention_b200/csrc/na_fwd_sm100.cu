@@ -47,7 +47,6 @@ namespace {
 constexpr int TC_THREADS = 384;
 constexpr int BLOCK_M = 128;     // query rows per block
 constexpr int CHUNK_N = 128;     // keys per chunk
-constexpr int HALF_BYTES = 128 * 128;  // one 128-row x 64-element bf16 box (16 KB)
 constexpr int REGS_LOADER = 56;        // warpgroup 0 after setmaxnreg.dec
 constexpr int REGS_SOFTMAX = 216;      // warpgroups 1 and 2 after setmaxnreg.inc
 constexpr int REGS_NEEDED = 128 * REGS_LOADER + 256 * REGS_SOFTMAX;  // must fit the launch
@@ -66,16 +65,41 @@ constexpr uint32_t INFO_END = 0xFFFFu;   // slot info: no more chunks
 // harmless to the fp32 accumulators -- while the reference rarely moves.
 constexpr float P_LIMIT = 16384.f;
 
-template <int D, bool F16 = false>
+// Input types of the kernel (template argument DT).
+constexpr int DT_BF16 = 0, DT_F16 = 1, DT_E4M3 = 2;
+// E4M3 inputs: P is formed against a reference P8_OFFSET log2 units below the
+// maximum it was set from, so typical weights land in the format's normal
+// range (>= 2^-6) instead of its coarse subnormals; rows are redone once their
+// sum (a bound of their largest P) exceeds P_LIMIT8, so P stays below the
+// format's largest value, 448.
+constexpr float P8_OFFSET = 4.f;
+constexpr float P_LIMIT8 = 256.f;
+
+template <int D, int DT = DT_BF16>
 struct TcCfg {
-  static constexpr int TILE_BYTES = 128 * D * 2;             // Q block or K/V chunk
-  static constexpr int NS = (D == 128) ? 5 : 8;              // ring slots
-  static constexpr int HALVES = D / 64;                      // 64-element boxes per row
+  static constexpr bool F16 = DT == DT_F16;
+  static constexpr bool E4M3 = DT == DT_E4M3;
+  static constexpr int ESZ = E4M3 ? 1 : 2;                   // bytes per input element
+  static constexpr int TILE_BYTES = 128 * D * ESZ;           // Q block or K/V chunk
+  // TMA boxes: 128 rows of BOX_ELEMS elements, BOX_ROW bytes per row (the
+  // swizzle span: 128 B, or 64 B for E4M3 at head_dim 64); NBOX boxes per row.
+  static constexpr int BOX_ELEMS = E4M3 ? D : 64;
+  static constexpr int BOX_ROW = BOX_ELEMS * ESZ;
+  static constexpr int NBOX = D / BOX_ELEMS;
+  static constexpr int BOX_BYTES = 128 * BOX_ROW;
+  static constexpr uint32_t LAYOUT = BOX_ROW == 128 ? 2u : 4u;   // SWIZZLE_128B / SWIZZLE_64B
+  static constexpr int SBO = 8 * BOX_ROW;                    // 8-row swizzle atom
+  static constexpr int MMA_K = E4M3 ? 32 : 16;               // K elements per MMA (32 bytes)
+  static constexpr int NS = E4M3 ? (D == 128 ? 10 : 16) : ((D == 128) ? 5 : 8);   // ring slots
+  static constexpr float PLIM = E4M3 ? P_LIMIT8 : P_LIMIT;
+  static constexpr float POFF = E4M3 ? P8_OFFSET : 0.f;
   static constexpr int TMEM_COLS = 512;
   static constexpr int S_COL0 = 0;
   static constexpr int O_COL0 = 256;
-  static constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(BLOCK_M, CHUNK_N, false, false, F16);
-  static constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(BLOCK_M, D, false, true, F16);
+  // Operand format code 0 is f16 for kind::f16 and E4M3 for kind::f8f6f4.
+  static constexpr uint32_t IDESC_QK =
+      ptx::idesc_bf16_f32(BLOCK_M, CHUNK_N, false, false, F16 || E4M3);
+  static constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(BLOCK_M, D, false, true, F16 || E4M3);
 };
 
 template <int NS>
@@ -93,10 +117,10 @@ struct Bars {
   ChunkGrid cg;      // and the chunk grid over their key box
 };
 
-template <int D>
+template <int D, int DT>
 constexpr size_t smem_bytes() {
-  return 1024 /* alignment slack */ + (size_t)(2 + TcCfg<D>::NS) * TcCfg<D>::TILE_BYTES +
-         sizeof(Bars<TcCfg<D>::NS>);
+  return 1024 /* alignment slack */ + (size_t)(2 + TcCfg<D, DT>::NS) * TcCfg<D, DT>::TILE_BYTES +
+         sizeof(Bars<TcCfg<D, DT>::NS>);
 }
 
 // Advance `it` to the first chunk (at or after it) that is non-empty for at
@@ -111,12 +135,13 @@ __device__ __forceinline__ void seek_pair(const ChunkGrid& cg, const int* kb, co
   st0 = st1 = CHUNK_EMPTY;
 }
 
-template <int D, bool F16>
+template <int D, int DT>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const TcLaunch P) {
-  using C = TcCfg<D, F16>;
+  using C = TcCfg<D, DT>;
   constexpr int NS = C::NS;
+  constexpr bool F16 = C::F16;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -184,9 +209,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       for (int b = 0; b < 2; ++b) {
         if (!bi[b].exists) continue;
         ptx::mbar_expect_tx(&bars->q_full[b], C::TILE_BYTES);
-        for (int h = 0; h < C::HALVES; ++h)
-          ptx::tma_load_5d(sQ + b * C::TILE_BYTES + h * HALF_BYTES, &tm_q, &bars->q_full[b],
-                           h * 64, bi[b].o[2], bi[b].o[1], bi[b].o[0], bh);
+        for (int h = 0; h < C::NBOX; ++h)
+          ptx::tma_load_5d(sQ + b * C::TILE_BYTES + h * C::BOX_BYTES, &tm_q, &bars->q_full[b],
+                           h * C::BOX_ELEMS, bi[b].o[2], bi[b].o[1], bi[b].o[0], bh);
       }
       ChunkIter it;
       iter_begin(cg, it);
@@ -203,9 +228,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (kv == 0) bars->info[slot] = (uint32_t)st0 | ((uint32_t)st1 << 2);
           if (!((P.debug_flags & 1) && seq == 0)) {  // testing hook: withhold chunk 0's K
             ptx::mbar_expect_tx(&bars->full[slot], C::TILE_BYTES);
-            for (int h = 0; h < C::HALVES; ++h)
-              ptx::tma_load_5d(ring + slot * C::TILE_BYTES + h * HALF_BYTES, kv ? &tm_v : &tm_k,
-                               &bars->full[slot], h * 64, it.a[2], it.a[1], it.a[0], bh);
+            for (int h = 0; h < C::NBOX; ++h)
+              ptx::tma_load_5d(ring + slot * C::TILE_BYTES + h * C::BOX_BYTES, kv ? &tm_v : &tm_k,
+                               &bars->full[slot], h * C::BOX_ELEMS, it.a[2], it.a[1], it.a[0], bh);
             ++issued[slot];
           }
           ++seq;
@@ -248,10 +273,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if constexpr (WARPWIDE) ptx::tc_commit_warp(bar); else ptx::tc_commit(bar);
       };
       auto mma_ss_i = [&](uint32_t d, uint64_t a, uint64_t b, uint32_t id, uint32_t acc) {
-        if constexpr (WARPWIDE) ptx::mma_ss_warp(d, a, b, id, acc); else ptx::mma_ss(d, a, b, id, acc);
+        if constexpr (C::E4M3) {
+          if constexpr (WARPWIDE) ptx::mma_ss_f8_warp(d, a, b, id, acc);
+          else ptx::mma_ss_f8(d, a, b, id, acc);
+        } else {
+          if constexpr (WARPWIDE) ptx::mma_ss_warp(d, a, b, id, acc);
+          else ptx::mma_ss(d, a, b, id, acc);
+        }
       };
       auto mma_ts_i = [&](uint32_t d, uint32_t a, uint64_t b, uint32_t id, uint32_t acc) {
-        if constexpr (WARPWIDE) ptx::mma_ts_warp(d, a, b, id, acc); else ptx::mma_ts(d, a, b, id, acc);
+        if constexpr (C::E4M3) {
+          if constexpr (WARPWIDE) ptx::mma_ts_f8_warp(d, a, b, id, acc);
+          else ptx::mma_ts_f8(d, a, b, id, acc);
+        } else {
+          if constexpr (WARPWIDE) ptx::mma_ts_warp(d, a, b, id, acc);
+          else ptx::mma_ts(d, a, b, id, acc);
+        }
       };
       bool ok = true;
       if (bi[0].exists) ok = wait_i(&bars->q_full[0], 0);
@@ -261,10 +298,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       auto issue_s = [&](int b, int kslot) {
         const uint32_t d_t = tmem + C::S_COL0 + b * 128;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-          const uint64_t ad = ptx::desc_sw128(sQa + b * C::TILE_BYTES + off, 16, 1024);
-          const uint64_t bd = ptx::desc_sw128(ringa + kslot * C::TILE_BYTES + off, 16, 1024);
+        for (int kk = 0; kk < D / C::MMA_K; ++kk) {
+          // K slice kk: bytes [32 kk, 32 kk + 32) of each row, inside box
+          // (32 kk) / BOX_ROW.
+          const uint32_t off = ((kk * 32) / C::BOX_ROW) * C::BOX_BYTES + (kk * 32) % C::BOX_ROW;
+          const uint64_t ad = ptx::desc_sw(sQa + b * C::TILE_BYTES + off, 16, C::SBO, C::LAYOUT);
+          const uint64_t bd = ptx::desc_sw(ringa + kslot * C::TILE_BYTES + off, 16, C::SBO, C::LAYOUT);
           mma_ss_i(d_t, ad, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
       };
@@ -273,9 +312,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint32_t d_t = tmem + C::O_COL0 + b * D;
         const uint32_t a_t = tmem + C::S_COL0 + b * 128;
 #pragma unroll
-        for (int kk = 0; kk < CHUNK_N / 16; ++kk) {
-          const uint64_t bd =
-              ptx::desc_sw128(ringa + vslot * C::TILE_BYTES + kk * 2048, HALF_BYTES, 1024);
+        for (int kk = 0; kk < CHUNK_N / C::MMA_K; ++kk) {
+          // keys [MMA_K kk, MMA_K (kk + 1)) of V (MN-major: boxes along the
+          // head dimension BOX_BYTES apart); P's 32 bytes of them are 8 columns.
+          const uint64_t bd = ptx::desc_sw(ringa + vslot * C::TILE_BYTES + kk * C::MMA_K * C::BOX_ROW,
+                                           C::BOX_BYTES, C::SBO, C::LAYOUT);
           mma_ts_i(d_t, a_t + kk * 8, bd, C::IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
         }
       };
@@ -447,7 +488,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               case 2: acc2 = ptx::f2_add(acc2, p); break;
               default: acc3 = ptx::f2_add(acc3, p); break;
             }
-            s[j] = ptx::pack_half2<F16>(p0, p1);
+            if constexpr (C::E4M3) {
+              // four keys per 32-bit column: pair j - 1 in bytes 0-1, pair j in 2-3
+              if (j & 1)
+                s[j >> 1] = ptx::pack_e4m3x4(__uint_as_float(s[2 * j - 2]),
+                                             __uint_as_float(s[2 * j - 1]), p0, p1);
+              else {
+                s[2 * j] = __float_as_uint(p0);   // kept until pair j + 1 is done
+                s[2 * j + 1] = __float_as_uint(p1);
+              }
+            } else {
+              s[j] = ptx::pack_half2<F16>(p0, p1);
+            }
           }
           float q0, q1, q2, q3, q4, q5, q6, q7;
           ptx::f2_split(acc0, q0, q1);
@@ -465,7 +517,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         float m_new = m, alpha = 1.f, sum;
         bool need = false;
         if (__any_sync(0xffffffffu, m == -INFINITY)) {
-          const float mx2 = row_max();
+          const float mx2 = row_max() - C::POFF;
           need = mx2 > m;
           m_new = need ? mx2 : m;
           const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
@@ -473,9 +525,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           sum = exp_pass(m_use);
         } else {
           sum = exp_pass(m);
-          if (__any_sync(0xffffffffu, !(sum <= P_LIMIT))) {
+          if (__any_sync(0xffffffffu, !(sum <= C::PLIM))) {
             load_scores();
-            const float mx2 = row_max();
+            const float mx2 = row_max() - C::POFF;
             need = mx2 > m;
             m_new = need ? mx2 : m;
             alpha = need ? ptx::ex2(m - m_new) : 1.f;
@@ -484,7 +536,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         const bool warp_need = __any_sync(0xffffffffu, need);
         ptx::tmem_st32(tS + 0, s0);
-        ptx::tmem_st32(tS + 32, s1);
+        if constexpr (!C::E4M3) ptx::tmem_st32(tS + 32, s1);
         if (warp_need && had_pv) {
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
@@ -563,10 +615,10 @@ __global__ void exp2_poly_selftest_kernel(const float* x, float* y, int n) {
 
 // ------------------------------------------------------------ host side --
 bool encode_map(CUtensorMap* m, const void* ptr, const TcLaunch& L, const int box[3]) {
-  return encode_grid_map_dil(m, ptr, L.f16, L.D, L.g.L, L.map, L.BH, L.N, box);
+  return encode_grid_map_dil(m, ptr, L.dt, L.D, L.g.L, L.map, L.BH, L.N, box);
 }
 
-template <int D, bool F16>
+template <int D, int DT>
 cudaError_t launch_d(const TcLaunch& L, cudaStream_t stream, char* err, int errlen) {
   CUtensorMap mq, mk, mv;
   if (!encode_map(&mq, L.q, L, L.t.qb) || !encode_map(&mk, L.k, L, L.kb) ||
@@ -574,7 +626,7 @@ cudaError_t launch_d(const TcLaunch& L, cudaStream_t stream, char* err, int errl
     snprintf(err, errlen, "cuTensorMapEncodeTiled failed (pointer alignment or shape)");
     return cudaErrorInvalidValue;
   }
-  const size_t smem = smem_bytes<D>();
+  const size_t smem = smem_bytes<D, DT>();
   static int attr_done[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -582,14 +634,14 @@ cudaError_t launch_d(const TcLaunch& L, cudaStream_t stream, char* err, int errl
     // setmaxnreg.inc waits for registers that the .dec of warpgroup 0 frees;
     // refuse to launch if the compiled register count could not cover the split.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, tc_fwd_kernel<D, F16>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, tc_fwd_kernel<D, DT>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs * TC_THREADS < REGS_NEEDED) {
       snprintf(err, errlen, "kernel compiled with %d registers/thread; the register split needs %d",
                fa.numRegs, (REGS_NEEDED + TC_THREADS - 1) / TC_THREADS);
       return cudaErrorInvalidConfiguration;
     }
-    e = cudaFuncSetAttribute(tc_fwd_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(tc_fwd_kernel<D, DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
@@ -597,22 +649,23 @@ cudaError_t launch_d(const TcLaunch& L, cudaStream_t stream, char* err, int errl
   const long long npairs = (L.t.nblocks + 1) / 2;
   const long long grid = npairs * L.BH;
   if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  tc_fwd_kernel<D, F16><<<(unsigned)grid, TC_THREADS, smem, stream>>>(mq, mk, mv, L);
+  tc_fwd_kernel<D, DT><<<(unsigned)grid, TC_THREADS, smem, stream>>>(mq, mk, mv, L);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-// [BH, X1, X2, X3, D] bf16 / f16 as a 5-d tensor (D, X3, X2, X1, BH),
-// 64-element inner box with 128-byte swizzle.
-bool encode_grid_map(CUtensorMap* m, const void* ptr, int f16, int D, const int L[3], int BH,
+// [BH, X1, X2, X3, D] bf16 / f16 / E4M3 as a 5-d tensor (D, X3, X2, X1, BH).
+// Inner box: 64 elements of 16-bit types, D elements of E4M3 (one row), with
+// the swizzle of its width in bytes (128 B, or 64 B for E4M3 at head_dim 64).
+bool encode_grid_map(CUtensorMap* m, const void* ptr, int dt, int D, const int L[3], int BH,
                      int N, const int box[3]) {
-  return encode_grid_map_dil(m, ptr, f16, D, L, identity_map(L), BH, N, box);
+  return encode_grid_map_dil(m, ptr, dt, D, L, identity_map(L), BH, N, box);
 }
 
 // Residue class of a dilated grid: coordinate x of dimension d steps map.dil[d]
 // tokens of the full grid, and the class starts at token full_token(map, 0, 0, 0).
-bool encode_grid_map_dil(CUtensorMap* m, const void* ptr, int f16, int D, const int L[3],
+bool encode_grid_map_dil(CUtensorMap* m, const void* ptr, int dt, int D, const int L[3],
                          const DilMap& map, int BH, int N, const int box[3]) {
   static PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   static std::once_flag once;
@@ -625,7 +678,8 @@ bool encode_grid_map_dil(CUtensorMap* m, const void* ptr, int f16, int D, const 
       enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
   if (!enc) return false;
-  const cuuint64_t es = 2;
+  const bool e4m3 = dt == 2;
+  const cuuint64_t es = e4m3 ? 1 : 2;
   cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)L[2], (cuuint64_t)L[1], (cuuint64_t)L[0],
                         (cuuint64_t)BH};
   const cuuint64_t row = (cuuint64_t)D * es;
@@ -634,12 +688,17 @@ bool encode_grid_map_dil(CUtensorMap* m, const void* ptr, int f16, int D, const 
                            (cuuint64_t)map.dil[0] * map.Lf[1] * map.Lf[2] * row,
                            (cuuint64_t)N * row};
   ptr = static_cast<const char*>(ptr) + (size_t)full_token(map, 0, 0, 0) * row;
-  cuuint32_t boxd[5] = {64, (cuuint32_t)box[2], (cuuint32_t)box[1], (cuuint32_t)box[0], 1};
+  const cuuint32_t inner = e4m3 ? (cuuint32_t)D : 64;
+  cuuint32_t boxd[5] = {inner, (cuuint32_t)box[2], (cuuint32_t)box[1], (cuuint32_t)box[0], 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  CUresult r = enc(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5,
-                   const_cast<void*>(ptr), dims, strides, boxd, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUtensorMapDataType ty = e4m3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                      : (dt == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  const CUtensorMapSwizzle sw =
+      inner * es == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUresult r = enc(m, ty, 5, const_cast<void*>(ptr), dims, strides, boxd, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -662,13 +721,13 @@ cudaError_t launch_tc(const TcLaunch& L0, cudaStream_t stream, char* err, int er
   }
   if (L.t.qb[0] * L.t.qb[1] * L.t.qb[2] != BLOCK_M || L.kb[0] * L.kb[1] * L.kb[2] != CHUNK_N)
     return cudaErrorNotSupported;
-  switch (L.D) {
-    case 64:
-      return L.f16 ? launch_d<64, true>(L, stream, err, errlen)
-                   : launch_d<64, false>(L, stream, err, errlen);
-    case 128:
-      return L.f16 ? launch_d<128, true>(L, stream, err, errlen)
-                   : launch_d<128, false>(L, stream, err, errlen);
+  switch (L.D * 4 + L.dt) {
+    case 64 * 4 + DT_BF16: return launch_d<64, DT_BF16>(L, stream, err, errlen);
+    case 64 * 4 + DT_F16: return launch_d<64, DT_F16>(L, stream, err, errlen);
+    case 64 * 4 + DT_E4M3: return launch_d<64, DT_E4M3>(L, stream, err, errlen);
+    case 128 * 4 + DT_BF16: return launch_d<128, DT_BF16>(L, stream, err, errlen);
+    case 128 * 4 + DT_F16: return launch_d<128, DT_F16>(L, stream, err, errlen);
+    case 128 * 4 + DT_E4M3: return launch_d<128, DT_E4M3>(L, stream, err, errlen);
     default: return cudaErrorNotSupported;
   }
 }

@@ -32,7 +32,7 @@ struct TcLaunch {
   int kb_log2[3];        // filled by launch_tc (chunk extents are powers of two)
   DilMap map;            // grid coordinates -> token of the full (undilated) grid
   int BH, N, D;          // N: tokens per head of the full grid
-  int f16;               // 1: f16 in/out, 0: bf16 in/out
+  int dt;                // inputs: 0 bf16, 1 f16 (out in the input type), 2 E4M3 (out bf16)
   float scale_log2;
   const void *q, *k, *v;
   void* out;
@@ -101,13 +101,14 @@ struct GatherLaunch {
 constexpr int GATHER_SMEM_BUDGET = 100 * 1024;
 cudaError_t launch_gather(const GatherLaunch& L, cudaStream_t stream);
 
-// 5-d TMA descriptor of a [BH, X1, X2, X3, D] bf16 / f16 tensor, 64-element
-// inner box of `box` tokens, 128-byte swizzle.
-bool encode_grid_map(CUtensorMap* m, const void* ptr, int f16, int D, const int L[3], int BH,
+// 5-d TMA descriptor of a [BH, X1, X2, X3, D] tensor of input type dt (0 bf16,
+// 1 f16: 64-element inner box, 128-byte swizzle; 2 E4M3: one row of D bytes,
+// 128- or 64-byte swizzle), `box` tokens.
+bool encode_grid_map(CUtensorMap* m, const void* ptr, int dt, int D, const int L[3], int BH,
                      int N, const int box[3]);
 // The same for a residue class of a dilated grid: the class's coordinates x
 // address token map.res + map.dil * x of the full grid (N tokens per head).
-bool encode_grid_map_dil(CUtensorMap* m, const void* ptr, int f16, int D, const int L[3],
+bool encode_grid_map_dil(CUtensorMap* m, const void* ptr, int dt, int D, const int L[3],
                          const DilMap& map, int BH, int N, const int box[3]);
 
 cudaError_t launch_simt(const SimtLaunch& L, cudaStream_t stream);

@@ -95,6 +95,8 @@ class OracleLib:
         lib.na_oracle_backward_sampled.restype = ctypes.c_int
         lib.na_oracle_f16_value.argtypes = [ctypes.c_uint16]
         lib.na_oracle_f16_value.restype = ctypes.c_double
+        lib.na_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.na_oracle_e4m3_value.restype = ctypes.c_double
         self.lib = lib
         self.path = path
 
@@ -149,15 +151,17 @@ class OracleLib:
         """Exact forward in fp64.
 
         q, k, v: arrays of shape [B, heads, *grid, d]; float32 values for
-        ``dtype="f32"``, uint16 bfloat16 bit patterns for ``dtype="bf16"`` or
-        float16 values for ``dtype="f16"`` (decoded by the C code from their
-        bit patterns).
+        ``dtype="f32"``, uint16 bfloat16 bit patterns for ``dtype="bf16"``,
+        float16 values for ``dtype="f16"`` or uint8 OFP8 E4M3 bit patterns for
+        ``dtype="e4m3"`` (the last two decoded by the C code from their bit
+        patterns).
         rows: None for every query, else int64 global row ids (bh * N + token).
         Returns (out [nrows, d] float64, lse [nrows] float64); with rows=None
         out is reshaped to q's shape and lse to q's shape without d.
         """
         grid, window, stride = _geom(grid, window, stride)
-        codes = {"f32": (np.float32, 0), "bf16": (np.uint16, 1), "f16": (np.float16, 2)}
+        codes = {"f32": (np.float32, 0), "bf16": (np.uint16, 1), "f16": (np.float16, 2),
+                 "e4m3": (np.uint8, 3)}
         if dtype not in codes:
             raise ValueError(f"unknown dtype {dtype!r}")
         want, code = codes[dtype]
@@ -202,7 +206,8 @@ class OracleLib:
         q, k, v, dout: arrays of shape [B, heads, *grid, d] in the encoding of
         ``forward``'s dtype.  Returns three float64 arrays of q's shape."""
         grid, window, stride = _geom(grid, window, stride)
-        codes = {"f32": (np.float32, 0), "bf16": (np.uint16, 1), "f16": (np.float16, 2)}
+        codes = {"f32": (np.float32, 0), "bf16": (np.uint16, 1), "f16": (np.float16, 2),
+                 "e4m3": (np.uint8, 3)}
         if dtype not in codes:
             raise ValueError(f"unknown dtype {dtype!r}")
         want, code = codes[dtype]
@@ -233,7 +238,8 @@ class OracleLib:
         sampled rows: (dq [len(qrows), d], dk [len(krows), d], dv [len(krows), d])
         in fp64; qrows / krows are token indices within the slice."""
         grid, window, stride = _geom(grid, window, stride)
-        codes = {"f32": (np.float32, 0), "bf16": (np.uint16, 1), "f16": (np.float16, 2)}
+        codes = {"f32": (np.float32, 0), "bf16": (np.uint16, 1), "f16": (np.float16, 2),
+                 "e4m3": (np.uint8, 3)}
         want, code = codes[dtype]
         arrs = [np.ascontiguousarray(a) for a in (q, k, v, dout)]
         for a in arrs:
@@ -261,6 +267,10 @@ class OracleLib:
     def f16_value(self, bits: int) -> float:
         """The oracle's decoding of one binary16 bit pattern."""
         return float(self.lib.na_oracle_f16_value(int(bits)))
+
+    def e4m3_value(self, bits: int) -> float:
+        """The oracle's decoding of one OFP8 E4M3 bit pattern."""
+        return float(self.lib.na_oracle_e4m3_value(int(bits)))
 
     # -- block counting ------------------------------------------------------
     def block_counts(self, grid, window, stride, block: int, mode=None):

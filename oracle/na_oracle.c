@@ -92,7 +92,7 @@
 
 #define NA_ORACLE_MAXDIM 3
 
-enum { IN_F32 = 0, IN_BF16 = 1, IN_F16 = 2 };
+enum { IN_F32 = 0, IN_BF16 = 1, IN_F16 = 2, IN_E4M3 = 3 };
 enum { WIN_CLAMPED = 0, WIN_TRUNCATED = 1, WIN_CAUSAL = 2 };
 
 /* ---------------------------------------------------------------- window -- */
@@ -228,9 +228,28 @@ double na_oracle_f16_value(uint16_t h) {
     return (h & 0x8000) ? -v : v;
 }
 
+/*
+ * Value of an OFP8 E4M3 bit pattern ("OCP 8-bit Floating Point
+ * Specification", E4M3 encoding): sign bit, 4-bit exponent field e (bias 7),
+ * 3-bit mantissa m.  e = 0: subnormal m * 2^-9; e = 15 with m = 7: NaN (the
+ * format has no infinities); otherwise (8 + m) * 2^(e - 10) = (1 + m/8) * 2^(e - 7).
+ */
+double na_oracle_e4m3_value(uint8_t b) {
+    const int e = (b >> 3) & 0xf, m = b & 0x7;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -9);
+    else if (e == 15 && m == 7)
+        v = NAN;
+    else
+        v = ldexp((double)(8 + m), e - 10);
+    return (b & 0x80) ? -v : v;
+}
+
 static inline double load_in(const void* p, int dtype, size_t idx) {
     if (dtype == IN_F32) return (double)((const float*)p)[idx];
     if (dtype == IN_F16) return na_oracle_f16_value(((const uint16_t*)p)[idx]);
+    if (dtype == IN_E4M3) return na_oracle_e4m3_value(((const uint8_t*)p)[idx]);
     uint32_t bits = (uint32_t)((const uint16_t*)p)[idx] << 16;
     float f;
     memcpy(&f, &bits, sizeof f);
@@ -320,7 +339,7 @@ int na_oracle_forward_dil(const void* q, const void* k, const void* v, int in_dt
                           long long nrows, double* out, double* lse, int nthreads) {
     long long N;
     if (!q || !k || !v || !out || !lse || BH < 1 || d < 1 || nrows < 0) return -1;
-    if (in_dtype != IN_F32 && in_dtype != IN_BF16 && in_dtype != IN_F16) return -1;
+    if (in_dtype < IN_F32 || in_dtype > IN_E4M3) return -1;
     if (check_geometry(ndim, L, w, s, mode, dil, &N)) return -1;
     if (!rows && nrows != BH * N) return -1;
     long long W = 1;
@@ -462,7 +481,7 @@ int na_oracle_backward_dil(const void* q, const void* k, const void* v, const vo
                            double* dq, double* dk, double* dv, int nthreads) {
     long long N;
     if (!q || !k || !v || !dout || !dq || !dk || !dv || BH < 1 || d < 1) return -1;
-    if (in_dtype != IN_F32 && in_dtype != IN_BF16 && in_dtype != IN_F16) return -1;
+    if (in_dtype < IN_F32 || in_dtype > IN_E4M3) return -1;
     if (check_geometry(ndim, L, w, s, mode, dil, &N)) return -1;
     long long W = 1;
     for (int a = 0; a < ndim; ++a) W *= w[a];
@@ -670,7 +689,7 @@ int na_oracle_backward_sampled(const void* q, const void* k, const void* v, cons
     long long N;
     if (!q || !k || !v || !dout || BH < 1 || bh < 0 || bh >= BH || d < 1) return -1;
     if ((nq && (!qrows || !dq)) || (nk && (!krows || !dk || !dv))) return -1;
-    if (in_dtype != IN_F32 && in_dtype != IN_BF16 && in_dtype != IN_F16) return -1;
+    if (in_dtype < IN_F32 || in_dtype > IN_E4M3) return -1;
     if (check_geometry(ndim, L, w, s, mode, NULL, &N)) return -1;
     for (long long r = 0; r < nq; ++r) if (qrows[r] < 0 || qrows[r] >= N) return -1;
     for (long long r = 0; r < nk; ++r) if (krows[r] < 0 || krows[r] >= N) return -1;

@@ -4,7 +4,8 @@ CUDA side of every test and of the benchmark.
 This module holds no attention arithmetic.  It only maps (seed, element index)
 to a standard-normal sample through a counter-based SplitMix64 generator and a
 Box-Muller transform (see ``gen.c``), then rounds to float32, bfloat16 or
-float16 (round-to-nearest-even; float16 by numpy's conversion).  Both sides
+float16 (round-to-nearest-even; float16 by numpy's conversion) or OFP8 E4M3
+(round-to-nearest-even, saturating at +-448).  Both sides
 receive the very same host buffers, so the oracle reads exactly the values
 that the GPU receives.
 """
@@ -46,6 +47,11 @@ def _load():
             lib.na_gen_normal_bf16.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_float,
                                                ctypes.c_void_p, ctypes.c_int]
             lib.na_gen_normal_bf16.restype = ctypes.c_int
+            lib.na_gen_normal_e4m3.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_float,
+                                               ctypes.c_void_p, ctypes.c_int]
+            lib.na_gen_normal_e4m3.restype = ctypes.c_int
+            lib.na_gen_round_e4m3.argtypes = [ctypes.c_void_p, ctypes.c_uint64, ctypes.c_void_p]
+            lib.na_gen_round_e4m3.restype = None
             lib.na_gen_splitmix64_at.argtypes = [ctypes.c_uint64, ctypes.c_uint64]
             lib.na_gen_splitmix64_at.restype = ctypes.c_uint64
             _lib = lib
@@ -76,6 +82,25 @@ def normal_bf16_bits(seed: int, shape, scale: float = 1.0, threads: int | None =
     return out
 
 
+def normal_e4m3_bits(seed: int, shape, scale: float = 1.0, threads: int | None = None) -> np.ndarray:
+    """uint8 array holding the OFP8 E4M3 (RNE, saturating at +-448) bit
+    patterns of the same samples."""
+    lib = _load()
+    out = np.empty(shape, dtype=np.uint8)
+    rc = lib.na_gen_normal_e4m3(seed, out.size, scale, out.ctypes.data, _threads(threads))
+    if rc != 0:
+        raise RuntimeError("na_gen_normal_e4m3 failed")
+    return out
+
+
+def round_e4m3_bits(values) -> np.ndarray:
+    """E4M3 bit patterns of float32 values (the generator's own rounding)."""
+    a = np.ascontiguousarray(np.asarray(values, dtype=np.float32))
+    out = np.empty(a.shape, dtype=np.uint8)
+    _load().na_gen_round_e4m3(a.ctypes.data, a.size, out.ctypes.data)
+    return out
+
+
 def splitmix64_at(seed: int, k: int) -> int:
     """k-th raw 64-bit output of a SplitMix64 sequence started at ``seed``."""
     return int(_load().na_gen_splitmix64_at(seed, k))
@@ -95,11 +120,13 @@ def qkv(seed_base: int, B: int, heads: int, grid, head_dim: int, dtype: str,
         threads: int | None = None):
     """(q, k, v) host arrays of shape [B, heads, *grid, head_dim].
 
-    ``dtype`` is "f32" (float32 arrays), "bf16" (uint16 bit-pattern arrays) or
-    "f16" (float16 arrays).  Streams ``seed_base + 0/1/2`` feed q, k and v.
+    ``dtype`` is "f32" (float32 arrays), "bf16" (uint16 bit-pattern arrays),
+    "f16" (float16 arrays) or "e4m3" (uint8 bit-pattern arrays).  Streams
+    ``seed_base + 0/1/2`` feed q, k and v.
     """
     shape = (B, heads, *tuple(grid), head_dim)
-    gens = {"f32": normal_f32, "bf16": normal_bf16_bits, "f16": normal_f16}
+    gens = {"f32": normal_f32, "bf16": normal_bf16_bits, "f16": normal_f16,
+            "e4m3": normal_e4m3_bits}
     if dtype not in gens:
         raise ValueError(f"unknown dtype {dtype!r}")
     gen = gens[dtype]

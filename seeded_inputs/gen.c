@@ -12,8 +12,9 @@
  * Because every element is a pure function of (seed, n), the array can be
  * filled by any number of threads in any order with identical results.
  *
- * Outputs: float32 (round-to-nearest from the double sample) or bfloat16
- * bit patterns (round-to-nearest-even from that float32).
+ * Outputs: float32 (round-to-nearest from the double sample), bfloat16
+ * bit patterns (round-to-nearest-even from that float32), or OFP8 E4M3 bit
+ * patterns (round-to-nearest-even from that float32, saturating at +-448).
  */
 #include <math.h>
 #include <pthread.h>
@@ -56,11 +57,32 @@ static inline uint16_t f32_to_bf16_rne(float f) {
     return (uint16_t)(u >> 16);
 }
 
+/* OFP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no
+ * infinities; largest finite 448 = 1.75 * 2^8; subnormals m * 2^-9) from a
+ * float32, rounding to nearest even and saturating out-of-range values. */
+static inline uint8_t f32_to_e4m3_rne(float f) {
+    const uint8_t sign = signbit(f) ? 0x80u : 0u;
+    const double a = fabs((double)f);
+    if (a != a) return 0x7fu;                 /* NaN */
+    if (a >= 448.0) return sign | 0x7eu;      /* saturate */
+    if (a < 0.015625) {                       /* below 2^-6: subnormal grid of 2^-9 */
+        const double q = rint(a * 512.0);     /* 0..8; 8 is the smallest normal */
+        return sign | (uint8_t)q;
+    }
+    int e;
+    const double m = frexp(a, &e);           /* a = m * 2^e, m in [0.5, 1) */
+    int ex = e - 1;                          /* a = (2m) * 2^ex, 2m in [1, 2) */
+    double q = rint((2.0 * m - 1.0) * 8.0);  /* 0..8 */
+    if (q == 8.0) { q = 0.0; ++ex; }
+    const int code = ((ex + 7) << 3) | (int)q;
+    return sign | (uint8_t)(code > 0x7e ? 0x7e : code);
+}
+
 typedef struct {
     uint64_t seed;
     uint64_t begin, end;
     float scale;
-    int kind;      /* 0 = float32, 1 = bf16 bits */
+    int kind;      /* 0 = float32, 1 = bf16 bits, 2 = E4M3 bits */
     void* out;
 } job_t;
 
@@ -70,10 +92,14 @@ static void* run_job(void* p) {
         float* o = (float*)j->out;
         for (uint64_t n = j->begin; n < j->end; ++n)
             o[n] = (float)(normal_at(j->seed, n) * j->scale);
-    } else {
+    } else if (j->kind == 1) {
         uint16_t* o = (uint16_t*)j->out;
         for (uint64_t n = j->begin; n < j->end; ++n)
             o[n] = f32_to_bf16_rne((float)(normal_at(j->seed, n) * j->scale));
+    } else {
+        uint8_t* o = (uint8_t*)j->out;
+        for (uint64_t n = j->begin; n < j->end; ++n)
+            o[n] = f32_to_e4m3_rne((float)(normal_at(j->seed, n) * j->scale));
     }
     return NULL;
 }
@@ -114,6 +140,16 @@ int na_gen_normal_f32(uint64_t seed, uint64_t count, float scale, float* out, in
 /* Same samples, rounded to bfloat16 (RNE), written as raw 16-bit patterns. */
 int na_gen_normal_bf16(uint64_t seed, uint64_t count, float scale, uint16_t* out, int nthreads) {
     return fill(seed, count, scale, 1, out, nthreads);
+}
+
+/* Same samples, rounded to OFP8 E4M3 (RNE, saturating at +-448), raw bytes. */
+int na_gen_normal_e4m3(uint64_t seed, uint64_t count, float scale, uint8_t* out, int nthreads) {
+    return fill(seed, count, scale, 2, out, nthreads);
+}
+
+/* E4M3 rounding of arbitrary float32 values (the same routine), for tests. */
+void na_gen_round_e4m3(const float* in, uint64_t count, uint8_t* out) {
+    for (uint64_t n = 0; n < count; ++n) out[n] = f32_to_e4m3_rne(in[n]);
 }
 
 /* Single raw SplitMix64 output, exposed so tests can check the published sequence. */

@@ -151,7 +151,8 @@ def pin_mask_bruteforce(lib):
 def pin_full_attention(lib):
     """window = whole grid: equals dense softmax attention (numpy matmuls)."""
     for grid, stride, d, dtype in [([7, 5], [2, 3], 16, "f32"), ([3, 4, 5], [1, 2, 5], 8, "f32"),
-                                   ([23], [1], 12, "bf16"), ([6, 7], [3, 1], 16, "f16")]:
+                                   ([23], [1], 12, "bf16"), ([6, 7], [3, 1], 16, "f16"),
+                                   ([5, 9], [1, 3], 16, "e4m3")]:
         B, H = 2, 1
         shape = (B, H, *grid, d)
         if dtype == "f32":
@@ -160,6 +161,9 @@ def pin_full_attention(lib):
         elif dtype == "f16":
             q, k, v = (seeded_inputs.normal_f16(85 + t, shape, threads=1) for t in range(3))
             qf, kf, vf = (a.astype(np.float64) for a in (q, k, v))
+        elif dtype == "e4m3":
+            q, k, v = (seeded_inputs.normal_e4m3_bits(87 + t, shape, threads=1) for t in range(3))
+            qf, kf, vf = (_e4m3_reference_values(a) for a in (q, k, v))
         else:
             q, k, v = (seeded_inputs.normal_bf16_bits(80 + t, shape, threads=1) for t in range(3))
             qf, kf, vf = (seeded_inputs.bf16_bits_to_f32(a) for a in (q, k, v))
@@ -332,6 +336,32 @@ def pin_f16_decoding(lib):
     assert np.array_equal(np.isnan(got), nan)
     assert np.array_equal(got[~nan], ref[~nan])
     assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+
+
+def _e4m3_reference_values(bits):
+    """float64 values of E4M3 bit patterns by torch's float8_e4m3fn conversion
+    (a library routine, independent of the oracle's decoder)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(bits, dtype=np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def pin_e4m3_decoding(lib):
+    """The oracle's OFP8 E4M3 decoding equals torch's float8_e4m3fn -> float64
+    conversion for all 256 bit patterns (the two NaN patterns decode to NaN),
+    and the format's landmarks hold: 0x7e = 448 (largest finite), 0x08 = 2^-6
+    (smallest normal), 0x01 = 2^-9 (smallest subnormal), 0x38 = 1."""
+    bits = np.arange(256, dtype=np.uint8)
+    ref = _e4m3_reference_values(bits)
+    got = np.array([lib.e4m3_value(int(b)) for b in bits])
+    nan = np.isnan(ref)
+    assert nan.sum() == 2
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+    assert lib.e4m3_value(0x7E) == 448.0 and lib.e4m3_value(0xFE) == -448.0
+    assert lib.e4m3_value(0x08) == 2.0 ** -6 and lib.e4m3_value(0x01) == 2.0 ** -9
+    assert lib.e4m3_value(0x38) == 1.0 and lib.e4m3_value(0x00) == 0.0
 
 
 # ------------------------------------------------- truncated / causal modes --
@@ -691,7 +721,8 @@ ALL_PINS = [
     pin_constant_values, pin_explicit_scale, pin_row_subset, pin_wsa_empty_blocks_golden,
     pin_block_counts_closed_forms, pin_ena_density_golden, pin_truncated_eq5, pin_causal_eq5,
     pin_modes_strided, pin_mode_mask_bruteforce, pin_causal_full_sdpa, pin_mode_uniform_queries,
-    pin_sa_empty_blocks_golden, pin_f16_decoding, pin_backward_finite_differences,
+    pin_sa_empty_blocks_golden, pin_f16_decoding, pin_e4m3_decoding,
+    pin_backward_finite_differences,
     pin_backward_full_attention_autograd, pin_backward_invariants, pin_backward_sampled_rows,
     pin_dilated_window_bruteforce, pin_dilated_mask_bruteforce, pin_dilated_residue_subgrids,
     pin_dilated_backward_subgrids,

@@ -250,6 +250,7 @@ def _backward_call(lib, ptr_over=None, B=1, heads=1, dims=(2, 64), grid=(8, 8), 
     (dict(window=(9, 3)), 1),
     (dict(stride=(4, 1)), 1),
     (dict(dtype=0, kernel="tc"), 2),                           # tensor cores with fp32
+    (dict(dtype=3), 2),                                        # no backward for E4M3
     (dict(B=1 << 16, heads=1 << 15), 2),                       # B * heads = 2^31 > 2^30
     (dict(dims=(3, 64), grid=(2048, 2048, 1024), window=(3, 3, 3)), 2),   # 2^32 tokens
     (dict(dims=(3, 64), grid=(2048, 1024, 1024), window=(3, 3, 3)), 2),   # exactly 2^31 tokens
@@ -286,3 +287,25 @@ def test_noalloc_refuses_token_counts_an_int_cannot_hold(grid, expect):
              None) == expect
     lib.na_last_error.restype = ctypes.c_char_p
     assert "2^31" in lib.na_last_error().decode()
+
+
+def test_e4m3_plans_on_the_tensor_cores_only():
+    """8-bit inputs: the tensor-core kernel is chosen even for windows the
+    window-gather kernel would take; the CUDA-core kernels and head_dim 32 are
+    refused on the host."""
+    import neighborhood_attention_b200 as na
+    plan = na.na_plan([16, 16], [3, 3], [1, 1], None, 64, na.NA_E4M3)
+    assert plan["kernel"] == "tc"
+    assert na.na_plan([30, 48, 80], [18, 24, 40], [6, 8, 8], [6, 8, 8], 128,
+                      na.NA_E4M3)["kernel"] == "tc"
+    for kernel in (na.NA_KERNEL_SIMT, na.NA_KERNEL_GATHER):
+        with pytest.raises(na.NaError) as e:
+            na.na_plan([16, 16], [5, 5], None, None, 64, na.NA_E4M3,
+                       options=na.make_options(kernel=kernel))
+        assert e.value.status == na.NA_ERR_UNSUPPORTED
+    with pytest.raises(na.NaError) as e:
+        na.na_plan([16, 16], [5, 5], None, None, 32, na.NA_E4M3)
+    assert e.value.status == na.NA_ERR_UNSUPPORTED
+    with pytest.raises(na.NaError) as e:
+        na.na_plan([16, 16], [5, 5], None, None, 64, 4)
+    assert e.value.status == na.NA_ERR_INVALID_ARG

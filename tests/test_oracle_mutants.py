@@ -52,6 +52,9 @@ MUTANTS = [
      "J->mode, NULL, t, mask);\n            const size_t qoff"),
     ("bwd_delta_from_v", "Di += load_in(J->dout, J->dtype, qoff + c) * o[c];",
      "Di += load_in(J->dout, J->dtype, qoff + c) * load_in(J->v, J->dtype, qoff + c);"),
+    ("e4m3_exponent_bias", "v = ldexp((double)(8 + m), e - 10);", "v = ldexp((double)(8 + m), e - 9);"),
+    ("e4m3_subnormal_as_normal", "v = ldexp((double)m, -9);", "v = ldexp((double)(8 + m), -10);"),
+    ("e4m3_read_as_f16_byte", "if (dtype == IN_E4M3) return", "if (dtype == -1) return"),
     # the sampled backward forgets the queries that only its key rows read
     ("sampled_stats_miss_key_queries",
      "if (window_holds(ndim, L, w, s, mode, qi, kj)) needed[t] = 1;", ""),
