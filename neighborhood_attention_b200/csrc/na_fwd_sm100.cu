@@ -345,6 +345,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int kslot = seq % NS, kseq = seq++;   // next K tile or the end marker
         ok = wait_i(&bars->full[vslot], (vseq / NS) & 1);
         if (!ok) break;
+        // The next K tile (loaded well ahead) is waited for here, before block
+        // 0's P, so that no barrier check sits between block 0's two products.
+        ok = wait_i(&bars->full[kslot], (kseq / NS) & 1);
+        if (!ok) break;
+        const uint32_t ninfo = bars->info[kslot];
         ptx::tc_fence_after();
         if (cinfo & 3u) {
           ok = wait_i(&bars->p_ready[0], ph0 & 1);
@@ -354,10 +359,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           issue_pv(0, vslot, acc0);
           acc0 = true;
         }
-        ok = wait_i(&bars->full[kslot], (kseq / NS) & 1);
-        if (!ok) break;
-        const uint32_t ninfo = bars->info[kslot];
-        ptx::tc_fence_after();
         const bool more = ninfo != INFO_END;
         if (more && (ninfo & 3u)) { issue_s(0, kslot); commit_i(&bars->s_full[0]); }
         if (cinfo >> 2) {
