@@ -46,7 +46,8 @@ def _decode(bits):
 
 def _run(c, qkv, kernel=na.NA_KERNEL_AUTO):
     q, k, v = (torch.from_numpy(a).view(torch.float8_e4m3fn).cuda() for a in qkv)
-    opts = na.make_options(kernel=kernel, window_mode=c.get("mode"), ndim=len(c["grid"]))
+    opts = na.make_options(kernel=kernel, window_mode=c.get("mode"), ndim=len(c["grid"]),
+                           dilation=c.get("dil"))
     out, lse = na.forward(q, k, v, c["window"], c["stride"], c.get("tile"), options=opts)
     na.na_sync_status()
     assert out.dtype == torch.bfloat16
@@ -66,14 +67,19 @@ def _sigma(c, qkv, rows):
     groups = {}
     for r, row in enumerate(rows):
         bh = int(row) // N
-        win = tuple(oracle.window(grid[i], c["window"][i], c["stride"][i],
-                                  (c.get("mode") or ["clamped"] * len(grid))[i], int(coords[r][i]))
-                    for i in range(len(grid)))
+        if c.get("dil"):     # each row on its own (small grids only)
+            win = int(row)
+        else:
+            win = tuple(oracle.window(grid[i], c["window"][i], c["stride"][i],
+                                      (c.get("mode") or ["clamped"] * len(grid))[i],
+                                      int(coords[r][i]))
+                        for i in range(len(grid)))
         groups.setdefault((bh, win), []).append(r)
     sig = np.empty((len(rows), d))
     for (bh, _), members in groups.items():
         t0 = int(rows[members[0]]) % N
-        keys = np.flatnonzero(oracle.mask_row(grid, c["window"], c["stride"], t0, c.get("mode")))
+        keys = np.flatnonzero(oracle.mask_row(grid, c["window"], c["stride"], t0, c.get("mode"),
+                                              c.get("dil")))
         ts = np.asarray(rows)[members] % N
         z = (q[bh, ts] @ k[bh, keys].T) * scale
         p = np.exp(z - z.max(axis=1, keepdims=True))
@@ -86,7 +92,7 @@ def _sigma(c, qkv, rows):
 def _check(c, qkv, o, l, rows, label):
     d = c["d"]
     ref_o, ref_l = oracle.forward(*qkv, c["grid"], c["window"], c["stride"], dtype="e4m3",
-                                  rows=rows, mode=c.get("mode"))
+                                  rows=rows, mode=c.get("mode"), dilation=c.get("dil"))
     go = o.reshape(-1, d)[rows]
     gl = l.reshape(-1)[rows]
     assert np.isfinite(go).all() and np.isfinite(gl).all(), f"{label}: non-finite output"
@@ -102,9 +108,9 @@ def _check(c, qkv, o, l, rows, label):
     assert dl <= 1e-3, f"{label}: max|dlse| {dl:.3e}"
 
 
-def _case(grid, window, stride, d, B=1, heads=2, tile=None, mode=None):
+def _case(grid, window, stride, d, B=1, heads=2, tile=None, mode=None, dil=None):
     return dict(B=B, heads=heads, grid=tuple(grid), window=tuple(window), stride=tuple(stride),
-                tile=tile, d=d, dtype="e4m3", mode=mode)
+                tile=tile, d=d, dtype="e4m3", mode=mode, dil=dil)
 
 
 SMALL = {
@@ -114,6 +120,9 @@ SMALL = {
     "gna2d_partial_d64": _case((50, 44), (20, 16), (5, 4), 64),
     "na1d_causal_d128": _case((600,), (97,), (1,), 128, mode=["causal"]),
     "full_attention_d64": _case((24, 20), (24, 20), (1, 1), 64),
+    # dilated windows (one launch per residue class, strided tensor maps)
+    "dilated2d_d128": _case((23, 34), (5, 8), (1, 2), 128, dil=(3, 2),
+                            mode=["clamped", "truncated"]),
 }
 
 
