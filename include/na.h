@@ -214,14 +214,17 @@ const char* na_last_error(void);
  */
 typedef struct {
   int kernel;               /* na_kernel actually chosen */
-  int qblock[3];            /* query block shape (3-d padded, outermost first); 1 x 1 x 1
-                               for the window-gather kernel (each query on its own) */
+  int qblock[3];            /* query block shape (3-d padded, outermost first); for the
+                               window-gather kernel its query tile (staged form) or
+                               1 x 1 x 1 (direct form: each query on its own) */
   int kvchunk[3];           /* key chunk shape; 1 x 1 x 1 for the window-gather kernel
                                (it reads exactly the window's keys) */
   int tile[3];              /* query tile shape used to order blocks */
   long long query_blocks;   /* blocks per head */
-  long long ctas;           /* CTAs per head (window-gather: head's rows / rows per CTA,
-                               rounded up; its CTAs may straddle heads) */
+  long long ctas;           /* CTAs per head (window-gather: its query tiles per head in
+                               the staged form, walked by a persistent grid; in the
+                               direct form the head's rows / rows per CTA, rounded up,
+                               CTAs straddling heads) */
   long long chunks_loaded;  /* key chunks staged per head */
   long long units_full;     /* (block, chunk) products with no mask */
   long long units_partial;  /* (block, chunk) products with an element mask */

@@ -7,6 +7,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <array>
 #include <map>
 #include <mutex>
@@ -51,6 +52,8 @@ struct Plan {
   // window-gather kernel: query tile staged per CTA (gq[0] == 0: direct reads),
   // its shared memory, and the K / V rows staged per head
   int gq[3] = {0, 0, 0};
+  int gqrows = 0, gkrows = 0;   // rows of a stage's Q region and of its K / V regions
+  int gnst = 0;                 // stages (1 or 2)
   int gsmem = 0;
   long long gstaged = 0;
 };
@@ -70,14 +73,25 @@ void gather_box_extent(const Geom& g, int d, int t, int& kmax, long long& sum) {
   }
 }
 
-// Query tile of the window-gather kernel: among boxes of 2^k queries (k <= 8)
-// whose largest key box fits the shared-memory budget, the one that stages
-// the fewest K / V rows per head, counting each CTA as 32 rows of fixed cost.
-// No fitting box (a wide window): gq stays 0 and the kernel reads directly.
+// Query tile and stage count of the window-gather kernel's staged form,
+// among boxes of 2^k queries (k <= 8) no wider than the grid needs.  A stage
+// holds a tile's queries and the K and V rows of its key box.  Preference, in
+// order: a tile that fills a round of the CTA's threads (or the whole grid)
+// with two stages that leave room for two CTAs per SM; the same with one
+// stage; any tile with two CTAs per SM; a full-round tile alone on its SM;
+// any tile that fits at all.  Two stages wherever they fit the tier's
+// budget.  Within the first tier that has one, the tile that stages the
+// fewest K / V rows per head, counting each tile as 32 rows of fixed cost.
+// No fitting tile (a wide window): gq stays 0 and the kernel reads K and V
+// directly.
 void choose_gather_tile(const Problem& P, Plan& plan) {
   const int esz = P.dtype == NA_F32 ? 4 : 2;
-  double best = 0;
-  bool found = false;
+  const long long ntok = (long long)P.g.L[0] * P.g.L[1] * P.g.L[2];
+  const long long fill = std::min<long long>(gather_tile_queries_per_round(P.D), ntok);
+  constexpr int TIERS = 5;
+  double best[TIERS] = {};
+  bool found[TIERS] = {};
+  Plan pick[TIERS];
   for (int lp = 8; lp >= 0; --lp) {
     for (int e0 = 0; e0 <= lp; ++e0)
       for (int e1 = 0; e0 + e1 <= lp; ++e1) {
@@ -85,7 +99,7 @@ void choose_gather_tile(const Problem& P, Plan& plan) {
         int t[3], km[3];
         long long sm[3];
         bool ok = true;
-        long long box = 1, staged = 1, tiles = 1;
+        long long box = 1, staged = 1, tiles = 1, tq = 1;
         for (int d = 0; d < 3 && ok; ++d) {
           t[d] = 1 << e[d];
           if (t[d] > 1 && t[d] / 2 >= P.g.L[d]) ok = false;   // no wider than needed
@@ -94,25 +108,45 @@ void choose_gather_tile(const Problem& P, Plan& plan) {
           box *= km[d];
           staged *= sm[d];
           tiles *= (P.g.L[d] + t[d] - 1) / t[d];
+          tq *= std::min(t[d], P.g.L[d]);
         }
         if (!ok) continue;
-        const long long bytes = 2 * box * P.D * esz;
-        if (bytes > GATHER_SMEM_BUDGET) continue;
+        const long long one = gather_smem_bytes(tq, box, P.D, esz, 1);
+        const long long two = gather_smem_bytes(tq, box, P.D, esz, 2);
+        const bool full = tq >= fill;
+        int tier, nst;
+        if (full && two <= GATHER_SMEM_TWO_PER_SM) tier = 0, nst = 2;
+        else if (full && one <= GATHER_SMEM_TWO_PER_SM) tier = 1, nst = 1;
+        else if (one <= GATHER_SMEM_TWO_PER_SM) tier = 2, nst = two <= GATHER_SMEM_TWO_PER_SM ? 2 : 1;
+        else if (full && one <= GATHER_SMEM_MAX) tier = 3, nst = two <= GATHER_SMEM_MAX ? 2 : 1;
+        else if (one <= GATHER_SMEM_MAX) tier = 4, nst = two <= GATHER_SMEM_MAX ? 2 : 1;
+        else continue;
         const double cost = (double)staged + 32.0 * (double)tiles;
-        if (!found || cost < best - 1e-9) {
-          found = true;
-          best = cost;
-          for (int d = 0; d < 3; ++d) plan.gq[d] = t[d];
-          plan.gsmem = (int)bytes;
-          plan.gstaged = staged;
+        if (!found[tier] || cost < best[tier] - 1e-9) {
+          found[tier] = true;
+          best[tier] = cost;
+          for (int d = 0; d < 3; ++d) pick[tier].gq[d] = t[d];
+          pick[tier].gqrows = (int)tq;
+          pick[tier].gkrows = (int)box;
+          pick[tier].gnst = nst;
+          pick[tier].gsmem = (int)(nst == 2 ? two : one);
+          pick[tier].gstaged = staged;
         }
       }
   }
-  if (!found) {
-    plan.gq[0] = plan.gq[1] = plan.gq[2] = 0;
-    plan.gsmem = 0;
-    plan.gstaged = 0;
+  for (int tier = 0; tier < TIERS; ++tier) {
+    if (!found[tier]) continue;
+    for (int d = 0; d < 3; ++d) plan.gq[d] = pick[tier].gq[d];
+    plan.gqrows = pick[tier].gqrows;
+    plan.gkrows = pick[tier].gkrows;
+    plan.gnst = pick[tier].gnst;
+    plan.gsmem = pick[tier].gsmem;
+    plan.gstaged = pick[tier].gstaged;
+    return;
   }
+  plan.gq[0] = plan.gq[1] = plan.gq[2] = 0;
+  plan.gqrows = plan.gkrows = plan.gnst = plan.gsmem = 0;
+  plan.gstaged = 0;
 }
 
 na_status read_problem(const int dims[2], const int* grid, const int* window, const int* stride,
@@ -502,7 +536,16 @@ na_status launch_forward(const Problem& P, const DilMap& map, long long BH, cons
       G.qt[d] = plan.gq[d];
       G.nt[d] = plan.gq[0] > 0 ? (P.g.L[d] + plan.gq[d] - 1) / plan.gq[d] : 0;
     }
+    G.qrows = plan.gqrows;
+    G.krows = plan.gkrows;
+    G.nstages = plan.gnst;
     G.smem_bytes = plan.gsmem;
+    G.status = nullptr;
+    G.timeout_ns = P.opt.wait_timeout_ns > 0 ? P.opt.wait_timeout_ns : default_timeout_ns();
+    if (plan.gq[0] > 0) {
+      st = status_word(&G.status);
+      if (st != NA_OK) return st;
+    }
     cudaError_t e = launch_gather(G, s);
     if (e == cudaErrorNotSupported) return fail(NA_ERR_UNSUPPORTED, "window-gather kernel: shape");
     if (e != cudaSuccess)

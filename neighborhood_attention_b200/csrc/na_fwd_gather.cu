@@ -3,23 +3,25 @@
 //
 // With a handful of keys per query the forward is bound by HBM traffic (q, k,
 // v read and out written once: a few FLOPs per byte), so this kernel moves
-// bytes, not tiles of scores.  A CTA owns a box of queries (a tile of the
-// grid).  It first stages the K and V rows of the tile's key box -- the union
-// of its queries' windows, itself a box -- into shared memory with 16-byte
-// asynchronous copies, coalesced along the grid's innermost dimension, each
-// row fetched once per tile.  Then each query is served by a group of G
-// consecutive threads, each holding one 16-byte slice of the head dimension:
-// the group walks the query's own window key by key (the product of its
-// per-dimension ranges, cut windows included) over the staged rows, reduces
-// the partial dot products with shuffles and keeps an online softmax in the
-// log2 domain.  The output slice goes out as one 16-byte store per thread,
-// coalesced across the group and across consecutive queries.  When even a
-// one-query tile's key box would not fit the shared-memory budget (a wide
-// window), the same walk reads K and V straight from global memory instead.
+// bytes, not tiles of scores.  The work is cut into query tiles (boxes of the
+// grid); a persistent grid of CTAs walks them.  A tile's query rows and the K
+// and V rows of its key box -- the union of its queries' windows, itself a
+// box -- arrive by bulk copies (one per run of rows adjacent in memory) into
+// a shared-memory stage; with two stages the next tile streams in while the
+// current one is computed.  Each query is served by a group of consecutive
+// threads, each holding 32 elements of the head dimension: the group walks
+// the query's own window key by key (the product of its per-dimension ranges,
+// cut windows included) over the staged rows, reduces the partial dot
+// products with shuffles and keeps an online softmax in the log2 domain.  The
+// output goes out as 16-byte stores.  When even a one-query tile's key box
+// would not fit in shared memory (a wide window), a direct form reads K and V
+// straight from global memory instead.
 //
 // The arithmetic is the restricted softmax attention of "pi-Attention",
 // section 3.1 eqs. (1)-(3) with the neighbourhood of section 3.2 (eq. (5) for
 // cut windows); the lse output is the log of eq. (2)'s denominator.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -179,105 +181,192 @@ __device__ __forceinline__ void load_q(const GatherLaunch& P, size_t off, float 
   for (int e = 0; e < slice_elems<T>(); ++e) qv[e] *= P.scale_log2;   // log2-domain scores
 }
 
-// Staged form: one CTA per query tile, the tile's key box in shared memory.
-// Each query is served by G = D / 32 threads holding 32 elements each (q and
-// the output accumulator as packed f32x2 pairs), so a key costs a thread four
-// (bf16 / f16) or eight (fp32) 16-byte shared-memory reads per operand and at
-// most two shuffles.  Row r's 16-byte slice s sits at slot s ^ (r mod slots):
-// the threads of a warp read different rows at the same logical slice, and
-// the swizzle spreads them over all banks.
-template <int D, int T>
-__global__ void __launch_bounds__(GATHER_THREADS) gather_tile_kernel(const GatherLaunch P) {
+// Staged form.  The grid is persistent: CTA b takes query tiles b, b + grid,
+// ... (numbered head-major, then row-major over the tile grid), so the CTAs
+// at work at any moment hold neighbouring tiles and share their halo rows
+// in L2.  A tile's rows -- its queries, and the K and V rows of its key box
+// (the union of its queries' windows, itself a box) -- arrive by bulk copies
+// into one of two stages while the CTA computes the tile before it from the
+// other: one copy per run of adjacent rows (a whole tile of a 1-D grid is
+// one run per tensor), completion counted in bytes on the stage's mbarrier.
+struct TileGeo {
+  int bh;
+  int o[3], nq[3];   // first query and extent of the tile per dimension
+  int lo[3], kx[3];  // first key and extent of its key box
+};
+
+__device__ __forceinline__ TileGeo tile_geo(const GatherLaunch& P, int t) {
+  TileGeo tg;
+  const int tiles = P.nt[0] * P.nt[1] * P.nt[2];
+  tg.bh = t / tiles;
+  int tix = t % tiles;
+  int tc[3];
+  tc[2] = tix % P.nt[2];
+  tix /= P.nt[2];
+  tc[1] = tix % P.nt[1];
+  tc[0] = tix / P.nt[1];
+  for (int d = 0; d < 3; ++d) {
+    tg.o[d] = tc[d] * P.qt[d];
+    tg.nq[d] = imin(P.qt[d], P.g.L[d] - tg.o[d]);
+    int a, b, c, e;
+    window_range(P.g.L[d], P.g.w[d], P.g.s[d], P.g.m[d], tg.o[d], a, b);
+    window_range(P.g.L[d], P.g.w[d], P.g.s[d], P.g.m[d], tg.o[d] + tg.nq[d] - 1, c, e);
+    tg.lo[d] = a;   // both window ends are monotone in the query coordinate
+    tg.kx[d] = e - a;
+  }
+  return tg;
+}
+
+// Bulk copies of one box of rows (extent n, origin a in grid coordinates)
+// into consecutive shared-memory rows, row-major over the box; the lanes of
+// one warp share the runs.
+template <int RB>
+__device__ __forceinline__ void copy_box(const GatherLaunch& P, size_t head, const int a[3],
+                                         const int n[3], const void* src, unsigned char* dst,
+                                         uint64_t* bar, int lane) {
+  const int rows = n[0] * n[1] * n[2];
+  const int len = P.map.dil[2] == 1 ? n[2] : 1;   // adjacent in memory along the innermost
+  for (int r = lane * len; r < rows; r += 32 * len) {
+    const int r2 = r % n[2], r1 = (r / n[2]) % n[1], r0 = r / (n[2] * n[1]);
+    const size_t tok = (size_t)full_token(P.map, a[0] + r0, a[1] + r1, a[2] + r2);
+    ptx::bulk_load(dst + (size_t)r * RB, static_cast<const char*>(src) + (head + tok) * RB,
+                   (uint32_t)(len * RB), bar);
+  }
+}
+
+template <int RB>
+__device__ __forceinline__ void issue_tile(const GatherLaunch& P, int t, unsigned char* stage,
+                                           uint64_t* bar, int lane) {
+  const TileGeo tg = tile_geo(P, t);
+  const int nqt = tg.nq[0] * tg.nq[1] * tg.nq[2];
+  const int rows = tg.kx[0] * tg.kx[1] * tg.kx[2];
+  if (lane == 0) ptx::mbar_expect_tx(bar, (uint32_t)((nqt + 2 * rows) * RB));
+  __syncwarp();
+  const size_t head = (size_t)tg.bh * (size_t)P.N;
+  unsigned char* sK = stage + (size_t)P.qrows * RB;
+  unsigned char* sV = sK + (size_t)P.krows * RB;
+  copy_box<RB>(P, head, tg.o, tg.nq, P.q, stage, bar, lane);
+  copy_box<RB>(P, head, tg.lo, tg.kx, P.k, sK, bar, lane);
+  copy_box<RB>(P, head, tg.lo, tg.kx, P.v, sV, bar, lane);
+}
+
+// s += q . k over the 32 elements a thread holds, for 16-bit inputs: each
+// product of two 16-bit values is formed exactly and added in fp32 by one
+// mixed-precision FMA, so neither operand is widened first.
+template <int T>
+__device__ __forceinline__ void dot_words(uint32_t qw, uint32_t kw, float& a0, float& a1) {
+  if constexpr (T == G_BF16)
+    asm("{\n\t.reg .b16 ql, qh, kl, kh;\n\t"
+        "mov.b32 {ql, qh}, %2;\n\t"
+        "mov.b32 {kl, kh}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, ql, kl, %0;\n\t"
+        "fma.rn.f32.bf16 %1, qh, kh, %1;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "r"(qw), "r"(kw));
+  else
+    asm("{\n\t.reg .b16 ql, qh, kl, kh;\n\t"
+        "mov.b32 {ql, qh}, %2;\n\t"
+        "mov.b32 {kl, kh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, ql, kl, %0;\n\t"
+        "fma.rn.f32.f16 %1, qh, kh, %1;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "r"(qw), "r"(kw));
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {   // 2^x, 0 at -inf
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// One tile from its stage.  Each query is served by G = D / 32 threads holding
+// 32 elements each, so a key costs a thread four (16-bit) or eight (fp32)
+// 16-byte shared-memory reads per operand and at most two shuffles.  Scores:
+// for 16-bit inputs q stays in its 16-bit form and every product is one
+// mixed-precision FMA (exact product, fp32 sum; the scale is applied to the
+// sum); fp32 inputs use scaled fp32 q.  Values: the fp32 accumulator as
+// packed pairs, one f32x2 FMA per two elements.  Register slot k of a thread
+// holds one of its slices in an order rotated per lane: rows sit a whole
+// number of 128-byte lines apart (head_dim >= 64 at 16 bits), so a 16-byte
+// read's bank group is its slice's, and the rotation gives the eight lanes of
+// each phase of a warp-wide read eight different bank groups.  ONED: a 1-D
+// grid (the two outer extents 1), whose coordinates need no division.
+template <int D, int T, bool ONED>
+__device__ __forceinline__ void compute_tile(const GatherLaunch& P, const TileGeo& tg,
+                                             const unsigned char* stage) {
   constexpr int VE = slice_elems<T>();       // elements per 16-byte slice
   constexpr int ESZ = T == G_F32 ? 4 : 2;
-  constexpr int SPR = D * ESZ / 16;          // slices per row (4 .. 32)
+  constexpr int RB = D * ESZ;                // bytes per row
+  constexpr int SPR = RB / 16;               // slices per row (4 .. 32)
   constexpr int E = 32;                      // elements per thread
-  constexpr int S = E / VE;                  // slices per thread
+  constexpr int S = E / VE;                  // slices per thread (4 or 8)
   constexpr int G = D / E;                   // threads per query (1, 2 or 4)
   constexpr int QPC = GATHER_THREADS / G;    // queries per round
   constexpr int KPS = 2;                     // keys per online-softmax step
-  static_assert(SPR % S == 0 && (SPR & (SPR - 1)) == 0, "slices");
-  extern __shared__ uint4 smem[];
-
+  constexpr bool MIX = T != G_F32;
+  static_assert(SPR % S == 0 && (S & (S - 1)) == 0, "slices");
+  const uint4* sQ = reinterpret_cast<const uint4*>(stage);
+  const uint4* sK = sQ + (size_t)P.qrows * SPR;
+  const uint4* sV = sK + (size_t)P.krows * SPR;
   const Geom& g = P.g;
-  const int tiles = P.nt[0] * P.nt[1] * P.nt[2];
-  const int bh = blockIdx.x / tiles;
-  int tix = blockIdx.x % tiles;
-  int o[3], nq[3], lo[3], kx[3];
-  {
-    int tc[3];
-    tc[2] = tix % P.nt[2];
-    tix /= P.nt[2];
-    tc[1] = tix % P.nt[1];
-    tc[0] = tix / P.nt[1];
-    for (int d = 0; d < 3; ++d) {
-      o[d] = tc[d] * P.qt[d];
-      nq[d] = imin(P.qt[d], g.L[d] - o[d]);
-      int a, b, c, e;
-      window_range(g.L[d], g.w[d], g.s[d], g.m[d], o[d], a, b);
-      window_range(g.L[d], g.w[d], g.s[d], g.m[d], o[d] + nq[d] - 1, c, e);
-      lo[d] = a;          // both window ends are monotone in the query coordinate
-      kx[d] = e - a;
-    }
-  }
-  const int rows = kx[0] * kx[1] * kx[2];
-  uint4* sK = smem;
-  uint4* sV = smem + (size_t)rows * SPR;
-  const size_t head = (size_t)bh * (size_t)P.N;
-
-  // Stage the key box: slice sl of row r of K and V, 16 bytes per copy.
-  for (int i = threadIdx.x; i < rows * SPR; i += GATHER_THREADS) {
-    const int r = i / SPR, sl = i % SPR;
-    const int r2 = r % kx[2], r1 = (r / kx[2]) % kx[1], r0 = r / (kx[2] * kx[1]);
-    const size_t tok = (size_t)full_token(P.map, lo[0] + r0, lo[1] + r1, lo[2] + r2);
-    const size_t off = (head + tok) * D * ESZ + (size_t)sl * 16;
-    const int slot = r * SPR + (sl ^ (r & (SPR - 1)));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                     static_cast<uint32_t>(__cvta_generic_to_shared(sK + slot))),
-                 "l"(static_cast<const char*>(P.k) + off)
-                 : "memory");
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                     static_cast<uint32_t>(__cvta_generic_to_shared(sV + slot))),
-                 "l"(static_cast<const char*>(P.v) + off)
-                 : "memory");
-  }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-  __syncthreads();
-
+  const int lane = threadIdx.x % 32;
   const int part = threadIdx.x % G;
-  const int tile_q = nq[0] * nq[1] * nq[2];
+  const int rot = S == 4 ? ((lane >> 1) & 3) : (lane & 7);
+  auto sl = [&](int k) { return part * S + ((k + rot) & (S - 1)); };   // slice in slot k
+  const size_t head = (size_t)tg.bh * (size_t)P.N;
+  const int tile_q = tg.nq[0] * tg.nq[1] * tg.nq[2];
+
   for (int q0 = 0; q0 < tile_q; q0 += QPC) {
     const int qi = q0 + threadIdx.x / G;
     const bool valid = qi < tile_q;
     const int qq = valid ? qi : 0;
-    int c[3];
-    c[2] = o[2] + qq % nq[2];
-    c[1] = o[1] + (qq / nq[2]) % nq[1];
-    c[0] = o[0] + qq / (nq[2] * nq[1]);
-    int wl[3], n[3];
-    for (int d = 0; d < 3; ++d) {
+    int c[3], wl[3], n[3];
+    if constexpr (ONED) {
+      c[0] = c[1] = 0;
+      c[2] = tg.o[2] + qq;
       int hi;
-      window_range(g.L[d], g.w[d], g.s[d], g.m[d], c[d], wl[d], hi);
-      n[d] = hi - wl[d];
-      wl[d] -= lo[d];     // box-relative
+      window_range(g.L[2], g.w[2], g.s[2], g.m[2], c[2], wl[2], hi);
+      n[2] = hi - wl[2];
+      wl[2] -= tg.lo[2];
+      n[0] = n[1] = 1;
+      wl[0] = wl[1] = 0;
+    } else {
+      c[2] = tg.o[2] + qq % tg.nq[2];
+      c[1] = tg.o[1] + (qq / tg.nq[2]) % tg.nq[1];
+      c[0] = tg.o[0] + qq / (tg.nq[2] * tg.nq[1]);
+      for (int d = 0; d < 3; ++d) {
+        int hi;
+        window_range(g.L[d], g.w[d], g.s[d], g.m[d], c[d], wl[d], hi);
+        n[d] = hi - wl[d];
+        wl[d] -= tg.lo[d];     // box-relative
+      }
     }
     const int W = valid ? n[0] * n[1] * n[2] : 0;
     const int Wmax = __reduce_max_sync(0xffffffffu, W);   // uniform trip count for the shuffles
     const size_t token = (size_t)full_token(P.map, c[0], c[1], c[2]);
-    const size_t row_off = (head + token) * D * ESZ + (size_t)part * S * 16;
+    const size_t row_off = (head + token) * RB;
 
-    uint64_t q2[E / 2], acc2[E / 2];
+    float acc[E];
+    uint32_t qw[MIX ? E / 2 : 1];
+    uint64_t q2[MIX ? 1 : E / 2];
 #pragma unroll
     for (int k = 0; k < S; ++k) {
-      float f[VE];
-      unpack<T>(load_slice(P.q, row_off + (size_t)k * 16), f);
+      const uint4 u = sQ[qq * SPR + sl(k)];
+      if constexpr (MIX) {
+        qw[k * 4 + 0] = u.x;
+        qw[k * 4 + 1] = u.y;
+        qw[k * 4 + 2] = u.z;
+        qw[k * 4 + 3] = u.w;
+      } else {
+        float f[VE];
+        unpack<T>(u, f);
 #pragma unroll
-      for (int i = 0; i < VE / 2; ++i)
-        q2[k * VE / 2 + i] = ptx::f2(f[2 * i] * P.scale_log2, f[2 * i + 1] * P.scale_log2);
+        for (int i = 0; i < VE / 2; ++i)
+          q2[k * VE / 2 + i] = ptx::f2(f[2 * i] * P.scale_log2, f[2 * i + 1] * P.scale_log2);
+      }
     }
 #pragma unroll
-    for (int i = 0; i < E / 2; ++i) acc2[i] = ptx::f2(0.f, 0.f);
+    for (int i = 0; i < E; ++i) acc[i] = 0.f;
     float m = -INFINITY, l = 0.f;
 
     int j0 = 0, j1 = 0, j2 = 0;   // odometer over the window, innermost last
@@ -290,32 +379,42 @@ __global__ void __launch_bounds__(GATHER_THREADS) gather_tile_kernel(const Gathe
         in[u] = base + u < W;
         r[u] = 0;
         if (in[u]) {
-          r[u] = ((wl[0] + j0) * kx[1] + (wl[1] + j1)) * kx[2] + wl[2] + j2;
-          if (++j2 == n[2]) {
-            j2 = 0;
-            if (++j1 == n[1]) {
-              j1 = 0;
-              ++j0;
+          if constexpr (ONED) {
+            r[u] = wl[2] + j2++;
+          } else {
+            r[u] = ((wl[0] + j0) * tg.kx[1] + (wl[1] + j1)) * tg.kx[2] + wl[2] + j2;
+            if (++j2 == n[2]) {
+              j2 = 0;
+              if (++j1 == n[1]) {
+                j1 = 0;
+                ++j0;
+              }
             }
           }
         }
-        uint64_t a[4] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f),
-                         ptx::f2(0.f, 0.f)};
+        if constexpr (MIX) {
+          float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k = 0; k < S; ++k) {
-          const int sl = part * S + k;
-          float f[VE];
-          unpack<T>(sK[r[u] * SPR + (sl ^ (r[u] & (SPR - 1)))], f);
-#pragma unroll
-          for (int i = 0; i < VE / 2; ++i) {
-            const int j = k * VE / 2 + i;
-            a[j & 3] = ptx::f2_fma(q2[j], ptx::f2(f[2 * i], f[2 * i + 1]), a[j & 3]);
+          for (int k = 0; k < S; ++k) {
+            const uint4 kv = sK[r[u] * SPR + sl(k)];
+            dot_words<T>(qw[k * 4 + 0], kv.x, a[0], a[1]);
+            dot_words<T>(qw[k * 4 + 1], kv.y, a[2], a[3]);
+            dot_words<T>(qw[k * 4 + 2], kv.z, a[0], a[1]);
+            dot_words<T>(qw[k * 4 + 3], kv.w, a[2], a[3]);
           }
+          s[u] = ((a[0] + a[1]) + (a[2] + a[3])) * P.scale_log2;   // log2-domain score
+        } else {
+          uint64_t a[2] = {ptx::f2(0.f, 0.f), ptx::f2(0.f, 0.f)};
+#pragma unroll
+          for (int k = 0; k < S; ++k) {
+            const uint4 kv = sK[r[u] * SPR + sl(k)];
+            a[0] = ptx::f2_fma(q2[2 * k], ptx::f2(__uint_as_float(kv.x), __uint_as_float(kv.y)), a[0]);
+            a[1] = ptx::f2_fma(q2[2 * k + 1], ptx::f2(__uint_as_float(kv.z), __uint_as_float(kv.w)), a[1]);
+          }
+          float x0, x1;
+          ptx::f2_split(ptx::f2_add(a[0], a[1]), x0, x1);
+          s[u] = x0 + x1;
         }
-        const uint64_t a01 = ptx::f2_add(a[0], a[1]), a23 = ptx::f2_add(a[2], a[3]);
-        float x0, x1;
-        ptx::f2_split(ptx::f2_add(a01, a23), x0, x1);
-        s[u] = x0 + x1;
       }
 #pragma unroll
       for (int off = G / 2; off > 0; off >>= 1) {
@@ -330,26 +429,32 @@ __global__ void __launch_bounds__(GATHER_THREADS) gather_tile_kernel(const Gathe
       }
       const float m_new = fmaxf(m, mb);
       if (m_new == -INFINITY) continue;   // no key of this row yet (uniform in the group)
-      const float alpha = exp2f(m - m_new);
+      const float alpha = ex2_approx(m - m_new);
       l *= alpha;
       const uint64_t alpha2 = ptx::f2(alpha, alpha);
 #pragma unroll
-      for (int i = 0; i < E / 2; ++i) acc2[i] = ptx::f2_mul(acc2[i], alpha2);
+      for (int i = 0; i < E / 2; ++i) {
+        uint64_t t = ptx::f2(acc[2 * i], acc[2 * i + 1]);
+        t = ptx::f2_mul(t, alpha2);
+        ptx::f2_split(t, acc[2 * i], acc[2 * i + 1]);
+      }
 #pragma unroll
       for (int u = 0; u < KPS; ++u) {
-        const float pu = exp2f(s[u] - m_new);   // 0 for a masked key
+        const float pu = ex2_approx(s[u] - m_new);   // 0 for a masked key
         l += pu;
         if (!in[u]) continue;
         const uint64_t p2 = ptx::f2(pu, pu);
 #pragma unroll
         for (int k = 0; k < S; ++k) {
-          const int sl = part * S + k;
           float f[VE];
-          unpack<T>(sV[r[u] * SPR + (sl ^ (r[u] & (SPR - 1)))], f);
+          unpack<T>(sV[r[u] * SPR + sl(k)], f);
 #pragma unroll
           for (int i = 0; i < VE / 2; ++i) {
-            const int j = k * VE / 2 + i;
-            acc2[j] = ptx::f2_fma(p2, ptx::f2(f[2 * i], f[2 * i + 1]), acc2[j]);
+            float& x0 = acc[k * VE + 2 * i];
+            float& x1 = acc[k * VE + 2 * i + 1];
+            uint64_t t = ptx::f2(x0, x1);
+            t = ptx::f2_fma(p2, ptx::f2(f[2 * i], f[2 * i + 1]), t);
+            ptx::f2_split(t, x0, x1);
           }
         }
       }
@@ -357,21 +462,68 @@ __global__ void __launch_bounds__(GATHER_THREADS) gather_tile_kernel(const Gathe
     }
 
     if (valid) {
-      const float inv_l = 1.f / l;
+      float inv_l, lg;
+      asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv_l) : "f"(l));
+      asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(l));
 #pragma unroll
       for (int k = 0; k < S; ++k) {
         float f[VE];
 #pragma unroll
-        for (int i = 0; i < VE / 2; ++i) {
-          ptx::f2_split(acc2[k * VE / 2 + i], f[2 * i], f[2 * i + 1]);
-          f[2 * i] *= inv_l;
-          f[2 * i + 1] *= inv_l;
-        }
-        *reinterpret_cast<uint4*>(static_cast<char*>(P.out) + row_off + (size_t)k * 16) =
+        for (int i = 0; i < VE; ++i) f[i] = acc[k * VE + i] * inv_l;
+        *reinterpret_cast<uint4*>(static_cast<char*>(P.out) + row_off + (size_t)sl(k) * 16) =
             pack<T>(f);
       }
-      if (part == 0) P.lse[head + token] = (m + log2f(l)) * 0.69314718055994530942f;
+      if (part == 0) P.lse[head + token] = (m + lg) * 0.69314718055994530942f;
     }
+  }
+}
+
+template <int D, int T, bool ONED>
+__global__ void __launch_bounds__(GATHER_THREADS, 2) gather_staged_kernel(const GatherLaunch P) {
+  constexpr int RB = D * (T == G_F32 ? 4 : 2);
+  extern __shared__ __align__(128) unsigned char smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // one mbarrier per stage
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 16);
+  unsigned char* stage0 = smem + GATHER_SMEM_HEADER;
+  const int stage_bytes = (P.qrows + 2 * P.krows) * RB;
+  const int nst = P.nstages;   // 1 or 2
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int total = P.BH * P.nt[0] * P.nt[1] * P.nt[2];   // the host keeps it below 2^30
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&full[0], 1);
+    ptx::mbar_init(&full[1], 1);
+    *abort_flag = *reinterpret_cast<volatile int*>(P.status) != 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  ptx::WaitCtl ctl;
+  ctl.abort = abort_flag;
+  ctl.status = P.status;
+  ctl.timeout_ns = (uint64_t)P.timeout_ns;
+
+  int t = blockIdx.x, i = 0, st = 0, par = 0;
+  bool ok = true;
+  if (warp == 0 && t < total) issue_tile<RB>(P, t, stage0, &full[0], lane);
+  for (; t < total; t += gridDim.x, ++i) {
+    st = nst == 2 ? (i & 1) : 0;
+    par = nst == 2 ? ((i >> 1) & 1) : (i & 1);
+    const bool more = t + (int)gridDim.x < total;
+    // Two stages: the other one was released by the barrier that ended the
+    // last tile, and the next tile streams in while this one is computed.
+    if (nst == 2 && warp == 0 && more)
+      issue_tile<RB>(P, t + gridDim.x, stage0 + (st ^ 1) * stage_bytes, &full[st ^ 1], lane);
+    ok = __syncthreads_and(ptx::wait(&full[st], par, ctl));
+    if (!ok) break;
+    compute_tile<D, T, ONED>(P, tile_geo(P, t), stage0 + st * stage_bytes);
+    __syncthreads();
+    // One stage: the next tile's copies start once every thread is done.
+    if (nst == 1 && warp == 0 && more) issue_tile<RB>(P, t + gridDim.x, stage0, &full[0], lane);
+  }
+  if (!ok && threadIdx.x == 0) {
+    // A wait gave up: the copies in flight land before shared memory goes away.
+    ptx::wait_drain(&full[st], par, ctl);
+    if (nst == 2 && t + (int)gridDim.x < total)
+      ptx::wait_drain(&full[st ^ 1], ((i + 1) >> 1) & 1, ctl);
   }
 }
 
@@ -425,19 +577,41 @@ __global__ void __launch_bounds__(GATHER_THREADS) gather_direct_kernel(const Gat
 template <int D, int T>
 cudaError_t launch_dt(const GatherLaunch& L, cudaStream_t stream) {
   if (L.qt[0] > 0) {
-    const long long blocks = (long long)L.BH * L.nt[0] * L.nt[1] * L.nt[2];
-    if (blocks <= 0 || blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    if (L.smem_bytes <= 0 || L.smem_bytes > GATHER_SMEM_BUDGET) return cudaErrorInvalidValue;
-    static int attr_done[64] = {0};
+    const long long tiles = (long long)L.BH * L.nt[0] * L.nt[1] * L.nt[2];
+    if (tiles <= 0 || tiles >= (1LL << 30)) return cudaErrorInvalidConfiguration;
+    const int esz = T == G_F32 ? 4 : 2;
+    if (L.qrows <= 0 || L.krows <= 0 || (L.nstages != 1 && L.nstages != 2) ||
+        L.smem_bytes > GATHER_SMEM_MAX ||
+        L.smem_bytes != gather_smem_bytes(L.qrows, L.krows, D, esz, L.nstages) || !L.status)
+      return cudaErrorInvalidValue;
+    const bool oned = L.g.L[0] == 1 && L.g.L[1] == 1;
+    auto kern = oned ? gather_staged_kernel<D, T, true> : gather_staged_kernel<D, T, false>;
+    // Per device: the shared-memory opt-in, the SM count, and the resident
+    // CTAs per SM at the last footprint launched.
+    static int attr_done[64] = {0}, sms[64] = {0}, occ_smem[64] = {0}, occ[64] = {0};
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-      const cudaError_t e = cudaFuncSetAttribute(
-          gather_tile_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, GATHER_SMEM_BUDGET);
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
+      for (auto f : {gather_staged_kernel<D, T, true>, gather_staged_kernel<D, T, false>}) {
+        e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, GATHER_SMEM_MAX);
+        if (e != cudaSuccess) return e;
+      }
+      e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
       if (e != cudaSuccess) return e;
       attr_done[dev] = 1;
     }
-    gather_tile_kernel<D, T><<<(unsigned)blocks, GATHER_THREADS, L.smem_bytes, stream>>>(L);
+    if (occ_smem[dev] != L.smem_bytes) {
+      int nb = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, gather_staged_kernel<D, T, false>,
+                                                        GATHER_THREADS, L.smem_bytes);
+      if (e != cudaSuccess) return e;
+      occ[dev] = nb > 0 ? nb : 1;
+      occ_smem[dev] = L.smem_bytes;
+    }
+    const long long grid = std::min(tiles, (long long)sms[dev] * occ[dev]);
+    kern<<<(unsigned)grid, GATHER_THREADS, L.smem_bytes, stream>>>(L);
   } else {
     const long long qpc = GATHER_THREADS / (D / slice_elems<T>());
     const long long rows = (long long)L.BH * L.g.L[0] * L.g.L[1] * L.g.L[2];

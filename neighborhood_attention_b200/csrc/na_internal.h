@@ -78,9 +78,11 @@ struct TcBwdLaunch {
 };
 
 // Window-gather kernel (CUDA cores): each query reads its own window's keys.
-// 256 threads, one 16-byte slice of the head dimension each: query rows served
-// at once per CTA.
+// 256 threads per CTA.  Direct form: one 16-byte slice of the head dimension
+// per thread, so query rows served at once per CTA =
 inline int gather_rows_per_cta(int D, int dtype) { return 256 / (D / (dtype == 0 ? 4 : 8)); }
+// Staged form: 32 head-dim elements per thread, so queries served per round =
+inline int gather_tile_queries_per_round(int D) { return 256 / (D / 32); }
 
 struct GatherLaunch {
   Geom g;
@@ -91,14 +93,26 @@ struct GatherLaunch {
   const void *q, *k, *v;
   void* out;
   float* lse;
-  int qt[3];             // query tile per CTA (a box of the grid); qt[0] == 0: no
-                         // staging, every key read straight from global memory
+  int qt[3];             // query tile (a box of the grid); qt[0] == 0: no staging,
+                         // every key read straight from global memory
   int nt[3];             // tiles per dimension
-  int smem_bytes;        // K and V rows of the largest key box of a tile
+  int qrows, krows;      // staged form: rows of a stage's Q region (the tile) and of
+                         // its K and V regions (the largest key box of a tile)
+  int nstages;           // staged form: 1 or 2 stages
+  int smem_bytes;        // staged form: header + the stages
+  int* status;           // device status word
+  long long timeout_ns;  // bound on every in-kernel wait
 };
 
-// Shared memory the staged form may use per CTA (two CTAs fit on an SM).
-constexpr int GATHER_SMEM_BUDGET = 100 * 1024;
+// Staged form: a barrier header, then one or two stages of (Q tile, K box,
+// V box).
+constexpr int GATHER_SMEM_HEADER = 128;
+// Footprints that let two CTAs share an SM, and one CTA's limit.
+constexpr int GATHER_SMEM_TWO_PER_SM = 110 * 1024;
+constexpr int GATHER_SMEM_MAX = 220 * 1024;
+inline long long gather_smem_bytes(long long qrows, long long krows, int D, int esz, int nst) {
+  return GATHER_SMEM_HEADER + nst * (qrows + 2 * krows) * D * esz;
+}
 cudaError_t launch_gather(const GatherLaunch& L, cudaStream_t stream);
 
 // 5-d TMA descriptor of a [BH, X1, X2, X3, D] tensor of input type dt (0 bf16,

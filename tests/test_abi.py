@@ -150,6 +150,26 @@ def test_auto_sends_narrow_windows_to_the_gather_kernel(window, dtype, expect):
         assert 40 * 48 <= p["chunks_loaded"] <= p["ctas"] * np.prod(window) * 256
 
 
+@pytest.mark.parametrize("grid,window,mode,d,dtype,tile", [
+    # 1-D causal, k = 4, head_dim 64: 128-query tiles fill a round of the CTA's
+    # 256 threads (two per query) and two stages of 50 KB leave room for two
+    # CTAs per SM
+    ((32768,), (5,), ["causal"], 64, "bf16", [1, 1, 128]),
+    # 2-D 5 x 5: a full 128-query tile, one stage (78 KB)
+    ((128, 128), (5, 5), None, 64, "bf16", [1, 8, 16]),
+    # a wide window: 64-query tiles with a 320-row key box fit one CTA per SM
+    ((600,), (257,), ["causal"], 128, "bf16", [1, 1, 64]),
+    # one query's 513-row key box fits no shared memory: the direct form
+    ((1200,), (513,), ["causal"], 128, "bf16", [1, 1, 1]),
+])
+def test_gather_tile_choice(grid, window, mode, d, dtype, tile):
+    import neighborhood_attention_b200 as na
+    dt = {"bf16": na.NA_BF16, "f16": na.NA_F16, "f32": na.NA_F32}[dtype]
+    opts = na.make_options(kernel=na.NA_KERNEL_GATHER, window_mode=mode, ndim=len(grid))
+    p = na.na_plan(list(grid), list(window), None, None, d, dt, options=opts)
+    assert p["kernel"] == "gather" and p["qblock"] == tile
+
+
 def test_gather_selector_takes_any_window_and_cut_modes():
     import neighborhood_attention_b200 as na
     opts = na.make_options(kernel=na.NA_KERNEL_GATHER, window_mode=["causal", "truncated"])

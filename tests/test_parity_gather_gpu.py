@@ -45,9 +45,12 @@ CASES = {
     "full1d": _case((40,), (40,), (1,), 64, dtype="f16"),
     # fp32, head_dim 128: a whole warp per query
     "f32_d128": _case((50, 6), (3, 5), (1, 1), 128, dtype="f32", mode=["causal", "clamped"]),
-    # one query's key box (257 rows of K and V at 256 bytes each) exceeds the
-    # shared-memory budget: the direct form, keys read from global memory
-    "direct1d_wide": _case((600,), (257,), (1,), 128, mode=["causal"]),
+    # a wide window whose staged tiles fit only one CTA per SM (64 queries,
+    # a 320-row key box at 256 bytes a row)
+    "wide1d_one_cta": _case((600,), (257,), (1,), 128, mode=["causal"]),
+    # one query's key box (513 rows of K and V at 256 bytes each) exceeds the
+    # shared-memory limit: the direct form, keys read from global memory
+    "direct1d_wide": _case((1200,), (513,), (1,), 128, mode=["causal"]),
 }
 
 
