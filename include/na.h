@@ -134,9 +134,11 @@ typedef struct {
   long long wait_timeout_ns;/* bound on each in-kernel wait; <= 0: 4 s (or env NA_WAIT_TIMEOUT_MS) */
   int debug_flags;          /* TESTING HOOK, not a supported option: leave it 0.  1: the
                                tensor-core forward kernel's loader withholds the first key
-                               chunk, so the consumer's bounded wait expires and the timeout
-                               path (NA_ERR_TIMEOUT from na_sync_status) is exercised without
-                               any fault or hang; the outputs of such a call are undefined. */
+                               chunk (the window-gather kernel's staged form: the copies of
+                               the first query tile), so the consumers' bounded waits expire
+                               and the timeout path (NA_ERR_TIMEOUT from na_sync_status) is
+                               exercised without any fault or hang; the outputs of such a
+                               call are undefined. */
   int window_mode[3];       /* na_window_mode of grid dimension i (i < ndim, the order of
                                `window`); entries from ndim on are ignored.  0 = clamped. */
   int dilation[3];          /* dilation of grid dimension i (i < ndim); 0 or 1 = none.  The

@@ -542,6 +542,7 @@ na_status launch_forward(const Problem& P, const DilMap& map, long long BH, cons
     G.smem_bytes = plan.gsmem;
     G.status = nullptr;
     G.timeout_ns = P.opt.wait_timeout_ns > 0 ? P.opt.wait_timeout_ns : default_timeout_ns();
+    G.debug_flags = P.opt.debug_flags;
     if (plan.gq[0] > 0) {
       st = status_word(&G.status);
       if (st != NA_OK) return st;

@@ -236,12 +236,16 @@ __device__ __forceinline__ void copy_box(const GatherLaunch& P, size_t head, con
 
 template <int RB>
 __device__ __forceinline__ void issue_tile(const GatherLaunch& P, int t, unsigned char* stage,
-                                           uint64_t* bar, int lane) {
+                                           uint64_t* bar, TileGeo* geo, int lane) {
   const TileGeo tg = tile_geo(P, t);
+  if (lane == 0) *geo = tg;   // published to the consumers by the arrive below
   const int nqt = tg.nq[0] * tg.nq[1] * tg.nq[2];
   const int rows = tg.kx[0] * tg.kx[1] * tg.kx[2];
   if (lane == 0) ptx::mbar_expect_tx(bar, (uint32_t)((nqt + 2 * rows) * RB));
   __syncwarp();
+  // Testing hook: CTA 0's first tile is announced but never copied, so the
+  // waits on it run out and the timeout path unwinds.
+  if ((P.debug_flags & 1) && t == 0) return;
   const size_t head = (size_t)tg.bh * (size_t)P.N;
   unsigned char* sK = stage + (size_t)P.qrows * RB;
   unsigned char* sV = sK + (size_t)P.krows * RB;
@@ -292,7 +296,7 @@ __device__ __forceinline__ float ex2_approx(float x) {   // 2^x, 0 at -inf
 // each phase of a warp-wide read eight different bank groups.  ONED: a 1-D
 // grid (the two outer extents 1), whose coordinates need no division.
 template <int D, int T, bool ONED>
-__device__ __forceinline__ void compute_tile(const GatherLaunch& P, const TileGeo& tg,
+__device__ __forceinline__ void compute_tile(const GatherLaunch& P, const TileGeo tg,
                                              const unsigned char* stage) {
   constexpr int VE = slice_elems<T>();       // elements per 16-byte slice
   constexpr int ESZ = T == G_F32 ? 4 : 2;
@@ -302,7 +306,7 @@ __device__ __forceinline__ void compute_tile(const GatherLaunch& P, const TileGe
   constexpr int S = E / VE;                  // slices per thread (4 or 8)
   constexpr int G = D / E;                   // threads per query (1, 2 or 4)
   constexpr int QPC = GATHER_THREADS / G;    // queries per round
-  constexpr int KPS = 2;                     // keys per online-softmax step
+  constexpr int KPS = 3;                     // keys per online-softmax step
   constexpr bool MIX = T != G_F32;
   static_assert(SPR % S == 0 && (S & (S - 1)) == 0, "slices");
   const uint4* sQ = reinterpret_cast<const uint4*>(stage);
@@ -325,7 +329,10 @@ __device__ __forceinline__ void compute_tile(const GatherLaunch& P, const TileGe
       c[0] = c[1] = 0;
       c[2] = tg.o[2] + qq;
       int hi;
-      window_range(g.L[2], g.w[2], g.s[2], g.m[2], c[2], wl[2], hi);
+      if (g.s[2] == 1)   // no division by the stride
+        window_range(g.L[2], g.w[2], 1, g.m[2], c[2], wl[2], hi);
+      else
+        window_range(g.L[2], g.w[2], g.s[2], g.m[2], c[2], wl[2], hi);
       n[2] = hi - wl[2];
       wl[2] -= tg.lo[2];
       n[0] = n[1] = 1;
@@ -478,20 +485,34 @@ __device__ __forceinline__ void compute_tile(const GatherLaunch& P, const TileGe
   }
 }
 
+// The staged form's CTA loop.  There is no CTA-wide barrier per tile: every
+// warp waits for a tile's stage to fill, computes its share of the tile and
+// counts itself done with the stage; the warp that finishes the stage last
+// refills it with the tile `nst` steps ahead.  With two stages a warp can run
+// a whole tile ahead of the slowest one.
 template <int D, int T, bool ONED>
 __global__ void __launch_bounds__(GATHER_THREADS, 2) gather_staged_kernel(const GatherLaunch P) {
   constexpr int RB = D * (T == G_F32 ? 4 : 2);
+  constexpr int NWARPS = GATHER_THREADS / 32;
   extern __shared__ __align__(128) unsigned char smem[];
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);   // one mbarrier per stage
+  // Header: a full barrier, a done count, an issue count and the geometry per stage.
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + 16);
+  int* done = reinterpret_cast<int*>(smem + 20);
+  int* issued = reinterpret_cast<int*>(smem + 28);
+  TileGeo* geo = reinterpret_cast<TileGeo*>(smem + 40);
+  static_assert(40 + 2 * sizeof(TileGeo) <= GATHER_SMEM_HEADER, "header");
   unsigned char* stage0 = smem + GATHER_SMEM_HEADER;
   const int stage_bytes = (P.qrows + 2 * P.krows) * RB;
   const int nst = P.nstages;   // 1 or 2
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int total = P.BH * P.nt[0] * P.nt[1] * P.nt[2];   // the host keeps it below 2^30
   if (threadIdx.x == 0) {
-    ptx::mbar_init(&full[0], 1);
-    ptx::mbar_init(&full[1], 1);
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      done[s] = 0;
+      issued[s] = 0;
+    }
     *abort_flag = *reinterpret_cast<volatile int*>(P.status) != 0;
     ptx::fence_mbar_init();
   }
@@ -501,30 +522,44 @@ __global__ void __launch_bounds__(GATHER_THREADS, 2) gather_staged_kernel(const 
   ctl.status = P.status;
   ctl.timeout_ns = (uint64_t)P.timeout_ns;
 
-  int t = blockIdx.x, i = 0, st = 0, par = 0;
-  bool ok = true;
-  if (warp == 0 && t < total) issue_tile<RB>(P, t, stage0, &full[0], lane);
-  for (; t < total; t += gridDim.x, ++i) {
-    st = nst == 2 ? (i & 1) : 0;
-    par = nst == 2 ? ((i >> 1) & 1) : (i & 1);
-    const bool more = t + (int)gridDim.x < total;
-    // Two stages: the other one was released by the barrier that ended the
-    // last tile, and the next tile streams in while this one is computed.
-    if (nst == 2 && warp == 0 && more)
-      issue_tile<RB>(P, t + gridDim.x, stage0 + (st ^ 1) * stage_bytes, &full[st ^ 1], lane);
-    ok = __syncthreads_and(ptx::wait(&full[st], par, ctl));
-    if (!ok) break;
-    compute_tile<D, T, ONED>(P, tile_geo(P, t), stage0 + st * stage_bytes);
-    __syncthreads();
-    // One stage: the next tile's copies start once every thread is done.
-    if (nst == 1 && warp == 0 && more) issue_tile<RB>(P, t + gridDim.x, stage0, &full[0], lane);
+  auto issue = [&](int tt, int s) {   // one warp, all lanes
+    issue_tile<RB>(P, tt, stage0 + s * stage_bytes, &full[s], &geo[s], lane);
+    if (lane == 0) ++issued[s];
+  };
+  if (warp == 0)
+    for (int s = 0; s < nst; ++s)
+      if (blockIdx.x + s * gridDim.x < (unsigned)total) issue(blockIdx.x + s * gridDim.x, s);
+
+  int i = 0;
+  for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+    const int st = nst == 2 ? (i & 1) : 0;
+    const int par = (nst == 2 ? i >> 1 : i) & 1;
+    if (!__all_sync(0xffffffffu, ptx::wait(&full[st], par, ctl))) break;
+    compute_tile<D, T, ONED>(P, geo[st], stage0 + st * stage_bytes);
+    // Release the stage; the last warp out refills it.
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+      __threadfence_block();   // this warp's reads of the stage before its count
+      last = atomicAdd(&done[st], 1) == NWARPS - 1;
+    }
+    if (__shfl_sync(0xffffffffu, last, 0)) {
+      if (lane == 0) done[st] = 0;
+      const int tn = t + nst * gridDim.x;
+      if (tn < total) {
+        __threadfence_block();
+        // Generic-proxy reads of the stage are ordered before the bulk copies' writes.
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue(tn, st);
+      }
+    }
   }
-  if (!ok && threadIdx.x == 0) {
-    // A wait gave up: the copies in flight land before shared memory goes away.
-    ptx::wait_drain(&full[st], par, ctl);
-    if (nst == 2 && t + (int)gridDim.x < total)
-      ptx::wait_drain(&full[st ^ 1], ((i + 1) >> 1) & 1, ctl);
-  }
+  // Every warp is out of its loop (a failed wait ends it early): copies still
+  // in flight land before the CTA's shared memory goes away.
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int s = 0; s < nst; ++s)
+      if (issued[s] > 0) ptx::wait_drain(&full[s], (issued[s] - 1) & 1, ctl);
 }
 
 // Direct form: no staging (a wide window); one query per thread group, every

@@ -102,11 +102,12 @@ struct GatherLaunch {
   int smem_bytes;        // staged form: header + the stages
   int* status;           // device status word
   long long timeout_ns;  // bound on every in-kernel wait
+  int debug_flags;       // testing hook: 1 = CTA 0's first tile gets no copies
 };
 
-// Staged form: a barrier header, then one or two stages of (Q tile, K box,
-// V box).
-constexpr int GATHER_SMEM_HEADER = 128;
+// Staged form: a header (barriers, tile geometry), then one or two stages of
+// (Q tile, K box, V box).
+constexpr int GATHER_SMEM_HEADER = 256;
 // Footprints that let two CTAs share an SM, and one CTA's limit.
 constexpr int GATHER_SMEM_TWO_PER_SM = 110 * 1024;
 constexpr int GATHER_SMEM_MAX = 220 * 1024;

@@ -106,3 +106,25 @@ def test_gather_uniform_queries_give_window_sizes():
                                                 dtype="bf16", mode=c["mode"])
     assert np.abs(l.reshape(-1) - ref_l.reshape(-1)).max() <= 1e-5
     assert np.abs(o.reshape(ref_o.shape) - ref_o).max() <= 1e-2
+
+
+def test_gather_bounded_wait_timeout_is_reported_and_recoverable():
+    """The testing hook announces the first query tile's copies but issues
+    none: the staged kernel's bounded waits expire, it unwinds (draining what
+    was issued), na_sync_status reports NA_ERR_TIMEOUT, and the next call on
+    the same context is correct."""
+    from gpu_parity import to_device
+    c = CASES["causal1d_k4"]
+    qkv = host_inputs(c, seed=7)
+    q, k, v = (to_device(a, c["dtype"]) for a in qkv)
+    opts = na.make_options(kernel=GATHER, window_mode=c["mode"], ndim=1,
+                           wait_timeout_ns=50_000_000, debug_flags=1)
+    assert na.na_plan(c["grid"], c["window"], c["stride"], None, c["d"], na.NA_BF16,
+                      options=opts)["qblock"] != [1, 1, 1]   # the staged form
+    na.forward(q, k, v, c["window"], c["stride"], options=opts)
+    with pytest.raises(na.NaError) as ei:
+        na.na_sync_status()
+    assert ei.value.status == na.NA_ERR_TIMEOUT
+    na.na_sync_status()  # cleared
+    o, l = run_gpu(c, qkv, kernel=GATHER)
+    assert_within(c, compare(c, qkv, o, l), "after-timeout")
