@@ -432,6 +432,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // Scores of the chunk into registers (and -inf outside the row's
         // window on partial chunks).
         auto load_scores = [&]() {
+          if (D == 64 && st == CHUNK_PARTIAL) {
+            // Scores outside the row's window become -inf in TMEM, one
+            // 32-key word at a time (a loop, not unrolled: the masked path
+            // stays small in the instruction cache); words no lane of the
+            // warp masks are skipped.
+            int lo[3], hi[3];
+            for (int d = 0; d < 3; ++d) {
+              lo[d] = imin(imax(wlo[d] - it.a[d], 0), P.kb[d]);
+              hi[d] = imin(imax(whi[d] - it.a[d], 0), P.kb[d]);
+            }
+            const int sh[3] = {P.kb_log2[1] + P.kb_log2[2], P.kb_log2[2], 0};
+#pragma unroll 1
+            for (int wd = 0; wd < 4; ++wd) {
+              uint32_t mw = 0xffffffffu;
+#pragma unroll
+              for (int d = 0; d < 3; ++d) mw &= dim_word_mask(wd, sh[d], P.kb[d], lo[d], hi[d]);
+              if (__any_sync(0xffffffffu, mw != 0xffffffffu)) {
+                uint32_t r[32];
+                ptx::tmem_ld32(tS + 32 * wd, r);
+                ptx::tmem_ld_wait();
+                ptx::reg_fence(r);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (!((mw >> j) & 1u)) r[j] = __float_as_uint(-INFINITY);
+                ptx::tmem_st32(tS + 32 * wd, r);
+              }
+            }
+            ptx::tmem_st_wait();
+          }
           ptx::tmem_ld32(tS + 0, s0);
           ptx::tmem_ld32(tS + 32, s1);
           ptx::tmem_ld32(tS + 64, s2);
@@ -441,12 +470,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           ptx::reg_fence(s1);
           ptx::reg_fence(s2);
           ptx::reg_fence(s3);
-          if (st == CHUNK_PARTIAL) {
+          if (D == 128 && st == CHUNK_PARTIAL) {
+            // At head_dim 128 the mask is applied in registers, built by
+            // the loop form (see chunk_key_mask_compact).
             uint32_t mk[4];
-            if constexpr (D == 128)
-              chunk_key_mask_compact(it.a, wlo, whi, P.kb, P.kb_log2, mk);
-            else
-              chunk_key_mask(it.a, wlo, whi, P.kb, P.kb_log2, mk);
+            chunk_key_mask_compact(it.a, wlo, whi, P.kb, P.kb_log2, mk);
 #pragma unroll
             for (int j = 0; j < 128; ++j)
               if (!((mk[j >> 5] >> (j & 31)) & 1u)) s[j] = __float_as_uint(-INFINITY);
@@ -514,25 +542,50 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // still in TMEM) only when a row's sum -- an upper bound of its largest
         // P -- exceeds P_LIMIT.  Without a reference yet (first chunk, or rows
         // masked so far) the chunk's own maximum becomes the reference first.
-        load_scores();
         float m_new = m, alpha = 1.f, sum;
         bool need = false;
-        if (__any_sync(0xffffffffu, m == -INFINITY)) {
-          const float mx2 = row_max() - C::POFF;
-          need = mx2 > m;
-          m_new = need ? mx2 : m;
-          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-          alpha = need ? ptx::ex2(m - m_use) : 1.f;
-          sum = exp_pass(m_use);
-        } else {
-          sum = exp_pass(m);
-          if (__any_sync(0xffffffffu, !(sum <= C::PLIM))) {
+        if constexpr (D == 64) {
+          // One copy of the score load, the row maximum and the exponential
+          // pass serves every path (the loop runs a second time only for a
+          // redo): at head_dim 64 the softmax loop's code then stays small
+          // enough for the instruction cache.
+          bool fresh = __any_sync(0xffffffffu, m == -INFINITY);
+#pragma unroll 1
+          for (;;) {
             load_scores();
+            float m_use = m;
+            if (fresh) {
+              const float mx2 = row_max() - C::POFF;
+              need = mx2 > m;
+              m_new = need ? mx2 : m;
+              m_use = (m_new == -INFINITY) ? 0.f : m_new;
+              alpha = need ? ptx::ex2(m - m_use) : 1.f;
+            }
+            sum = exp_pass(m_use);
+            if (fresh || !__any_sync(0xffffffffu, !(sum <= C::PLIM))) break;
+            fresh = true;
+          }
+        } else {
+          // At head_dim 128 the straight-line form (a copy of the pass per
+          // path) schedules better and the loop's code fits either way.
+          load_scores();
+          if (__any_sync(0xffffffffu, m == -INFINITY)) {
             const float mx2 = row_max() - C::POFF;
             need = mx2 > m;
             m_new = need ? mx2 : m;
-            alpha = need ? ptx::ex2(m - m_new) : 1.f;
-            sum = exp_pass(m_new);
+            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+            alpha = need ? ptx::ex2(m - m_use) : 1.f;
+            sum = exp_pass(m_use);
+          } else {
+            sum = exp_pass(m);
+            if (__any_sync(0xffffffffu, !(sum <= C::PLIM))) {
+              load_scores();
+              const float mx2 = row_max() - C::POFF;
+              need = mx2 > m;
+              m_new = need ? mx2 : m;
+              alpha = need ? ptx::ex2(m - m_new) : 1.f;
+              sum = exp_pass(m_new);
+            }
           }
         }
         const bool warp_need = __any_sync(0xffffffffu, need);
