@@ -294,8 +294,10 @@ __device__ __forceinline__ float ex2_approx(float x) {   // 2^x, 0 at -inf
 // number of 128-byte lines apart (head_dim >= 64 at 16 bits), so a 16-byte
 // read's bank group is its slice's, and the rotation gives the eight lanes of
 // each phase of a warp-wide read eight different bank groups.  ONED: a 1-D
-// grid (the two outer extents 1), whose coordinates need no division.
-template <int D, int T, bool ONED>
+// grid (the two outer extents 1), whose coordinates need no division.  KPS:
+// keys per online-softmax step (3 or 5, whichever wastes fewer slots on the
+// window; each step costs a rescale of the accumulator).
+template <int D, int T, bool ONED, int KPS>
 __device__ __forceinline__ void compute_tile(const GatherLaunch& P, const TileGeo tg,
                                              const unsigned char* stage) {
   constexpr int VE = slice_elems<T>();       // elements per 16-byte slice
@@ -306,7 +308,6 @@ __device__ __forceinline__ void compute_tile(const GatherLaunch& P, const TileGe
   constexpr int S = E / VE;                  // slices per thread (4 or 8)
   constexpr int G = D / E;                   // threads per query (1, 2 or 4)
   constexpr int QPC = GATHER_THREADS / G;    // queries per round
-  constexpr int KPS = 3;                     // keys per online-softmax step
   constexpr bool MIX = T != G_F32;
   static_assert(SPR % S == 0 && (S & (S - 1)) == 0, "slices");
   const uint4* sQ = reinterpret_cast<const uint4*>(stage);
@@ -490,7 +491,7 @@ __device__ __forceinline__ void compute_tile(const GatherLaunch& P, const TileGe
 // counts itself done with the stage; the warp that finishes the stage last
 // refills it with the tile `nst` steps ahead.  With two stages a warp can run
 // a whole tile ahead of the slowest one.
-template <int D, int T, bool ONED>
+template <int D, int T, bool ONED, int KPS>
 __global__ void __launch_bounds__(GATHER_THREADS, 2) gather_staged_kernel(const GatherLaunch P) {
   constexpr int RB = D * (T == G_F32 ? 4 : 2);
   constexpr int NWARPS = GATHER_THREADS / 32;
@@ -535,7 +536,7 @@ __global__ void __launch_bounds__(GATHER_THREADS, 2) gather_staged_kernel(const 
     const int st = nst == 2 ? (i & 1) : 0;
     const int par = (nst == 2 ? i >> 1 : i) & 1;
     if (!__all_sync(0xffffffffu, ptx::wait(&full[st], par, ctl))) break;
-    compute_tile<D, T, ONED>(P, geo[st], stage0 + st * stage_bytes);
+    compute_tile<D, T, ONED, KPS>(P, geo[st], stage0 + st * stage_bytes);
     // Release the stage; the last warp out refills it.
     __syncwarp();
     int last = 0;
@@ -620,7 +621,12 @@ cudaError_t launch_dt(const GatherLaunch& L, cudaStream_t stream) {
         L.smem_bytes != gather_smem_bytes(L.qrows, L.krows, D, esz, L.nstages) || !L.status)
       return cudaErrorInvalidValue;
     const bool oned = L.g.L[0] == 1 && L.g.L[1] == 1;
-    auto kern = oned ? gather_staged_kernel<D, T, true> : gather_staged_kernel<D, T, false>;
+    const int wk = L.g.w[0] * L.g.w[1] * L.g.w[2];   // keys of a whole window
+    const bool k5 = (wk + 4) / 5 * 5 - wk < (wk + 2) / 3 * 3 - wk;   // fewer wasted slots
+    using Kern = void (*)(GatherLaunch);
+    const Kern kerns[4] = {gather_staged_kernel<D, T, false, 3>, gather_staged_kernel<D, T, false, 5>,
+                           gather_staged_kernel<D, T, true, 3>, gather_staged_kernel<D, T, true, 5>};
+    const Kern kern = kerns[(oned ? 2 : 0) + (k5 ? 1 : 0)];
     // Per device: the shared-memory opt-in, the SM count, and the resident
     // CTAs per SM at the last footprint launched.
     static int attr_done[64] = {0}, sms[64] = {0}, occ_smem[64] = {0}, occ[64] = {0};
@@ -629,7 +635,7 @@ cudaError_t launch_dt(const GatherLaunch& L, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!attr_done[dev]) {
-      for (auto f : {gather_staged_kernel<D, T, true>, gather_staged_kernel<D, T, false>}) {
+      for (const Kern f : kerns) {
         e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, GATHER_SMEM_MAX);
         if (e != cudaSuccess) return e;
       }
@@ -639,8 +645,8 @@ cudaError_t launch_dt(const GatherLaunch& L, cudaStream_t stream) {
     }
     if (occ_smem[dev] != L.smem_bytes) {
       int nb = 0;
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, gather_staged_kernel<D, T, false>,
-                                                        GATHER_THREADS, L.smem_bytes);
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kerns[0], GATHER_THREADS,
+                                                        L.smem_bytes);
       if (e != cudaSuccess) return e;
       occ[dev] = nb > 0 ? nb : 1;
       occ_smem[dev] = L.smem_bytes;
