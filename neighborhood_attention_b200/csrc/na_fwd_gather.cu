@@ -186,9 +186,10 @@ __device__ __forceinline__ void load_q(const GatherLaunch& P, size_t off, float 
 // at work at any moment hold neighbouring tiles and share their halo rows
 // in L2.  A tile's rows -- its queries, and the K and V rows of its key box
 // (the union of its queries' windows, itself a box) -- arrive by bulk copies
-// into one of two stages while the CTA computes the tile before it from the
-// other: one copy per run of adjacent rows (a whole tile of a 1-D grid is
-// one run per tensor), completion counted in bytes on the stage's mbarrier.
+// into a stage of shared memory: one copy per run of adjacent rows (a whole
+// tile of a 1-D grid is one run per tensor), completion counted in bytes on
+// the stage's mbarrier.  With two stages (where they fit) the next tile
+// streams in while the CTA computes the current one from the other.
 struct TileGeo {
   int bh;
   int o[3], nq[3];   // first query and extent of the tile per dimension
