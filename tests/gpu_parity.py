@@ -97,7 +97,7 @@ def tile_tokens(grid, tile, tcoord):
                     dtype=np.int64)
 
 
-def survey_tiles(grid, tile):
+def corner_edge_interior_tiles(grid, tile):
     """Tile coordinates of a 3-D tile grid sampled at its 8 corner tiles, 4 tiles
     on its edges (two coordinates at a border, one inside) and 4 interior
     tiles: the places where clamped windows differ most, and the bulk."""

@@ -166,12 +166,12 @@ def test_backward_sliding_tile_full_size_tiles_of_every_head():
     window's P rounded to bf16 as the operand of dV (2^-9 P_ij per key,
     averaging over the W keys of the window)."""
     c = _case((30, 48, 80), (18, 24, 40), (6, 8, 8), 128, heads=24, tile=(6, 8, 8))
-    from gpu_parity import survey_tiles, tile_tokens
+    from gpu_parity import corner_edge_interior_tiles, tile_tokens
     host, (dq, dk, dv), dod = _full_size_grads(c, 9100)
     q, k, v, do = host
     N = int(np.prod(c["grid"]))
     W = int(np.prod(c["window"]))
-    corners, edges, interior = survey_tiles(c["grid"], c["tile"])
+    corners, edges, interior = corner_edge_interior_tiles(c["grid"], c["tile"])
     qrows = np.concatenate([tile_tokens(c["grid"], c["tile"], t)[::48]
                             for t in corners + edges + interior])
     key_tiles = corners + edges + interior[:2] + corners[::-1] + edges[:2]

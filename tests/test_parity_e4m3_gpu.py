@@ -36,7 +36,7 @@ if not torch.cuda.is_available():  # pragma: no cover - CPU machines skip the mo
 import neighborhood_attention_b200 as na  # noqa: E402
 import oracle  # noqa: E402
 import seeded_inputs  # noqa: E402
-from gpu_parity import CONFIGS, sample_rows, survey_tiles, tile_tokens  # noqa: E402
+from gpu_parity import CONFIGS, sample_rows, corner_edge_interior_tiles, tile_tokens  # noqa: E402
 
 
 def _decode(bits):
@@ -143,7 +143,7 @@ def test_e4m3_sliding_tile_full_size_tiles():
     qkv = seeded_inputs.qkv(7400, c["B"], c["heads"], c["grid"], c["d"], "e4m3")
     o, l = _run(c, qkv)
     N = int(np.prod(c["grid"]))
-    corners, edges, interior = survey_tiles(c["grid"], c["tile"])
+    corners, edges, interior = corner_edge_interior_tiles(c["grid"], c["tile"])
     toks = np.concatenate([tile_tokens(c["grid"], c["tile"], t)
                            for t in corners + edges + interior])
     BH = c["B"] * c["heads"]

@@ -17,7 +17,7 @@ if not torch.cuda.is_available():  # pragma: no cover - CPU machines skip the mo
 
 import neighborhood_attention_b200 as na  # noqa: E402
 from gpu_parity import (CONFIGS, assert_within, compare, host_inputs, run_gpu,  # noqa: E402
-                        sample_rows, seed_for, survey_tiles, tile_tokens)
+                        sample_rows, seed_for, corner_edge_interior_tiles, tile_tokens)
 
 SIMT, TC = na.NA_KERNEL_SIMT, na.NA_KERNEL_TC
 
@@ -88,7 +88,7 @@ def test_sliding_tile_full_size_tiles_of_every_head():
     c = CONFIGS[4]
     qkv = host_inputs(c, seed_for(4))
     N = int(np.prod(c["grid"]))
-    corners, edges, interior = survey_tiles(c["grid"], c["tile"])
+    corners, edges, interior = corner_edge_interior_tiles(c["grid"], c["tile"])
     toks = np.concatenate([tile_tokens(c["grid"], c["tile"], t)
                            for t in corners + edges + interior])
     BH = c["B"] * c["heads"]
