@@ -329,3 +329,60 @@ def test_e4m3_plans_on_the_tensor_cores_only():
     with pytest.raises(na.NaError) as e:
         na.na_plan([16, 16], [5, 5], None, None, 64, 4)
     assert e.value.status == na.NA_ERR_INVALID_ARG
+
+
+def _gather_box_extent(L, w, s, mode, t):
+    """Largest key-box extent along one dimension over query tiles of extent t
+    (the union of the windows of the tile's first and last query), from the
+    oracle's window rule."""
+    import oracle
+    best = 0
+    for o in range(0, L, t):
+        n = min(t, L - o)
+        lo, _ = oracle.window(L, w, s, mode, o)
+        _, hi = oracle.window(L, w, s, mode, o + n - 1)
+        best = max(best, hi - lo)
+    return best
+
+
+def test_gather_tiles_fit_shared_memory_on_random_problems():
+    """On random 1-, 2- and 3-D problems the window-gather plan's query tile is
+    a box of 2^k <= 256 queries no wider than the grid needs whose staged rows
+    (the tile's queries plus its largest K and V key boxes) fit one CTA's
+    shared memory (220 KB with a 256-byte header); when it falls back to
+    direct reads, not even a one-query tile fits."""
+    import numpy as np
+    import neighborhood_attention_b200 as na
+    rng = np.random.default_rng(1234)
+    modes = ["clamped", "truncated", "causal"]
+    for _ in range(60):
+        nd = int(rng.integers(1, 4))
+        grid = [int(rng.integers(1, 70)) for _ in range(nd)]
+        window = [int(rng.integers(1, g + 1)) for g in grid]
+        stride = [int(rng.integers(1, w + 1)) for w in window]
+        mode = [modes[int(rng.integers(0, 3))] for _ in range(nd)]
+        d = int(rng.choice([32, 64, 128]))
+        dtype, esz = [(na.NA_BF16, 2), (na.NA_F16, 2), (na.NA_F32, 4)][int(rng.integers(0, 3))]
+        opts = na.make_options(kernel=na.NA_KERNEL_GATHER, window_mode=mode, ndim=nd)
+        p = na.na_plan(grid, window, stride, None, d, dtype, options=opts)
+        assert p["kernel"] == "gather"
+        g3 = [1] * (3 - nd) + grid
+        w3 = [1] * (3 - nd) + window
+        s3 = [1] * (3 - nd) + stride
+        m3 = ["clamped"] * (3 - nd) + mode
+        t = p["qblock"]
+
+        def footprint(tile):
+            q = int(np.prod([min(tile[i], g3[i]) for i in range(3)]))
+            k = int(np.prod([_gather_box_extent(g3[i], w3[i], s3[i], m3[i], tile[i])
+                             for i in range(3)]))
+            return 256 + (q + 2 * k) * d * esz
+
+        # the direct form reports CTAs of several query rows each; the staged
+        # form one CTA-unit per tile (a 1 x 1 x 1 tile: one per token)
+        if t == [1, 1, 1] and p["ctas"] < int(np.prod(grid)):
+            assert footprint([1, 1, 1]) > 220 * 1024, (grid, window, stride, mode, d)
+            continue
+        assert all(x >= 1 and (x & (x - 1)) == 0 for x in t) and int(np.prod(t)) <= 256
+        assert all(t[i] == 1 or t[i] // 2 < g3[i] for i in range(3)), (t, g3)
+        assert footprint(t) <= 220 * 1024, (grid, window, stride, mode, d, t)
