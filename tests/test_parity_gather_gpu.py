@@ -128,3 +128,33 @@ def test_gather_bounded_wait_timeout_is_reported_and_recoverable():
     na.na_sync_status()  # cleared
     o, l = run_gpu(c, qkv, kernel=GATHER)
     assert_within(c, compare(c, qkv, o, l), "after-timeout")
+
+
+def _random_case(seed):
+    """A seeded random problem: 1-3 dimensions, any window mode, stride and
+    dilation the API accepts, every input type and head_dim."""
+    rng = np.random.default_rng(seed)
+    nd = int(rng.integers(1, 4))
+    cap = {1: 400, 2: 40, 3: 14}[nd]
+    grid = [int(rng.integers(3, cap + 1)) for _ in range(nd)]
+    dil = [int(rng.integers(1, 3)) if g >= 8 else 1 for g in grid]
+    window = [int(rng.integers(1, max(1, g // dl) + 1)) for g, dl in zip(grid, dil)]
+    stride = [int(rng.integers(1, w + 1)) for w in window]
+    mode = [["clamped", "truncated", "causal"][int(rng.integers(0, 3))] for _ in range(nd)]
+    d = int(rng.choice([32, 64, 128]))
+    dtype = ["bf16", "f16", "f32"][int(rng.integers(0, 3))]
+    c = _case(grid, window, stride, d, dtype=dtype, heads=int(rng.integers(1, 3)), mode=mode)
+    if any(x > 1 for x in dil):
+        c["dil"] = tuple(dil)
+    return c
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_gather_random_problems(seed):
+    """Seeded random problems through the window-gather kernel (staged or
+    direct form, one or two stages, three or five keys per step, as the plan
+    picks), every output against the oracle."""
+    c = _random_case(4100 + seed)
+    qkv = host_inputs(c, seed=4200 + seed)
+    o, l = run_gpu(c, qkv, kernel=GATHER)
+    assert_within(c, compare(c, qkv, o, l), f"random {seed}: {c}")
