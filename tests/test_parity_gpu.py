@@ -165,3 +165,31 @@ def test_bounded_wait_timeout_is_reported_and_recoverable():
     na.na_sync_status()  # cleared
     o, l = run_gpu(c, qkv, kernel=TC)
     assert_within(c, compare(c, qkv, o, l), "after-timeout")
+
+
+def _random_tc_case(seed):
+    """A seeded random problem for the tensor-core kernel: 1-3 dimensions,
+    windows from a few keys to the whole grid (partial chunks on most
+    blocks), any stride and window mode, bf16 or f16, head_dim 64 or 128."""
+    rng = np.random.default_rng(seed)
+    nd = int(rng.integers(1, 4))
+    cap = {1: 1500, 2: 48, 3: 14}[nd]
+    grid = [int(rng.integers(4, cap + 1)) for _ in range(nd)]
+    window = [int(rng.integers(2, g + 1)) for g in grid]
+    stride = [int(rng.integers(1, w + 1)) for w in window]
+    mode = [["clamped", "truncated", "causal"][int(rng.integers(0, 3))] for _ in range(nd)]
+    c = _case(grid, window, stride, int(rng.choice([64, 128])),
+              dtype=["bf16", "f16"][int(rng.integers(0, 2))], heads=int(rng.integers(1, 3)))
+    c["mode"] = mode
+    return c
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_tc_random_problems(seed):
+    """Seeded random problems through the tensor-core kernel (full and
+    partial chunks, masked in tensor memory at head_dim 64 and in registers
+    at 128), every output against the oracle."""
+    c = _random_tc_case(5100 + seed)
+    qkv = host_inputs(c, seed=5200 + seed)
+    o, l = run_gpu(c, qkv, kernel=TC)
+    assert_within(c, compare(c, qkv, o, l), f"random {seed}: {c}")
