@@ -211,3 +211,27 @@ def test_backward_local3d_full_size_sampled():
         b, h = divmod(bh, c["heads"])
         got = [_rows_of(t, b, h, N, c["d"], rows) for t in (dq, dk, dv)]
         _assert_close(c, got, (rq, rk, rv), f"local3d bh={bh}")
+
+
+def _random_bwd_case(seed):
+    """A seeded random backward problem: 1-3 dimensions, any window mode and
+    stride, bf16 or f16 at head_dim 64 / 128 (tensor cores) or fp32 at 32."""
+    rng = np.random.default_rng(seed)
+    nd = int(rng.integers(1, 4))
+    cap = {1: 600, 2: 30, 3: 10}[nd]
+    grid = [int(rng.integers(3, cap + 1)) for _ in range(nd)]
+    window = [int(rng.integers(1, g + 1)) for g in grid]
+    stride = [int(rng.integers(1, w + 1)) for w in window]
+    mode = [["clamped", "truncated", "causal"][int(rng.integers(0, 3))] for _ in range(nd)]
+    kind = int(rng.integers(0, 3))
+    d, dtype = [(64, "bf16"), (128, "f16"), (32, "f32")][kind]
+    return _case(grid, window, stride, d, dtype=dtype, heads=int(rng.integers(1, 3)), mode=mode)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_backward_random_problems(seed):
+    """Seeded random problems through the default backward path, dq / dk / dv
+    against the oracle's gradients."""
+    c = _random_bwd_case(6100 + seed)
+    got, ref = _run(c, seed=6200 + seed)
+    _assert_close(c, got, ref, f"random {seed}: {c}")
