@@ -196,3 +196,22 @@ def test_e4m3_refusals():
     with pytest.raises(na.NaError) as e:
         na.forward(q32, q32, q32, (3, 3))
     assert e.value.status == na.NA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_e4m3_random_problems(seed):
+    """Seeded random problems with E4M3 inputs (1-3 dimensions, any window
+    mode and stride, head_dim 64 or 128), every row against the oracle."""
+    rng = np.random.default_rng(7700 + seed)
+    nd = int(rng.integers(1, 4))
+    cap = {1: 900, 2: 40, 3: 12}[nd]
+    grid = tuple(int(rng.integers(4, cap + 1)) for _ in range(nd))
+    window = tuple(int(rng.integers(2, g + 1)) for g in grid)
+    stride = tuple(int(rng.integers(1, w + 1)) for w in window)
+    mode = [["clamped", "truncated", "causal"][int(rng.integers(0, 3))] for _ in range(nd)]
+    c = _case(grid, window, stride, int(rng.choice([64, 128])), heads=int(rng.integers(1, 3)),
+              mode=mode)
+    qkv = seeded_inputs.qkv(7800 + seed, c["B"], c["heads"], c["grid"], c["d"], "e4m3")
+    o, l = _run(c, qkv)
+    rows = np.arange(c["B"] * c["heads"] * int(np.prod(c["grid"])), dtype=np.int64)
+    _check(c, qkv, o, l, rows, f"random {seed}: {c}")
